@@ -1,0 +1,127 @@
+/*
+ * kda.h - C ABI of the B200 (sm_100a) Kimi Delta Attention library (libkda.so).
+ *
+ * The operator (Kimi Linear summary page, th.news.hada.io topic 31936):
+ *   per (sequence, head), state S in R^{dk x dv}, channel-wise gate alpha_t = exp(log_alpha_t),
+ *       S_t = (I - beta_t k_t k_t^T) Diag(alpha_t) S_{t-1} + beta_t k_t v_t^T,   o_t = S_t^T q_t.
+ *   - section "From linear attention to Gated DeltaNet": the delta rule and the gate;
+ *   - section "Fine-grained memory control of KDA": the diagonal (channel-wise) gate inside a
+ *     DPLR transition consistent with the delta rule;
+ *   - section "Reduced computation vs general DPLR": both DPLR vectors tied to k, so a chunk
+ *     needs only two decayed Gram matrices (k-k and q-k);
+ *   - section "Chunkwise parallel algorithm": fixed-length chunks passing their final state on,
+ *     WY packing of the rank-1 updates, the UT transform (I + A)^-1 by forward substitution,
+ *     and an output mixing the inter-chunk state with intra-chunk parallel work.
+ * No output scale is applied (the pages give none).  log_alpha is a natural log and must be <= 0.
+ *
+ * Conventions shared by every entry point
+ *   - All tensor pointers are DEVICE pointers owned by the caller.  The library allocates no
+ *     device memory per call; the caller passes any workspace.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t passed as void*; NULL = legacy default
+ *     stream).  Errors that the host can detect are returned before anything is launched.
+ *     Errors found on the device (malformed cu_seqlens, a bounded wait that ran out) are
+ *     written to a status word inside the workspace and read back with kda_get_status().
+ *   - Layouts are dense, row-major, token-major:
+ *       q, k, log_alpha : [B, T, H, dk]      v, o : [B, T, H, dv]      beta : [B, T, H]
+ *       states h0, h_T, S : [N, H, dk, dv] fp32, S[i][j] with i the key channel.
+ *   - Every pointer must be 16-byte aligned.
+ *   - The result is deterministic: two calls with the same inputs give identical bits.
+ */
+#ifndef KDA_H
+#define KDA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define KDA_API __attribute__((visibility("default")))
+#else
+#define KDA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Element type of q, k, v and o.  log_alpha, beta and every state are always fp32. */
+typedef enum { KDA_F32 = 0, KDA_BF16 = 1 } kda_dtype;
+
+/* Status codes.  0 is success; all errors are negative. */
+enum {
+    KDA_OK = 0,
+    KDA_ERR_NULL_ARG = -1,            /* a required pointer is NULL */
+    KDA_ERR_BAD_SHAPE = -2,           /* a size is <= 0, inconsistent, or too large */
+    KDA_ERR_BAD_DTYPE = -3,           /* dtype is not a kda_dtype */
+    KDA_ERR_MISALIGNED = -4,          /* a pointer is not 16-byte aligned */
+    KDA_ERR_UNSUPPORTED = -5,         /* valid but not implemented (head dim, chunk size) */
+    KDA_ERR_BAD_SEQLENS = -6,         /* device-detected: cu_seqlens not 0..T non-decreasing */
+    KDA_ERR_WORKSPACE_TOO_SMALL = -7, /* workspace_bytes < kda_chunk_fwd_workspace_size() */
+    KDA_ERR_CUDA = -8,                /* a CUDA runtime call failed (launch or query) */
+    KDA_ERR_TIMEOUT = -9,             /* device-detected: a bounded wait gave up */
+    KDA_ERR_ALIASING = -10            /* o overlaps an input, or h_T partially overlaps h0 */
+};
+
+/* Bytes of device workspace kda_chunk_fwd needs for these sizes (dtype-dependent).  It holds
+ * the device status word, the varlen chunk table and the per-chunk WY operands handed from
+ * the intra-chunk kernel to the state-passing kernel.  Returns 0 for unsupported sizes.
+ * num_seqs is N (= B without cu_seqlens). */
+KDA_API size_t kda_chunk_fwd_workspace_size(int B, int T, int H, int dk, int dv, int num_seqs,
+                                    int chunk_size, kda_dtype dtype);
+
+/* Chunkwise-parallel KDA forward (prefill).
+ *   q, k      : [B, T, H, dk] dtype           v : [B, T, H, dv] dtype
+ *   log_alpha : [B, T, H, dk] fp32 (<= 0)     beta : [B, T, H] fp32
+ *   h0        : [N, H, dk, dv] fp32 initial states, or NULL for zero states
+ *   cu_seqlens: device int32 [N + 1] token offsets of N packed sequences (then B must be 1,
+ *               cu_seqlens[0] = 0, non-decreasing, cu_seqlens[N] = T; chunks never cross a
+ *               sequence boundary), or NULL (then N = B and each batch row is one sequence).
+ *   chunk_size: must be 64.
+ *   o         : [B, T, H, dv] dtype output; must not overlap any input.
+ *   h_T       : [N, H, dk, dv] fp32 final states, or NULL.  h_T == h0 (exact alias) is
+ *               allowed and continues a sequence in place; any other overlap is rejected.
+ *   workspace : device buffer of at least kda_chunk_fwd_workspace_size(...) bytes, 256-byte
+ *               aligned; contents on entry are ignored.  Must not be shared by calls that
+ *               can run concurrently.
+ * Supported: dk = dv = 128 with dtype BF16 (tensor-core path) or F32; dk = dv = 64 with F32 or
+ * BF16 (CUDA-core path).  Returns KDA_OK once the work is enqueued. */
+KDA_API int kda_chunk_fwd(const void *q, const void *k, const void *v, const float *log_alpha,
+                  const float *beta, const float *h0, const int32_t *cu_seqlens, int num_seqs,
+                  int B, int T, int H, int dk, int dv, int chunk_size, kda_dtype dtype, void *o,
+                  float *h_T, void *workspace, size_t workspace_bytes, void *stream);
+
+/* One recurrent decode step for N*H independent states, updated in place:
+ *   S' = Diag(exp(log_alpha)) S;  u = beta (v - S'^T k);  S <- S' + k u^T;  o = S^T q.
+ *   q, k      : [N, H, dk] dtype     v, o : [N, H, dv] dtype
+ *   log_alpha : [N, H, dk] fp32      beta : [N, H] fp32      S : [N, H, dk, dv] fp32 in/out
+ * Supported: dk = dv in {64, 128}.  Needs no workspace and detects no device errors. */
+KDA_API int kda_decode_step(const void *q, const void *k, const void *v, const float *log_alpha,
+                    const float *beta, float *S, int N, int H, int dk, int dv, kda_dtype dtype,
+                    void *o, void *stream);
+
+/* Synchronizes `stream`, reads the device status word kept in `workspace` by the last
+ * kda_chunk_fwd that used it, clears it, and returns it (KDA_OK, KDA_ERR_BAD_SEQLENS or
+ * KDA_ERR_TIMEOUT), or KDA_ERR_CUDA if the synchronization itself failed. */
+KDA_API int kda_get_status(void *workspace, void *stream);
+
+/* Static, human-readable name of a status code. */
+KDA_API const char *kda_status_string(int status);
+
+/* Diagnostics (not needed to compute anything): per-kernel device timing for benchmarks and
+ * profiling.  After kda_trace_begin(max_kernels), each kernel the library launches (up to
+ * max_kernels of them) is bracketed by a pair of CUDA events recorded on its stream.
+ * kda_trace_end() synchronizes the device, stops recording, writes up to `capacity` entries of
+ * (kernel id, milliseconds) into kernel_ids / ms and returns how many kernels were recorded (or
+ * KDA_ERR_CUDA).  Kernel ids: 0 varlen chunk table, 1 intra-chunk WY kernel (tensor cores),
+ * 2 state-passing kernel (tensor cores), 3 chunkwise kernel (CUDA cores), 4 decode step.
+ * Process-wide and not thread-safe; events are owned by the library. */
+KDA_API int kda_trace_begin(int max_kernels);
+KDA_API int kda_trace_end(int *kernel_ids, float *ms, int capacity);
+
+/* Library version as an integer (major * 10000 + minor * 100 + patch). */
+KDA_API int kda_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KDA_H */

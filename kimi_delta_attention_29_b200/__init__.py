@@ -1,0 +1,135 @@
+"""B200 (sm_100a) Kimi Delta Attention: chunkwise prefill and recurrent decode.
+
+The Python functions below share their names with the C ABI in include/kda.h and only
+marshal arguments (tensor pointers, sizes, the current CUDA stream) into libkda.so.  torch is
+used for device memory and streams; every step of the method runs in the library's kernels.
+"""
+from __future__ import annotations
+
+import ctypes
+
+from . import _lib
+from ._lib import KdaError, status_string  # noqa: F401
+
+__all__ = ["kda_chunk_fwd", "kda_chunk_fwd_workspace_size", "kda_decode_step", "kda_get_status",
+           "kda_status_string", "kda_trace_begin", "kda_trace_end", "KdaError", "Workspace"]
+
+
+def _torch():
+    import torch
+    return torch
+
+
+def _dtype_code(dt) -> int:
+    torch = _torch()
+    if dt == torch.bfloat16:
+        return _lib.KDA_BF16
+    if dt == torch.float32:
+        return _lib.KDA_F32
+    return 99  # rejected by the library as KDA_ERR_BAD_DTYPE
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not t.is_contiguous():
+        raise ValueError("KDA tensors must be contiguous (dense row-major layout)")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream, device):
+    torch = _torch()
+    s = stream if stream is not None else torch.cuda.current_stream(device)
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def kda_status_string(code: int) -> str:
+    return status_string(code)
+
+
+def kda_chunk_fwd_workspace_size(B: int, T: int, H: int, dk: int, dv: int, num_seqs: int,
+                                 chunk_size: int = 64, dtype=None) -> int:
+    torch = _torch()
+    code = _dtype_code(dtype if dtype is not None else torch.bfloat16)
+    return int(_lib.load().kda_chunk_fwd_workspace_size(B, T, H, dk, dv, num_seqs, chunk_size, code))
+
+
+class Workspace:
+    """A reusable device workspace for kda_chunk_fwd (grows on demand, never shrinks)."""
+
+    def __init__(self, device="cuda"):
+        self.device = device
+        self.buf = None
+
+    def get(self, nbytes: int):
+        torch = _torch()
+        if self.buf is None or self.buf.numel() < nbytes:
+            self.buf = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=self.device)
+        return self.buf
+
+
+def kda_chunk_fwd(q, k, v, log_alpha, beta, h0=None, cu_seqlens=None, chunk_size: int = 64, o=None,
+                  h_T=None, output_final_state: bool = True, workspace=None, stream=None):
+    """Chunkwise KDA forward.  q, k [B,T,H,dk], v [B,T,H,dv] (bf16 or fp32), log_alpha [B,T,H,dk]
+    fp32, beta [B,T,H] fp32, h0 [N,H,dk,dv] fp32 or None, cu_seqlens int32 [N+1] (device) or None.
+    Returns (o, h_T); h_T is None when output_final_state is False and none was passed."""
+    torch = _torch()
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    N = B if cu_seqlens is None else cu_seqlens.numel() - 1
+    if o is None:
+        o = torch.empty((B, T, H, dv), dtype=q.dtype, device=q.device)
+    if h_T is None and output_final_state:
+        h_T = torch.empty((N, H, dk, dv), dtype=torch.float32, device=q.device)
+    code = _dtype_code(q.dtype)
+    need = int(_lib.load().kda_chunk_fwd_workspace_size(B, T, H, dk, dv, N, chunk_size, code))
+    if isinstance(workspace, Workspace):
+        ws = workspace.get(need)
+    elif workspace is None:
+        ws = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
+    else:
+        ws = workspace
+    rc = _lib.load().kda_chunk_fwd(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(h0), _ptr(cu_seqlens), N, B, T, H,
+        dk, dv, chunk_size, code, _ptr(o), _ptr(h_T), _ptr(ws), ws.numel() * ws.element_size(),
+        _stream(stream, q.device))
+    if rc != _lib.KDA_OK:
+        raise KdaError(rc, "kda_chunk_fwd")
+    return o, h_T
+
+
+def kda_get_status(workspace, stream=None) -> int:
+    buf = workspace.buf if isinstance(workspace, Workspace) else workspace
+    return int(_lib.load().kda_get_status(_ptr(buf), _stream(stream, buf.device)))
+
+
+def kda_decode_step(q, k, v, log_alpha, beta, S, o=None, stream=None):
+    """One recurrent step on S [N,H,dk,dv] fp32 (updated in place).  q, k [N,H,dk], v [N,H,dv],
+    log_alpha [N,H,dk] fp32, beta [N,H] fp32.  Returns o [N,H,dv]."""
+    torch = _torch()
+    N, H, dk = q.shape
+    dv = v.shape[-1]
+    if o is None:
+        o = torch.empty((N, H, dv), dtype=q.dtype, device=q.device)
+    rc = _lib.load().kda_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(S), N, H,
+                                     dk, dv, _dtype_code(q.dtype), _ptr(o), _stream(stream, q.device))
+    if rc != _lib.KDA_OK:
+        raise KdaError(rc, "kda_decode_step")
+    return o
+
+
+def kda_trace_begin(max_kernels: int) -> None:
+    """Start per-kernel device timing for the next `max_kernels` library kernels (diagnostics)."""
+    rc = _lib.load().kda_trace_begin(int(max_kernels))
+    if rc != _lib.KDA_OK:
+        raise KdaError(rc, "kda_trace_begin")
+
+
+def kda_trace_end(capacity: int = 4096) -> list[tuple[str, float]]:
+    """Synchronize, stop tracing and return [(kernel name, milliseconds), ...] in launch order."""
+    ids = (ctypes.c_int * capacity)()
+    ms = (ctypes.c_float * capacity)()
+    n = _lib.load().kda_trace_end(ids, ms, capacity)
+    if n < 0:
+        raise KdaError(n, "kda_trace_end")
+    return [(_lib.KERNEL_NAMES.get(ids[i], str(ids[i])), float(ms[i])) for i in range(min(n, capacity))]

@@ -1,0 +1,228 @@
+// C ABI of the KDA library: argument validation (before any launch), workspace sizing and
+// dispatch to the kernels.  See include/kda.h for the contract of every entry point.
+#include <cstdint>
+#include <cstring>
+#include <vector>
+
+#include "kda_common.cuh"
+
+namespace {
+
+constexpr size_t kStatusBytes = 256;  // status word + padding at the head of the workspace
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+struct Range {
+    uintptr_t lo, hi;  // [lo, hi)
+};
+Range range_of(const void *p, size_t bytes) {
+    const uintptr_t a = reinterpret_cast<uintptr_t>(p);
+    return Range{a, a + bytes};
+}
+bool overlaps(const Range &a, const Range &b) {
+    return a.lo < b.hi && b.lo < a.hi && a.lo != a.hi && b.lo != b.hi;
+}
+
+bool supported_dims(int dk, int dv) { return (dk == 128 && dv == 128) || (dk == 64 && dv == 64); }
+
+bool uses_tensor_cores(int dk, int dv, kda_dtype dtype) {
+    return dtype == KDA_BF16 && dk == 128 && dv == 128;
+}
+
+size_t elem_size(kda_dtype d) { return d == KDA_BF16 ? 2 : 4; }
+
+// Shape checks common to the prefill entry points.  Returns KDA_OK or an error code.
+int check_prefill_shape(int B, int T, int H, int dk, int dv, int num_seqs, bool varlen, int chunk) {
+    if (B <= 0 || T < 0 || H <= 0 || dk <= 0 || dv <= 0 || num_seqs <= 0) return KDA_ERR_BAD_SHAPE;
+    if (varlen ? (B != 1) : (num_seqs != B)) return KDA_ERR_BAD_SHAPE;
+    const int64_t tokens = (int64_t)B * T;
+    if (tokens * H * (int64_t)(dk > dv ? dk : dv) > ((int64_t)1 << 40)) return KDA_ERR_BAD_SHAPE;
+    if (tokens > INT32_MAX || (int64_t)num_seqs * H > INT32_MAX / 4) return KDA_ERR_BAD_SHAPE;
+    if (chunk != kda::kChunk) return KDA_ERR_UNSUPPORTED;
+    if (!supported_dims(dk, dv)) return KDA_ERR_UNSUPPORTED;
+    return KDA_OK;
+}
+
+}  // namespace
+
+// ------------------------------------------------------------------ per-kernel timing diagnostics
+namespace kda {
+namespace {
+struct TraceState {
+    bool on = false;
+    int capacity = 0, used = 0;
+    std::vector<cudaEvent_t> ev;  // 2 per kernel
+    std::vector<int> ids;
+};
+TraceState g_trace;
+}  // namespace
+
+void trace_before(int kernel_id, cudaStream_t stream) {
+    if (!g_trace.on || g_trace.used >= g_trace.capacity) return;
+    g_trace.ids[g_trace.used] = kernel_id;
+    cudaEventRecord(g_trace.ev[2 * g_trace.used], stream);
+}
+void trace_after(cudaStream_t stream) {
+    if (!g_trace.on || g_trace.used >= g_trace.capacity) return;
+    cudaEventRecord(g_trace.ev[2 * g_trace.used + 1], stream);
+    ++g_trace.used;
+}
+}  // namespace kda
+
+extern "C" {
+
+int kda_trace_begin(int max_kernels) {
+    using kda::g_trace;
+    if (max_kernels <= 0) return KDA_ERR_BAD_SHAPE;
+    if ((int)g_trace.ev.size() < 2 * max_kernels) {
+        const size_t old = g_trace.ev.size();
+        g_trace.ev.resize(2 * (size_t)max_kernels);
+        for (size_t i = old; i < g_trace.ev.size(); ++i)
+            if (cudaEventCreate(&g_trace.ev[i]) != cudaSuccess) {
+                g_trace.ev.resize(i);
+                return KDA_ERR_CUDA;
+            }
+    }
+    g_trace.ids.assign(max_kernels, -1);
+    g_trace.capacity = max_kernels;
+    g_trace.used = 0;
+    g_trace.on = true;
+    return KDA_OK;
+}
+
+int kda_trace_end(int *kernel_ids, float *ms, int capacity) {
+    using kda::g_trace;
+    g_trace.on = false;
+    if (cudaDeviceSynchronize() != cudaSuccess) return KDA_ERR_CUDA;
+    const int n = g_trace.used;
+    for (int i = 0; i < n && i < capacity; ++i) {
+        float t = 0.f;
+        if (cudaEventElapsedTime(&t, g_trace.ev[2 * i], g_trace.ev[2 * i + 1]) != cudaSuccess) return KDA_ERR_CUDA;
+        if (kernel_ids) kernel_ids[i] = g_trace.ids[i];
+        if (ms) ms[i] = t;
+    }
+    return n;
+}
+
+
+int kda_version(void) { return 100; }
+
+const char *kda_status_string(int status) {
+    switch (status) {
+        case KDA_OK: return "KDA_OK";
+        case KDA_ERR_NULL_ARG: return "KDA_ERR_NULL_ARG: a required pointer is NULL";
+        case KDA_ERR_BAD_SHAPE: return "KDA_ERR_BAD_SHAPE: a size is invalid or inconsistent";
+        case KDA_ERR_BAD_DTYPE: return "KDA_ERR_BAD_DTYPE: unknown element type";
+        case KDA_ERR_MISALIGNED: return "KDA_ERR_MISALIGNED: a pointer is not 16-byte aligned";
+        case KDA_ERR_UNSUPPORTED: return "KDA_ERR_UNSUPPORTED: head dim or chunk size not implemented";
+        case KDA_ERR_BAD_SEQLENS: return "KDA_ERR_BAD_SEQLENS: cu_seqlens is not 0..T non-decreasing";
+        case KDA_ERR_WORKSPACE_TOO_SMALL: return "KDA_ERR_WORKSPACE_TOO_SMALL: workspace below the required size";
+        case KDA_ERR_CUDA: return "KDA_ERR_CUDA: a CUDA runtime call failed";
+        case KDA_ERR_TIMEOUT: return "KDA_ERR_TIMEOUT: a bounded device wait gave up";
+        case KDA_ERR_ALIASING: return "KDA_ERR_ALIASING: an output overlaps an input";
+        default: return "KDA: unknown status";
+    }
+}
+
+size_t kda_chunk_fwd_workspace_size(int B, int T, int H, int dk, int dv, int num_seqs, int chunk_size,
+                                    kda_dtype dtype) {
+    if (dtype != KDA_F32 && dtype != KDA_BF16) return 0;
+    // Varlen-ness does not change validity here beyond B; size for the larger (varlen) table.
+    const bool varlen = (B == 1 && num_seqs > 1);
+    if (check_prefill_shape(B, T, H, dk, dv, num_seqs, varlen, chunk_size) != KDA_OK) return 0;
+    // The tensor-core path's layout starts with the same 256-byte status block.
+    if (uses_tensor_cores(dk, dv, dtype)) return kda::prefill_tc_workspace_bytes(B, T, H, num_seqs, true);
+    return kStatusBytes;
+}
+
+int kda_chunk_fwd(const void *q, const void *k, const void *v, const float *log_alpha, const float *beta,
+                  const float *h0, const int32_t *cu_seqlens, int num_seqs, int B, int T, int H, int dk,
+                  int dv, int chunk_size, kda_dtype dtype, void *o, float *h_T, void *workspace,
+                  size_t workspace_bytes, void *stream_) {
+    if (dtype != KDA_F32 && dtype != KDA_BF16) return KDA_ERR_BAD_DTYPE;
+    if (!q || !k || !v || !log_alpha || !beta || !o || !workspace) return KDA_ERR_NULL_ARG;
+    const bool varlen = cu_seqlens != nullptr;
+    int rc = check_prefill_shape(B, T, H, dk, dv, num_seqs, varlen, chunk_size);
+    if (rc != KDA_OK) return rc;
+    const void *ptrs[] = {q, k, v, log_alpha, beta, h0, cu_seqlens, o, h_T};
+    for (const void *p : ptrs)
+        if (p && !aligned16(p)) return KDA_ERR_MISALIGNED;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return KDA_ERR_MISALIGNED;
+
+    const size_t es = elem_size(dtype);
+    const size_t tok = (size_t)B * T * H;
+    const size_t sbytes = (size_t)num_seqs * H * dk * dv * sizeof(float);
+    const Range ro = range_of(o, tok * dv * es);
+    const Range inputs[] = {range_of(q, tok * dk * es), range_of(k, tok * dk * es), range_of(v, tok * dv * es),
+                            range_of(log_alpha, tok * dk * 4), range_of(beta, tok * 4),
+                            range_of(h0, h0 ? sbytes : 0),
+                            range_of(cu_seqlens, cu_seqlens ? (size_t)(num_seqs + 1) * 4 : 0)};
+    for (const Range &r : inputs)
+        if (overlaps(ro, r)) return KDA_ERR_ALIASING;
+    if (h_T) {
+        const Range rh = range_of(h_T, sbytes);
+        if (overlaps(rh, ro)) return KDA_ERR_ALIASING;
+        for (int i = 0; i < 5; ++i)
+            if (overlaps(rh, inputs[i])) return KDA_ERR_ALIASING;
+        if (overlaps(rh, inputs[6])) return KDA_ERR_ALIASING;
+        if (h0 && h_T != h0 && overlaps(rh, inputs[5])) return KDA_ERR_ALIASING;
+    }
+    const size_t need = kda_chunk_fwd_workspace_size(B, T, H, dk, dv, num_seqs, chunk_size, dtype);
+    if (need == 0) return KDA_ERR_BAD_SHAPE;
+    if (workspace_bytes < need) return KDA_ERR_WORKSPACE_TOO_SMALL;
+
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+    int *status = static_cast<int *>(workspace);
+    cudaError_t e;
+    if (uses_tensor_cores(dk, dv, dtype)) {
+        e = kda::launch_prefill_tc(q, k, v, log_alpha, beta, h0, cu_seqlens, num_seqs, B, T, H, o, h_T,
+                                   workspace, workspace_bytes, stream);
+    } else {
+        e = cudaMemsetAsync(workspace, 0, kStatusBytes, stream);
+        if (e == cudaSuccess)
+            e = kda::launch_prefill_simt(q, k, v, log_alpha, beta, h0, cu_seqlens, num_seqs, B, T, H, dk, dv,
+                                     dtype, o, h_T, status, stream);
+    }
+    return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+int kda_decode_step(const void *q, const void *k, const void *v, const float *log_alpha, const float *beta,
+                    float *S, int N, int H, int dk, int dv, kda_dtype dtype, void *o, void *stream_) {
+    if (dtype != KDA_F32 && dtype != KDA_BF16) return KDA_ERR_BAD_DTYPE;
+    if (!q || !k || !v || !log_alpha || !beta || !S || !o) return KDA_ERR_NULL_ARG;
+    if (N <= 0 || H <= 0 || dk <= 0 || dv <= 0) return KDA_ERR_BAD_SHAPE;
+    if ((int64_t)N * H > (int64_t)INT32_MAX) return KDA_ERR_BAD_SHAPE;
+    if (!supported_dims(dk, dv)) return KDA_ERR_UNSUPPORTED;
+    const void *ptrs[] = {q, k, v, log_alpha, beta, S, o};
+    for (const void *p : ptrs)
+        if (!aligned16(p)) return KDA_ERR_MISALIGNED;
+    const size_t es = elem_size(dtype), units = (size_t)N * H;
+    const Range ro = range_of(o, units * dv * es), rs = range_of(S, units * dk * dv * 4);
+    const Range inputs[] = {range_of(q, units * dk * es), range_of(k, units * dk * es),
+                            range_of(v, units * dv * es), range_of(log_alpha, units * dk * 4),
+                            range_of(beta, units * 4)};
+    if (overlaps(ro, rs)) return KDA_ERR_ALIASING;
+    for (const Range &r : inputs)
+        if (overlaps(ro, r) || overlaps(rs, r)) return KDA_ERR_ALIASING;
+    cudaError_t e = kda::launch_decode(q, k, v, log_alpha, beta, S, N, H, dk, dv, dtype, o,
+                                       static_cast<cudaStream_t>(stream_));
+    return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+int kda_get_status(void *workspace, void *stream_) {
+    if (!workspace) return KDA_ERR_NULL_ARG;
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+    int host = 0;
+    if (cudaMemcpyAsync(&host, workspace, sizeof(int), cudaMemcpyDeviceToHost, stream) != cudaSuccess)
+        return KDA_ERR_CUDA;
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return KDA_ERR_CUDA;
+    if (host != 0) {
+        const int zero = 0;
+        if (cudaMemcpyAsync(workspace, &zero, sizeof(int), cudaMemcpyHostToDevice, stream) != cudaSuccess)
+            return KDA_ERR_CUDA;
+        if (cudaStreamSynchronize(stream) != cudaSuccess) return KDA_ERR_CUDA;
+    }
+    return host;
+}
+
+}  // extern "C"

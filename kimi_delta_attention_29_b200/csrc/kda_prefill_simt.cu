@@ -1,0 +1,272 @@
+// Chunkwise KDA forward on CUDA cores, fp32 arithmetic (the fp32-dtype path, and the path for
+// head dim 64).  Same chunkwise algorithm as the tensor-core path, without tensor cores.
+//
+// Kimi Linear summary page (th.news.hada.io topic 31936), section "Chunkwise parallel
+// algorithm": the sequence is cut into 64-token chunks; each chunk's final state seeds the next;
+// the chunk's rank-1 updates are packed through the lower-triangular inverse
+// T = (I + A)^-1 found by forward substitution (UT transform); the output merges the
+// inter-chunk state term with the intra-chunk term.  Section "Reduced computation vs general
+// DPLR": with both DPLR vectors tied to k only two decayed Gram matrices are needed,
+//     A[r][i] = beta_r sum_c k_rc k_ic e^{G_rc - G_ic}  (i < r),
+//     P[r][i] =        sum_c q_rc k_ic e^{G_rc - G_ic}  (i <= r),   G_r = sum_{s<=r} log_alpha_s.
+// Per chunk with incoming state S:  Delta = T Diag(beta) (V - (K o e^G) S),
+//     O = (Q o e^G) S + P Delta,    S <- Diag(e^{G_last}) S + (K o e^{G_last - G})^T Delta.
+// (Delta = U - W S with the WY factors U = T Diag(beta) V, W = T Diag(beta) (K o e^G); this path
+//  applies T to V - (K o e^G) S directly, which is the same product taken in the other order.)
+//
+// Decay factors (section "Reduced computation vs general DPLR": fine-grained decay inside a
+// chunk needs log-domain care): e^{G_rc - G_ic} is split at a reference point per 16-row block,
+// E_b = G at row 16b + 7, as  e^{G_r - E_b(r)} * e^{E_b(r) - E_b(i)} * e^{E_b(i) - G_i};
+// each factor stays within e^{+-8 max|log_alpha|} or below 1, so nothing overflows fp32 even when
+// G falls far below -88 within a chunk.
+//
+// One CTA of 256 threads owns (sequence, head, 32 value columns); value columns evolve
+// independently, so the slices need no communication.
+#include "kda_common.cuh"
+
+namespace kda {
+namespace {
+
+constexpr int kC = kChunk;    // 64 rows per chunk
+constexpr int kNV = 32;       // value columns per CTA
+constexpr int kThreads = 256;
+constexpr int kBlocks = kC / 16;
+
+template <int DK>
+struct SimtSmem {
+    static constexpr int DKP = DK + 1;  // padded row stride (bank-conflict free column walks)
+    static constexpr int CP = kC + 1;
+    static constexpr size_t floats =
+        3 * (size_t)kC * DKP          // Xo (k, then k e^{G-E}), Xq (q e^{G-E}), Y (G, then k e^{E-G})
+        + (size_t)kBlocks * kBlocks * DK  // Cf[b][a][c] = e^{E_b - E_a}
+        + 2 * (size_t)kBlocks * DK        // eb = e^{E_b}, gle = e^{G_last - E_b}
+        + DK                              // egl = e^{G_last}
+        + 3 * (size_t)kC * kNV            // Vs, X1, Dl
+        + (size_t)DK * kNV                // Ss
+        + 3 * (size_t)kC * CP             // Am, Pm, Tm
+        + kC;                             // beta
+    static constexpr size_t bytes = floats * sizeof(float);
+};
+
+template <int DK, typename T>
+__global__ void __launch_bounds__(kThreads, 1)
+kda_prefill_simt_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
+                        const float *__restrict__ log_alpha, const float *__restrict__ beta,
+                        const float *__restrict__ h0, const int32_t *__restrict__ cu_seqlens,
+                        int num_seqs, int T_len, int H, T *__restrict__ o, float *__restrict__ h_T,
+                        int *status) {
+    constexpr int DV = DK;
+    using SM = SimtSmem<DK>;
+    constexpr int DKP = SM::DKP, CP = SM::CP;
+    extern __shared__ float smem[];
+    float *Xo = smem;
+    float *Xq = Xo + kC * DKP;
+    float *Y = Xq + kC * DKP;
+    float *Cf = Y + kC * DKP;
+    float *eb = Cf + kBlocks * kBlocks * DK;
+    float *gle = eb + kBlocks * DK;
+    float *egl = gle + kBlocks * DK;
+    float *Vs = egl + DK;
+    float *X1 = Vs + kC * kNV;
+    float *Dl = X1 + kC * kNV;
+    float *Ss = Dl + kC * kNV;
+    float *Am = Ss + DK * kNV;
+    float *Pm = Am + kC * CP;
+    float *Tm = Pm + kC * CP;
+    float *bt = Tm + kC * CP;
+
+    constexpr int slices = DV / kNV;
+    int bid = blockIdx.x;
+    const int slice = bid % slices;
+    bid /= slices;
+    const int h = bid % H;
+    const int n = bid / H;
+    const int j0 = slice * kNV;
+    const int tid = threadIdx.x;
+
+    int64_t start, len;
+    if (cu_seqlens) {
+        const int a = __ldg(cu_seqlens + n), b = __ldg(cu_seqlens + n + 1);
+        const bool bad = a < 0 || b < a || b > T_len || (n == 0 && a != 0) ||
+                         (n == num_seqs - 1 && b != T_len);
+        if (bad) {
+            if (tid == 0) set_status(status, KDA_ERR_BAD_SEQLENS);
+            return;
+        }
+        start = a;
+        len = b - a;
+    } else {
+        start = (int64_t)n * T_len;
+        len = T_len;
+    }
+
+    const size_t state_off = ((size_t)n * H + h) * DK * DV;
+    for (int idx = tid; idx < DK * kNV; idx += kThreads) {
+        const int c = idx / kNV, j = idx % kNV;
+        Ss[idx] = h0 ? h0[state_off + (size_t)c * DV + j0 + j] : 0.f;
+    }
+
+    for (int64_t c0 = 0; c0 < len; c0 += kC) {
+        const int L = (len - c0) < kC ? (int)(len - c0) : kC;
+        __syncthreads();
+        // 1. gather the chunk (rows >= L padded with the neutral token k=q=v=beta=log_alpha=0)
+        for (int idx = tid; idx < kC * DK; idx += kThreads) {
+            const int r = idx / DK, c = idx % DK;
+            float kv = 0.f, qv = 0.f, lv = 0.f;
+            if (r < L) {
+                const size_t off = ((size_t)(start + c0 + r) * H + h) * DK + c;
+                kv = Elem<T>::load(k + off);
+                qv = Elem<T>::load(q + off);
+                lv = __ldg(log_alpha + off);
+            }
+            Xo[r * DKP + c] = kv;
+            Xq[r * DKP + c] = qv;
+            Y[r * DKP + c] = lv;
+        }
+        for (int idx = tid; idx < kC * kNV; idx += kThreads) {
+            const int r = idx / kNV, j = idx % kNV;
+            Vs[idx] = r < L ? Elem<T>::load(v + ((size_t)(start + c0 + r) * H + h) * DV + j0 + j) : 0.f;
+        }
+        if (tid < kC) bt[tid] = tid < L ? __ldg(beta + (size_t)(start + c0 + tid) * H + h) : 0.f;
+        __syncthreads();
+
+        // 2. per-channel cumulative log-gate and the block-referenced decay factors
+        for (int c = tid; c < DK; c += kThreads) {
+            float acc = 0.f;
+            for (int r = 0; r < kC; ++r) {
+                acc += Y[r * DKP + c];
+                Y[r * DKP + c] = acc;
+            }
+            float E[kBlocks];
+#pragma unroll
+            for (int b = 0; b < kBlocks; ++b) E[b] = Y[(16 * b + 7) * DKP + c];
+            const float gl = acc;
+#pragma unroll
+            for (int b = 0; b < kBlocks; ++b) {
+#pragma unroll
+                for (int a = 0; a < kBlocks; ++a) Cf[(b * kBlocks + a) * DK + c] = a <= b ? expf(E[b] - E[a]) : 0.f;
+                eb[b * DK + c] = expf(E[b]);
+                gle[b * DK + c] = expf(gl - E[b]);
+            }
+            egl[c] = expf(gl);
+            for (int r = 0; r < kC; ++r) {
+                const float Eb = E[r / 16];
+                const float g = Y[r * DKP + c];
+                const float kk = Xo[r * DKP + c];
+                const float F = expf(g - Eb);
+                Xo[r * DKP + c] = kk * F;
+                Xq[r * DKP + c] *= F;
+                Y[r * DKP + c] = kk * expf(Eb - g);
+            }
+        }
+        __syncthreads();
+
+        // 3. decayed Gram matrices A (strict lower, times beta_r) and P (inclusive lower)
+        for (int p = tid; p < kC * kC; p += kThreads) {
+            const int r = p / kC, i = p % kC;
+            float sa = 0.f, sp = 0.f;
+            if (i <= r) {
+                const float *cf = Cf + ((r / 16) * kBlocks + i / 16) * DK;
+                for (int c = 0; c < DK; ++c) {
+                    const float yi = Y[i * DKP + c] * cf[c];
+                    sa = fmaf(Xo[r * DKP + c], yi, sa);
+                    sp = fmaf(Xq[r * DKP + c], yi, sp);
+                }
+            }
+            Am[r * CP + i] = i < r ? bt[r] * sa : 0.f;
+            Pm[r * CP + i] = i <= r ? sp : 0.f;
+        }
+        __syncthreads();
+
+        // 4. UT transform: T = (I + A)^-1 by forward substitution, one row at a time
+        for (int r = 0; r < kC; ++r) {
+            if (tid < kC) {
+                const int j = tid;
+                float t = (j == r) ? 1.f : 0.f;
+                if (j < r)
+                    for (int i = j; i < r; ++i) t = fmaf(-Am[r * CP + i], Tm[i * CP + j], t);
+                Tm[r * CP + j] = (j <= r) ? t : 0.f;
+            }
+            __syncthreads();
+        }
+
+        // 5. X1 = V - (K o e^G) S      (K o e^G)_r = Xo_r * e^{E_b(r)}
+        for (int idx = tid; idx < kC * kNV; idx += kThreads) {
+            const int r = idx / kNV, j = idx % kNV;
+            const float *e = eb + (r / 16) * DK;
+            float acc = Vs[idx];
+            for (int c = 0; c < DK; ++c) acc = fmaf(-Xo[r * DKP + c] * e[c], Ss[c * kNV + j], acc);
+            X1[idx] = acc;
+        }
+        __syncthreads();
+        // 6. Delta = T Diag(beta) X1
+        for (int idx = tid; idx < kC * kNV; idx += kThreads) {
+            const int r = idx / kNV, j = idx % kNV;
+            float acc = 0.f;
+            for (int i = 0; i <= r; ++i) acc = fmaf(Tm[r * CP + i] * bt[i], X1[i * kNV + j], acc);
+            Dl[idx] = acc;
+        }
+        __syncthreads();
+        // 7. O = (Q o e^G) S + P Delta
+        for (int idx = tid; idx < kC * kNV; idx += kThreads) {
+            const int r = idx / kNV, j = idx % kNV;
+            if (r >= L) continue;
+            const float *e = eb + (r / 16) * DK;
+            float acc = 0.f;
+            for (int c = 0; c < DK; ++c) acc = fmaf(Xq[r * DKP + c] * e[c], Ss[c * kNV + j], acc);
+            for (int i = 0; i <= r; ++i) acc = fmaf(Pm[r * CP + i], Dl[i * kNV + j], acc);
+            Elem<T>::store(o + ((size_t)(start + c0 + r) * H + h) * DV + j0 + j, acc);
+        }
+        __syncthreads();
+        // 8. S <- Diag(e^{G_last}) S + (K o e^{G_last - G})^T Delta;  (K o e^{G_last-G})_i = Y_i e^{G_last - E_b(i)}
+        for (int idx = tid; idx < DK * kNV; idx += kThreads) {
+            const int c = idx / kNV, j = idx % kNV;
+            float acc = egl[c] * Ss[idx];
+            for (int i = 0; i < kC; ++i) acc = fmaf(Y[i * DKP + c] * gle[(i / 16) * DK + c], Dl[i * kNV + j], acc);
+            Ss[idx] = acc;
+        }
+    }
+    __syncthreads();
+    if (h_T) {
+        for (int idx = tid; idx < DK * kNV; idx += kThreads) {
+            const int c = idx / kNV, j = idx % kNV;
+            h_T[state_off + (size_t)c * DV + j0 + j] = Ss[idx];
+        }
+    }
+}
+
+template <int DK, typename T>
+cudaError_t launch_t(const void *q, const void *k, const void *v, const float *la, const float *beta,
+                     const float *h0, const int32_t *cu, int num_seqs, int T_len, int H, void *o,
+                     float *h_T, int *status, cudaStream_t stream) {
+    auto kern = kda_prefill_simt_kernel<DK, T>;
+    const size_t smem = SimtSmem<DK>::bytes;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const unsigned grid = (unsigned)num_seqs * (unsigned)H * (unsigned)(DK / kNV);
+    trace_before(kKernSimt, stream);
+    kern<<<grid, kThreads, smem, stream>>>(static_cast<const T *>(q), static_cast<const T *>(k),
+                                           static_cast<const T *>(v), la, beta, h0, cu, num_seqs, T_len,
+                                           H, static_cast<T *>(o), h_T, status);
+    trace_after(stream);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_prefill_simt(const void *q, const void *k, const void *v, const float *log_alpha,
+                                const float *beta, const float *h0, const int32_t *cu_seqlens,
+                                int num_seqs, int B, int T, int H, int dk, int dv, kda_dtype dtype,
+                                void *o, float *h_T, int *status, cudaStream_t stream) {
+    (void)B;
+    (void)dv;
+    if (dk == 128)
+        return dtype == KDA_BF16
+                   ? launch_t<128, __nv_bfloat16>(q, k, v, log_alpha, beta, h0, cu_seqlens, num_seqs, T, H, o, h_T, status, stream)
+                   : launch_t<128, float>(q, k, v, log_alpha, beta, h0, cu_seqlens, num_seqs, T, H, o, h_T, status, stream);
+    return dtype == KDA_BF16
+               ? launch_t<64, __nv_bfloat16>(q, k, v, log_alpha, beta, h0, cu_seqlens, num_seqs, T, H, o, h_T, status, stream)
+               : launch_t<64, float>(q, k, v, log_alpha, beta, h0, cu_seqlens, num_seqs, T, H, o, h_T, status, stream);
+}
+
+}  // namespace kda

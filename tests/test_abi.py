@@ -1,0 +1,113 @@
+"""C-ABI checks that need no GPU: the library loads, exports every entry point include/kda.h
+declares, and rejects invalid arguments on the host before anything is launched."""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from kimi_delta_attention_29_b200 import _lib
+from kimi_delta_attention_29_b200 import build as kbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    kbuild.build()
+    return _lib.load()
+
+
+def declared_functions() -> list[str]:
+    names = []
+    for h in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if h.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", h)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names += re.findall(r"\b(kda_\w+)\s*\(", text)
+    return sorted(set(names))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert set(_lib.EXPORTED) <= set(names)
+    for name in names:
+        assert hasattr(lib, name), f"{name} declared in include/ but not exported by libkda.so"
+
+
+def test_status_strings_and_version(lib):
+    assert lib.kda_version() >= 100
+    for code in range(0, -11, -1):
+        s = _lib.status_string(code)
+        assert s.startswith("KDA_")
+    assert "unknown" in _lib.status_string(-999)
+
+
+def test_workspace_size_queries(lib):
+    ws = lib.kda_chunk_fwd_workspace_size
+    assert ws(1, 131072, 32, 128, 128, 1, 64, _lib.KDA_BF16) > 4 * 2**30       # WY records for 2048 chunks
+    assert ws(1, 256, 2, 64, 64, 1, 64, _lib.KDA_F32) == 256                     # CUDA-core path: status only
+    assert ws(1, 256, 2, 64, 64, 1, 32, _lib.KDA_F32) == 0                       # chunk 32 unsupported
+    assert ws(1, 256, 2, 96, 96, 1, 64, _lib.KDA_BF16) == 0                      # head dim 96 unsupported
+    assert ws(1, 256, 2, 128, 128, 1, 64, 7) == 0                                # bad dtype
+    assert ws(2, 256, 2, 128, 128, 3, 64, _lib.KDA_BF16) == 0                    # N != B without varlen
+
+
+# Fake, 256-byte aligned device addresses: every call below must fail validation before it touches them.
+A = 1 << 20
+
+
+def _fwd(lib, **kw):
+    args = dict(q=A, k=2 * A, v=3 * A, la=4 * A, beta=5 * A, h0=None, cu=None, N=1, B=1, T=128, H=2, dk=128,
+                dv=128, chunk=64, dtype=_lib.KDA_BF16, o=6 * A, hT=7 * A, ws=8 * A, ws_bytes=1 << 40, stream=None)
+    args.update(kw)
+    c = ctypes.c_void_p
+    return lib.kda_chunk_fwd(c(args["q"]), c(args["k"]), c(args["v"]), c(args["la"]), c(args["beta"]),
+                             c(args["h0"]), c(args["cu"]), args["N"], args["B"], args["T"], args["H"],
+                             args["dk"], args["dv"], args["chunk"], args["dtype"], c(args["o"]), c(args["hT"]),
+                             c(args["ws"]), args["ws_bytes"], c(args["stream"]))
+
+
+def test_chunk_fwd_rejects_on_host(lib):
+    assert _fwd(lib, dtype=5) == _lib.KDA_ERR_BAD_DTYPE
+    assert _fwd(lib, q=None) == _lib.KDA_ERR_NULL_ARG
+    assert _fwd(lib, ws=None) == _lib.KDA_ERR_NULL_ARG
+    assert _fwd(lib, B=0) == _lib.KDA_ERR_BAD_SHAPE
+    assert _fwd(lib, T=-1) == _lib.KDA_ERR_BAD_SHAPE
+    assert _fwd(lib, N=2) == _lib.KDA_ERR_BAD_SHAPE                      # N != B without cu_seqlens
+    assert _fwd(lib, B=2, N=2, cu=9 * A) == _lib.KDA_ERR_BAD_SHAPE      # varlen needs B = 1
+    assert _fwd(lib, chunk=32) == _lib.KDA_ERR_UNSUPPORTED
+    assert _fwd(lib, dk=128, dv=64) == _lib.KDA_ERR_UNSUPPORTED
+    assert _fwd(lib, dk=96, dv=96) == _lib.KDA_ERR_UNSUPPORTED
+    assert _fwd(lib, v=3 * A + 8) == _lib.KDA_ERR_MISALIGNED
+    assert _fwd(lib, ws=8 * A + 16) == _lib.KDA_ERR_MISALIGNED          # workspace needs 256-byte alignment
+    assert _fwd(lib, o=A) == _lib.KDA_ERR_ALIASING                       # o on top of q
+    assert _fwd(lib, hT=3 * A) == _lib.KDA_ERR_ALIASING                  # h_T on top of v
+    assert _fwd(lib, h0=7 * A + 1024, hT=7 * A) == _lib.KDA_ERR_ALIASING  # partial h0 / h_T overlap
+    assert _fwd(lib, ws_bytes=1024) == _lib.KDA_ERR_WORKSPACE_TOO_SMALL
+
+
+def test_decode_rejects_on_host(lib):
+    c = ctypes.c_void_p
+
+    def dec(q=A, k=2 * A, v=3 * A, la=4 * A, beta=5 * A, S=6 * A, N=4, H=2, dk=128, dv=128,
+            dtype=_lib.KDA_BF16, o=8 * A):
+        return lib.kda_decode_step(c(q), c(k), c(v), c(la), c(beta), c(S), N, H, dk, dv, dtype, c(o), c(None))
+
+    assert dec(dtype=3) == _lib.KDA_ERR_BAD_DTYPE
+    assert dec(S=None) == _lib.KDA_ERR_NULL_ARG
+    assert dec(N=0) == _lib.KDA_ERR_BAD_SHAPE
+    assert dec(dk=32, dv=32) == _lib.KDA_ERR_UNSUPPORTED
+    assert dec(o=8 * A + 4) == _lib.KDA_ERR_MISALIGNED
+    assert dec(o=6 * A) == _lib.KDA_ERR_ALIASING                         # o inside S
+    assert dec(S=A) == _lib.KDA_ERR_ALIASING                             # S on top of q
+
+
+def test_binding_refuses_noncontiguous():
+    import torch
+    import kimi_delta_attention_29_b200 as kda
+    x = torch.zeros(4, 8)[:, ::2]
+    with pytest.raises(ValueError):
+        kda._ptr(x)
