@@ -1,0 +1,381 @@
+#!/usr/bin/env python
+"""KDA benchmark: long-context chunkwise prefill on B200 (plus the recurrent decode workload).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl kda|reference]
+
+Step = one kda_chunk_fwd over the long-context batch (B=1, H=32, T=131072, d_k=d_v=128, bf16 q/k/v,
+fp32 gates, h0 ~ N(0, 0.02)): chunk prep + state passing + output + final state.  Inputs (6.4 GB
+per step) are larger than L2, so no flush is needed between steps.  Timing: W untimed warm-up steps,
+then K steps between a barrier + synchronize on both sides, CUDA events on the launching stream,
+max over ranks.  N > 1 runs independent replicas (weak scaling, no data-path collective).
+
+--impl reference times the fp64 CPU oracle (test infrastructure) on a bounded sample of the same
+workload on the host cores; rank 0 alone runs it.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "KDA prefill tokens/s (H=32,d=128,T=128K) & % roofline; decode HBM GB/s"
+UNIT = "tokens/s"
+
+# Algorithmic traffic (bytes) and work, per token-head of the prefill (bf16 q,k,v,o; fp32 gates):
+#   q, k, v 3 x 256 B, log_alpha 512 B, beta 4 B, o 256 B.
+PREFILL_BYTES_PER_TOKEN_HEAD = 768 + 512 + 4 + 256
+PREFILL_FLOP_PER_TOKEN_HEAD = 180224          # five C x d and three d x d products per token at C=64, d=128
+STATE_BYTES = 128 * 128 * 4                    # one fp32 state (h0 read or h_T write)
+REC_WRITE_BYTES = 74240                        # WY record bytes the intra-chunk kernel writes per chunk-head
+REC_READ_BYTES = 32768 + 16384 + 8192 + 512 + 16384  # record bytes the state kernel needs per chunk-head
+DECODE_BYTES_PER_STATE = 2 * STATE_BYTES + 3 * 256 + 512 + 4 + 256  # S read+write, q/k/v, gates, beta, o
+
+
+def parse_args():
+    p = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=10)
+    p.add_argument("--warmup", type=int, default=3)
+    p.add_argument("--impl", choices=["kda", "reference"], default="kda")
+    p.add_argument("--e2e-steps", type=int, default=2)
+    p.add_argument("--decode-steps", type=int, default=1024)
+    p.add_argument("--no-decode", action="store_true")
+    p.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle sample")
+    return p.parse_args()
+
+
+def dist_env():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("LOCAL_RANK", "0")),
+            int(os.environ.get("WORLD_SIZE", "1")))
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            pk = json.load(f)
+        return dict(hbm_gbs=float(pk["hbm_gbs"]), bf16_tflops=float(pk["bf16_tflops"]),
+                    bf16_tflops_sustained=float(pk.get("bf16_tflops_sustained", pk["bf16_tflops"])),
+                    source="measured")
+    return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, source="fallback")
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling while the timed region runs."""
+
+    FIELDS = ["index", "clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.active",
+              "clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
+              "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(prefix="kda_clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={','.join(self.FIELDS)}", "--format=csv,noheader,nounits",
+                 "-lms", "200", "-i", str(self.gpu)], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                cols = [c.strip() for c in line.split(",")]
+                if len(cols) < len(self.FIELDS):
+                    continue
+                try:
+                    sm.append(float(cols[1]))
+                    mx.append(float(cols[2]))
+                except ValueError:
+                    continue
+                for name, val in zip(names, cols[5:9]):
+                    if val.lower().startswith("active"):
+                        reasons.add(name)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- CPU oracle timing
+def oracle_sample(target_s: float, seed: int = 0):
+    """Time the fp64 oracle on the first T_s tokens (all 32 heads) of the long-context workload,
+    T_s sized so the timed call takes about target_s seconds.  Returns a cpu_baseline dict."""
+    import torch
+
+    import oracle
+    from kimi_delta_attention_29_b200 import inputs as gen
+
+    shp = gen.LONG
+
+    def run(T_s):
+        x = gen.make_prefill(1, T_s, shp.H, shp.dk, shp.dv, shp.dtype, shp.gate_shift, shp.h0_std, seed, "cpu")
+        f = lambda t: t.float().numpy()
+        args = (f(x["q"]), f(x["k"]), f(x["v"]), f(x["log_alpha"]), f(x["beta"]), f(x["h0"]))
+        t0 = time.perf_counter()
+        oracle.recurrent(*args)
+        return time.perf_counter() - t0
+
+    probe_T = 256
+    t_probe = run(probe_T)
+    T_s = int(max(64, min(shp.T, probe_T * target_s / max(t_probe, 1e-3))) // 64 * 64)
+    dt = run(T_s)
+    cores = oracle.num_threads()
+    return {"value": T_s / dt, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"fp64 recurrent oracle on tokens 0..{T_s - 1} of B=1,H=32,T=131072,d=128 "
+                      f"(all 32 heads, h0 included); {dt:.1f} s on {cores} threads",
+            "seconds": dt, "tokens": T_s}
+
+
+def config_dict():
+    return {"workload": "long_B1_H32_T131072_d128", "model": "KDA operator (chunkwise prefill)", "B": 1,
+            "T": 131072, "H": 32, "dk": 128, "dv": 128, "chunk": 64, "global_batch": 1, "seq_len": 131072,
+            "gates": "log_alpha=-softplus(N(0,1)+2), beta=sigmoid(N(0,1)), h0~N(0,0.02)",
+            "l2": "no flush: inputs (6.4 GB per step) are larger than the 126 MB L2",
+            "parallelism": "replicas (independent problems per GPU)"}
+
+
+def reference_arm(args):
+    rank, _, world = dist_env()
+    if rank != 0:
+        return 0
+    for _ in range(args.warmup):
+        oracle_sample(max(1.0, args.cpu_seconds / 4))
+    samples = [oracle_sample(max(1.0, args.cpu_seconds / 2)) for _ in range(args.steps)]
+    tok = sum(s["tokens"] for s in samples)
+    sec = sum(s["seconds"] for s in samples)
+    value = tok / sec
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * 131072 / value,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": config_dict(),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": samples[0]["cores"], "kind": "oracle",
+                             "sample": f"{args.steps} steps, each the fp64 oracle on the first "
+                                       f"{samples[0]['tokens']} tokens x 32 heads of the workload"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------------- GPU arm
+def kernel_stats(traces):
+    out = {}
+    for name, ms in traces:
+        d = out.setdefault(name, {"launches": 0, "total_ms": 0.0})
+        d["launches"] += 1
+        d["total_ms"] += ms
+    total = sum(d["total_ms"] for d in out.values()) or 1.0
+    for d in out.values():
+        d["avg_ms"] = d["total_ms"] / d["launches"]
+        d["share"] = d["total_ms"] / total
+    return out
+
+
+def gpu_arm(args):
+    import torch
+    import torch.distributed as dist
+
+    import kimi_delta_attention_29_b200 as kda
+    from kimi_delta_attention_29_b200 import inputs as gen
+
+    rank, local_rank, world = dist_env()
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        t = torch.tensor([x], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    peaks = load_peaks()
+    shp = gen.LONG
+    x = gen.make_prefill_for(shp, seed=rank, device=dev)
+    B, T, H, D = shp.B, shp.T, shp.H, shp.dk
+    o = torch.empty(B, T, H, D, dtype=shp.dtype, device=dev)
+    hT = torch.empty(B, H, D, D, dtype=torch.float32, device=dev)
+    ws = kda.Workspace(dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        kda.kda_chunk_fwd(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], x["h0"], None, o=o, h_T=hT,
+                          workspace=ws, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    assert kda.kda_get_status(ws) == 0, "device status after warm-up"
+
+    clocks = ClockSampler(dev.index)
+    barrier()
+    torch.cuda.synchronize(dev)
+    clocks.start()
+    time.sleep(0.3)
+    kda.kda_trace_begin(16 * args.steps + 16)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for _ in range(args.steps):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    traces = kda.kda_trace_end()
+    barrier()
+    clk = clocks.stop()
+    elapsed_ms = max_over_ranks(ev0.elapsed_time(ev1))
+    ms_per_step = elapsed_ms / args.steps
+    tokens_per_step = B * T
+    value = world * tokens_per_step * args.steps / (elapsed_ms / 1e3)
+
+    # per-kernel timing (live, CUDA events around each library kernel in the timed region)
+    kst = kernel_stats(traces)
+    dominant = max(kst, key=lambda n: kst[n]["total_ms"])
+    token_heads = B * T * H
+    chunk_heads = B * ((T + 63) // 64) * H
+    kbytes = {
+        "kda_tc_prep_kernel": token_heads * (768 + 512 + 4) + chunk_heads * REC_WRITE_BYTES,
+        "kda_tc_state_kernel": chunk_heads * REC_READ_BYTES + token_heads * 256 + 2 * B * H * STATE_BYTES,
+    }
+    peak_bw = peaks["hbm_gbs"]
+    achieved = kbytes.get(dominant, 0) / (kst[dominant]["avg_ms"] / 1e3) / 1e9
+    roofline = {"kernel": dominant, "bound": "hbm", "achieved": achieved, "peak": peak_bw, "unit": "GB/s",
+                "frac": achieved / peak_bw, "traffic": None, "peak_source": peaks["source"],
+                "algorithmic_bytes_per_launch": kbytes.get(dominant, 0), "avg_ms": kst[dominant]["avg_ms"]}
+    op_bytes = token_heads * PREFILL_BYTES_PER_TOKEN_HEAD + 2 * B * H * STATE_BYTES
+    op_flop = token_heads * PREFILL_FLOP_PER_TOKEN_HEAD
+    op_gbs = op_bytes / (ms_per_step / 1e3) / 1e9
+    op_tflops = op_flop / (ms_per_step / 1e3) / 1e12
+    operator_roofline = {"bytes_per_step": op_bytes, "achieved_gbs": op_gbs, "hbm_frac": op_gbs / peak_bw,
+                         "flop_per_step": op_flop, "achieved_tflops": op_tflops,
+                         "tensor_frac": op_tflops / peaks["bf16_tflops_sustained"],
+                         "note": "whole call (all kernels) against the operator's algorithmic bytes / FLOPs; "
+                                 "tensor_frac against the sustained bf16 peak"}
+
+    # end to end through the public API with host buffers: pinned H2D of the step's inputs, the call,
+    # D2H of the results (o and h_T), all inside the timed region
+    host = {kk: x[kk].cpu().pin_memory() for kk in ("q", "k", "v", "log_alpha", "beta", "h0")}
+    o_h = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+    hT_h = torch.empty(hT.shape, dtype=hT.dtype, pin_memory=True)
+    dx = {kk: torch.empty_like(x[kk]) for kk in host}
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = o_h.numel() * o_h.element_size() + hT_h.numel() * hT_h.element_size()
+
+    def e2e_step():
+        for kk in host:
+            dx[kk].copy_(host[kk], non_blocking=True)
+        kda.kda_chunk_fwd(dx["q"], dx["k"], dx["v"], dx["log_alpha"], dx["beta"], dx["h0"], None, o=o, h_T=hT,
+                          workspace=ws, stream=stream)
+        o_h.copy_(o, non_blocking=True)
+        hT_h.copy_(hT, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize(dev)
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1)) / args.e2e_steps
+    e2e = {"value": world * tokens_per_step / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+           "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": args.e2e_steps}
+    del host, dx, o_h, hT_h
+
+    decode = None
+    if not args.no_decode:
+        decode = decode_bench(args, dev, stream, peaks, barrier, max_over_ranks)
+
+    cpu_baseline = None
+    if rank == 0 and world == 1:
+        cpu_baseline = oracle_sample(args.cpu_seconds)
+
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config_dict(),
+            "roofline": roofline, "operator_roofline": operator_roofline, "cpu_baseline": cpu_baseline,
+            "e2e": e2e, "gpu_launches": len(traces), "clocks": clk, "decode": decode,
+            "kernels": kst, "peaks": peaks}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def decode_bench(args, dev, stream, peaks, barrier, max_over_ranks):
+    """256 x 32 fp32 states (128 x 128), `decode_steps` single-token steps, state updated in place."""
+    import torch
+
+    import kimi_delta_attention_29_b200 as kda
+    from kimi_delta_attention_29_b200 import inputs as gen
+
+    shp = gen.DECODE
+    S = gen.make_decode_state(shp.N, shp.H, shp.dk, shp.dv, std=shp.s0_std, seed=0, device=dev)
+    pool = [gen.make_decode_token(shp.N, shp.H, shp.dk, shp.dv, dtype=shp.dtype, seed=1000 + s, device=dev)
+            for s in range(8)]
+    o = torch.empty(shp.N, shp.H, shp.dv, dtype=shp.dtype, device=dev)
+
+    def step(s):
+        t = pool[s % len(pool)]
+        kda.kda_decode_step(t["q"], t["k"], t["v"], t["log_alpha"], t["beta"], S, o=o, stream=stream)
+
+    for s in range(16):
+        step(s)
+    torch.cuda.synchronize(dev)
+    barrier()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for s in range(args.decode_steps):
+        step(s)
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    ms = max_over_ranks(ev0.elapsed_time(ev1)) / args.decode_steps
+    nbytes = shp.N * shp.H * DECODE_BYTES_PER_STATE
+    gbs = nbytes / (ms / 1e3) / 1e9
+    return {"workload": shp.name, "steps": args.decode_steps, "ms_per_step": ms,
+            "tokens_per_s": shp.N / (ms / 1e3), "hbm_gbs": gbs, "peak_gbs": peaks["hbm_gbs"],
+            "frac": gbs / peaks["hbm_gbs"], "bytes_per_step": nbytes,
+            "note": "inputs cycle through 8 pre-drawn token sets; the 512 MiB state streams from HBM each step"}
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        return reference_arm(args)
+    return gpu_arm(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())
