@@ -89,6 +89,30 @@ KDA_API int kda_chunk_fwd(const void *q, const void *k, const void *v, const flo
                   int B, int T, int H, int dk, int dv, int chunk_size, kda_dtype dtype, void *o,
                   float *h_T, void *workspace, size_t workspace_bytes, void *stream);
 
+/* kda_chunk_fwd for callers that cannot allocate device memory (the paper has no counterpart;
+ * this is a deployment convenience).  Some callers cannot call cudaMalloc: a plugin whose host
+ * framework hands it only its input and output buffers, or an engine that has already reserved
+ * all free device memory for its own pool.  This entry point takes the same arguments as
+ * kda_chunk_fwd minus the workspace and uses instead a fixed 64 MiB scratch array that the
+ * library holds in device memory on every GPU that loads it, until the process exits.
+ *   - It allocates nothing (no cudaMalloc / cudaFree, no allocating library call).
+ *   - Sizes whose kda_chunk_fwd_workspace_size() exceeds 64 MiB are rejected with
+ *     KDA_ERR_WORKSPACE_TOO_SMALL before anything is launched.  For the tensor-core path
+ *     (bf16, d = 128) that is roughly num_chunks * H <= 896, where num_chunks = ceil(B*T/64) + N;
+ *     e.g. H = 32 heads up to T = 1728 tokens for one sequence.
+ *   - The first call on a device looks up the scratch's device address for that device (with
+ *     that device current) and caches it; make that first call before any stream capture.
+ *   - All calls share the one scratch array, which keeps the last call's contents (the status
+ *     word is cleared at the start of every call).  Calls that overlap on the GPU (on different
+ *     streams, or from different host threads) race on it and must be serialized by the caller.
+ *   - Device-detected errors (malformed cu_seqlens, timeouts) are recorded in the shared scratch
+ *     and cannot be read back through this entry point.
+ * Returns the same codes as kda_chunk_fwd otherwise. */
+KDA_API int kda_chunk_fwd_noalloc(const void *q, const void *k, const void *v, const float *log_alpha,
+                                  const float *beta, const float *h0, const int32_t *cu_seqlens,
+                                  int num_seqs, int B, int T, int H, int dk, int dv, int chunk_size,
+                                  kda_dtype dtype, void *o, float *h_T, void *stream);
+
 /* One recurrent decode step for N*H independent states, updated in place:
  *   S' = Diag(exp(log_alpha)) S;  u = beta (v - S'^T k);  S <- S' + k u^T;  o = S^T q.
  *   q, k      : [N, H, dk] dtype     v, o : [N, H, dv] dtype
