@@ -48,7 +48,10 @@ def parse_args():
     p.add_argument("--e2e-steps", type=int, default=2)
     p.add_argument("--decode-steps", type=int, default=1024)
     p.add_argument("--no-decode", action="store_true")
-    p.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle sample")
+    p.add_argument("--cpu-seconds", type=float, default=12.0,
+                   help="target CPU time of the oracle sample (0 skips the CPU baseline)")
+    p.add_argument("--seq-len", type=int, default=131072,
+                   help="override T of the long-context workload (small cases for profiler captures)")
     return p.parse_args()
 
 
@@ -149,11 +152,11 @@ def oracle_sample(target_s: float, seed: int = 0):
             "seconds": dt, "tokens": T_s}
 
 
-def config_dict():
-    return {"workload": "long_B1_H32_T131072_d128", "model": "KDA operator (chunkwise prefill)", "B": 1,
-            "T": 131072, "H": 32, "dk": 128, "dv": 128, "chunk": 64, "global_batch": 1, "seq_len": 131072,
+def config_dict(T: int = 131072):
+    return {"workload": f"long_B1_H32_T{T}_d128", "model": "KDA operator (chunkwise prefill)", "B": 1,
+            "T": T, "H": 32, "dk": 128, "dv": 128, "chunk": 64, "global_batch": 1, "seq_len": T,
             "gates": "log_alpha=-softplus(N(0,1)+2), beta=sigmoid(N(0,1)), h0~N(0,0.02)",
-            "l2": "no flush: inputs (6.4 GB per step) are larger than the 126 MB L2",
+            "l2": f"no flush: inputs ({T * 32 * 1284 / 1e9:.2f} GB per step) are larger than the 126 MB L2",
             "parallelism": "replicas (independent problems per GPU)"}
 
 
@@ -219,7 +222,8 @@ def gpu_arm(args):
         return float(t.item())
 
     peaks = load_peaks()
-    shp = gen.LONG
+    import dataclasses
+    shp = dataclasses.replace(gen.LONG, T=args.seq_len)
     x = gen.make_prefill_for(shp, seed=rank, device=dev)
     B, T, H, D = shp.B, shp.T, shp.H, shp.dk
     o = torch.empty(B, T, H, D, dtype=shp.dtype, device=dev)
@@ -297,19 +301,21 @@ def gpu_arm(args):
         o_h.copy_(o, non_blocking=True)
         hT_h.copy_(hT, non_blocking=True)
 
-    e2e_step()
-    torch.cuda.synchronize(dev)
-    barrier()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(args.e2e_steps):
+    e2e = None
+    if args.e2e_steps > 0:
         e2e_step()
-    e1.record(stream)
-    torch.cuda.synchronize(dev)
-    barrier()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1)) / args.e2e_steps
-    e2e = {"value": world * tokens_per_step / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
-           "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": args.e2e_steps}
+        torch.cuda.synchronize(dev)
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier()
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1)) / args.e2e_steps
+        e2e = {"value": world * tokens_per_step / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": args.e2e_steps}
     del host, dx, o_h, hT_h
 
     decode = None
@@ -317,12 +323,12 @@ def gpu_arm(args):
         decode = decode_bench(args, dev, stream, peaks, barrier, max_over_ranks)
 
     cpu_baseline = None
-    if rank == 0 and world == 1:
+    if rank == 0 and world == 1 and args.cpu_seconds > 0:
         cpu_baseline = oracle_sample(args.cpu_seconds)
 
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config_dict(),
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config_dict(T),
             "roofline": roofline, "operator_roofline": operator_roofline, "cpu_baseline": cpu_baseline,
             "e2e": e2e, "gpu_launches": len(traces), "clocks": clk, "decode": decode,
             "kernels": kst, "peaks": peaks}
