@@ -48,10 +48,10 @@ constexpr int C = kChunk;
 constexpr uint32_t REC_AQ = 0;        // [W; Q o e^G]: K-major sw128, 128 rows x 128 (2 atoms x 16 KiB)
 constexpr uint32_t REC_KH = 32768;    // K o e^{G_63 - G}: MN-major sw128, 64 k-rows x 128 (2 blocks x 8 KiB)
 constexpr uint32_t REC_P = 49152;     // P: K-major sw128, 64 rows x 64 (8 KiB)
-constexpr uint32_t REC_U = 57344;     // U: bf16 row-major [64][128] (16 KiB)
+constexpr uint32_t REC_U = 57344;     // U: bf16, four [64][32] blocks (one per 32-column slice), 64-byte swizzle
 constexpr uint32_t REC_GL = 73728;    // e^{G_63}: fp32 [128]
 constexpr uint32_t REC_BYTES = 74752;
-constexpr uint32_t REC_TX = 32768 + 16384 + 8192 + 512;  // bytes the state kernel copies per chunk
+constexpr uint32_t REC_TX = 32768 + 16384 + 8192 + 512 + 4096;  // bytes one state CTA copies per chunk
 
 struct TcLayout {
     size_t base_off, table_off, rec_off, total;
@@ -79,6 +79,11 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 __device__ __forceinline__ float2 unpack_bf16(uint32_t u) {
     const __nv_bfloat162 v = *reinterpret_cast<const __nv_bfloat162 *>(&u);
     return __bfloat1622float2(v);
+}
+// Byte offset of the 16-byte chunk x (elements 8x..8x+7) of k-row kr of a tile with 64-byte rows stored
+// with the 64-byte swizzle (MN-major sw64 operands, and the U slices of a record).
+__device__ __forceinline__ uint32_t sw64_chunk(uint32_t kr, uint32_t x) {
+    return kr * 64u + ((x ^ ((kr >> 1) & 3u)) << 4);
 }
 __device__ __forceinline__ float2 expv(float2 x) { return make_float2(__expf(x.x), __expf(x.y)); }
 __device__ __forceinline__ float2 sub2(float2 a, float2 b) { return make_float2(a.x - b.x, a.y - b.y); }
@@ -134,10 +139,22 @@ __global__ void __launch_bounds__(1024) kda_chunk_table_kernel(const int32_t *__
 }
 
 // ============================================================================ intra-chunk kernel
-constexpr int kPrepThreads = 128;
+// 256 threads per (chunk, head).  Warp w owns key channels [64 (w & 1), 64 (w & 1) + 64) as pairs
+// (lane l -> channels c0 = 64 (w & 1) + 2 l, c0 + 1) for the 16 rows of key block qr = w >> 1, so
+// every row a thread touches shares one decay reference.  Log-gates are kept in base-2 units
+// (scaled by log2 e on load) so each decay factor is a single ex2.
+constexpr int kPrepThreads = 256;
 constexpr uint32_t PREP_X0 = 0, PREP_X1 = 32768, PREP_R = 65536, PREP_KT = 81920, PREP_SMALL = 98304;
-constexpr uint32_t PREP_SMEM = PREP_SMALL + (64 + 512 + 128 + 128) * 4 + 16 + 1024;
+constexpr uint32_t PREP_SMEM = PREP_SMALL + (64 + 512 + 512 + 128) * 4 + 16 + 1024;
 constexpr uint32_t kPrepTmemCols = 256;
+constexpr int kAS = 68;  // fp32 row stride of the 64 x 64 A / T tile (16-byte aligned rows)
+
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+__device__ __forceinline__ float2 ex2v(float2 x) { return make_float2(ex2(x.x), ex2(x.y)); }
 
 __global__ void __launch_bounds__(kPrepThreads, 2)
 kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
@@ -148,17 +165,17 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
     uint8_t *sm = align1024(smem_raw);
     uint8_t *X0 = sm + PREP_X0;   // Gram strip operand (strips 0 then 2)
     uint8_t *X1 = sm + PREP_X1;   // Gram strip operand (strips 1 then 3)
-    uint8_t *Rimg = sm + PREP_R;  // K o e^{E_b(i) - G_i}: K-major 64 x 128
-    uint8_t *KT = sm + PREP_KT;   // K o e^G: MN-major 64 k-rows x 128
+    uint8_t *Rimg = sm + PREP_R;  // K o 2^{E_b(i) - G_i}: K-major 64 x 128
+    uint8_t *KT = sm + PREP_KT;   // K o 2^G: MN-major 64 k-rows x 128
     float *s_beta = reinterpret_cast<float *>(sm + PREP_SMALL);
-    float *s_E = s_beta + 64;  // [4][128]
-    float *s_tot = s_E + 512;  // [128]
-    float *s_gl = s_tot + 128; // [128]
+    float *s_E = s_beta + 64;   // [4][128] block references (base 2)
+    float *s_tot = s_E + 512;   // [4][128] per-block gate sums (base 2)
+    float *s_gl = s_tot + 512;  // [128]    G_63 (base 2)
     uint64_t *mbar = reinterpret_cast<uint64_t *>(s_gl + 128);
     uint32_t *s_tmem = reinterpret_cast<uint32_t *>(mbar + 1);
-    // reused after the Gram matrices are read out
-    float *Asm = reinterpret_cast<float *>(X0);              // [64][65] fp32: A, then T in place
-    float *Mscr = reinterpret_cast<float *>(X0 + 16640);     // [16][48] fp32 scratch
+    // reused once the Gram matrices are read out
+    float *Asm = reinterpret_cast<float *>(X0);              // [64][kAS] fp32: A, then T in place
+    float *Mscr = reinterpret_cast<float *>(X0 + 17408);     // [16][48] fp32 scratch
     uint8_t *TB = X0 + 20480;                                // T Diag(beta): K-major 64 x 64
     uint8_t *Vimg = X1;                                      // V: MN-major 64 k-rows x 128
 
@@ -178,8 +195,9 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
     uint8_t *rec = records + ((size_t)chunk * H + h) * REC_BYTES;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int c0 = 2 * ((warp & 1) * 32 + lane);  // this thread's two key channels
-    const int hr = warp >> 1;                     // rows 32 hr .. 32 hr + 31
+    const int c0 = 64 * (warp & 1) + 2 * lane;  // this thread's two key channels
+    const int qr = warp >> 1;                   // key block: rows 16 qr .. 16 qr + 15
+    constexpr float kLog2e = 1.4426950408889634f;
 
     if (tid == 0) {
         mbar_init(mbar, 1);
@@ -190,14 +208,14 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
         tmem_relinquish();
     }
 
-    // ---- load this thread's k, q (bf16 pairs) and log-gates (fp32 pairs) for its 32 rows
+    // ---- load k, q (bf16 pairs) and log-gates (fp32 pairs) of this thread's 16 rows
     const size_t tok_stride = (size_t)H * D;
     const size_t off0 = ((size_t)t0 * H + h) * D + c0;
-    float2 g[32];
-    uint32_t kk[32], qq[32];
+    float2 g[16];
+    uint32_t kk[16], qq[16];
 #pragma unroll
-    for (int m = 0; m < 32; ++m) {
-        const int r = 32 * hr + m;
+    for (int m = 0; m < 16; ++m) {
+        const int r = 16 * qr + m;
         if (r < L) {
             const size_t off = off0 + (size_t)r * tok_stride;
             g[m] = __ldcs(reinterpret_cast<const float2 *>(log_alpha + off));
@@ -211,68 +229,59 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
     }
     if (tid < 64) s_beta[tid] = tid < L ? __ldg(beta + ((size_t)t0 + tid) * H + h) : 0.f;
 
-    // ---- chunk-local cumulative log-gate G (fp32), halves joined through shared memory
+    // ---- chunk-local cumulative log2-gate G (fp32): block-local prefix, then block offsets
+    g[0] = make_float2(g[0].x * kLog2e, g[0].y * kLog2e);
 #pragma unroll
-    for (int m = 1; m < 32; ++m) g[m] = make_float2(g[m].x + g[m - 1].x, g[m].y + g[m - 1].y);
-    if (hr == 0) {
-        s_tot[c0] = g[31].x;
-        s_tot[c0 + 1] = g[31].y;
-    }
+    for (int m = 1; m < 16; ++m) g[m] = make_float2(fmaf(g[m].x, kLog2e, g[m - 1].x), fmaf(g[m].y, kLog2e, g[m - 1].y));
+    s_tot[qr * D + c0] = g[15].x;
+    s_tot[qr * D + c0 + 1] = g[15].y;
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *s_tmem;
-    if (hr == 1) {
-        const float2 t = make_float2(s_tot[c0], s_tot[c0 + 1]);
+    {
+        float2 base = make_float2(0.f, 0.f);
 #pragma unroll
-        for (int m = 0; m < 32; ++m) g[m] = make_float2(g[m].x + t.x, g[m].y + t.y);
+        for (int b = 0; b < 3; ++b)
+            if (b < qr) base = make_float2(base.x + s_tot[b * D + c0], base.y + s_tot[b * D + c0 + 1]);
+#pragma unroll
+        for (int m = 0; m < 16; ++m) g[m] = make_float2(g[m].x + base.x, g[m].y + base.y);
     }
-    s_E[(2 * hr) * D + c0] = g[7].x;
-    s_E[(2 * hr) * D + c0 + 1] = g[7].y;
-    s_E[(2 * hr + 1) * D + c0] = g[23].x;
-    s_E[(2 * hr + 1) * D + c0 + 1] = g[23].y;
-    if (hr == 1) {
-        s_gl[c0] = g[31].x;
-        s_gl[c0 + 1] = g[31].y;
+    const float2 Eown = g[7];  // reference of this block: G at row 16 qr + 7
+    s_E[qr * D + c0] = Eown.x;
+    s_E[qr * D + c0 + 1] = Eown.y;
+    if (qr == 3) {
+        s_gl[c0] = g[15].x;
+        s_gl[c0 + 1] = g[15].y;
     }
     __syncthreads();
 
-    float2 E[4];
-#pragma unroll
-    for (int b = 0; b < 4; ++b) E[b] = make_float2(s_E[b * D + c0], s_E[b * D + c0 + 1]);
     const float2 gl = make_float2(s_gl[c0], s_gl[c0 + 1]);
-    // references of this thread's own two blocks (b = 2 hr + bi), selected without dynamic indexing
-    const float2 Eown[2] = {hr ? E[2] : E[0], hr ? E[3] : E[1]};
-    // per own block: cross-block factors e^{E_b - E_a} (a <= b, else 0), e^{E_b}, e^{G_63 - E_b}
-    float2 Cba[2][4], eE[2], eGL[2];
+    // cross-block factors 2^{E_own - E_a} for a <= own block (else 0), 2^{E_own}, 2^{G_63 - E_own}
+    float2 Cs[4];
 #pragma unroll
-    for (int bi = 0; bi < 2; ++bi) {
-        const int b = 2 * hr + bi;
-#pragma unroll
-        for (int a = 0; a < 4; ++a) Cba[bi][a] = a <= b ? expv(sub2(Eown[bi], E[a])) : make_float2(0.f, 0.f);
-        eE[bi] = expv(Eown[bi]);
-        eGL[bi] = expv(sub2(gl, Eown[bi]));
-    }
+    for (int a = 0; a < 4; ++a)
+        Cs[a] = a <= qr ? ex2v(sub2(Eown, make_float2(s_E[a * D + c0], s_E[a * D + c0 + 1]))) : make_float2(0.f, 0.f);
+    const float2 eE = ex2v(Eown), eGL = ex2v(sub2(gl, Eown));
 
-    // ---- phase A: operands for Gram strips 0 and 1, R, K o e^G (smem); Q o e^G and K o e^{G63-G} (record)
+    // ---- phase A: strips 0 and 1, R, K o 2^G (smem); Q o 2^G and K o 2^{G63-G} (record)
 #pragma unroll
-    for (int m = 0; m < 32; ++m) {
-        const int r = 32 * hr + m, bi = m >> 4;
-        const float2 F = expv(sub2(g[m], Eown[bi]));
-        const float2 Rf = expv(sub2(Eown[bi], g[m]));
+    for (int m = 0; m < 16; ++m) {
+        const int r = 16 * qr + m;
+        const float2 F = ex2v(sub2(g[m], Eown));
+        const float2 Rf = ex2v(sub2(Eown, g[m]));
         const float2 kf = unpack_bf16(kk[m]), qf = unpack_bf16(qq[m]);
         const float2 kF = mul2(kf, F), qF = mul2(qf, F);
-        const float2 c_0 = Cba[bi][0], c_1 = Cba[bi][1];
-        *reinterpret_cast<uint32_t *>(X0 + sw128_off(r, c0, 128)) = pack_bf16(kF.x * c_0.x, kF.y * c_0.y);
-        *reinterpret_cast<uint32_t *>(X0 + sw128_off(64 + r, c0, 128)) = pack_bf16(qF.x * c_0.x, qF.y * c_0.y);
-        *reinterpret_cast<uint32_t *>(X1 + sw128_off(r, c0, 128)) = pack_bf16(kF.x * c_1.x, kF.y * c_1.y);
-        *reinterpret_cast<uint32_t *>(X1 + sw128_off(64 + r, c0, 128)) = pack_bf16(qF.x * c_1.x, qF.y * c_1.y);
+        *reinterpret_cast<uint32_t *>(X0 + sw128_off(r, c0, 128)) = pack_bf16(kF.x * Cs[0].x, kF.y * Cs[0].y);
+        *reinterpret_cast<uint32_t *>(X0 + sw128_off(64 + r, c0, 128)) = pack_bf16(qF.x * Cs[0].x, qF.y * Cs[0].y);
+        *reinterpret_cast<uint32_t *>(X1 + sw128_off(r, c0, 128)) = pack_bf16(kF.x * Cs[1].x, kF.y * Cs[1].y);
+        *reinterpret_cast<uint32_t *>(X1 + sw128_off(64 + r, c0, 128)) = pack_bf16(qF.x * Cs[1].x, qF.y * Cs[1].y);
         *reinterpret_cast<uint32_t *>(Rimg + sw128_off(r, c0, 64)) = pack_bf16(kf.x * Rf.x, kf.y * Rf.y);
-        *reinterpret_cast<uint32_t *>(KT + sw128_off(r, c0, 64)) = pack_bf16(kF.x * eE[bi].x, kF.y * eE[bi].y);
-        *reinterpret_cast<uint32_t *>(rec + REC_AQ + sw128_off(64 + r, c0, 128)) =
-            pack_bf16(qF.x * eE[bi].x, qF.y * eE[bi].y);
+        *reinterpret_cast<uint32_t *>(KT + sw128_off(r, c0, 64)) = pack_bf16(kF.x * eE.x, kF.y * eE.y);
+        *reinterpret_cast<uint32_t *>(rec + REC_AQ + sw128_off(64 + r, c0, 128)) = pack_bf16(qF.x * eE.x, qF.y * eE.y);
         *reinterpret_cast<uint32_t *>(rec + REC_KH + sw128_off(r, c0, 64)) =
-            pack_bf16(kf.x * Rf.x * eGL[bi].x, kf.y * Rf.y * eGL[bi].y);
+            pack_bf16(kf.x * Rf.x * eGL.x, kf.y * Rf.y * eGL.y);
+        g[m] = F;  // keep the row factor for strips 2 and 3
     }
     fence_async_smem();
     __syncthreads();
@@ -295,20 +304,18 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
 
     bool ok = mbar_wait(mbar, 0);
     ok = __syncthreads_and(ok);
-    // ---- phase B: strips 2 and 3 (only rows 32..63 are non-zero)
+    // ---- phase B: strips 2 and 3 (only key blocks 2 and 3 are non-zero)
     if (ok) {
 #pragma unroll
-        for (int m = 0; m < 32; ++m) {
-            const int r = 32 * hr + m, bi = m >> 4;
+        for (int m = 0; m < 16; ++m) {
+            const int r = 16 * qr + m;
             uint32_t k2 = 0, q2 = 0, k3 = 0, q3 = 0;
-            if (hr == 1) {
-                const float2 F = expv(sub2(g[m], Eown[bi]));
-                const float2 kF = mul2(unpack_bf16(kk[m]), F), qF = mul2(unpack_bf16(qq[m]), F);
-                const float2 c_2 = Cba[bi][2], c_3 = Cba[bi][3];
-                k2 = pack_bf16(kF.x * c_2.x, kF.y * c_2.y);
-                q2 = pack_bf16(qF.x * c_2.x, qF.y * c_2.y);
-                k3 = pack_bf16(kF.x * c_3.x, kF.y * c_3.y);
-                q3 = pack_bf16(qF.x * c_3.x, qF.y * c_3.y);
+            if (qr >= 2) {
+                const float2 kF = mul2(unpack_bf16(kk[m]), g[m]), qF = mul2(unpack_bf16(qq[m]), g[m]);
+                k2 = pack_bf16(kF.x * Cs[2].x, kF.y * Cs[2].y);
+                q2 = pack_bf16(qF.x * Cs[2].x, qF.y * Cs[2].y);
+                k3 = pack_bf16(kF.x * Cs[3].x, kF.y * Cs[3].y);
+                q3 = pack_bf16(qF.x * Cs[3].x, qF.y * Cs[3].y);
             }
             *reinterpret_cast<uint32_t *>(X0 + sw128_off(r, c0, 128)) = k2;
             *reinterpret_cast<uint32_t *>(X0 + sw128_off(64 + r, c0, 128)) = q2;
@@ -333,9 +340,9 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
         mma_commit(mbar);
     }
     // V tile for U = T Diag(beta) V, fetched while strips 2 and 3 run
-    uint4 vreg[8];
+    uint4 vreg[4];
 #pragma unroll
-    for (int s = 0; s < 8; ++s) {
+    for (int s = 0; s < 4; ++s) {
         const int idx = tid + kPrepThreads * s, row = idx >> 4, ch = idx & 15;
         vreg[s] = row < L ? __ldcs(reinterpret_cast<const uint4 *>(v + ((size_t)(t0 + row) * H + h) * D + ch * 8))
                           : make_uint4(0u, 0u, 0u, 0u);
@@ -347,39 +354,42 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
         tc_fence_after();
         // V -> MN-major operand image (X1 is free: strip 3 has completed)
 #pragma unroll
-        for (int s = 0; s < 8; ++s) {
+        for (int s = 0; s < 4; ++s) {
             const int idx = tid + kPrepThreads * s, row = idx >> 4, ch = idx & 15;
             *reinterpret_cast<uint4 *>(Vimg + sw128_off(row, ch * 8, 64)) = vreg[s];
         }
-        // Gram read-out: TMEM lanes 0..63 hold k-rows (A), 64..127 hold q-rows (P)
-        const int row = (warp & 1) * 32 + lane;
-        const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+        // Gram read-out: TMEM lanes 0..63 hold k-rows (A), 64..127 q-rows (P); warps w and w+4
+        // share a lane quadrant and take column halves.
+        const int quad = warp & 3, hc = warp >> 2;
+        const int row = (quad & 1) * 32 + lane;
+        float vals[32];
+        tmem_ld32(tmem + ((uint32_t)(quad * 32) << 16) + 32 * hc, vals);
+        tmem_wait_ld();
+        if (quad < 2) {
+            const float br = s_beta[row];
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-            float vals[32];
-            tmem_ld32(tmem + lane_base + 32 * half, vals);
-            tmem_wait_ld();
-            if (warp < 2) {
-                const float br = s_beta[row];
+            for (int x = 0; x < 8; ++x) {
+                float4 w4;
+                const int col = 32 * hc + 4 * x;
+                w4.x = col + 0 < row ? br * vals[4 * x + 0] : 0.f;
+                w4.y = col + 1 < row ? br * vals[4 * x + 1] : 0.f;
+                w4.z = col + 2 < row ? br * vals[4 * x + 2] : 0.f;
+                w4.w = col + 3 < row ? br * vals[4 * x + 3] : 0.f;
+                *reinterpret_cast<float4 *>(Asm + row * kAS + col) = w4;
+            }
+        } else {
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const int col = 32 * half + i;
-                    Asm[row * 65 + col] = col < row ? br * vals[i] : 0.f;
+            for (int cq = 0; cq < 4; ++cq) {
+                uint32_t w[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int col = 32 * hc + 8 * cq + 2 * e;
+                    w[e] = pack_bf16(col <= row ? vals[8 * cq + 2 * e] : 0.f,
+                                     col + 1 <= row ? vals[8 * cq + 2 * e + 1] : 0.f);
                 }
-            } else {
-#pragma unroll
-                for (int cq = 0; cq < 4; ++cq) {
-                    uint32_t w[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int col = 32 * half + 8 * cq + 2 * e;
-                        w[e] = pack_bf16(col <= row ? vals[8 * cq + 2 * e] : 0.f,
-                                         col + 1 <= row ? vals[8 * cq + 2 * e + 1] : 0.f);
-                    }
-                    const int chunk16 = 4 * half + cq;
-                    *reinterpret_cast<uint4 *>(rec + REC_P + row * 128 + ((chunk16 ^ (row & 7)) << 4)) =
-                        make_uint4(w[0], w[1], w[2], w[3]);
-                }
+                const int chunk16 = 4 * hc + cq;
+                *reinterpret_cast<uint4 *>(rec + REC_P + row * 128 + ((chunk16 ^ (row & 7)) << 4)) =
+                    make_uint4(w[0], w[1], w[2], w[3]);
             }
         }
     }
@@ -395,41 +405,55 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
             for (int rr = 0; rr < 16; ++rr) {
                 float s = 0.f;
 #pragma unroll
-                for (int ii = 0; ii < rr; ++ii) s = fmaf(Asm[(o + rr) * 65 + o + ii], x[ii], s);
+                for (int i4 = 0; i4 < (rr + 3) / 4; ++i4) {
+                    const float4 a4 = *reinterpret_cast<const float4 *>(Asm + (o + rr) * kAS + o + 4 * i4);
+                    if (4 * i4 + 0 < rr) s = fmaf(a4.x, x[4 * i4 + 0], s);
+                    if (4 * i4 + 1 < rr) s = fmaf(a4.y, x[4 * i4 + 1], s);
+                    if (4 * i4 + 2 < rr) s = fmaf(a4.z, x[4 * i4 + 2], s);
+                    if (4 * i4 + 3 < rr) s = fmaf(a4.w, x[4 * i4 + 3], s);
+                }
                 x[rr] = rr == j ? 1.f : (rr > j ? -s : 0.f);
             }
-            __syncwarp();
-            asm volatile("bar.sync 1, 64;" ::: "memory");
+            asm volatile("bar.sync 1, 64;" ::: "memory");  // every A_bb entry read before T_bb lands
 #pragma unroll
-            for (int rr = 0; rr < 16; ++rr) Asm[(o + rr) * 65 + o + j] = x[rr];
+            for (int rr = 0; rr < 16; ++rr) Asm[(o + rr) * kAS + o + j] = x[rr];
         }
         __syncthreads();
         for (int b = 1; b < 4; ++b) {  // block row b: T_ba = -T_bb sum_{c=a}^{b-1} A_bc T_ca
             const int ncol = 16 * b, o = 16 * b;
             for (int e = tid; e < 16 * ncol; e += kPrepThreads) {
                 const int rr = e / ncol, col = e % ncol;
+                const float *arow = Asm + (o + rr) * kAS;
                 float s = 0.f;
-                for (int i = col & ~15; i < o; ++i) s = fmaf(Asm[(o + rr) * 65 + i], Asm[i * 65 + col], s);
+                for (int i = col & ~15; i < o; i += 4) {
+                    const float4 a4 = *reinterpret_cast<const float4 *>(arow + i);
+                    s = fmaf(a4.x, Asm[(i + 0) * kAS + col], s);
+                    s = fmaf(a4.y, Asm[(i + 1) * kAS + col], s);
+                    s = fmaf(a4.z, Asm[(i + 2) * kAS + col], s);
+                    s = fmaf(a4.w, Asm[(i + 3) * kAS + col], s);
+                }
                 Mscr[rr * 48 + col] = s;
             }
             __syncthreads();
             for (int e = tid; e < 16 * ncol; e += kPrepThreads) {
                 const int rr = e / ncol, col = e % ncol;
                 float s = 0.f;
-                for (int jj = 0; jj <= rr; ++jj) s = fmaf(Asm[(o + rr) * 65 + o + jj], Mscr[jj * 48 + col], s);
-                Asm[(o + rr) * 65 + col] = -s;
+                for (int jj = 0; jj <= rr; ++jj) s = fmaf(Asm[(o + rr) * kAS + o + jj], Mscr[jj * 48 + col], s);
+                Asm[(o + rr) * kAS + col] = -s;
             }
             __syncthreads();
         }
         // T Diag(beta) -> bf16 K-major operand (64 x 64)
         for (int e = tid; e < 64 * 8; e += kPrepThreads) {
             const int r = e >> 3, j = e & 7;
+            const float4 t0v = *reinterpret_cast<const float4 *>(Asm + r * kAS + 8 * j);
+            const float4 t1v = *reinterpret_cast<const float4 *>(Asm + r * kAS + 8 * j + 4);
+            const float tv[8] = {t0v.x, t0v.y, t0v.z, t0v.w, t1v.x, t1v.y, t1v.z, t1v.w};
             uint32_t w[4];
 #pragma unroll
             for (int x = 0; x < 4; ++x) {
                 const int i0 = 8 * j + 2 * x;
-                w[x] = pack_bf16(i0 <= r ? Asm[r * 65 + i0] * s_beta[i0] : 0.f,
-                                 i0 + 1 <= r ? Asm[r * 65 + i0 + 1] * s_beta[i0 + 1] : 0.f);
+                w[x] = pack_bf16(i0 <= r ? tv[2 * x] * s_beta[i0] : 0.f, i0 + 1 <= r ? tv[2 * x + 1] * s_beta[i0 + 1] : 0.f);
             }
             *reinterpret_cast<uint4 *>(TB + r * 128 + ((j ^ (r & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
         }
@@ -451,30 +475,30 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
         }
         mma_commit(mbar);
     }
-    if (ok) reinterpret_cast<float *>(rec + REC_GL)[tid] = __expf(s_gl[tid]);
+    if (ok && tid < D) reinterpret_cast<float *>(rec + REC_GL)[tid] = ex2(s_gl[tid]);
     if (ok) ok = mbar_wait(mbar, 0);
     ok = __syncthreads_and(ok);
     if (ok) {
         tc_fence_after();
-        // M=64 accumulator layout: row 16 w + l lives in TMEM lane 32 w + l (l < 16)
-        const int r = 16 * warp + lane;
-        const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+        // M=64 accumulator layout: row 16 q + l lives in TMEM lane 32 q + l (l < 16).  Warps 0-3 read
+        // W (columns 0..127), warps 4-7 read U (columns 128..255) of their lane quadrant.
+        const int quad = warp & 3, part = warp >> 2;
+        const int r = 16 * quad + lane;
+        const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
 #pragma unroll 1
-        for (int cb = 0; cb < 8; ++cb) {
+        for (int cb = 0; cb < 4; ++cb) {
             float vals[32];
-            tmem_ld32(tmem + lane_base + 32 * cb, vals);
+            tmem_ld32(tmem + lane_base + 128 * part + 32 * cb, vals);
             tmem_wait_ld();
             if (lane < 16) {
 #pragma unroll
                 for (int x = 0; x < 4; ++x) {
                     const uint4 w = make_uint4(pack_bf16(vals[8 * x + 0], vals[8 * x + 1]), pack_bf16(vals[8 * x + 2], vals[8 * x + 3]),
                                                pack_bf16(vals[8 * x + 4], vals[8 * x + 5]), pack_bf16(vals[8 * x + 6], vals[8 * x + 7]));
-                    if (cb < 4) {
-                        const int col = 32 * cb + 8 * x;
-                        *reinterpret_cast<uint4 *>(rec + REC_AQ + sw128_off(r, col, 128)) = w;
-                    } else {
-                        const int col = 32 * (cb - 4) + 8 * x;
-                        *reinterpret_cast<uint4 *>(rec + REC_U + (r * D + col) * 2) = w;
+                    if (part == 0) {
+                        *reinterpret_cast<uint4 *>(rec + REC_AQ + sw128_off(r, 32 * cb + 8 * x, 128)) = w;
+                    } else {  // U, one contiguous 64 x 32 block per 32-column slice
+                        *reinterpret_cast<uint4 *>(rec + REC_U + cb * 4096 + sw64_chunk(r, x)) = w;
                     }
                 }
             }
@@ -488,15 +512,44 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
 }
 
 // ============================================================================ state-passing kernel
+// One CTA per (sequence, head, 32 value columns).  Warps 0-3 own the 128 state rows (TMEM lanes)
+// and keep the fp32 master state in registers; thread 0 issues the MMAs on the recurrence's
+// critical path right after a named barrier.  Warp 4 streams the chunk records into a 3-stage
+// shared-memory ring with bulk copies and issues the output MMAs, which stay off the critical path:
+//   critical:  D_w = W S  (M=64)  ->  Delta = U - D_w  ->  D_b = K^T Delta (M=128)  ->  S = g S + D_b
+//   output:    D_o[i%2] = Q~ S + P Delta  (M=64), read out while the next chunk's K^T Delta runs.
+// S and Delta operand images are double-buffered so the output MMAs of chunk i may still read
+// them while chunk i+1 proceeds.
 constexpr int kNV = 32;            // value columns per CTA
 constexpr int kStages = 3;
-constexpr uint32_t ST_AQ = 0, ST_KH = 32768, ST_AC = 49152, ST_GL = 65536, ST_BYTES = 66560;
-constexpr uint32_t ST_SIMG = kStages * ST_BYTES;     // S (bf16) operand: K-major 32 x 128
-constexpr uint32_t ST_DIMG = ST_SIMG + 8192;         // Delta operand: K-major 32 x 64
-constexpr uint32_t ST_BAR = ST_DIMG + 4096;
-constexpr uint32_t STATE_SMEM = ST_BAR + 128 + 1024;
-constexpr int kStateThreads = 160;  // warps 0-3: TMEM lanes / state rows; warp 4: copies + MMA issue
-constexpr uint32_t kStateTmemCols = 64;
+constexpr uint32_t ST_AQ = 0, ST_KH = 32768, ST_P = 49152, ST_U = 57344, ST_GL = 61440, ST_BYTES = 62464;
+constexpr uint32_t ST_SIMG = kStages * ST_BYTES;     // 2 x S (bf16) operand: MN-major sw64, 128 k-rows x 32
+constexpr uint32_t ST_DIMG = ST_SIMG + 2 * 8192;     // 2 x Delta operand: MN-major sw64, 64 k-rows x 32
+constexpr uint32_t ST_BAR = ST_DIMG + 2 * 4096;
+constexpr uint32_t STATE_SMEM = ST_BAR + 256 + 1024;
+constexpr int kStateThreads = 160;
+constexpr uint32_t kStateTmemCols = 128;  // D_w [0,32) | D_b [32,64) | D_o[0] [64,96) | D_o[1] [96,128)
+
+// 64-byte-swizzled operand descriptor (MN-major tiles 32 bf16 wide).
+__device__ __forceinline__ uint64_t smem_desc_sw64(uint32_t start, uint32_t sbo) {
+    uint64_t d = 0;
+    d |= (uint64_t)((start >> 4) & 0x3FFFu);
+    d |= (uint64_t)1 << 16;  // leading byte offset (unused: the tile is one 32-element atom wide)
+    d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+    d |= (uint64_t)1 << 46;
+    d |= (uint64_t)4 << 61;  // 64-byte swizzle
+    return d;
+}
+// Named barrier over the 128 compute threads that also ANDs a per-thread flag.
+__device__ __forceinline__ bool bar_and(int id, bool pred) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.and.pred q, %2, 128, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)pred), "r"(id)
+        : "memory");
+    return r != 0;
+}
 
 __global__ void __launch_bounds__(kStateThreads, 1)
 kda_tc_state_kernel(const uint8_t *__restrict__ records, const float *__restrict__ h0,
@@ -504,14 +557,17 @@ kda_tc_state_kernel(const uint8_t *__restrict__ records, const float *__restrict
                     __nv_bfloat16 *__restrict__ o, float *__restrict__ h_T, int *status) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = align1024(smem_raw);
-    uint8_t *Simg = sm + ST_SIMG;
-    uint8_t *Dimg = sm + ST_DIMG;
-    uint64_t *full = reinterpret_cast<uint64_t *>(sm + ST_BAR);  // [kStages]
-    uint64_t *s_ready = full + kStages;
-    uint64_t *d_ready = s_ready + 1;
-    uint64_t *a_done = d_ready + 1;
-    uint64_t *bc_done = a_done + 1;
-    uint32_t *s_tmem = reinterpret_cast<uint32_t *>(bc_done + 1);
+    uint8_t *Simg = sm + ST_SIMG;  // [2][8 KiB], chunk i reads image i % 2
+    uint8_t *Dimg = sm + ST_DIMG;  // [2][4 KiB], chunk i writes image i % 2
+    // Every barrier below can run at most one phase ahead of the threads that wait on it, so the
+    // parity waits are unambiguous: per-stage full/empty, per-buffer output and hand-off barriers.
+    uint64_t *full = reinterpret_cast<uint64_t *>(sm + ST_BAR);  // [kStages] record landed
+    uint64_t *empty = full + kStages;   // [kStages] MMA-b and the output MMAs of the stage's chunk done
+    uint64_t *bar_w = empty + kStages;  // W S done
+    uint64_t *bar_b = bar_w + 1;        // K^T Delta done
+    uint64_t *bar_o = bar_b + 1;        // [2] output MMAs of chunk i done (i % 2)
+    uint64_t *d_ready = bar_o + 2;      // [2] Delta of chunk i written and MMA-b issued (i % 2)
+    uint32_t *s_tmem = reinterpret_cast<uint32_t *>(d_ready + 2);
 
     int bid = blockIdx.x;
     const int slice = bid % (D / kNV);
@@ -529,32 +585,36 @@ kda_tc_state_kernel(const uint8_t *__restrict__ records, const float *__restrict
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
     if (tid == 0) {
-        for (int s = 0; s < kStages; ++s) mbar_init(&full[s], 1);
-        mbar_init(s_ready, 128);
-        mbar_init(d_ready, 64);
-        mbar_init(a_done, 1);
-        mbar_init(bc_done, 1);
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 2);
+        }
+        mbar_init(bar_w, 1);
+        mbar_init(bar_b, 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&bar_o[b], 1);
+            mbar_init(&d_ready[b], 1);
+        }
         mbar_fence_init();
     }
     if (warp == 0) {
         tmem_alloc(s_tmem, kStateTmemCols);
         tmem_relinquish();
     }
-    // zero the upper half of each [0; P] operand (rows 0..63 of a 128-row K-major tile)
-    for (int e = tid; e < kStages * 512; e += kStateThreads) {
-        const int s = e / 512, x = e % 512;
-        reinterpret_cast<uint4 *>(sm + s * ST_BYTES + ST_AC)[x] = make_uint4(0u, 0u, 0u, 0u);
-    }
-    fence_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *s_tmem;
-    bool ok = true;
+    const uint32_t D_W = tmem + 0, D_B = tmem + 32, D_O = tmem + 64;
+    // MMA shapes: [M, N=32]; A K-major unless noted, B (S, Delta) MN-major
+    const uint32_t id_w = idesc_bf16_f32(64, kNV, 0, 1);   // W S, Q~ S, P Delta
+    const uint32_t id_b = idesc_bf16_f32(128, kNV, 1, 1);  // K^T Delta (K^ stored MN-major)
+    const uint32_t sm_base = smem_u32(sm);
 
     if (warp == 4) {
-        // ------------------------------------------------ copies + MMA issue (one thread)
+        // ------------------------------------------------ bulk copies + output MMAs (one thread)
         if (lane == 0) {
+            bool ok = true;
             auto issue_load = [&](int i) {
                 const int s = i % kStages;
                 uint8_t *st = sm + s * ST_BYTES;
@@ -562,38 +622,34 @@ kda_tc_state_kernel(const uint8_t *__restrict__ records, const float *__restrict
                 mbar_arrive_expect_tx(&full[s], REC_TX);
                 bulk_g2s(st + ST_AQ, rec + REC_AQ, 32768, &full[s]);
                 bulk_g2s(st + ST_KH, rec + REC_KH, 16384, &full[s]);
-                bulk_g2s(st + ST_AC + 8192, rec + REC_P, 8192, &full[s]);
+                bulk_g2s(st + ST_P, rec + REC_P, 8192, &full[s]);
+                bulk_g2s(st + ST_U, rec + REC_U + slice * 4096, 4096, &full[s]);
                 bulk_g2s(st + ST_GL, rec + REC_GL, 512, &full[s]);
             };
             for (int i = 0; i < kStages && i < nchunks; ++i) issue_load(i);
-            const uint32_t id_a = idesc_bf16_f32(128, kNV, 0, 0);
-            const uint32_t id_b = idesc_bf16_f32(128, kNV, 1, 0);
             for (int i = 0; i < nchunks && ok; ++i) {
                 const int s = i % kStages;
-                const uint32_t st = smem_u32(sm + s * ST_BYTES);
-                ok = mbar_wait(&full[s], (i / kStages) & 1) && mbar_wait(s_ready, i & 1);
-                if (!ok) break;
-                if (i >= 1 && i + kStages - 1 < nchunks) issue_load(i + kStages - 1);  // reuses chunk i-1's stage
-                tc_fence_after();
-#pragma unroll
-                for (int ks = 0; ks < 8; ++ks) {
-                    const uint64_t ad = smem_desc_sw128(st + ST_AQ + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
-                    const uint64_t bd = smem_desc_sw128(smem_u32(Simg) + (ks >> 2) * 4096 + (ks & 3) * 32, 16, 1024);
-                    mma_bf16_ss(tmem + 0, ad, bd, id_a, ks > 0);
-                }
-                mma_commit(a_done);
-                ok = mbar_wait(d_ready, i & 1);
+                const uint32_t st = sm_base + s * ST_BYTES;
+                const uint32_t simg = smem_u32(Simg) + (i & 1) * 8192;
+                ok = mbar_wait(&d_ready[i & 1], (i >> 1) & 1);
                 if (!ok) break;
                 tc_fence_after();
 #pragma unroll
-                for (int ks = 0; ks < 4; ++ks) {
-                    const uint64_t bd = smem_desc_sw128(smem_u32(Dimg) + ks * 32, 16, 1024);
-                    const uint64_t akh = smem_desc_sw128(st + ST_KH + ks * 2048, 8192, 1024);
-                    mma_bf16_ss(tmem + kNV, akh, bd, id_b, ks > 0);
-                    const uint64_t ac = smem_desc_sw128(st + ST_AC + ks * 32, 16, 1024);
-                    mma_bf16_ss(tmem + 0, ac, bd, id_a, 1);
+                for (int ks = 0; ks < 8; ++ks)  // Q~ S  (Q~ = rows 64..127 of the [W; Q~] image)
+                    mma_bf16_ss(D_O + 32 * (i & 1),
+                                smem_desc_sw128(st + ST_AQ + 8192 + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024),
+                                smem_desc_sw64(simg + ks * 1024, 512), id_w, ks > 0);
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)  // + P Delta
+                    mma_bf16_ss(D_O + 32 * (i & 1), smem_desc_sw128(st + ST_P + ks * 32, 16, 1024),
+                                smem_desc_sw64(smem_u32(Dimg) + (i & 1) * 4096 + ks * 1024, 512), id_w, 1);
+                mma_commit(&bar_o[i & 1]);
+                mma_commit(&empty[s]);
+                if (i + kStages < nchunks) {  // refill stage s once MMA-b and these MMAs are done
+                    ok = mbar_wait(&empty[s], (i / kStages) & 1);
+                    if (!ok) break;
+                    issue_load(i + kStages);
                 }
-                mma_commit(bc_done);
             }
             if (!ok) set_status(status, KDA_ERR_TIMEOUT);
         }
@@ -602,6 +658,7 @@ kda_tc_state_kernel(const uint8_t *__restrict__ records, const float *__restrict
         // ------------------------------------------------ warps 0-3: state row t = tid (TMEM lane)
         const int t = tid;
         const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+        const int r16 = 16 * warp + lane;  // row of an M=64 accumulator held by this lane (lane < 16)
         const size_t soff = (((size_t)n * H + h) * D + t) * D + j0;
         float S[kNV];
 #pragma unroll
@@ -610,79 +667,150 @@ kda_tc_state_kernel(const uint8_t *__restrict__ records, const float *__restrict
             S[4 * x] = w.x; S[4 * x + 1] = w.y; S[4 * x + 2] = w.z; S[4 * x + 3] = w.w;
         }
 #pragma unroll
-        for (int j = 0; j < kNV; ++j)
-            *reinterpret_cast<__nv_bfloat16 *>(Simg + sw128_off(j, t, kNV)) = __float2bfloat16_rn(S[j]);
+        for (int x = 0; x < 4; ++x)
+            *reinterpret_cast<uint4 *>(Simg + sw64_chunk(t, x)) =
+                make_uint4(pack_bf16(S[8 * x], S[8 * x + 1]), pack_bf16(S[8 * x + 2], S[8 * x + 3]),
+                           pack_bf16(S[8 * x + 4], S[8 * x + 5]), pack_bf16(S[8 * x + 6], S[8 * x + 7]));
         fence_async_smem();
-        mbar_arrive(s_ready);
+        bool ok = bar_and(1, true);
 
-        for (int i = 0; i < nchunks && ok; ++i) {
-            const int s = i % kStages;
-            const uint8_t *st = sm + s * ST_BYTES;
-            const int chunk = c_begin + i;
+        auto write_o = [&](int i) {  // output rows of chunk i from D_o[i % 2] (M=64 layout)
             int64_t t0;
             int L;
             if (table) {
-                const int4 e = table[chunk];
+                const int4 e = table[c_begin + i];
                 t0 = e.y;
                 L = e.z;
             } else {
                 t0 = (int64_t)n * T_len + (int64_t)i * C;
                 L = min(C, T_len - i * C);
             }
-            if (warp < 2) {
-                // Delta = U - W S for chunk row t
-                const uint8_t *urow = records + ((size_t)chunk * H + h) * REC_BYTES + REC_U + (t * D + j0) * 2;
-                uint4 u4[4];
+            float ov[32];
+            tmem_ld32(D_O + 32 * (i & 1) + lane_base, ov);
+            tmem_wait_ld();
+            // Lanes 0..15 hold rows 16 w + l; lanes l and l + 16 split the row's four 16-byte
+            // chunks so that each store instruction fills whole 32-byte sectors.
+            uint32_t pk[16];
 #pragma unroll
-                for (int x = 0; x < 4; ++x) u4[x] = *reinterpret_cast<const uint4 *>(urow + 16 * x);
-                bool w_ok = mbar_wait(a_done, i & 1);
-                if (!__all_sync(0xffffffffu, w_ok)) { ok = false; break; }
+            for (int e = 0; e < 16; ++e) pk[e] = pack_bf16(ov[2 * e], ov[2 * e + 1]);
+            const bool upper = lane >= 16;
+            const int row = 16 * warp + (lane & 15);
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+                uint32_t w[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const uint32_t mine = pk[8 * k + e];         // chunk 2k of this lane's row
+                    const uint32_t odd = pk[8 * k + 4 + e];      // chunk 2k + 1
+                    const uint32_t from_low = __shfl_sync(0xffffffffu, odd, lane & 15);
+                    w[e] = upper ? from_low : mine;
+                }
+                if (row < L) {
+                    __nv_bfloat16 *orow = o + ((size_t)(t0 + row) * H + h) * D + j0;
+                    reinterpret_cast<uint4 *>(orow)[2 * k + (upper ? 1 : 0)] = make_uint4(w[0], w[1], w[2], w[3]);
+                }
+            }
+        };
+
+        for (int i = 0; i < nchunks && ok; ++i) {
+            const int s = i % kStages;
+            const uint8_t *st = sm + s * ST_BYTES;
+            const uint32_t st_u = sm_base + s * ST_BYTES;
+            const uint32_t simg = smem_u32(Simg) + (i & 1) * 8192;
+            uint8_t *dimg = Dimg + (i & 1) * 4096;
+            // (1) W S on the critical path
+            bool w_ok = mbar_wait(&full[s], (i / kStages) & 1);
+            if (t == 0 && w_ok) {
+                tc_fence_after();
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks)
+                    mma_bf16_ss(D_W, smem_desc_sw128(st_u + ST_AQ + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024),
+                                smem_desc_sw64(simg + ks * 1024, 512), id_w, ks > 0);
+                mma_commit(bar_w);
+            }
+            // every read of stage s by these threads happens before d_ready (the stage may be refilled after)
+            const float gl = reinterpret_cast<const float *>(st + ST_GL)[t];
+            // (2) Delta = U - W S  (rows 16 w + l, l < 16)
+            w_ok = w_ok && mbar_wait(bar_w, i & 1);
+            if (__all_sync(0xffffffffu, w_ok)) {
                 tc_fence_after();
                 float ws[32];
-                tmem_ld32(tmem + lane_base + 0, ws);
+                tmem_ld32(D_W + lane_base, ws);
                 tmem_wait_ld();
+                if (lane < 16) {
 #pragma unroll
-                for (int x = 0; x < 4; ++x) {
-                    const uint32_t uw[4] = {u4[x].x, u4[x].y, u4[x].z, u4[x].w};
+                    for (int x = 0; x < 4; ++x) {
+                        const uint4 u4 = *reinterpret_cast<const uint4 *>(st + ST_U + sw64_chunk(r16, x));
+                        const uint32_t uw[4] = {u4.x, u4.y, u4.z, u4.w};
+                        uint32_t dw[4];
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float2 uf = unpack_bf16(uw[e]);
-                        const int j = 8 * x + 2 * e;
-                        *reinterpret_cast<__nv_bfloat16 *>(Dimg + sw128_off(j, t, kNV)) = __float2bfloat16_rn(uf.x - ws[j]);
-                        *reinterpret_cast<__nv_bfloat16 *>(Dimg + sw128_off(j + 1, t, kNV)) = __float2bfloat16_rn(uf.y - ws[j + 1]);
+                        for (int e = 0; e < 4; ++e) {
+                            const float2 uf = unpack_bf16(uw[e]);
+                            dw[e] = pack_bf16(uf.x - ws[8 * x + 2 * e], uf.y - ws[8 * x + 2 * e + 1]);
+                        }
+                        *reinterpret_cast<uint4 *>(dimg + sw64_chunk(r16, x)) = make_uint4(dw[0], dw[1], dw[2], dw[3]);
                     }
                 }
-                tc_fence_before();
-                fence_async_smem();
-                mbar_arrive(d_ready);
+            } else {
+                w_ok = false;
             }
-            bool w_ok = mbar_wait(&full[s], (i / kStages) & 1) && mbar_wait(bc_done, i & 1);
-            if (!__all_sync(0xffffffffu, w_ok)) { ok = false; break; }
-            tc_fence_after();
-            float upd[32], ov[32];
-            tmem_ld32(tmem + lane_base + kNV, upd);
-            if (warp >= 2) tmem_ld32(tmem + lane_base + 0, ov);
-            tmem_wait_ld();
-            const float gl = reinterpret_cast<const float *>(st + ST_GL)[t];
-#pragma unroll
-            for (int j = 0; j < kNV; ++j) S[j] = fmaf(gl, S[j], upd[j]);
-            if (warp >= 2) {
-                const int r = t - 64;
-                if (r < L) {
-                    __nv_bfloat16 *orow = o + ((size_t)(t0 + r) * H + h) * D + j0;
-#pragma unroll
-                    for (int x = 0; x < 4; ++x)
-                        reinterpret_cast<uint4 *>(orow)[x] =
-                            make_uint4(pack_bf16(ov[8 * x], ov[8 * x + 1]), pack_bf16(ov[8 * x + 2], ov[8 * x + 3]),
-                                       pack_bf16(ov[8 * x + 4], ov[8 * x + 5]), pack_bf16(ov[8 * x + 6], ov[8 * x + 7]));
-                }
-            }
-#pragma unroll
-            for (int j = 0; j < kNV; ++j)
-                *reinterpret_cast<__nv_bfloat16 *>(Simg + sw128_off(j, t, kNV)) = __float2bfloat16_rn(S[j]);
             tc_fence_before();
             fence_async_smem();
-            mbar_arrive(s_ready);
+            ok = bar_and(2, w_ok);
+            if (!ok) break;
+            // (3) K^T Delta on the critical path; warp 4 then issues this chunk's output MMAs
+            if (t == 0) {
+                tc_fence_after();
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    mma_bf16_ss(D_B, smem_desc_sw128(st_u + ST_KH + ks * 2048, 8192, 1024),
+                                smem_desc_sw64(smem_u32(dimg) + ks * 1024, 512), id_b, ks > 0);
+                mma_commit(bar_b);
+                mma_commit(&empty[s]);
+                mbar_arrive(&d_ready[i & 1]);
+            }
+            // (4) while K^T Delta runs: output rows of the previous chunk; this also retires the
+            //     MMAs that read S image (i+1) % 2 before step (5) overwrites it
+            w_ok = true;
+            if (i > 0) {
+                w_ok = mbar_wait(&bar_o[(i - 1) & 1], ((i - 1) >> 1) & 1);
+                if (__all_sync(0xffffffffu, w_ok)) {
+                    tc_fence_after();
+                    write_o(i - 1);
+                } else {
+                    w_ok = false;
+                }
+            }
+            // (5) S <- e^{G_63} S + K^T Delta; bf16 copy into the other S image
+            w_ok = w_ok && mbar_wait(bar_b, i & 1);
+            if (__all_sync(0xffffffffu, w_ok)) {
+                tc_fence_after();
+                float upd[32];
+                tmem_ld32(D_B + lane_base, upd);
+                tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < kNV; ++j) S[j] = fmaf(gl, S[j], upd[j]);
+                uint8_t *snext = Simg + ((i + 1) & 1) * 8192;
+#pragma unroll
+                for (int x = 0; x < 4; ++x)
+                    *reinterpret_cast<uint4 *>(snext + sw64_chunk(t, x)) =
+                        make_uint4(pack_bf16(S[8 * x], S[8 * x + 1]), pack_bf16(S[8 * x + 2], S[8 * x + 3]),
+                                   pack_bf16(S[8 * x + 4], S[8 * x + 5]), pack_bf16(S[8 * x + 6], S[8 * x + 7]));
+            } else {
+                w_ok = false;
+            }
+            tc_fence_before();
+            fence_async_smem();
+            ok = bar_and(1, w_ok);
+        }
+        if (ok && nchunks > 0) {  // output rows of the last chunk
+            bool w_ok = mbar_wait(&bar_o[(nchunks - 1) & 1], ((nchunks - 1) >> 1) & 1);
+            if (__all_sync(0xffffffffu, w_ok)) {
+                tc_fence_after();
+                write_o(nchunks - 1);
+            } else {
+                ok = false;
+            }
         }
         if (!ok) {
             if (lane == 0) set_status(status, KDA_ERR_TIMEOUT);
