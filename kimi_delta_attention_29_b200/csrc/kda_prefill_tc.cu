@@ -156,6 +156,47 @@ __device__ __forceinline__ float ex2(float x) {
 }
 __device__ __forceinline__ float2 ex2v(float2 x) { return make_float2(ex2(x.x), ex2(x.y)); }
 
+// Block row b of the UT transform, in place in the 64 x 64 fp32 tile Asm (row stride kAS):
+// rows 16b..16b+15 hold A_b* to the left of the already inverted diagonal block T_bb, rows above
+// hold finished T.  Computes T_ba = -T_bb sum_{c=a}^{b-1} A_bc T_ca for every a < b.  Thread
+// (rr, cb) = (tid / 16, tid % 16) owns row rr of the block row and column cb of each 16-wide
+// block a; upper triangles are stored as zeros, so every sum runs over whole 16-blocks.
+template <int b>
+__device__ __forceinline__ void subst_block_row(float *Asm, float *Mscr, int tid) {
+    constexpr int o = 16 * b;
+    const int rr = tid >> 4, cb = tid & 15;
+    // stage 1: M[rr][16a + cb] = sum_{i = 16a}^{16b-1} A[o + rr][i] T[i][16a + cb]
+    float arow[o];
+#pragma unroll
+    for (int q4 = 0; q4 < o / 4; ++q4) {
+        const float4 a4 = *reinterpret_cast<const float4 *>(Asm + (o + rr) * kAS + 4 * q4);
+        arow[4 * q4] = a4.x; arow[4 * q4 + 1] = a4.y; arow[4 * q4 + 2] = a4.z; arow[4 * q4 + 3] = a4.w;
+    }
+#pragma unroll
+    for (int a = 0; a < b; ++a) {
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int i = 16 * a; i < o; ++i) acc[i & 3] = fmaf(arow[i], Asm[i * kAS + 16 * a + cb], acc[i & 3]);
+        Mscr[rr * 48 + 16 * a + cb] = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+    }
+    __syncthreads();
+    // stage 2: T[o + rr][16a + cb] = -sum_jj T_bb[rr][jj] M[jj][16a + cb]  (T_bb lower triangular)
+    float trow[16];
+#pragma unroll
+    for (int q4 = 0; q4 < 4; ++q4) {
+        const float4 t4 = *reinterpret_cast<const float4 *>(Asm + (o + rr) * kAS + o + 4 * q4);
+        trow[4 * q4] = t4.x; trow[4 * q4 + 1] = t4.y; trow[4 * q4 + 2] = t4.z; trow[4 * q4 + 3] = t4.w;
+    }
+#pragma unroll
+    for (int a = 0; a < b; ++a) {
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int jj = 0; jj < 16; ++jj) acc[jj & 3] = fmaf(trow[jj], Mscr[jj * 48 + 16 * a + cb], acc[jj & 3]);
+        Asm[(o + rr) * kAS + 16 * a + cb] = -((acc[0] + acc[1]) + (acc[2] + acc[3]));
+    }
+    __syncthreads();
+}
+
 __global__ void __launch_bounds__(kPrepThreads, 2)
 kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
                    const __nv_bfloat16 *__restrict__ v, const float *__restrict__ log_alpha,
@@ -419,30 +460,9 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
             for (int rr = 0; rr < 16; ++rr) Asm[(o + rr) * kAS + o + j] = x[rr];
         }
         __syncthreads();
-        for (int b = 1; b < 4; ++b) {  // block row b: T_ba = -T_bb sum_{c=a}^{b-1} A_bc T_ca
-            const int ncol = 16 * b, o = 16 * b;
-            for (int e = tid; e < 16 * ncol; e += kPrepThreads) {
-                const int rr = e / ncol, col = e % ncol;
-                const float *arow = Asm + (o + rr) * kAS;
-                float s = 0.f;
-                for (int i = col & ~15; i < o; i += 4) {
-                    const float4 a4 = *reinterpret_cast<const float4 *>(arow + i);
-                    s = fmaf(a4.x, Asm[(i + 0) * kAS + col], s);
-                    s = fmaf(a4.y, Asm[(i + 1) * kAS + col], s);
-                    s = fmaf(a4.z, Asm[(i + 2) * kAS + col], s);
-                    s = fmaf(a4.w, Asm[(i + 3) * kAS + col], s);
-                }
-                Mscr[rr * 48 + col] = s;
-            }
-            __syncthreads();
-            for (int e = tid; e < 16 * ncol; e += kPrepThreads) {
-                const int rr = e / ncol, col = e % ncol;
-                float s = 0.f;
-                for (int jj = 0; jj <= rr; ++jj) s = fmaf(Asm[(o + rr) * kAS + o + jj], Mscr[jj * 48 + col], s);
-                Asm[(o + rr) * kAS + col] = -s;
-            }
-            __syncthreads();
-        }
+        subst_block_row<1>(Asm, Mscr, tid);
+        subst_block_row<2>(Asm, Mscr, tid);
+        subst_block_row<3>(Asm, Mscr, tid);
         // T Diag(beta) -> bf16 K-major operand (64 x 64)
         for (int e = tid; e < 64 * 8; e += kPrepThreads) {
             const int r = e >> 3, j = e & 7;
