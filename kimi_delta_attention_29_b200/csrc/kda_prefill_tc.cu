@@ -76,6 +76,9 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<const uint32_t *>(&v);
 }
+__device__ __forceinline__ __nv_bfloat162 as_bf2(uint32_t u) {
+    return *reinterpret_cast<const __nv_bfloat162 *>(&u);
+}
 __device__ __forceinline__ float2 unpack_bf16(uint32_t u) {
     const __nv_bfloat162 v = *reinterpret_cast<const __nv_bfloat162 *>(&u);
     return __bfloat1622float2(v);
@@ -305,23 +308,27 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
         Cs[a] = a <= qr ? ex2v(sub2(Eown, make_float2(s_E[a * D + c0], s_E[a * D + c0 + 1]))) : make_float2(0.f, 0.f);
     const float2 eE = ex2v(Eown), eGL = ex2v(sub2(gl, Eown));
 
-    // ---- phase A: strips 0 and 1, R, K o 2^G (smem); Q o 2^G and K o 2^{G63-G} (record)
+    // ---- phase A: strips 0 and 1, R, K o 2^G (smem); Q o 2^G and K o 2^{G63-G} (record).
+    // The factors are rounded to bf16 and applied with packed bf16 multiplies on the bf16 inputs.
 #pragma unroll
     for (int m = 0; m < 16; ++m) {
         const int r = 16 * qr + m;
         const float2 F = ex2v(sub2(g[m], Eown));
         const float2 Rf = ex2v(sub2(Eown, g[m]));
-        const float2 kf = unpack_bf16(kk[m]), qf = unpack_bf16(qq[m]);
-        const float2 kF = mul2(kf, F), qF = mul2(qf, F);
-        *reinterpret_cast<uint32_t *>(X0 + sw128_off(r, c0, 128)) = pack_bf16(kF.x * Cs[0].x, kF.y * Cs[0].y);
-        *reinterpret_cast<uint32_t *>(X0 + sw128_off(64 + r, c0, 128)) = pack_bf16(qF.x * Cs[0].x, qF.y * Cs[0].y);
-        *reinterpret_cast<uint32_t *>(X1 + sw128_off(r, c0, 128)) = pack_bf16(kF.x * Cs[1].x, kF.y * Cs[1].y);
-        *reinterpret_cast<uint32_t *>(X1 + sw128_off(64 + r, c0, 128)) = pack_bf16(qF.x * Cs[1].x, qF.y * Cs[1].y);
-        *reinterpret_cast<uint32_t *>(Rimg + sw128_off(r, c0, 64)) = pack_bf16(kf.x * Rf.x, kf.y * Rf.y);
-        *reinterpret_cast<uint32_t *>(KT + sw128_off(r, c0, 64)) = pack_bf16(kF.x * eE.x, kF.y * eE.y);
-        *reinterpret_cast<uint32_t *>(rec + REC_AQ + sw128_off(64 + r, c0, 128)) = pack_bf16(qF.x * eE.x, qF.y * eE.y);
-        *reinterpret_cast<uint32_t *>(rec + REC_KH + sw128_off(r, c0, 64)) =
-            pack_bf16(kf.x * Rf.x * eGL.x, kf.y * Rf.y * eGL.y);
+        const __nv_bfloat162 k2 = as_bf2(kk[m]), q2 = as_bf2(qq[m]);
+        const __nv_bfloat162 f0 = __floats2bfloat162_rn(F.x * Cs[0].x, F.y * Cs[0].y);
+        const __nv_bfloat162 f1 = __floats2bfloat162_rn(F.x * Cs[1].x, F.y * Cs[1].y);
+        const __nv_bfloat162 fe = __floats2bfloat162_rn(F.x * eE.x, F.y * eE.y);
+        const __nv_bfloat162 fr = __floats2bfloat162_rn(Rf.x, Rf.y);
+        const __nv_bfloat162 frg = __floats2bfloat162_rn(Rf.x * eGL.x, Rf.y * eGL.y);
+        *reinterpret_cast<__nv_bfloat162 *>(X0 + sw128_off(r, c0, 128)) = __hmul2(k2, f0);
+        *reinterpret_cast<__nv_bfloat162 *>(X0 + sw128_off(64 + r, c0, 128)) = __hmul2(q2, f0);
+        *reinterpret_cast<__nv_bfloat162 *>(X1 + sw128_off(r, c0, 128)) = __hmul2(k2, f1);
+        *reinterpret_cast<__nv_bfloat162 *>(X1 + sw128_off(64 + r, c0, 128)) = __hmul2(q2, f1);
+        *reinterpret_cast<__nv_bfloat162 *>(Rimg + sw128_off(r, c0, 64)) = __hmul2(k2, fr);
+        *reinterpret_cast<__nv_bfloat162 *>(KT + sw128_off(r, c0, 64)) = __hmul2(k2, fe);
+        *reinterpret_cast<__nv_bfloat162 *>(rec + REC_AQ + sw128_off(64 + r, c0, 128)) = __hmul2(q2, fe);
+        *reinterpret_cast<__nv_bfloat162 *>(rec + REC_KH + sw128_off(r, c0, 64)) = __hmul2(k2, frg);
         g[m] = F;  // keep the row factor for strips 2 and 3
     }
     fence_async_smem();
@@ -350,18 +357,19 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
 #pragma unroll
         for (int m = 0; m < 16; ++m) {
             const int r = 16 * qr + m;
-            uint32_t k2 = 0, q2 = 0, k3 = 0, q3 = 0;
+            __nv_bfloat162 k2 = as_bf2(0u), q2 = k2, k3 = k2, q3 = k2;
             if (qr >= 2) {
-                const float2 kF = mul2(unpack_bf16(kk[m]), g[m]), qF = mul2(unpack_bf16(qq[m]), g[m]);
-                k2 = pack_bf16(kF.x * Cs[2].x, kF.y * Cs[2].y);
-                q2 = pack_bf16(qF.x * Cs[2].x, qF.y * Cs[2].y);
-                k3 = pack_bf16(kF.x * Cs[3].x, kF.y * Cs[3].y);
-                q3 = pack_bf16(qF.x * Cs[3].x, qF.y * Cs[3].y);
+                const __nv_bfloat162 f2 = __floats2bfloat162_rn(g[m].x * Cs[2].x, g[m].y * Cs[2].y);
+                const __nv_bfloat162 f3 = __floats2bfloat162_rn(g[m].x * Cs[3].x, g[m].y * Cs[3].y);
+                k2 = __hmul2(as_bf2(kk[m]), f2);
+                q2 = __hmul2(as_bf2(qq[m]), f2);
+                k3 = __hmul2(as_bf2(kk[m]), f3);
+                q3 = __hmul2(as_bf2(qq[m]), f3);
             }
-            *reinterpret_cast<uint32_t *>(X0 + sw128_off(r, c0, 128)) = k2;
-            *reinterpret_cast<uint32_t *>(X0 + sw128_off(64 + r, c0, 128)) = q2;
-            *reinterpret_cast<uint32_t *>(X1 + sw128_off(r, c0, 128)) = k3;
-            *reinterpret_cast<uint32_t *>(X1 + sw128_off(64 + r, c0, 128)) = q3;
+            *reinterpret_cast<__nv_bfloat162 *>(X0 + sw128_off(r, c0, 128)) = k2;
+            *reinterpret_cast<__nv_bfloat162 *>(X0 + sw128_off(64 + r, c0, 128)) = q2;
+            *reinterpret_cast<__nv_bfloat162 *>(X1 + sw128_off(r, c0, 128)) = k3;
+            *reinterpret_cast<__nv_bfloat162 *>(X1 + sw128_off(64 + r, c0, 128)) = q3;
         }
         fence_async_smem();
     }
