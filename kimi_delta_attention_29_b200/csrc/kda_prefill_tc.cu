@@ -51,7 +51,7 @@ constexpr uint32_t REC_P = 49152;     // P: K-major sw128, 64 rows x 64 (8 KiB)
 constexpr uint32_t REC_U = 57344;     // U: bf16, four [64][32] blocks (one per 32-column slice), 64-byte swizzle
 constexpr uint32_t REC_GL = 73728;    // e^{G_63}: fp32 [128]
 constexpr uint32_t REC_BYTES = 74752;
-constexpr uint32_t REC_TX = 32768 + 16384 + 8192 + 512 + 4096;  // bytes one state CTA copies per chunk
+constexpr uint32_t REC_TX = 32768 + 16384 + 8192 + 4096 + 512;  // bytes one state CTA copies per chunk
 
 struct TcLayout {
     size_t base_off, table_off, rec_off, total;
@@ -540,23 +540,23 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
 }
 
 // ============================================================================ state-passing kernel
-// One CTA per (sequence, head, 32 value columns).  Warps 0-3 own the 128 state rows (TMEM lanes)
-// and keep the fp32 master state in registers; thread 0 issues the MMAs on the recurrence's
-// critical path right after a named barrier.  Warp 4 streams the chunk records into a 3-stage
-// shared-memory ring with bulk copies and issues the output MMAs, which stay off the critical path:
-//   critical:  D_w = W S  (M=64)  ->  Delta = U - D_w  ->  D_b = K^T Delta (M=128)  ->  S = g S + D_b
-//   output:    D_o[i%2] = Q~ S + P Delta  (M=64), read out while the next chunk's K^T Delta runs.
-// S and Delta operand images are double-buffered so the output MMAs of chunk i may still read
-// them while chunk i+1 proceeds.
+// One CTA per (sequence, head, 32 value columns); the value columns of S evolve independently.
+// Warps 0-3 own the 128 state rows (TMEM lanes) and keep the fp32 master state in registers,
+// warp 4 streams the chunk records into a 2-stage shared-memory ring with bulk copies, warp 5
+// issues every MMA.  Warps 0-3 and 5 meet at two named barriers per chunk.  Per chunk i:
+//   D_a[i%2]  = [W; Q~] S        (M=128, N=32, K=128)   rows 0..63 -> Delta = U - W S
+//   D_b       = K^T Delta        (M=128, N=32, K=64)    -> S <- e^{G_63} S + D_b
+//   D_a[i%2] += [0; P] Delta     (M=128, N=32, K=64)    rows 64..127 = output, read during chunk i+1
+// Only the first two products are on the recurrence's critical path.
 constexpr int kNV = 32;            // value columns per CTA
-constexpr int kStages = 3;
-constexpr uint32_t ST_AQ = 0, ST_KH = 32768, ST_P = 49152, ST_U = 57344, ST_GL = 61440, ST_BYTES = 62464;
-constexpr uint32_t ST_SIMG = kStages * ST_BYTES;     // 2 x S (bf16) operand: MN-major sw64, 128 k-rows x 32
-constexpr uint32_t ST_DIMG = ST_SIMG + 2 * 8192;     // 2 x Delta operand: MN-major sw64, 64 k-rows x 32
-constexpr uint32_t ST_BAR = ST_DIMG + 2 * 4096;
+constexpr int kStages = 2;
+constexpr uint32_t ST_AQ = 0, ST_KH = 32768, ST_AC = 49152, ST_U = 65536, ST_GL = 69632, ST_BYTES = 70656;
+constexpr uint32_t ST_SIMG = kStages * ST_BYTES;  // S (bf16): MN-major sw64, 128 k-rows x 32 (8 KiB)
+constexpr uint32_t ST_DIMG = ST_SIMG + 8192;      // Delta (bf16): MN-major sw64, 64 k-rows x 32 (4 KiB)
+constexpr uint32_t ST_BAR = ST_DIMG + 4096;
 constexpr uint32_t STATE_SMEM = ST_BAR + 256 + 1024;
-constexpr int kStateThreads = 160;
-constexpr uint32_t kStateTmemCols = 128;  // D_w [0,32) | D_b [32,64) | D_o[0] [64,96) | D_o[1] [96,128)
+constexpr int kStateThreads = 192;        // warps 0-3 state rows, warp 4 copies, warp 5 MMAs
+constexpr uint32_t kStateTmemCols = 128;  // D_a[0] [0,32) | D_a[1] [32,64) | D_b [64,96)
 
 // 64-byte-swizzled operand descriptor (MN-major tiles 32 bf16 wide).
 __device__ __forceinline__ uint64_t smem_desc_sw64(uint32_t start, uint32_t sbo) {
@@ -568,11 +568,11 @@ __device__ __forceinline__ uint64_t smem_desc_sw64(uint32_t start, uint32_t sbo)
     d |= (uint64_t)4 << 61;  // 64-byte swizzle
     return d;
 }
-// Named barrier over the 128 compute threads that also ANDs a per-thread flag.
-__device__ __forceinline__ bool bar_and(int id, bool pred) {
+// Named barrier over warps 0-3 and 5 (160 threads) that also ANDs a per-thread flag.
+__device__ __forceinline__ bool bar_and160(int id, bool pred) {
     uint32_t r;
     asm volatile(
-        "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.and.pred q, %2, 128, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+        "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.and.pred q, %2, 160, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
         : "=r"(r)
         : "r"((uint32_t)pred), "r"(id)
         : "memory");
@@ -585,17 +585,16 @@ kda_tc_state_kernel(const uint8_t *__restrict__ records, const float *__restrict
                     __nv_bfloat16 *__restrict__ o, float *__restrict__ h_T, int *status) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = align1024(smem_raw);
-    uint8_t *Simg = sm + ST_SIMG;  // [2][8 KiB], chunk i reads image i % 2
-    uint8_t *Dimg = sm + ST_DIMG;  // [2][4 KiB], chunk i writes image i % 2
-    // Every barrier below can run at most one phase ahead of the threads that wait on it, so the
-    // parity waits are unambiguous: per-stage full/empty, per-buffer output and hand-off barriers.
+    uint8_t *Simg = sm + ST_SIMG;
+    uint8_t *Dimg = sm + ST_DIMG;
+    // Each barrier completes once per chunk (per use of a stage) and cannot complete a second
+    // time before its waiters have seen the first, so the parity waits are unambiguous.
     uint64_t *full = reinterpret_cast<uint64_t *>(sm + ST_BAR);  // [kStages] record landed
-    uint64_t *empty = full + kStages;   // [kStages] MMA-b and the output MMAs of the stage's chunk done
-    uint64_t *bar_w = empty + kStages;  // W S done
+    uint64_t *empty = full + kStages;   // [kStages] the three products of the stage's chunk are done
+    uint64_t *bar_w = empty + kStages;  // [W; Q~] S done
     uint64_t *bar_b = bar_w + 1;        // K^T Delta done
-    uint64_t *bar_o = bar_b + 1;        // [2] output MMAs of chunk i done (i % 2)
-    uint64_t *d_ready = bar_o + 2;      // [2] Delta of chunk i written and MMA-b issued (i % 2)
-    uint32_t *s_tmem = reinterpret_cast<uint32_t *>(d_ready + 2);
+    uint64_t *bar_c = bar_b + 1;        // [0; P] Delta done (and every earlier product)
+    uint32_t *s_tmem = reinterpret_cast<uint32_t *>(bar_c + 1);
 
     int bid = blockIdx.x;
     const int slice = bid % (D / kNV);
@@ -615,32 +614,30 @@ kda_tc_state_kernel(const uint8_t *__restrict__ records, const float *__restrict
     if (tid == 0) {
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], 2);
+            mbar_init(&empty[s], 1);
         }
         mbar_init(bar_w, 1);
         mbar_init(bar_b, 1);
-        for (int b = 0; b < 2; ++b) {
-            mbar_init(&bar_o[b], 1);
-            mbar_init(&d_ready[b], 1);
-        }
+        mbar_init(bar_c, 1);
         mbar_fence_init();
     }
     if (warp == 0) {
         tmem_alloc(s_tmem, kStateTmemCols);
         tmem_relinquish();
     }
+    for (int e = tid; e < kStages * 512; e += kStateThreads) {  // zero half of each [0; P] operand
+        const int s = e / 512, x = e % 512;
+        reinterpret_cast<uint4 *>(sm + s * ST_BYTES + ST_AC)[x] = make_uint4(0u, 0u, 0u, 0u);
+    }
+    fence_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *s_tmem;
-    const uint32_t D_W = tmem + 0, D_B = tmem + 32, D_O = tmem + 64;
-    // MMA shapes: [M, N=32]; A K-major unless noted, B (S, Delta) MN-major
-    const uint32_t id_w = idesc_bf16_f32(64, kNV, 0, 1);   // W S, Q~ S, P Delta
-    const uint32_t id_b = idesc_bf16_f32(128, kNV, 1, 1);  // K^T Delta (K^ stored MN-major)
-    const uint32_t sm_base = smem_u32(sm);
+    const uint32_t D_A = tmem + 0, D_B = tmem + 64;
 
     if (warp == 4) {
-        // ------------------------------------------------ bulk copies + output MMAs (one thread)
+        // ------------------------------------------------ bulk copies (one thread)
         if (lane == 0) {
             bool ok = true;
             auto issue_load = [&](int i) {
@@ -650,43 +647,66 @@ kda_tc_state_kernel(const uint8_t *__restrict__ records, const float *__restrict
                 mbar_arrive_expect_tx(&full[s], REC_TX);
                 bulk_g2s(st + ST_AQ, rec + REC_AQ, 32768, &full[s]);
                 bulk_g2s(st + ST_KH, rec + REC_KH, 16384, &full[s]);
-                bulk_g2s(st + ST_P, rec + REC_P, 8192, &full[s]);
+                bulk_g2s(st + ST_AC + 8192, rec + REC_P, 8192, &full[s]);
                 bulk_g2s(st + ST_U, rec + REC_U + slice * 4096, 4096, &full[s]);
                 bulk_g2s(st + ST_GL, rec + REC_GL, 512, &full[s]);
             };
             for (int i = 0; i < kStages && i < nchunks; ++i) issue_load(i);
-            for (int i = 0; i < nchunks && ok; ++i) {
-                const int s = i % kStages;
-                const uint32_t st = sm_base + s * ST_BYTES;
-                const uint32_t simg = smem_u32(Simg) + (i & 1) * 8192;
-                ok = mbar_wait(&d_ready[i & 1], (i >> 1) & 1);
-                if (!ok) break;
-                tc_fence_after();
-#pragma unroll
-                for (int ks = 0; ks < 8; ++ks)  // Q~ S  (Q~ = rows 64..127 of the [W; Q~] image)
-                    mma_bf16_ss(D_O + 32 * (i & 1),
-                                smem_desc_sw128(st + ST_AQ + 8192 + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024),
-                                smem_desc_sw64(simg + ks * 1024, 512), id_w, ks > 0);
-#pragma unroll
-                for (int ks = 0; ks < 4; ++ks)  // + P Delta
-                    mma_bf16_ss(D_O + 32 * (i & 1), smem_desc_sw128(st + ST_P + ks * 32, 16, 1024),
-                                smem_desc_sw64(smem_u32(Dimg) + (i & 1) * 4096 + ks * 1024, 512), id_w, 1);
-                mma_commit(&bar_o[i & 1]);
-                mma_commit(&empty[s]);
-                if (i + kStages < nchunks) {  // refill stage s once MMA-b and these MMAs are done
-                    ok = mbar_wait(&empty[s], (i / kStages) & 1);
-                    if (!ok) break;
-                    issue_load(i + kStages);
-                }
+            for (int i = 0; i + kStages < nchunks && ok; ++i) {
+                ok = mbar_wait(&empty[i % kStages], (i / kStages) & 1);
+                if (ok) issue_load(i + kStages);
             }
             if (!ok) set_status(status, KDA_ERR_TIMEOUT);
         }
         __syncwarp();
+    } else if (warp == 5) {
+        // ------------------------------------------------ MMA issue (one thread)
+        const uint32_t id_a = idesc_bf16_f32(128, kNV, 0, 1);  // [W; Q~] S, [0; P] Delta
+        const uint32_t id_b = idesc_bf16_f32(128, kNV, 1, 1);  // K^T Delta (K^ stored MN-major)
+        const uint64_t d_s = smem_desc_sw64(smem_u32(Simg), 512);
+        const uint64_t d_d = smem_desc_sw64(smem_u32(Dimg), 512);
+        bool ok = bar_and160(1, true);
+        for (int i = 0; i < nchunks && ok; ++i) {
+            const int s = i % kStages;
+            const uint32_t st = smem_u32(sm + s * ST_BYTES);
+            const uint64_t d_aq = smem_desc_sw128(st + ST_AQ, 16, 1024);
+            const uint64_t d_kh = smem_desc_sw128(st + ST_KH, 8192, 1024);
+            const uint64_t d_ac = smem_desc_sw128(st + ST_AC, 16, 1024);
+            const uint32_t d_a = D_A + 32 * (i & 1);
+            bool w_ok = true;
+            if (lane == 0) {
+                w_ok = mbar_wait(&full[s], (i / kStages) & 1);
+                if (w_ok) {
+                    tc_fence_after();
+#pragma unroll
+                    for (int ks = 0; ks < 8; ++ks)  // descriptor start fields advance in 16-byte units
+                        mma_bf16_ss(d_a, d_aq + (uint64_t)(((ks >> 2) * 16384 + (ks & 3) * 32) >> 4),
+                                    d_s + (uint64_t)((ks * 1024) >> 4), id_a, ks > 0);
+                    mma_commit(bar_w);
+                }
+            }
+            ok = bar_and160(2, __shfl_sync(0xffffffffu, w_ok, 0));
+            if (!ok) break;
+            if (lane == 0) {
+                tc_fence_after();
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    mma_bf16_ss(D_B, d_kh + (uint64_t)((ks * 2048) >> 4), d_d + (uint64_t)((ks * 1024) >> 4), id_b,
+                                ks > 0);
+                mma_commit(bar_b);
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    mma_bf16_ss(d_a, d_ac + (uint64_t)((ks * 32) >> 4), d_d + (uint64_t)((ks * 1024) >> 4), id_a, 1);
+                mma_commit(bar_c);
+                mma_commit(&empty[s]);
+            }
+            __syncwarp();
+            ok = bar_and160(1, true);
+        }
     } else {
         // ------------------------------------------------ warps 0-3: state row t = tid (TMEM lane)
         const int t = tid;
         const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-        const int r16 = 16 * warp + lane;  // row of an M=64 accumulator held by this lane (lane < 16)
         const size_t soff = (((size_t)n * H + h) * D + t) * D + j0;
         float S[kNV];
 #pragma unroll
@@ -694,15 +714,19 @@ kda_tc_state_kernel(const uint8_t *__restrict__ records, const float *__restrict
             const float4 w = h0 ? *reinterpret_cast<const float4 *>(h0 + soff + 4 * x) : make_float4(0.f, 0.f, 0.f, 0.f);
             S[4 * x] = w.x; S[4 * x + 1] = w.y; S[4 * x + 2] = w.z; S[4 * x + 3] = w.w;
         }
+        auto store_S_image = [&]() {
 #pragma unroll
-        for (int x = 0; x < 4; ++x)
-            *reinterpret_cast<uint4 *>(Simg + sw64_chunk(t, x)) =
-                make_uint4(pack_bf16(S[8 * x], S[8 * x + 1]), pack_bf16(S[8 * x + 2], S[8 * x + 3]),
-                           pack_bf16(S[8 * x + 4], S[8 * x + 5]), pack_bf16(S[8 * x + 6], S[8 * x + 7]));
+            for (int x = 0; x < 4; ++x)
+                *reinterpret_cast<uint4 *>(Simg + sw64_chunk(t, x)) =
+                    make_uint4(pack_bf16(S[8 * x], S[8 * x + 1]), pack_bf16(S[8 * x + 2], S[8 * x + 3]),
+                               pack_bf16(S[8 * x + 4], S[8 * x + 5]), pack_bf16(S[8 * x + 6], S[8 * x + 7]));
+        };
+        store_S_image();
         fence_async_smem();
-        bool ok = bar_and(1, true);
+        bool ok = bar_and160(1, true);
 
-        auto write_o = [&](int i) {  // output rows of chunk i from D_o[i % 2] (M=64 layout)
+        // output rows of chunk i: D_a[i % 2] rows 64..127, read by warps 2 and 3 (row = t - 64)
+        auto write_o = [&](int i) {
             int64_t t0;
             int L;
             if (table) {
@@ -714,61 +738,59 @@ kda_tc_state_kernel(const uint8_t *__restrict__ records, const float *__restrict
                 L = min(C, T_len - i * C);
             }
             float ov[32];
-            tmem_ld32(D_O + 32 * (i & 1) + lane_base, ov);
+            tmem_ld32(D_A + 32 * (i & 1) + lane_base, ov);
             tmem_wait_ld();
-            // Lanes 0..15 hold rows 16 w + l; lanes l and l + 16 split the row's four 16-byte
-            // chunks so that each store instruction fills whole 32-byte sectors.
-            uint32_t pk[16];
+            uint32_t pk[16];  // four 16-byte chunks (4 words each) of this lane's row
 #pragma unroll
             for (int e = 0; e < 16; ++e) pk[e] = pack_bf16(ov[2 * e], ov[2 * e + 1]);
-            const bool upper = lane >= 16;
-            const int row = 16 * warp + (lane & 15);
+            // Lanes l and l ^ 1 (rows 2p and 2p+1 of the chunk) trade 16-byte chunks so that every
+            // store instruction fills whole 32-byte sectors: for chunk pair (2c, 2c+1), the first
+            // store writes both chunks of the even row, the second both chunks of the odd row.
+            const bool odd = lane & 1;
+            const int row = t - 64;
+            const int even_row = row & ~1, odd_row = row | 1;
 #pragma unroll
-            for (int k = 0; k < 2; ++k) {
-                uint32_t w[4];
+            for (int c = 0; c < 2; ++c) {
+                uint4 mine, theirs;
+                uint32_t mv[4], tv[4];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    const uint32_t mine = pk[8 * k + e];         // chunk 2k of this lane's row
-                    const uint32_t odd = pk[8 * k + 4 + e];      // chunk 2k + 1
-                    const uint32_t from_low = __shfl_sync(0xffffffffu, odd, lane & 15);
-                    w[e] = upper ? from_low : mine;
+                    const uint32_t give = odd ? pk[8 * c + e] : pk[8 * c + 4 + e];  // even gives 2c+1, odd gives 2c
+                    tv[e] = __shfl_xor_sync(0xffffffffu, give, 1);
+                    mv[e] = odd ? pk[8 * c + 4 + e] : pk[8 * c + e];
                 }
-                if (row < L) {
-                    __nv_bfloat16 *orow = o + ((size_t)(t0 + row) * H + h) * D + j0;
-                    reinterpret_cast<uint4 *>(orow)[2 * k + (upper ? 1 : 0)] = make_uint4(w[0], w[1], w[2], w[3]);
-                }
+                mine = make_uint4(mv[0], mv[1], mv[2], mv[3]);
+                theirs = make_uint4(tv[0], tv[1], tv[2], tv[3]);
+                const int chunk16 = 2 * c + (odd ? 1 : 0);
+                // store 1: the even row (even lane: its own chunk 2c, odd lane: the even row's 2c+1)
+                if (even_row < L)
+                    reinterpret_cast<uint4 *>(o + ((size_t)(t0 + even_row) * H + h) * D + j0)[chunk16] = odd ? theirs : mine;
+                // store 2: the odd row (even lane: the odd row's chunk 2c, odd lane: its own 2c+1)
+                if (odd_row < L)
+                    reinterpret_cast<uint4 *>(o + ((size_t)(t0 + odd_row) * H + h) * D + j0)[chunk16] = odd ? mine : theirs;
             }
         };
 
         for (int i = 0; i < nchunks && ok; ++i) {
             const int s = i % kStages;
             const uint8_t *st = sm + s * ST_BYTES;
-            const uint32_t st_u = sm_base + s * ST_BYTES;
-            const uint32_t simg = smem_u32(Simg) + (i & 1) * 8192;
-            uint8_t *dimg = Dimg + (i & 1) * 4096;
-            // (1) W S on the critical path
+            const uint32_t d_a = D_A + 32 * (i & 1);
+            // (1) stage data this thread reads (before the stage can be refilled)
             bool w_ok = mbar_wait(&full[s], (i / kStages) & 1);
-            if (t == 0 && w_ok) {
-                tc_fence_after();
-#pragma unroll
-                for (int ks = 0; ks < 8; ++ks)
-                    mma_bf16_ss(D_W, smem_desc_sw128(st_u + ST_AQ + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024),
-                                smem_desc_sw64(simg + ks * 1024, 512), id_w, ks > 0);
-                mma_commit(bar_w);
-            }
-            // every read of stage s by these threads happens before d_ready (the stage may be refilled after)
             const float gl = reinterpret_cast<const float *>(st + ST_GL)[t];
-            // (2) Delta = U - W S  (rows 16 w + l, l < 16)
+            // (2) warps 0-1: Delta = U - W S once the previous chunk's [0; P] Delta no longer reads
+            //     the Delta image; warps 2-3: output of the previous chunk
+            if (i > 0) w_ok = w_ok && mbar_wait(bar_c, (i - 1) & 1);
             w_ok = w_ok && mbar_wait(bar_w, i & 1);
             if (__all_sync(0xffffffffu, w_ok)) {
                 tc_fence_after();
-                float ws[32];
-                tmem_ld32(D_W + lane_base, ws);
-                tmem_wait_ld();
-                if (lane < 16) {
+                if (warp < 2) {
+                    float ws[32];
+                    tmem_ld32(d_a + lane_base, ws);
+                    tmem_wait_ld();
 #pragma unroll
                     for (int x = 0; x < 4; ++x) {
-                        const uint4 u4 = *reinterpret_cast<const uint4 *>(st + ST_U + sw64_chunk(r16, x));
+                        const uint4 u4 = *reinterpret_cast<const uint4 *>(st + ST_U + sw64_chunk(t, x));
                         const uint32_t uw[4] = {u4.x, u4.y, u4.z, u4.w};
                         uint32_t dw[4];
 #pragma unroll
@@ -776,41 +798,20 @@ kda_tc_state_kernel(const uint8_t *__restrict__ records, const float *__restrict
                             const float2 uf = unpack_bf16(uw[e]);
                             dw[e] = pack_bf16(uf.x - ws[8 * x + 2 * e], uf.y - ws[8 * x + 2 * e + 1]);
                         }
-                        *reinterpret_cast<uint4 *>(dimg + sw64_chunk(r16, x)) = make_uint4(dw[0], dw[1], dw[2], dw[3]);
+                        *reinterpret_cast<uint4 *>(Dimg + sw64_chunk(t, x)) = make_uint4(dw[0], dw[1], dw[2], dw[3]);
                     }
+                } else if (i > 0) {
+                    write_o(i - 1);
                 }
             } else {
                 w_ok = false;
             }
             tc_fence_before();
             fence_async_smem();
-            ok = bar_and(2, w_ok);
+            ok = bar_and160(2, w_ok);
             if (!ok) break;
-            // (3) K^T Delta on the critical path; warp 4 then issues this chunk's output MMAs
-            if (t == 0) {
-                tc_fence_after();
-#pragma unroll
-                for (int ks = 0; ks < 4; ++ks)
-                    mma_bf16_ss(D_B, smem_desc_sw128(st_u + ST_KH + ks * 2048, 8192, 1024),
-                                smem_desc_sw64(smem_u32(dimg) + ks * 1024, 512), id_b, ks > 0);
-                mma_commit(bar_b);
-                mma_commit(&empty[s]);
-                mbar_arrive(&d_ready[i & 1]);
-            }
-            // (4) while K^T Delta runs: output rows of the previous chunk; this also retires the
-            //     MMAs that read S image (i+1) % 2 before step (5) overwrites it
-            w_ok = true;
-            if (i > 0) {
-                w_ok = mbar_wait(&bar_o[(i - 1) & 1], ((i - 1) >> 1) & 1);
-                if (__all_sync(0xffffffffu, w_ok)) {
-                    tc_fence_after();
-                    write_o(i - 1);
-                } else {
-                    w_ok = false;
-                }
-            }
-            // (5) S <- e^{G_63} S + K^T Delta; bf16 copy into the other S image
-            w_ok = w_ok && mbar_wait(bar_b, i & 1);
+            // (3) S <- e^{G_63} S + K^T Delta and its bf16 operand image
+            w_ok = mbar_wait(bar_b, i & 1);
             if (__all_sync(0xffffffffu, w_ok)) {
                 tc_fence_after();
                 float upd[32];
@@ -818,24 +819,19 @@ kda_tc_state_kernel(const uint8_t *__restrict__ records, const float *__restrict
                 tmem_wait_ld();
 #pragma unroll
                 for (int j = 0; j < kNV; ++j) S[j] = fmaf(gl, S[j], upd[j]);
-                uint8_t *snext = Simg + ((i + 1) & 1) * 8192;
-#pragma unroll
-                for (int x = 0; x < 4; ++x)
-                    *reinterpret_cast<uint4 *>(snext + sw64_chunk(t, x)) =
-                        make_uint4(pack_bf16(S[8 * x], S[8 * x + 1]), pack_bf16(S[8 * x + 2], S[8 * x + 3]),
-                                   pack_bf16(S[8 * x + 4], S[8 * x + 5]), pack_bf16(S[8 * x + 6], S[8 * x + 7]));
+                store_S_image();
             } else {
                 w_ok = false;
             }
             tc_fence_before();
             fence_async_smem();
-            ok = bar_and(1, w_ok);
+            ok = bar_and160(1, w_ok);
         }
-        if (ok && nchunks > 0) {  // output rows of the last chunk
-            bool w_ok = mbar_wait(&bar_o[(nchunks - 1) & 1], ((nchunks - 1) >> 1) & 1);
+        if (ok && nchunks > 0) {  // output of the last chunk
+            bool w_ok = mbar_wait(bar_c, (nchunks - 1) & 1);
             if (__all_sync(0xffffffffu, w_ok)) {
                 tc_fence_after();
-                write_o(nchunks - 1);
+                if (warp >= 2) write_o(nchunks - 1);
             } else {
                 ok = false;
             }
