@@ -196,6 +196,43 @@ def kernel_stats(traces):
     return out
 
 
+def reduce_max(x: float, world: int, device) -> float:
+    """Max of a per-rank scalar over all ranks (a timing collective, not part of the data path)."""
+    if world == 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(units_per_step_per_rank: float, steps: int, world: int, elapsed_ms_max: float) -> float:
+    """Units per second for the whole job: every rank processes its own units (weak scaling) and the
+    job takes as long as its slowest rank."""
+    return world * units_per_step_per_rank * steps / (elapsed_ms_max / 1e3)
+
+
+def ncu_traffic(kernel: str, units: int):
+    """DRAM bytes per launch of `kernel` for `units` work units, scaled from the committed ncu capture
+    in profiles/ncu_traffic.json, or None when the kernel's source changed since that capture."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        rec = json.load(f).get(kernel)
+    if not rec:
+        return None
+    src = os.path.join(ROOT, rec["source"])
+    if not os.path.exists(src):
+        return None
+    with open(src, "rb") as f:
+        if hashlib.sha256(f.read()).hexdigest() != rec["source_sha256"]:
+            return None
+    return rec["dram_bytes"] / rec["units"] * units
+
+
 def gpu_arm(args):
     import torch
     import torch.distributed as dist
@@ -215,11 +252,7 @@ def gpu_arm(args):
             dist.barrier()
 
     def max_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        t = torch.tensor([x], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return reduce_max(x, world, dev)
 
     peaks = load_peaks()
     import dataclasses
@@ -258,7 +291,7 @@ def gpu_arm(args):
     elapsed_ms = max_over_ranks(ev0.elapsed_time(ev1))
     ms_per_step = elapsed_ms / args.steps
     tokens_per_step = B * T
-    value = world * tokens_per_step * args.steps / (elapsed_ms / 1e3)
+    value = whole_job_rate(tokens_per_step, args.steps, world, elapsed_ms)
 
     # per-kernel timing (live, CUDA events around each library kernel in the timed region)
     kst = kernel_stats(traces)
@@ -272,7 +305,9 @@ def gpu_arm(args):
     peak_bw = peaks["hbm_gbs"]
     achieved = kbytes.get(dominant, 0) / (kst[dominant]["avg_ms"] / 1e3) / 1e9
     roofline = {"kernel": dominant, "bound": "hbm", "achieved": achieved, "peak": peak_bw, "unit": "GB/s",
-                "frac": achieved / peak_bw, "traffic": None, "peak_source": peaks["source"],
+                "frac": achieved / peak_bw, "traffic": ncu_traffic(dominant, chunk_heads), "peak_source": peaks["source"],
+                "traffic_note": "DRAM read+write bytes per launch from profiles/ncu_traffic.json (a T=8192 capture "
+                                "of the same kernel source, scaled by chunk-heads); null if the source changed",
                 "algorithmic_bytes_per_launch": kbytes.get(dominant, 0), "avg_ms": kst[dominant]["avg_ms"]}
     op_bytes = token_heads * PREFILL_BYTES_PER_TOKEN_HEAD + 2 * B * H * STATE_BYTES
     op_flop = token_heads * PREFILL_FLOP_PER_TOKEN_HEAD
@@ -370,9 +405,10 @@ def decode_bench(args, dev, stream, peaks, barrier, max_over_ranks):
     ms = max_over_ranks(ev0.elapsed_time(ev1)) / args.decode_steps
     nbytes = shp.N * shp.H * DECODE_BYTES_PER_STATE
     gbs = nbytes / (ms / 1e3) / 1e9
+    traffic = ncu_traffic("kda_decode_kernel", shp.N * shp.H)
     return {"workload": shp.name, "steps": args.decode_steps, "ms_per_step": ms,
             "tokens_per_s": shp.N / (ms / 1e3), "hbm_gbs": gbs, "peak_gbs": peaks["hbm_gbs"],
-            "frac": gbs / peaks["hbm_gbs"], "bytes_per_step": nbytes,
+            "frac": gbs / peaks["hbm_gbs"], "bytes_per_step": nbytes, "traffic": traffic,
             "note": "inputs cycle through 8 pre-drawn token sets; the 512 MiB state streams from HBM each step"}
 
 

@@ -88,9 +88,7 @@ __device__ __forceinline__ float2 unpack_bf16(uint32_t u) {
 __device__ __forceinline__ uint32_t sw64_chunk(uint32_t kr, uint32_t x) {
     return kr * 64u + ((x ^ ((kr >> 1) & 3u)) << 4);
 }
-__device__ __forceinline__ float2 expv(float2 x) { return make_float2(__expf(x.x), __expf(x.y)); }
 __device__ __forceinline__ float2 sub2(float2 a, float2 b) { return make_float2(a.x - b.x, a.y - b.y); }
-__device__ __forceinline__ float2 mul2(float2 a, float2 b) { return make_float2(a.x * b.x, a.y * b.y); }
 
 // ============================================================================ chunk table (varlen)
 // One CTA: validates cu_seqlens (0 = cu[0] <= cu[1] <= ... <= cu[N] = T), then writes the chunk
