@@ -17,22 +17,23 @@
 //
 // Two kernels:
 //  1. kda_tc_prep_kernel - one CTA per (chunk, head), all chunks in parallel.  Everything that does not
-//     depend on the state: log-gate cumsum, decay factors, the two Gram matrices (tcgen05, M=128 with
-//     k-rows and q-rows stacked, one N=16 strip per 16-row key block so each strip can use its own
-//     decay reference), the UT transform in fp32 on CUDA cores (blocked forward substitution), and
-//     W, U (tcgen05, M=64, N=128).  It writes [W; Q o e^G], K o e^{G_63-G}, P, U and e^{G_63} for the
-//     chunk as ready-to-use 128-byte-swizzled operand images ("records") in the workspace.
+//     depend on the state: log-gate cumsum, decay factors, the two Gram matrices (tcgen05, formed
+//     transposed: one M=64, N=32 product per 16-row block with k-rows and q-rows side by side, so
+//     each block can use its own decay reference), the UT transform in fp32 on CUDA cores (blocked
+//     forward substitution), and W, U (tcgen05, M=64, N=128).  It writes [W; Q o e^G],
+//     K o e^{G_63-G}, P, U and e^{G_63} for the chunk as ready-to-use swizzled operand images
+//     ("records") in the workspace.
 //  2. kda_tc_state_kernel - one CTA per (sequence, head, 32 value columns); the value columns of S
 //     evolve independently.  It walks the sequence's chunks in order, bulk-copying each record into
-//     a 3-stage shared-memory ring, and runs per chunk: D_a = [W; Q~] S (M=128, N=32, K=128),
+//     a 2-stage shared-memory ring, and runs per chunk: D_a = [W; Q~] S (M=128, N=32, K=128),
 //     Delta = U - D_a[0:64], D_b = K^T Delta (M=128, K=64), D_a[64:128] += P Delta, then
 //     S <- e^{G_63} S + D_b with the fp32 master state in registers and a bf16 copy as MMA operand.
 //
-// Decay references (secondary chunking): key block a (rows 16a..16a+15) uses E_a = G at row 16a+7.
-// The Gram strip of key block a is (K_r e^{G_r - E_a}) . (K_i e^{E_a - G_i}) for rows r >= 16a; with
-// E_b(r) the row's own reference, e^{G_r - E_a} = e^{G_r - E_b(r)} e^{E_b(r) - E_a}: the first factor
-// lies within e^{+-8 max|log_alpha|}, the second is <= 1, so no operand overflows even when G falls
-// far below the fp32 exponent range inside one chunk.  Factors that underflow belong to terms below
+// Decay references (secondary chunking): block b (rows 16b..16b+15) uses E_b = G at row 16b+7.
+// For a row r of block b and a key row i <= r, e^{G_r - G_i} = e^{G_r - E_b} e^{E_b - G_i}: the first
+// factor lies within e^{+-8 max|log_alpha|}; for i in block a <= b the second is e^{E_a - G_i}
+// (bounded the same way) times e^{E_b - E_a} <= 1, so no operand overflows even when G falls far
+// below the fp32 exponent range inside one chunk.  Factors that underflow belong to terms below
 // 1e-38 and are dropped harmlessly.
 #include "kda_common.cuh"
 #include "kda_sm100.cuh"
@@ -47,7 +48,7 @@ constexpr int C = kChunk;
 // Record of one (chunk, head) in the workspace.
 constexpr uint32_t REC_AQ = 0;        // [W; Q o e^G]: K-major sw128, 128 rows x 128 (2 atoms x 16 KiB)
 constexpr uint32_t REC_KH = 32768;    // K o e^{G_63 - G}: MN-major sw128, 64 k-rows x 128 (2 blocks x 8 KiB)
-constexpr uint32_t REC_P = 49152;     // P: K-major sw128, 64 rows x 64 (8 KiB)
+constexpr uint32_t REC_P = 49152;     // P as an MN-major operand (P^T rows): sw128, 64 k-rows x 64 (8 KiB)
 constexpr uint32_t REC_U = 57344;     // U: bf16, four [64][32] blocks (one per 32-column slice), 64-byte swizzle
 constexpr uint32_t REC_GL = 73728;    // e^{G_63}: fp32 [128]
 constexpr uint32_t REC_BYTES = 74752;
@@ -144,11 +145,31 @@ __global__ void __launch_bounds__(1024) kda_chunk_table_kernel(const int32_t *__
 // (lane l -> channels c0 = 64 (w & 1) + 2 l, c0 + 1) for the 16 rows of key block qr = w >> 1, so
 // every row a thread touches shares one decay reference.  Log-gates are kept in base-2 units
 // (scaled by log2 e on load) so each decay factor is a single ex2.
+//
+// The Gram matrices are formed transposed, one product per 16-row query/key block b (rows r):
+//   [A; P]^T[i][r] = sum_c (K_i o 2^{E_b - G_i})_c (X_r)_c,   X_r = [K_r; Q_r] o 2^{G_r - E_b},
+// so the block-dependent decay reference sits on the 64-row side R^(b) = K o 2^{E_b - G} and all four
+// products (M=64, N=32, K=128) go to the tensor pipe in one batch.  R^(b) is only needed for rows
+// i < 16 b + 16 (i > r is masked), so the four operands are packed back to back with 16, 32, 48 and
+// 64 rows; the product for block b reads 64 rows from the start of R^(b) and the rows past its own
+// belong to R^(b+1) (finite values whose outputs are masked).  For i in key block a <= b,
+// 2^{E_b - G_i} = 2^{E_a - G_i} 2^{E_b - E_a} with the second factor <= 1.
 constexpr int kPrepThreads = 256;
-constexpr uint32_t PREP_X0 = 0, PREP_X1 = 32768, PREP_R = 65536, PREP_KT = 81920, PREP_SMALL = 98304;
+constexpr uint32_t PREP_X = 0;             // X: K-major sw128, 4 blocks x (16 k-rows, 16 q-rows) x 128
+constexpr uint32_t PREP_R = 32768;         // R^(0..3): K-major sw128, 160 rows x 128
+constexpr uint32_t PREP_KT = 73728;        // K o 2^G: MN-major 64 k-rows x 128
+constexpr uint32_t PREP_V = 90112;         // V: MN-major 64 k-rows x 128
+constexpr uint32_t PREP_SMALL = 106496;
 constexpr uint32_t PREP_SMEM = PREP_SMALL + (64 + 512 + 512 + 128) * 4 + 16 + 1024;
+constexpr uint32_t kXAtom = 128 * 128;     // X: bytes per 64-channel atom column
+constexpr uint32_t kRRows = 160;
+constexpr uint32_t kRAtom = kRRows * 128;  // R: bytes per 64-channel atom column
 constexpr uint32_t kPrepTmemCols = 256;
 constexpr int kAS = 68;  // fp32 row stride of the 64 x 64 A / T tile (16-byte aligned rows)
+constexpr int kMS = 52;  // fp32 row stride of the 16 x 48 substitution scratch
+
+// first row of R^(b) inside the packed R image
+__host__ __device__ constexpr int r_first_row(int b) { return 8 * b * (b + 1); }
 
 __device__ __forceinline__ float ex2(float x) {
     float y;
@@ -156,44 +177,60 @@ __device__ __forceinline__ float ex2(float x) {
     return y;
 }
 __device__ __forceinline__ float2 ex2v(float2 x) { return make_float2(ex2(x.x), ex2(x.y)); }
+__device__ __forceinline__ __nv_bfloat162 bf2_of(float2 f) { return __floats2bfloat162_rn(f.x, f.y); }
+__device__ __forceinline__ void st_bf2(uint8_t *p, __nv_bfloat162 v) { *reinterpret_cast<__nv_bfloat162 *>(p) = v; }
 
-// Block row b of the UT transform, in place in the 64 x 64 fp32 tile Asm (row stride kAS):
-// rows 16b..16b+15 hold A_b* to the left of the already inverted diagonal block T_bb, rows above
-// hold finished T.  Computes T_ba = -T_bb sum_{c=a}^{b-1} A_bc T_ca for every a < b.  Thread
-// (rr, cb) = (tid / 16, tid % 16) owns row rr of the block row and column cb of each 16-wide
-// block a; upper triangles are stored as zeros, so every sum runs over whole 16-blocks.
-template <int b>
-__device__ __forceinline__ void subst_block_row(float *Asm, float *Mscr, int tid) {
-    constexpr int o = 16 * b;
-    const int rr = tid >> 4, cb = tid & 15;
-    // stage 1: M[rr][16a + cb] = sum_{i = 16a}^{16b-1} A[o + rr][i] T[i][16a + cb]
-    float arow[o];
+// Block row b of the UT transform, in place in the 64 x 64 fp32 tile Asm (row stride kAS): rows
+// 16b..16b+15 hold A_b* to the left of the already inverted diagonal block T_bb, rows above hold
+// finished T, upper triangles are zeros.  Computes T_ba = -T_bb sum_{c=a}^{b-1} A_bc T_ca for a < b.
+// Warps 2a, 2a+1 take key block a; a thread owns row rr = lane % 16 of the block row and four
+// adjacent columns 16a + 4 cq of it, so each shared load feeds four FMAs.
+template <int b, int a>
+__device__ __forceinline__ void subst_stage1(const float *Asm, float *Mscr, int rr, int cq) {
+    constexpr int o = 16 * b, i0 = 16 * a;
+    float arow[o - i0];
 #pragma unroll
-    for (int q4 = 0; q4 < o / 4; ++q4) {
-        const float4 a4 = *reinterpret_cast<const float4 *>(Asm + (o + rr) * kAS + 4 * q4);
+    for (int q4 = 0; q4 < (o - i0) / 4; ++q4) {
+        const float4 a4 = *reinterpret_cast<const float4 *>(Asm + (o + rr) * kAS + i0 + 4 * q4);
         arow[4 * q4] = a4.x; arow[4 * q4 + 1] = a4.y; arow[4 * q4 + 2] = a4.z; arow[4 * q4 + 3] = a4.w;
     }
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-    for (int a = 0; a < b; ++a) {
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int i = 16 * a; i < o; ++i) acc[i & 3] = fmaf(arow[i], Asm[i * kAS + 16 * a + cb], acc[i & 3]);
-        Mscr[rr * 48 + 16 * a + cb] = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+    for (int i = i0; i < o; ++i) {
+        const float4 t4 = *reinterpret_cast<const float4 *>(Asm + i * kAS + i0 + 4 * cq);
+        const float av = arow[i - i0];
+        acc.x = fmaf(av, t4.x, acc.x); acc.y = fmaf(av, t4.y, acc.y);
+        acc.z = fmaf(av, t4.z, acc.z); acc.w = fmaf(av, t4.w, acc.w);
+    }
+    *reinterpret_cast<float4 *>(Mscr + rr * kMS + i0 + 4 * cq) = acc;
+}
+template <int b>
+__device__ __forceinline__ void subst_block_row(float *Asm, float *Mscr, int warp, int lane) {
+    constexpr int o = 16 * b;
+    const int a = warp >> 1, rr = lane & 15, cq = ((warp & 1) << 1) | (lane >> 4);
+    // stage 1: M[rr][16a + 4cq ..] = sum_{i = 16a}^{16b-1} A[o + rr][i] T[i][16a + 4cq ..]
+    if (a < b) {
+        if (a == 0) subst_stage1<b, 0>(Asm, Mscr, rr, cq);
+        if constexpr (b > 1) { if (a == 1) subst_stage1<b, 1>(Asm, Mscr, rr, cq); }
+        if constexpr (b > 2) { if (a == 2) subst_stage1<b, 2>(Asm, Mscr, rr, cq); }
     }
     __syncthreads();
-    // stage 2: T[o + rr][16a + cb] = -sum_jj T_bb[rr][jj] M[jj][16a + cb]  (T_bb lower triangular)
-    float trow[16];
+    // stage 2: T[o + rr][16a + 4cq ..] = -sum_jj T_bb[rr][jj] M[jj][16a + 4cq ..]
+    if (a < b) {
+        float trow[16];
 #pragma unroll
-    for (int q4 = 0; q4 < 4; ++q4) {
-        const float4 t4 = *reinterpret_cast<const float4 *>(Asm + (o + rr) * kAS + o + 4 * q4);
-        trow[4 * q4] = t4.x; trow[4 * q4 + 1] = t4.y; trow[4 * q4 + 2] = t4.z; trow[4 * q4 + 3] = t4.w;
-    }
+        for (int q4 = 0; q4 < 4; ++q4) {
+            const float4 t4 = *reinterpret_cast<const float4 *>(Asm + (o + rr) * kAS + o + 4 * q4);
+            trow[4 * q4] = t4.x; trow[4 * q4 + 1] = t4.y; trow[4 * q4 + 2] = t4.z; trow[4 * q4 + 3] = t4.w;
+        }
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-    for (int a = 0; a < b; ++a) {
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int jj = 0; jj < 16; ++jj) acc[jj & 3] = fmaf(trow[jj], Mscr[jj * 48 + 16 * a + cb], acc[jj & 3]);
-        Asm[(o + rr) * kAS + 16 * a + cb] = -((acc[0] + acc[1]) + (acc[2] + acc[3]));
+        for (int jj = 0; jj < 16; ++jj) {
+            const float4 m4 = *reinterpret_cast<const float4 *>(Mscr + jj * kMS + 16 * a + 4 * cq);
+            acc.x = fmaf(trow[jj], m4.x, acc.x); acc.y = fmaf(trow[jj], m4.y, acc.y);
+            acc.z = fmaf(trow[jj], m4.z, acc.z); acc.w = fmaf(trow[jj], m4.w, acc.w);
+        }
+        *reinterpret_cast<float4 *>(Asm + (o + rr) * kAS + 16 * a + 4 * cq) = make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
     }
     __syncthreads();
 }
@@ -205,10 +242,10 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
                    const int4 *__restrict__ table, uint8_t *__restrict__ records, int *status) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = align1024(smem_raw);
-    uint8_t *X0 = sm + PREP_X0;   // Gram strip operand (strips 0 then 2)
-    uint8_t *X1 = sm + PREP_X1;   // Gram strip operand (strips 1 then 3)
-    uint8_t *Rimg = sm + PREP_R;  // K o 2^{E_b(i) - G_i}: K-major 64 x 128
-    uint8_t *KT = sm + PREP_KT;   // K o 2^G: MN-major 64 k-rows x 128
+    uint8_t *X = sm + PREP_X;     // [K; Q] o 2^{G - E_b}, per block b: 16 k-rows then 16 q-rows
+    uint8_t *Rimg = sm + PREP_R;  // R^(b) = K o 2^{E_b - G}, packed
+    uint8_t *KT = sm + PREP_KT;   // K o 2^G
+    uint8_t *Vimg = sm + PREP_V;  // V
     float *s_beta = reinterpret_cast<float *>(sm + PREP_SMALL);
     float *s_E = s_beta + 64;   // [4][128] block references (base 2)
     float *s_tot = s_E + 512;   // [4][128] per-block gate sums (base 2)
@@ -216,10 +253,9 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
     uint64_t *mbar = reinterpret_cast<uint64_t *>(s_gl + 128);
     uint32_t *s_tmem = reinterpret_cast<uint32_t *>(mbar + 1);
     // reused once the Gram matrices are read out
-    float *Asm = reinterpret_cast<float *>(X0);              // [64][kAS] fp32: A, then T in place
-    float *Mscr = reinterpret_cast<float *>(X0 + 17408);     // [16][48] fp32 scratch
-    uint8_t *TB = X0 + 20480;                                // T Diag(beta): K-major 64 x 64
-    uint8_t *Vimg = X1;                                      // V: MN-major 64 k-rows x 128
+    float *Asm = reinterpret_cast<float *>(X);           // [64][kAS] fp32: A, then T in place
+    float *Mscr = reinterpret_cast<float *>(X + 17408);  // [16][kMS] fp32 scratch
+    uint8_t *TB = X + 21504;                             // T Diag(beta): K-major 64 x 64
 
     const int chunk = blockIdx.x / H, h = blockIdx.x % H;
     int64_t t0;
@@ -299,14 +335,14 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
     __syncthreads();
 
     const float2 gl = make_float2(s_gl[c0], s_gl[c0 + 1]);
-    // cross-block factors 2^{E_own - E_a} for a <= own block (else 0), 2^{E_own}, 2^{G_63 - E_own}
-    float2 Cs[4];
+    // 2^{E_b - E_own} for the later blocks b > own (<= 1), 2^{E_own}, 2^{G_63 - E_own}
+    float2 Cr[4];
 #pragma unroll
-    for (int a = 0; a < 4; ++a)
-        Cs[a] = a <= qr ? ex2v(sub2(Eown, make_float2(s_E[a * D + c0], s_E[a * D + c0 + 1]))) : make_float2(0.f, 0.f);
+    for (int b = 0; b < 4; ++b)
+        Cr[b] = b > qr ? ex2v(sub2(make_float2(s_E[b * D + c0], s_E[b * D + c0 + 1]), Eown)) : make_float2(1.f, 1.f);
     const float2 eE = ex2v(Eown), eGL = ex2v(sub2(gl, Eown));
 
-    // ---- phase A: strips 0 and 1, R, K o 2^G (smem); Q o 2^G and K o 2^{G63-G} (record).
+    // ---- operands: X, R^(b) for b >= own block, K o 2^G (smem); Q o 2^G and K o 2^{G63-G} (record).
     // The factors are rounded to bf16 and applied with packed bf16 multiplies on the bf16 inputs.
 #pragma unroll
     for (int m = 0; m < 16; ++m) {
@@ -314,129 +350,85 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
         const float2 F = ex2v(sub2(g[m], Eown));
         const float2 Rf = ex2v(sub2(Eown, g[m]));
         const __nv_bfloat162 k2 = as_bf2(kk[m]), q2 = as_bf2(qq[m]);
-        const __nv_bfloat162 f0 = __floats2bfloat162_rn(F.x * Cs[0].x, F.y * Cs[0].y);
-        const __nv_bfloat162 f1 = __floats2bfloat162_rn(F.x * Cs[1].x, F.y * Cs[1].y);
-        const __nv_bfloat162 fe = __floats2bfloat162_rn(F.x * eE.x, F.y * eE.y);
-        const __nv_bfloat162 fr = __floats2bfloat162_rn(Rf.x, Rf.y);
-        const __nv_bfloat162 frg = __floats2bfloat162_rn(Rf.x * eGL.x, Rf.y * eGL.y);
-        *reinterpret_cast<__nv_bfloat162 *>(X0 + sw128_off(r, c0, 128)) = __hmul2(k2, f0);
-        *reinterpret_cast<__nv_bfloat162 *>(X0 + sw128_off(64 + r, c0, 128)) = __hmul2(q2, f0);
-        *reinterpret_cast<__nv_bfloat162 *>(X1 + sw128_off(r, c0, 128)) = __hmul2(k2, f1);
-        *reinterpret_cast<__nv_bfloat162 *>(X1 + sw128_off(64 + r, c0, 128)) = __hmul2(q2, f1);
-        *reinterpret_cast<__nv_bfloat162 *>(Rimg + sw128_off(r, c0, 64)) = __hmul2(k2, fr);
-        *reinterpret_cast<__nv_bfloat162 *>(KT + sw128_off(r, c0, 64)) = __hmul2(k2, fe);
-        *reinterpret_cast<__nv_bfloat162 *>(rec + REC_AQ + sw128_off(64 + r, c0, 128)) = __hmul2(q2, fe);
-        *reinterpret_cast<__nv_bfloat162 *>(rec + REC_KH + sw128_off(r, c0, 64)) = __hmul2(k2, frg);
-        g[m] = F;  // keep the row factor for strips 2 and 3
+        const __nv_bfloat162 fx = bf2_of(F);
+        const __nv_bfloat162 fe = bf2_of(make_float2(F.x * eE.x, F.y * eE.y));
+        const __nv_bfloat162 frg = bf2_of(make_float2(Rf.x * eGL.x, Rf.y * eGL.y));
+        st_bf2(X + sw128_off(32 * qr + m, c0, 128), __hmul2(k2, fx));
+        st_bf2(X + sw128_off(32 * qr + 16 + m, c0, 128), __hmul2(q2, fx));
+        st_bf2(KT + sw128_off(r, c0, 64), __hmul2(k2, fe));
+        st_bf2(rec + REC_AQ + sw128_off(64 + r, c0, 128), __hmul2(q2, fe));
+        st_bf2(rec + REC_KH + sw128_off(r, c0, 64), __hmul2(k2, frg));
+#pragma unroll
+        for (int b = 0; b < 4; ++b)
+            if (b >= qr)
+                st_bf2(Rimg + sw128_off(r_first_row(b) + r, c0, kRRows),
+                       __hmul2(k2, bf2_of(make_float2(Rf.x * Cr[b].x, Rf.y * Cr[b].y))));
     }
     fence_async_smem();
     __syncthreads();
 
-    const uint32_t id_gram = idesc_bf16_f32(128, 16, 0, 0);
     if (tid == 0) {
         tc_fence_after();
+        const uint32_t id_gram = idesc_bf16_f32(64, 32, 0, 0);
+        const uint32_t xs = smem_u32(X), rs = smem_u32(Rimg);
 #pragma unroll
-        for (int a = 0; a < 2; ++a) {
-            const uint32_t xa = smem_u32(a == 0 ? X0 : X1);
+        for (int b = 0; b < 4; ++b) {
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks) {
-                const uint64_t ad = smem_desc_sw128(xa + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
-                const uint64_t bd = smem_desc_sw128(smem_u32(Rimg) + (ks >> 2) * 8192 + a * 2048 + (ks & 3) * 32, 16, 1024);
-                mma_bf16_ss(tmem + 16 * a, ad, bd, id_gram, ks > 0);
+                const uint64_t ad = smem_desc_sw128(rs + (ks >> 2) * kRAtom + r_first_row(b) * 128 + (ks & 3) * 32, 16, 1024);
+                const uint64_t bd = smem_desc_sw128(xs + (ks >> 2) * kXAtom + 32 * b * 128 + (ks & 3) * 32, 16, 1024);
+                mma_bf16_ss(tmem + 32 * b, ad, bd, id_gram, ks > 0);
             }
         }
         mma_commit(mbar);
     }
-
-    bool ok = mbar_wait(mbar, 0);
-    ok = __syncthreads_and(ok);
-    // ---- phase B: strips 2 and 3 (only key blocks 2 and 3 are non-zero)
-    if (ok) {
-#pragma unroll
-        for (int m = 0; m < 16; ++m) {
-            const int r = 16 * qr + m;
-            __nv_bfloat162 k2 = as_bf2(0u), q2 = k2, k3 = k2, q3 = k2;
-            if (qr >= 2) {
-                const __nv_bfloat162 f2 = __floats2bfloat162_rn(g[m].x * Cs[2].x, g[m].y * Cs[2].y);
-                const __nv_bfloat162 f3 = __floats2bfloat162_rn(g[m].x * Cs[3].x, g[m].y * Cs[3].y);
-                k2 = __hmul2(as_bf2(kk[m]), f2);
-                q2 = __hmul2(as_bf2(qq[m]), f2);
-                k3 = __hmul2(as_bf2(kk[m]), f3);
-                q3 = __hmul2(as_bf2(qq[m]), f3);
-            }
-            *reinterpret_cast<__nv_bfloat162 *>(X0 + sw128_off(r, c0, 128)) = k2;
-            *reinterpret_cast<__nv_bfloat162 *>(X0 + sw128_off(64 + r, c0, 128)) = q2;
-            *reinterpret_cast<__nv_bfloat162 *>(X1 + sw128_off(r, c0, 128)) = k3;
-            *reinterpret_cast<__nv_bfloat162 *>(X1 + sw128_off(64 + r, c0, 128)) = q3;
-        }
-        fence_async_smem();
-    }
-    __syncthreads();
-    if (ok && tid == 0) {
-        tc_fence_after();
-#pragma unroll
-        for (int a = 2; a < 4; ++a) {
-            const uint32_t xa = smem_u32(a == 2 ? X0 : X1);
-#pragma unroll
-            for (int ks = 0; ks < 8; ++ks) {
-                const uint64_t ad = smem_desc_sw128(xa + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
-                const uint64_t bd = smem_desc_sw128(smem_u32(Rimg) + (ks >> 2) * 8192 + a * 2048 + (ks & 3) * 32, 16, 1024);
-                mma_bf16_ss(tmem + 16 * a, ad, bd, id_gram, ks > 0);
-            }
-        }
-        mma_commit(mbar);
-    }
-    // V tile for U = T Diag(beta) V, fetched while strips 2 and 3 run
-    uint4 vreg[4];
+    // V tile for U = T Diag(beta) V, fetched and laid out while the Gram products run
 #pragma unroll
     for (int s = 0; s < 4; ++s) {
         const int idx = tid + kPrepThreads * s, row = idx >> 4, ch = idx & 15;
-        vreg[s] = row < L ? __ldcs(reinterpret_cast<const uint4 *>(v + ((size_t)(t0 + row) * H + h) * D + ch * 8))
-                          : make_uint4(0u, 0u, 0u, 0u);
+        const uint4 v4 = row < L ? __ldcs(reinterpret_cast<const uint4 *>(v + ((size_t)(t0 + row) * H + h) * D + ch * 8))
+                                 : make_uint4(0u, 0u, 0u, 0u);
+        *reinterpret_cast<uint4 *>(Vimg + sw128_off(row, ch * 8, 64)) = v4;
     }
-    if (ok) ok = mbar_wait(mbar, 1);
+    fence_async_smem();
+    if (tid < D) reinterpret_cast<float *>(rec + REC_GL)[tid] = ex2(s_gl[tid]);
+    bool ok = mbar_wait(mbar, 0);
     ok = __syncthreads_and(ok);
 
     if (ok) {
         tc_fence_after();
-        // V -> MN-major operand image (X1 is free: strip 3 has completed)
-#pragma unroll
-        for (int s = 0; s < 4; ++s) {
-            const int idx = tid + kPrepThreads * s, row = idx >> 4, ch = idx & 15;
-            *reinterpret_cast<uint4 *>(Vimg + sw128_off(row, ch * 8, 64)) = vreg[s];
-        }
-        // Gram read-out: TMEM lanes 0..63 hold k-rows (A), 64..127 q-rows (P); warps w and w+4
-        // share a lane quadrant and take column halves.
+        // Gram read-out.  The M=64 accumulator of block b holds row i = 16 quad + l in TMEM lane
+        // 32 quad + l (l < 16), columns 32b + j: A^T[i][16b + j] (j < 16), P^T[i][16b + j - 16].
+        // Warps w and w + 4 share a lane quadrant and take blocks b = w / 4 and w / 4 + 2.
         const int quad = warp & 3, hc = warp >> 2;
-        const int row = (quad & 1) * 32 + lane;
-        float vals[32];
-        tmem_ld32(tmem + ((uint32_t)(quad * 32) << 16) + 32 * hc, vals);
-        tmem_wait_ld();
-        if (quad < 2) {
-            const float br = s_beta[row];
+        const int i = 16 * quad + lane;
 #pragma unroll
-            for (int x = 0; x < 8; ++x) {
-                float4 w4;
-                const int col = 32 * hc + 4 * x;
-                w4.x = col + 0 < row ? br * vals[4 * x + 0] : 0.f;
-                w4.y = col + 1 < row ? br * vals[4 * x + 1] : 0.f;
-                w4.z = col + 2 < row ? br * vals[4 * x + 2] : 0.f;
-                w4.w = col + 3 < row ? br * vals[4 * x + 3] : 0.f;
-                *reinterpret_cast<float4 *>(Asm + row * kAS + col) = w4;
+        for (int bb = 0; bb < 2; ++bb) {
+            const int b = hc + 2 * bb;
+            float vals[32];
+            if (b >= quad) {  // blocks left of the diagonal block are all masked
+                tmem_ld32(tmem + ((uint32_t)(quad * 32) << 16) + 32 * b, vals);
+                tmem_wait_ld();
+            } else {
+#pragma unroll
+                for (int j = 0; j < 32; ++j) vals[j] = 0.f;
             }
-        } else {
+            if (lane < 16) {
 #pragma unroll
-            for (int cq = 0; cq < 4; ++cq) {
-                uint32_t w[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int col = 32 * hc + 8 * cq + 2 * e;
-                    w[e] = pack_bf16(col <= row ? vals[8 * cq + 2 * e] : 0.f,
-                                     col + 1 <= row ? vals[8 * cq + 2 * e + 1] : 0.f);
+                for (int j = 0; j < 16; ++j) {
+                    const int r = 16 * b + j;
+                    Asm[r * kAS + i] = i < r ? s_beta[r] * vals[j] : 0.f;
                 }
-                const int chunk16 = 4 * hc + cq;
-                *reinterpret_cast<uint4 *>(rec + REC_P + row * 128 + ((chunk16 ^ (row & 7)) << 4)) =
-                    make_uint4(w[0], w[1], w[2], w[3]);
+                uint32_t w[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const int r = 16 * b + 2 * e;
+                    w[e] = pack_bf16(i <= r ? vals[16 + 2 * e] : 0.f, i <= r + 1 ? vals[17 + 2 * e] : 0.f);
+                }
+                // P^T: MN-major sw128, K-row i, 16-byte chunks 2b and 2b + 1 along r
+                uint8_t *prow = rec + REC_P + i * 128;
+                *reinterpret_cast<uint4 *>(prow + (((2 * b) ^ (i & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+                *reinterpret_cast<uint4 *>(prow + (((2 * b + 1) ^ (i & 7)) << 4)) = make_uint4(w[4], w[5], w[6], w[7]);
             }
         }
     }
@@ -466,9 +458,9 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
             for (int rr = 0; rr < 16; ++rr) Asm[(o + rr) * kAS + o + j] = x[rr];
         }
         __syncthreads();
-        subst_block_row<1>(Asm, Mscr, tid);
-        subst_block_row<2>(Asm, Mscr, tid);
-        subst_block_row<3>(Asm, Mscr, tid);
+        subst_block_row<1>(Asm, Mscr, warp, lane);
+        subst_block_row<2>(Asm, Mscr, warp, lane);
+        subst_block_row<3>(Asm, Mscr, warp, lane);
         // T Diag(beta) -> bf16 K-major operand (64 x 64)
         for (int e = tid; e < 64 * 8; e += kPrepThreads) {
             const int r = e >> 3, j = e & 7;
@@ -501,8 +493,7 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
         }
         mma_commit(mbar);
     }
-    if (ok && tid < D) reinterpret_cast<float *>(rec + REC_GL)[tid] = ex2(s_gl[tid]);
-    if (ok) ok = mbar_wait(mbar, 0);
+    if (ok) ok = mbar_wait(mbar, 1);
     ok = __syncthreads_and(ok);
     if (ok) {
         tc_fence_after();
@@ -659,8 +650,8 @@ kda_tc_state_kernel(const uint8_t *__restrict__ records, const float *__restrict
         __syncwarp();
     } else if (warp == 5) {
         // ------------------------------------------------ MMA issue (one thread)
-        const uint32_t id_a = idesc_bf16_f32(128, kNV, 0, 1);  // [W; Q~] S, [0; P] Delta
-        const uint32_t id_b = idesc_bf16_f32(128, kNV, 1, 1);  // K^T Delta (K^ stored MN-major)
+        const uint32_t id_a = idesc_bf16_f32(128, kNV, 0, 1);  // [W; Q~] S
+        const uint32_t id_b = idesc_bf16_f32(128, kNV, 1, 1);  // K^T Delta (K^ stored MN-major), [0; P] Delta
         const uint64_t d_s = smem_desc_sw64(smem_u32(Simg), 512);
         const uint64_t d_d = smem_desc_sw64(smem_u32(Dimg), 512);
         bool ok = bar_and160(1, true);
@@ -669,7 +660,7 @@ kda_tc_state_kernel(const uint8_t *__restrict__ records, const float *__restrict
             const uint32_t st = smem_u32(sm + s * ST_BYTES);
             const uint64_t d_aq = smem_desc_sw128(st + ST_AQ, 16, 1024);
             const uint64_t d_kh = smem_desc_sw128(st + ST_KH, 8192, 1024);
-            const uint64_t d_ac = smem_desc_sw128(st + ST_AC, 16, 1024);
+            const uint64_t d_ac = smem_desc_sw128(st + ST_AC, 8192, 1024);  // MN-major: zero atom, then P
             const uint32_t d_a = D_A + 32 * (i & 1);
             bool w_ok = true;
             if (lane == 0) {
@@ -694,7 +685,7 @@ kda_tc_state_kernel(const uint8_t *__restrict__ records, const float *__restrict
                 mma_commit(bar_b);
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)
-                    mma_bf16_ss(d_a, d_ac + (uint64_t)((ks * 32) >> 4), d_d + (uint64_t)((ks * 1024) >> 4), id_a, 1);
+                    mma_bf16_ss(d_a, d_ac + (uint64_t)((ks * 2048) >> 4), d_d + (uint64_t)((ks * 1024) >> 4), id_b, 1);
                 mma_commit(bar_c);
                 mma_commit(&empty[s]);
             }
