@@ -160,7 +160,7 @@ constexpr uint32_t PREP_R = 32768;         // R^(0..3): K-major sw128, 160 rows 
 constexpr uint32_t PREP_KT = 73728;        // K o 2^G: MN-major 64 k-rows x 128
 constexpr uint32_t PREP_V = 90112;         // V: MN-major 64 k-rows x 128
 constexpr uint32_t PREP_SMALL = 106496;
-constexpr uint32_t PREP_SMEM = PREP_SMALL + (64 + 512 + 512 + 128) * 4 + 16 + 1024;
+constexpr uint32_t PREP_SMEM = PREP_SMALL + (64 + 512 + 512 + 128) * 4 + 32 + 1024;
 constexpr uint32_t kXAtom = 128 * 128;     // X: bytes per 64-channel atom column
 constexpr uint32_t kRRows = 160;
 constexpr uint32_t kRAtom = kRRows * 128;  // R: bytes per 64-channel atom column
@@ -239,7 +239,7 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
 kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
                    const __nv_bfloat16 *__restrict__ v, const float *__restrict__ log_alpha,
                    const float *__restrict__ beta, int T_len, int H, int nc, const int *__restrict__ n_chunks,
-                   const int4 *__restrict__ table, uint8_t *__restrict__ records, int *status) {
+                   const int4 *__restrict__ table, uint8_t *__restrict__ records, int *status, int pf_dist) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = align1024(smem_raw);
     uint8_t *X = sm + PREP_X;     // [K; Q] o 2^{G - E_b}, per block b: 16 k-rows then 16 q-rows
@@ -250,8 +250,8 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
     float *s_E = s_beta + 64;   // [4][128] block references (base 2)
     float *s_tot = s_E + 512;   // [4][128] per-block gate sums (base 2)
     float *s_gl = s_tot + 512;  // [128]    G_63 (base 2)
-    uint64_t *mbar = reinterpret_cast<uint64_t *>(s_gl + 128);
-    uint32_t *s_tmem = reinterpret_cast<uint32_t *>(mbar + 1);
+    uint64_t *mbar = reinterpret_cast<uint64_t *>(s_gl + 128);  // [0] W/U, [1] Gram (4 issuers)
+    uint32_t *s_tmem = reinterpret_cast<uint32_t *>(mbar + 2);
     // reused once the Gram matrices are read out
     float *Asm = reinterpret_cast<float *>(X);           // [64][kAS] fp32: A, then T in place
     float *Mscr = reinterpret_cast<float *>(X + 17408);  // [16][kMS] fp32 scratch
@@ -273,12 +273,40 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
     uint8_t *rec = records + ((size_t)chunk * H + h) * REC_BYTES;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    {   // L2 prefetch of the inputs of the CTA that starts about when this one ends
+        const int64_t nb = (int64_t)blockIdx.x + pf_dist;
+        if (nb < (int64_t)gridDim.x) {
+            const int chunk2 = (int)(nb / H), h2 = (int)(nb % H);
+            int64_t t2 = 0;
+            int L2 = 0;
+            if (table) {
+                if (chunk2 < *n_chunks) {
+                    const int4 e2 = table[chunk2];
+                    t2 = e2.y;
+                    L2 = e2.z;
+                }
+            } else {
+                const int n2 = chunk2 / nc, cc2 = chunk2 % nc;
+                t2 = (int64_t)n2 * T_len + (int64_t)cc2 * C;
+                L2 = min(C, T_len - cc2 * C);
+            }
+            const int which = tid >> 6, row = tid & 63;
+            if (row < L2) {
+                const size_t off = ((size_t)(t2 + row) * H + h2) * D;
+                const void *p = which == 0 ? (const void *)(q + off) : which == 1 ? (const void *)(k + off)
+                              : which == 2 ? (const void *)(v + off) : (const void *)(log_alpha + off);
+                const uint32_t bytes = which == 3 ? 512u : 256u;
+                asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+            }
+        }
+    }
     const int c0 = 64 * (warp & 1) + 2 * lane;  // this thread's two key channels
     const int qr = warp >> 1;                   // key block: rows 16 qr .. 16 qr + 15
     constexpr float kLog2e = 1.4426950408889634f;
 
     if (tid == 0) {
         mbar_init(mbar, 1);
+        mbar_init(mbar + 1, 4);
         mbar_fence_init();
     }
     if (warp == 0) {
@@ -306,6 +334,18 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
         }
     }
     if (tid < 64) s_beta[tid] = tid < L ? __ldg(beta + ((size_t)t0 + tid) * H + h) : 0.f;
+#pragma unroll
+    for (int s = 0; s < 4; ++s) {  // V tile straight into its operand image, asynchronously
+        const int idx = tid + kPrepThreads * s, row = idx >> 4, ch = idx & 15;
+        uint8_t *dst = Vimg + sw128_off(row, ch * 8, 64);
+        if (row < L) {
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)),
+                         "l"(v + ((size_t)(t0 + row) * H + h) * D + ch * 8) : "memory");
+        } else {
+            *reinterpret_cast<uint4 *>(dst) = make_uint4(0u, 0u, 0u, 0u);
+        }
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
 
     // ---- chunk-local cumulative log2-gate G (fp32): block-local prefix, then block offsets
     g[0] = make_float2(g[0].x * kLog2e, g[0].y * kLog2e);
@@ -367,32 +407,21 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
     fence_async_smem();
     __syncthreads();
 
-    if (tid == 0) {
+    if (warp < 4 && lane == 0) {  // block b = warp: four issuers overlap their issue latency
         tc_fence_after();
         const uint32_t id_gram = idesc_bf16_f32(64, 32, 0, 0);
-        const uint32_t xs = smem_u32(X), rs = smem_u32(Rimg);
+        const int b = warp;
+        const uint32_t ra = smem_u32(Rimg) + r_first_row(b) * 128, xa = smem_u32(X) + 32 * b * 128;
 #pragma unroll
-        for (int b = 0; b < 4; ++b) {
-#pragma unroll
-            for (int ks = 0; ks < 8; ++ks) {
-                const uint64_t ad = smem_desc_sw128(rs + (ks >> 2) * kRAtom + r_first_row(b) * 128 + (ks & 3) * 32, 16, 1024);
-                const uint64_t bd = smem_desc_sw128(xs + (ks >> 2) * kXAtom + 32 * b * 128 + (ks & 3) * 32, 16, 1024);
-                mma_bf16_ss(tmem + 32 * b, ad, bd, id_gram, ks > 0);
-            }
+        for (int ks = 0; ks < 8; ++ks) {
+            const uint64_t ad = smem_desc_sw128(ra + (ks >> 2) * kRAtom + (ks & 3) * 32, 16, 1024);
+            const uint64_t bd = smem_desc_sw128(xa + (ks >> 2) * kXAtom + (ks & 3) * 32, 16, 1024);
+            mma_bf16_ss(tmem + 32 * b, ad, bd, id_gram, ks > 0);
         }
-        mma_commit(mbar);
+        mma_commit(mbar + 1);
     }
-    // V tile for U = T Diag(beta) V, fetched and laid out while the Gram products run
-#pragma unroll
-    for (int s = 0; s < 4; ++s) {
-        const int idx = tid + kPrepThreads * s, row = idx >> 4, ch = idx & 15;
-        const uint4 v4 = row < L ? __ldcs(reinterpret_cast<const uint4 *>(v + ((size_t)(t0 + row) * H + h) * D + ch * 8))
-                                 : make_uint4(0u, 0u, 0u, 0u);
-        *reinterpret_cast<uint4 *>(Vimg + sw128_off(row, ch * 8, 64)) = v4;
-    }
-    fence_async_smem();
     if (tid < D) reinterpret_cast<float *>(rec + REC_GL)[tid] = ex2(s_gl[tid]);
-    bool ok = mbar_wait(mbar, 0);
+    bool ok = mbar_wait(mbar + 1, 0);
     ok = __syncthreads_and(ok);
 
     if (ok) {
@@ -475,6 +504,7 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
             }
             *reinterpret_cast<uint4 *>(TB + r * 128 + ((j ^ (r & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
         }
+        asm volatile("cp.async.wait_all;" ::: "memory");  // this thread's V copies have landed
         fence_async_smem();
     }
     __syncthreads();
@@ -493,7 +523,7 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
         }
         mma_commit(mbar);
     }
-    if (ok) ok = mbar_wait(mbar, 1);
+    if (ok) ok = mbar_wait(mbar, 0);
     ok = __syncthreads_and(ok);
     if (ok) {
         tc_fence_after();
@@ -525,6 +555,7 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
     }
     tc_fence_before();
     __syncthreads();
+    asm volatile("cp.async.wait_all;" ::: "memory");  // after a failed wait: no copy outlives the CTA
     if (warp == 0) tmem_dealloc(tmem, kPrepTmemCols);
 }
 
@@ -865,6 +896,12 @@ cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(kda_tc_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)STATE_SMEM);
     if (e != cudaSuccess) return e;
+    // The intra-chunk kernel runs two CTAs per SM; each prefetches into L2 the inputs of the CTA
+    // two waves later, which starts about when it ends.
+    int dev = 0, nsm = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    const int pf = 2 * nsm;
     const auto *qb = static_cast<const __nv_bfloat16 *>(q);
     const auto *kb = static_cast<const __nv_bfloat16 *>(k);
     const auto *vb = static_cast<const __nv_bfloat16 *>(v);
@@ -877,7 +914,7 @@ cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const
         if (lay.max_chunks > 0) {
             trace_before(kKernTcPrep, stream);
             kda_tc_prep_kernel<<<(unsigned)(lay.max_chunks * H), kPrepThreads, PREP_SMEM, stream>>>(
-                qb, kb, vb, log_alpha, beta, T, H, 0, status + 1, table, records, status);
+                qb, kb, vb, log_alpha, beta, T, H, 0, status + 1, table, records, status, pf);
             trace_after(stream);
             if ((e = cudaGetLastError()) != cudaSuccess) return e;
         }
@@ -891,7 +928,7 @@ cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const
     if (nc > 0) {
         trace_before(kKernTcPrep, stream);
         kda_tc_prep_kernel<<<(unsigned)((int64_t)B * nc * H), kPrepThreads, PREP_SMEM, stream>>>(
-            qb, kb, vb, log_alpha, beta, T, H, nc, nullptr, nullptr, records, status);
+            qb, kb, vb, log_alpha, beta, T, H, nc, nullptr, nullptr, records, status, pf);
         trace_after(stream);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
