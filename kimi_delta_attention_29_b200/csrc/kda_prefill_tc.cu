@@ -80,9 +80,9 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 __device__ __forceinline__ __nv_bfloat162 as_bf2(uint32_t u) {
     return *reinterpret_cast<const __nv_bfloat162 *>(&u);
 }
+// bf16 -> fp32 is exact: the bf16 bits are the high half of the fp32 word.
 __device__ __forceinline__ float2 unpack_bf16(uint32_t u) {
-    const __nv_bfloat162 v = *reinterpret_cast<const __nv_bfloat162 *>(&u);
-    return __bfloat1622float2(v);
+    return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xFFFF0000u));
 }
 // Byte offset of the 16-byte chunk x (elements 8x..8x+7) of k-row kr of a tile with 64-byte rows stored
 // with the 64-byte swizzle (MN-major sw64 operands, and the U slices of a record).
@@ -443,10 +443,16 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
                 for (int j = 0; j < 32; ++j) vals[j] = 0.f;
             }
             if (lane < 16) {
+                float br[16];  // beta of the block's rows, loaded before the stores below
+#pragma unroll
+                for (int j4 = 0; j4 < 4; ++j4) {
+                    const float4 b4 = *reinterpret_cast<const float4 *>(s_beta + 16 * b + 4 * j4);
+                    br[4 * j4] = b4.x; br[4 * j4 + 1] = b4.y; br[4 * j4 + 2] = b4.z; br[4 * j4 + 3] = b4.w;
+                }
 #pragma unroll
                 for (int j = 0; j < 16; ++j) {
                     const int r = 16 * b + j;
-                    Asm[r * kAS + i] = i < r ? s_beta[r] * vals[j] : 0.f;
+                    Asm[r * kAS + i] = i < r ? br[j] * vals[j] : 0.f;
                 }
                 uint32_t w[8];
 #pragma unroll
@@ -490,19 +496,30 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
         subst_block_row<1>(Asm, Mscr, warp, lane);
         subst_block_row<2>(Asm, Mscr, warp, lane);
         subst_block_row<3>(Asm, Mscr, warp, lane);
-        // T Diag(beta) -> bf16 K-major operand (64 x 64)
-        for (int e = tid; e < 64 * 8; e += kPrepThreads) {
-            const int r = e >> 3, j = e & 7;
-            const float4 t0v = *reinterpret_cast<const float4 *>(Asm + r * kAS + 8 * j);
-            const float4 t1v = *reinterpret_cast<const float4 *>(Asm + r * kAS + 8 * j + 4);
-            const float tv[8] = {t0v.x, t0v.y, t0v.z, t0v.w, t1v.x, t1v.y, t1v.z, t1v.w};
-            uint32_t w[4];
+        {   // T Diag(beta) -> bf16 K-major operand (64 x 64): rows tid / 8 and tid / 8 + 32, columns 8 (tid % 8) + 0..7
+            const int j = tid & 7, r0 = tid >> 3;
+            const float4 b0 = *reinterpret_cast<const float4 *>(s_beta + 8 * j);
+            const float4 b1 = *reinterpret_cast<const float4 *>(s_beta + 8 * j + 4);
+            const float bj[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+            float tv[2][8];  // all loads before the stores (the two tiles share shared memory)
 #pragma unroll
-            for (int x = 0; x < 4; ++x) {
-                const int i0 = 8 * j + 2 * x;
-                w[x] = pack_bf16(i0 <= r ? tv[2 * x] * s_beta[i0] : 0.f, i0 + 1 <= r ? tv[2 * x + 1] * s_beta[i0 + 1] : 0.f);
+            for (int hh = 0; hh < 2; ++hh) {
+                const float4 t0v = *reinterpret_cast<const float4 *>(Asm + (r0 + 32 * hh) * kAS + 8 * j);
+                const float4 t1v = *reinterpret_cast<const float4 *>(Asm + (r0 + 32 * hh) * kAS + 8 * j + 4);
+                tv[hh][0] = t0v.x; tv[hh][1] = t0v.y; tv[hh][2] = t0v.z; tv[hh][3] = t0v.w;
+                tv[hh][4] = t1v.x; tv[hh][5] = t1v.y; tv[hh][6] = t1v.z; tv[hh][7] = t1v.w;
             }
-            *reinterpret_cast<uint4 *>(TB + r * 128 + ((j ^ (r & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                const int r = r0 + 32 * hh;
+                uint32_t w[4];
+#pragma unroll
+                for (int x = 0; x < 4; ++x) {
+                    const int i0 = 8 * j + 2 * x;
+                    w[x] = pack_bf16(i0 <= r ? tv[hh][2 * x] * bj[2 * x] : 0.f, i0 + 1 <= r ? tv[hh][2 * x + 1] * bj[2 * x + 1] : 0.f);
+                }
+                *reinterpret_cast<uint4 *>(TB + r * 128 + ((j ^ (r & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+            }
         }
         asm volatile("cp.async.wait_all;" ::: "memory");  // this thread's V copies have landed
         fence_async_smem();
@@ -807,10 +824,13 @@ kda_tc_state_kernel(const uint8_t *__restrict__ records, const float *__restrict
                 if (warp < 2) {
                     float ws[32];
                     tmem_ld32(d_a + lane_base, ws);
+                    uint4 u4s[4];  // all loads first: the Delta stores below could alias them
+#pragma unroll
+                    for (int x = 0; x < 4; ++x) u4s[x] = *reinterpret_cast<const uint4 *>(st + ST_U + sw64_chunk(t, x));
                     tmem_wait_ld();
 #pragma unroll
                     for (int x = 0; x < 4; ++x) {
-                        const uint4 u4 = *reinterpret_cast<const uint4 *>(st + ST_U + sw64_chunk(t, x));
+                        const uint4 u4 = u4s[x];
                         const uint32_t uw[4] = {u4.x, u4.y, u4.z, u4.w};
                         uint32_t dw[4];
 #pragma unroll
