@@ -580,11 +580,13 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
 // One CTA per (sequence, head, 32 value columns); the value columns of S evolve independently.
 // Warps 0-3 own the 128 state rows (TMEM lanes) and keep the fp32 master state in registers,
 // warp 4 streams the chunk records into a 2-stage shared-memory ring with bulk copies, warp 5
-// issues every MMA.  Warps 0-3 and 5 meet at two named barriers per chunk.  Per chunk i:
-//   D_a[i%2]  = [W; Q~] S        (M=128, N=32, K=128)   rows 0..63 -> Delta = U - W S
-//   D_b       = K^T Delta        (M=128, N=32, K=64)    -> S <- e^{G_63} S + D_b
-//   D_a[i%2] += [0; P] Delta     (M=128, N=32, K=64)    rows 64..127 = output, read during chunk i+1
-// Only the first two products are on the recurrence's critical path.
+// issues every MMA.  Per chunk i:
+//   D_a[i%2]  = [W; Q~] S        (M=128, N=32, K=128)   rows 0..63 -> Delta = U - W S (warps 0-1)
+//   D_b       = K^T Delta        (M=128, N=32, K=64)    -> S <- e^{G_63} S + D_b (warps 0-3)
+//   D_a[i%2] += [0; P] Delta     (M=128, N=32, K=64)    rows 64..127 = output, stored by warps 2-3
+//                                                        while chunk i+1 computes Delta and K^T Delta
+// Only the first two products are on the recurrence's critical path.  Warps 0, 1 and 5 meet at a
+// named barrier when Delta is ready, warps 0-3 and 5 at another when the next state image is.
 constexpr int kNV = 32;            // value columns per CTA
 constexpr int kStages = 2;
 constexpr uint32_t ST_AQ = 0, ST_KH = 32768, ST_AC = 49152, ST_U = 65536, ST_GL = 69632, ST_BYTES = 70656;
@@ -605,16 +607,19 @@ __device__ __forceinline__ uint64_t smem_desc_sw64(uint32_t start, uint32_t sbo)
     d |= (uint64_t)4 << 61;  // 64-byte swizzle
     return d;
 }
-// Named barrier over warps 0-3 and 5 (160 threads) that also ANDs a per-thread flag.
-__device__ __forceinline__ bool bar_and160(int id, bool pred) {
+// Named barrier over `count` threads that also ANDs a per-thread flag.  Barrier 1: warps 0-3 and 5
+// (160 threads); barrier 2: warps 0, 1 and 5 (96 threads).
+__device__ __forceinline__ bool bar_and(int id, int count, bool pred) {
     uint32_t r;
     asm volatile(
-        "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.and.pred q, %2, 160, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+        "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.and.pred q, %2, %3, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
         : "=r"(r)
-        : "r"((uint32_t)pred), "r"(id)
+        : "r"((uint32_t)pred), "r"(id), "r"(count)
         : "memory");
     return r != 0;
 }
+__device__ __forceinline__ bool bar_and160(bool pred) { return bar_and(1, 160, pred); }
+__device__ __forceinline__ bool bar_and96(bool pred) { return bar_and(2, 96, pred); }
 
 __global__ void __launch_bounds__(kStateThreads, 1)
 kda_tc_state_kernel(const uint8_t *__restrict__ records, const float *__restrict__ h0,
@@ -702,7 +707,7 @@ kda_tc_state_kernel(const uint8_t *__restrict__ records, const float *__restrict
         const uint32_t id_b = idesc_bf16_f32(128, kNV, 1, 1);  // K^T Delta (K^ stored MN-major), [0; P] Delta
         const uint64_t d_s = smem_desc_sw64(smem_u32(Simg), 512);
         const uint64_t d_d = smem_desc_sw64(smem_u32(Dimg), 512);
-        bool ok = bar_and160(1, true);
+        bool ok = bar_and160(true);
         for (int i = 0; i < nchunks && ok; ++i) {
             const int s = i % kStages;
             const uint32_t st = smem_u32(sm + s * ST_BYTES);
@@ -722,9 +727,9 @@ kda_tc_state_kernel(const uint8_t *__restrict__ records, const float *__restrict
                     mma_commit(bar_w);
                 }
             }
-            ok = bar_and160(2, __shfl_sync(0xffffffffu, w_ok, 0));
-            if (!ok) break;
-            if (lane == 0) {
+            // Delta is in shared memory (warps 0-1); a failure anywhere is carried to barrier 1
+            const bool d_ok = bar_and96(__shfl_sync(0xffffffffu, w_ok, 0));
+            if (d_ok && lane == 0) {
                 tc_fence_after();
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)
@@ -738,7 +743,7 @@ kda_tc_state_kernel(const uint8_t *__restrict__ records, const float *__restrict
                 mma_commit(&empty[s]);
             }
             __syncwarp();
-            ok = bar_and160(1, true);
+            ok = bar_and160(d_ok);
         }
     } else {
         // ------------------------------------------------ warps 0-3: state row t = tid (TMEM lane)
@@ -760,7 +765,7 @@ kda_tc_state_kernel(const uint8_t *__restrict__ records, const float *__restrict
         };
         store_S_image();
         fence_async_smem();
-        bool ok = bar_and160(1, true);
+        bool ok = bar_and160(true);
 
         // output rows of chunk i: D_a[i % 2] rows 64..127, read by warps 2 and 3 (row = t - 64)
         auto write_o = [&](int i) {
@@ -847,11 +852,12 @@ kda_tc_state_kernel(const uint8_t *__restrict__ records, const float *__restrict
                 w_ok = false;
             }
             tc_fence_before();
-            fence_async_smem();
-            ok = bar_and160(2, w_ok);
-            if (!ok) break;
+            if (warp < 2) {  // hand Delta to the MMA warp; warps 2-3 go on (their output stores overlap K^T Delta)
+                fence_async_smem();
+                w_ok = bar_and96(w_ok);
+            }
             // (3) S <- e^{G_63} S + K^T Delta and its bf16 operand image
-            w_ok = mbar_wait(bar_b, i & 1);
+            w_ok = w_ok && mbar_wait(bar_b, i & 1);
             if (__all_sync(0xffffffffu, w_ok)) {
                 tc_fence_after();
                 float upd[32];
@@ -865,7 +871,7 @@ kda_tc_state_kernel(const uint8_t *__restrict__ records, const float *__restrict
             }
             tc_fence_before();
             fence_async_smem();
-            ok = bar_and160(1, w_ok);
+            ok = bar_and160(w_ok);
         }
         if (ok && nchunks > 0) {  // output of the last chunk
             bool w_ok = mbar_wait(bar_c, (nchunks - 1) & 1);
