@@ -35,6 +35,11 @@
 // (bounded the same way) times e^{E_b - E_a} <= 1, so no operand overflows even when G falls far
 // below the fp32 exponent range inside one chunk.  Factors that underflow belong to terms below
 // 1e-38 and are dropped harmlessly.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
 #include "kda_common.cuh"
 #include "kda_sm100.cuh"
 
@@ -160,7 +165,7 @@ constexpr uint32_t PREP_R = 32768;         // R^(0..3): K-major sw128, 160 rows 
 constexpr uint32_t PREP_KT = 73728;        // K o 2^G: MN-major 64 k-rows x 128
 constexpr uint32_t PREP_V = 90112;         // V: MN-major 64 k-rows x 128
 constexpr uint32_t PREP_SMALL = 106496;
-constexpr uint32_t PREP_SMEM = PREP_SMALL + (64 + 512 + 512 + 128) * 4 + 32 + 1024;
+constexpr uint32_t PREP_SMEM = PREP_SMALL + (64 + 512 + 512 + 128) * 4 + 48 + 1024;
 constexpr uint32_t kXAtom = 128 * 128;     // X: bytes per 64-channel atom column
 constexpr uint32_t kRRows = 160;
 constexpr uint32_t kRAtom = kRRows * 128;  // R: bytes per 64-channel atom column
@@ -236,7 +241,9 @@ __device__ __forceinline__ void subst_block_row(float *Asm, float *Mscr, int war
 }
 
 __global__ void __launch_bounds__(kPrepThreads, 2)
-kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
+kda_tc_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
+                   const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
                    const __nv_bfloat16 *__restrict__ v, const float *__restrict__ log_alpha,
                    const float *__restrict__ beta, int T_len, int H, int nc, const int *__restrict__ n_chunks,
                    const int4 *__restrict__ table, uint8_t *__restrict__ records, int *status, int pf_dist) {
@@ -250,8 +257,12 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
     float *s_E = s_beta + 64;   // [4][128] block references (base 2)
     float *s_tot = s_E + 512;   // [4][128] per-block gate sums (base 2)
     float *s_gl = s_tot + 512;  // [128]    G_63 (base 2)
-    uint64_t *mbar = reinterpret_cast<uint64_t *>(s_gl + 128);  // [0] W/U, [1] Gram (4 issuers)
-    uint32_t *s_tmem = reinterpret_cast<uint32_t *>(mbar + 2);
+    uint64_t *mbar = reinterpret_cast<uint64_t *>(s_gl + 128);  // [0] W/U, [1] Gram (4 issuers), [2] q k g, [3] V
+    uint32_t *s_tmem = reinterpret_cast<uint32_t *>(mbar + 4);
+    // input tiles, landed by TMA where the Gram operands are built later
+    const uint8_t *Qin = X;            // q: [64 rows][128] bf16
+    const uint8_t *Kin = X + 16384;    // k: [64 rows][128] bf16
+    const uint8_t *Gin = Rimg;         // log_alpha: [64 rows][128] fp32
     // reused once the Gram matrices are read out
     float *Asm = reinterpret_cast<float *>(X);           // [64][kAS] fp32: A, then T in place
     float *Mscr = reinterpret_cast<float *>(X + 17408);  // [16][kMS] fp32 scratch
@@ -307,45 +318,43 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
     if (tid == 0) {
         mbar_init(mbar, 1);
         mbar_init(mbar + 1, 4);
+        mbar_init(mbar + 2, 1);
+        mbar_init(mbar + 3, 1);
         mbar_fence_init();
+        // rows past the chunk (next sequence) are masked below; rows past the tensor are zero-filled
+        const int ti = (int)t0;
+        mbar_arrive_expect_tx(mbar + 2, 16384 + 16384 + 32768);
+        tma_load_3d(sm + PREP_X, &tm_q, 0, h, ti, mbar + 2);
+        tma_load_3d(sm + PREP_X + 16384, &tm_k, 0, h, ti, mbar + 2);
+        tma_load_3d(Rimg, &tm_g, 0, h, ti, mbar + 2);
+        mbar_arrive_expect_tx(mbar + 3, 16384);  // V straight into its MN-major sw128 operand image
+        tma_load_3d(Vimg, &tm_v, 0, h, ti, mbar + 3);
+        tma_load_3d(Vimg + 8192, &tm_v, 64, h, ti, mbar + 3);
     }
     if (warp == 0) {
         tmem_alloc(s_tmem, kPrepTmemCols);
         tmem_relinquish();
     }
+    if (tid < 64) s_beta[tid] = tid < L ? __ldg(beta + ((size_t)t0 + tid) * H + h) : 0.f;
+    __syncthreads();  // barriers initialised before anyone waits on them
 
-    // ---- load k, q (bf16 pairs) and log-gates (fp32 pairs) of this thread's 16 rows
-    const size_t tok_stride = (size_t)H * D;
-    const size_t off0 = ((size_t)t0 * H + h) * D + c0;
+    // ---- k, q (bf16 pairs) and log-gates (fp32 pairs) of this thread's 16 rows, from the landed tiles
+    const bool in_ok = mbar_wait(mbar + 2, 0);
     float2 g[16];
     uint32_t kk[16], qq[16];
 #pragma unroll
     for (int m = 0; m < 16; ++m) {
         const int r = 16 * qr + m;
         if (r < L) {
-            const size_t off = off0 + (size_t)r * tok_stride;
-            g[m] = __ldcs(reinterpret_cast<const float2 *>(log_alpha + off));
-            kk[m] = __ldcs(reinterpret_cast<const unsigned int *>(k + off));
-            qq[m] = __ldcs(reinterpret_cast<const unsigned int *>(q + off));
+            g[m] = *reinterpret_cast<const float2 *>(Gin + (r * D + c0) * 4);
+            kk[m] = *reinterpret_cast<const uint32_t *>(Kin + (r * D + c0) * 2);
+            qq[m] = *reinterpret_cast<const uint32_t *>(Qin + (r * D + c0) * 2);
         } else {
             g[m] = make_float2(0.f, 0.f);
             kk[m] = 0u;
             qq[m] = 0u;
         }
     }
-    if (tid < 64) s_beta[tid] = tid < L ? __ldg(beta + ((size_t)t0 + tid) * H + h) : 0.f;
-#pragma unroll
-    for (int s = 0; s < 4; ++s) {  // V tile straight into its operand image, asynchronously
-        const int idx = tid + kPrepThreads * s, row = idx >> 4, ch = idx & 15;
-        uint8_t *dst = Vimg + sw128_off(row, ch * 8, 64);
-        if (row < L) {
-            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)),
-                         "l"(v + ((size_t)(t0 + row) * H + h) * D + ch * 8) : "memory");
-        } else {
-            *reinterpret_cast<uint4 *>(dst) = make_uint4(0u, 0u, 0u, 0u);
-        }
-    }
-    asm volatile("cp.async.commit_group;" ::: "memory");
 
     // ---- chunk-local cumulative log2-gate G (fp32): block-local prefix, then block offsets
     g[0] = make_float2(g[0].x * kLog2e, g[0].y * kLog2e);
@@ -421,7 +430,7 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
         mma_commit(mbar + 1);
     }
     if (tid < D) reinterpret_cast<float *>(rec + REC_GL)[tid] = ex2(s_gl[tid]);
-    bool ok = mbar_wait(mbar + 1, 0);
+    bool ok = mbar_wait(mbar + 1, 0) && in_ok;
     ok = __syncthreads_and(ok);
 
     if (ok) {
@@ -521,12 +530,12 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
                 *reinterpret_cast<uint4 *>(TB + r * 128 + ((j ^ (r & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
             }
         }
-        asm volatile("cp.async.wait_all;" ::: "memory");  // this thread's V copies have landed
         fence_async_smem();
     }
     __syncthreads();
 
     // ---- W = T Diag(beta) (K o e^G), U = T Diag(beta) V  (M=64, N=128, K=64)
+    if (ok && tid == 0) ok = mbar_wait(mbar + 3, 0);  // V tile landed
     if (ok && tid == 0) {
         tc_fence_after();
         const uint32_t id_wu = idesc_bf16_f32(64, 128, 0, 1);
@@ -572,7 +581,6 @@ kda_tc_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__r
     }
     tc_fence_before();
     __syncthreads();
-    asm volatile("cp.async.wait_all;" ::: "memory");  // after a failed wait: no copy outlives the CTA
     if (warp == 0) tmem_dealloc(tmem, kPrepTmemCols);
 }
 
@@ -896,6 +904,34 @@ kda_tc_state_kernel(const uint8_t *__restrict__ records, const float *__restrict
     if (warp == 0) tmem_dealloc(tmem, kStateTmemCols);
 }
 
+// cuTensorMapEncodeTiled, fetched from the driver once (the library does not link libcuda).
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult qr;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &qr) == cudaSuccess &&
+            qr == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// Tensor map over a [tokens][H][128] tensor whose box is `box0` channels x 1 head x 64 tokens.
+cudaError_t encode_token_map(CUtensorMap *map, const void *base, CUtensorMapDataType dt, uint32_t esize,
+                             uint64_t tokens, int H, uint32_t box0, CUtensorMapSwizzle swizzle) {
+    const PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+    if (!enc) return cudaErrorNotSupported;
+    const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)tokens};
+    const cuuint64_t strides[2] = {(cuuint64_t)D * esize, (cuuint64_t)H * D * esize};
+    const cuuint32_t box[3] = {box0, 1u, (cuuint32_t)C};
+    const cuuint32_t estr[3] = {1u, 1u, 1u};
+    const CUresult r = enc(map, dt, 3, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                           swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 }  // namespace
 
 size_t prefill_tc_workspace_bytes(int B, int T, int H, int num_seqs, bool varlen) {
@@ -928,6 +964,15 @@ cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const
     if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
     if ((e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
     const int pf = 2 * nsm;
+    // TMA maps of the intra-chunk kernel's input tiles (q, k, V: bf16; log_alpha: fp32)
+    const uint64_t tokens = (uint64_t)B * T;
+    CUtensorMap tm_q, tm_k, tm_v, tm_g;
+    if (tokens > 0 &&
+        ((e = encode_token_map(&tm_q, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, tokens, H, D, CU_TENSOR_MAP_SWIZZLE_NONE)) != cudaSuccess ||
+        (e = encode_token_map(&tm_k, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, tokens, H, D, CU_TENSOR_MAP_SWIZZLE_NONE)) != cudaSuccess ||
+        (e = encode_token_map(&tm_v, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, tokens, H, 64, CU_TENSOR_MAP_SWIZZLE_128B)) != cudaSuccess ||
+        (e = encode_token_map(&tm_g, log_alpha, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, tokens, H, D, CU_TENSOR_MAP_SWIZZLE_NONE)) != cudaSuccess))
+        return e;
     const auto *qb = static_cast<const __nv_bfloat16 *>(q);
     const auto *kb = static_cast<const __nv_bfloat16 *>(k);
     const auto *vb = static_cast<const __nv_bfloat16 *>(v);
@@ -940,7 +985,7 @@ cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const
         if (lay.max_chunks > 0) {
             trace_before(kKernTcPrep, stream);
             kda_tc_prep_kernel<<<(unsigned)(lay.max_chunks * H), kPrepThreads, PREP_SMEM, stream>>>(
-                qb, kb, vb, log_alpha, beta, T, H, 0, status + 1, table, records, status, pf);
+                tm_q, tm_k, tm_v, tm_g, qb, kb, vb, log_alpha, beta, T, H, 0, status + 1, table, records, status, pf);
             trace_after(stream);
             if ((e = cudaGetLastError()) != cudaSuccess) return e;
         }
@@ -954,7 +999,7 @@ cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const
     if (nc > 0) {
         trace_before(kKernTcPrep, stream);
         kda_tc_prep_kernel<<<(unsigned)((int64_t)B * nc * H), kPrepThreads, PREP_SMEM, stream>>>(
-            qb, kb, vb, log_alpha, beta, T, H, nc, nullptr, nullptr, records, status, pf);
+            tm_q, tm_k, tm_v, tm_g, qb, kb, vb, log_alpha, beta, T, H, nc, nullptr, nullptr, records, status, pf);
         trace_after(stream);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }

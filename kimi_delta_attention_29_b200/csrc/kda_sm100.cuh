@@ -64,6 +64,18 @@ __device__ __forceinline__ void bulk_g2s(void *dst_smem, const void *src_gmem, u
                  : "memory");
 }
 
+// Tensor-map (TMA) tile load of a 3-D box at coordinates (x, y, z), completion signalled as
+// transaction bytes on `bar`.  The innermost coordinate x times the element size must be a multiple
+// of 16 bytes; boxes reaching past the tensor's bounds are zero-filled.
+__device__ __forceinline__ void tma_load_3d(void *dst_smem, const void *tensor_map, int x, int y, int z,
+                                            uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(
+            smem_u32(dst_smem)),
+        "l"(tensor_map), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
+        : "memory");
+}
+
 // Generic-proxy shared-memory writes -> visible to the async proxy (tensor core operand reads).
 __device__ __forceinline__ void fence_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
