@@ -22,7 +22,8 @@
 //     each block can use its own decay reference), the UT transform in fp32 on CUDA cores (blocked
 //     forward substitution), and W, U (tcgen05, M=64, N=128).  It writes [W; Q o e^G],
 //     K o e^{G_63-G}, P, U and e^{G_63} for the chunk as ready-to-use swizzled operand images
-//     ("records") in the workspace.
+//     ("records") in the workspace.  Its q, k, log-gate and V tiles arrive by TMA (tensor maps
+//     encoded per call), V directly in the swizzled layout the W/U product reads.
 //  2. kda_tc_state_kernel - one CTA per (sequence, head, 32 value columns); the value columns of S
 //     evolve independently.  It walks the sequence's chunks in order, bulk-copying each record into
 //     a 2-stage shared-memory ring, and runs per chunk: D_a = [W; Q~] S (M=128, N=32, K=128),
@@ -243,10 +244,8 @@ __device__ __forceinline__ void subst_block_row(float *Asm, float *Mscr, int war
 __global__ void __launch_bounds__(kPrepThreads, 2)
 kda_tc_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
-                   const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
-                   const __nv_bfloat16 *__restrict__ v, const float *__restrict__ log_alpha,
                    const float *__restrict__ beta, int T_len, int H, int nc, const int *__restrict__ n_chunks,
-                   const int4 *__restrict__ table, uint8_t *__restrict__ records, int *status, int pf_dist) {
+                   const int4 *__restrict__ table, uint8_t *__restrict__ records, int *status) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = align1024(smem_raw);
     uint8_t *X = sm + PREP_X;     // [K; Q] o 2^{G - E_b}, per block b: 16 k-rows then 16 q-rows
@@ -284,33 +283,6 @@ kda_tc_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     uint8_t *rec = records + ((size_t)chunk * H + h) * REC_BYTES;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    {   // L2 prefetch of the inputs of the CTA that starts about when this one ends
-        const int64_t nb = (int64_t)blockIdx.x + pf_dist;
-        if (nb < (int64_t)gridDim.x) {
-            const int chunk2 = (int)(nb / H), h2 = (int)(nb % H);
-            int64_t t2 = 0;
-            int L2 = 0;
-            if (table) {
-                if (chunk2 < *n_chunks) {
-                    const int4 e2 = table[chunk2];
-                    t2 = e2.y;
-                    L2 = e2.z;
-                }
-            } else {
-                const int n2 = chunk2 / nc, cc2 = chunk2 % nc;
-                t2 = (int64_t)n2 * T_len + (int64_t)cc2 * C;
-                L2 = min(C, T_len - cc2 * C);
-            }
-            const int which = tid >> 6, row = tid & 63;
-            if (row < L2) {
-                const size_t off = ((size_t)(t2 + row) * H + h2) * D;
-                const void *p = which == 0 ? (const void *)(q + off) : which == 1 ? (const void *)(k + off)
-                              : which == 2 ? (const void *)(v + off) : (const void *)(log_alpha + off);
-                const uint32_t bytes = which == 3 ? 512u : 256u;
-                asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
-            }
-        }
-    }
     const int c0 = 64 * (warp & 1) + 2 * lane;  // this thread's two key channels
     const int qr = warp >> 1;                   // key block: rows 16 qr .. 16 qr + 15
     constexpr float kLog2e = 1.4426950408889634f;
@@ -958,12 +930,6 @@ cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(kda_tc_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)STATE_SMEM);
     if (e != cudaSuccess) return e;
-    // The intra-chunk kernel runs two CTAs per SM; each prefetches into L2 the inputs of the CTA
-    // two waves later, which starts about when it ends.
-    int dev = 0, nsm = 0;
-    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
-    if ((e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
-    const int pf = 2 * nsm;
     // TMA maps of the intra-chunk kernel's input tiles (q, k, V: bf16; log_alpha: fp32)
     const uint64_t tokens = (uint64_t)B * T;
     CUtensorMap tm_q, tm_k, tm_v, tm_g;
@@ -973,9 +939,6 @@ cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const
         (e = encode_token_map(&tm_v, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, tokens, H, 64, CU_TENSOR_MAP_SWIZZLE_128B)) != cudaSuccess ||
         (e = encode_token_map(&tm_g, log_alpha, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, tokens, H, D, CU_TENSOR_MAP_SWIZZLE_NONE)) != cudaSuccess))
         return e;
-    const auto *qb = static_cast<const __nv_bfloat16 *>(q);
-    const auto *kb = static_cast<const __nv_bfloat16 *>(k);
-    const auto *vb = static_cast<const __nv_bfloat16 *>(v);
     auto *ob = static_cast<__nv_bfloat16 *>(o);
     if (cu_seqlens) {
         trace_before(kKernChunkTable, stream);
@@ -985,7 +948,7 @@ cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const
         if (lay.max_chunks > 0) {
             trace_before(kKernTcPrep, stream);
             kda_tc_prep_kernel<<<(unsigned)(lay.max_chunks * H), kPrepThreads, PREP_SMEM, stream>>>(
-                tm_q, tm_k, tm_v, tm_g, qb, kb, vb, log_alpha, beta, T, H, 0, status + 1, table, records, status, pf);
+                tm_q, tm_k, tm_v, tm_g, beta, T, H, 0, status + 1, table, records, status);
             trace_after(stream);
             if ((e = cudaGetLastError()) != cudaSuccess) return e;
         }
@@ -999,7 +962,7 @@ cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const
     if (nc > 0) {
         trace_before(kKernTcPrep, stream);
         kda_tc_prep_kernel<<<(unsigned)((int64_t)B * nc * H), kPrepThreads, PREP_SMEM, stream>>>(
-            tm_q, tm_k, tm_v, tm_g, qb, kb, vb, log_alpha, beta, T, H, nc, nullptr, nullptr, records, status, pf);
+            tm_q, tm_k, tm_v, tm_g, beta, T, H, nc, nullptr, nullptr, records, status);
         trace_after(stream);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
