@@ -58,7 +58,8 @@ enum {
     KDA_ERR_WORKSPACE_TOO_SMALL = -7, /* workspace_bytes < kda_chunk_fwd_workspace_size() */
     KDA_ERR_CUDA = -8,                /* a CUDA runtime call failed (launch or query) */
     KDA_ERR_TIMEOUT = -9,             /* device-detected: a bounded wait gave up */
-    KDA_ERR_ALIASING = -10            /* o overlaps an input, or h_T partially overlaps h0 */
+    KDA_ERR_ALIASING = -10,           /* o overlaps an input, or h_T partially overlaps h0 */
+    KDA_ERR_BAD_SLOT = -11            /* device-detected: a state-pool slot index is out of range */
 };
 
 /* Bytes of device workspace kda_chunk_fwd needs for these sizes (dtype-dependent).  It holds
@@ -122,6 +123,35 @@ KDA_API int kda_decode_step(const void *q, const void *k, const void *v, const f
                     const float *beta, float *S, int N, int H, int dk, int dv, kda_dtype dtype,
                     void *o, void *stream);
 
+/* Multi-token recurrent decode over a pool of states (batched serving, speculative verification).
+ * Kimi Linear summary page (th.news.hada.io topic 31936), sections "Kimi Linear model composition"
+ * and the long-context decoding results: KDA layers keep a fixed-size per-head state in place of a
+ * KV cache, so serving reads and rewrites that state per step; this entry point advances each state
+ * by several tokens per read, and addresses states through slot indices so a serving engine can keep
+ * them in one pool.  The page describes no such interface; the recurrence is the one of
+ * kda_decode_step, applied Tq times.
+ * For each sequence n in [0, N) and head h, starting from S = S_pool[slot_in[n], h]:
+ *   for t = 0 .. Tq-1 (token (n, t)):
+ *     S' = Diag(exp(log_alpha[n,t,h])) S;  u = beta[n,t,h] (v[n,t,h] - S'^T k[n,t,h]);  S <- S' + k u^T;
+ *     o[n,t,h] = S^T q[n,t,h]
+ *   S_pool[slot_out[n], h] = S.
+ *   q, k      : [N, Tq, H, dk] dtype     v, o : [N, Tq, H, dv] dtype
+ *   log_alpha : [N, Tq, H, dk] fp32      beta : [N, Tq, H] fp32
+ *   S_pool    : [num_slots, H, dk, dv] fp32, read at slot_in and written at slot_out
+ *   slot_in, slot_out : device int32 [N], or NULL for slot n.  slot_out may equal slot_in (commit in
+ *               place) or name other slots (keep the input states, e.g. to verify draft tokens before
+ *               committing them).  No slot may be written for two sequences, nor written for one
+ *               sequence and read for another; such calls race (undefined results).
+ *   status    : device int32, or NULL.  A sequence whose slot_in or slot_out is outside
+ *               [0, num_slots) is skipped (nothing is read or written for it, its o rows are left
+ *               untouched) and KDA_ERR_BAD_SLOT is stored in *status if it still holds 0; read it
+ *               back with kda_get_status(status, stream).
+ * Supported: dk = dv in {64, 128}.  Needs no workspace.  Asynchronous on `stream`. */
+KDA_API int kda_decode_multi(const void *q, const void *k, const void *v, const float *log_alpha,
+                             const float *beta, float *S_pool, int num_slots, const int32_t *slot_in,
+                             const int32_t *slot_out, int N, int Tq, int H, int dk, int dv, kda_dtype dtype,
+                             void *o, int *status, void *stream);
+
 /* Synchronizes `stream`, reads the device status word kept in `workspace` by the last
  * kda_chunk_fwd that used it, clears it, and returns it (KDA_OK, KDA_ERR_BAD_SEQLENS or
  * KDA_ERR_TIMEOUT), or KDA_ERR_CUDA if the synchronization itself failed. */
@@ -136,7 +166,8 @@ KDA_API const char *kda_status_string(int status);
  * kda_trace_end() synchronizes the device, stops recording, writes up to `capacity` entries of
  * (kernel id, milliseconds) into kernel_ids / ms and returns how many kernels were recorded (or
  * KDA_ERR_CUDA).  Kernel ids: 0 varlen chunk table, 1 intra-chunk WY kernel (tensor cores),
- * 2 state-passing kernel (tensor cores), 3 chunkwise kernel (CUDA cores), 4 decode step.
+ * 2 state-passing kernel (tensor cores), 3 chunkwise kernel (CUDA cores), 4 decode step,
+ * 5 multi-token decode.
  * Process-wide and not thread-safe; events are owned by the library. */
 KDA_API int kda_trace_begin(int max_kernels);
 KDA_API int kda_trace_end(int *kernel_ids, float *ms, int capacity);

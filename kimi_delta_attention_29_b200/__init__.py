@@ -98,6 +98,25 @@ def kda_chunk_fwd(q, k, v, log_alpha, beta, h0=None, cu_seqlens=None, chunk_size
     return o, h_T
 
 
+def kda_decode_multi(q, k, v, log_alpha, beta, S_pool, slot_in=None, slot_out=None, o=None, status=None,
+                     stream=None):
+    """Tq recurrent steps per sequence on a slot-indexed state pool.  q, k [N,Tq,H,dk], v [N,Tq,H,dv]
+    (bf16 or fp32), log_alpha [N,Tq,H,dk] fp32, beta [N,Tq,H] fp32, S_pool [P,H,dk,dv] fp32 (read at
+    slot_in, written at slot_out), slot_in / slot_out int32 [N] on the device or None (slot n),
+    status: int32 device tensor receiving KDA_ERR_BAD_SLOT, or None.  Returns o [N,Tq,H,dv]."""
+    torch = _torch()
+    N, Tq, H, dk = q.shape
+    dv = v.shape[-1]
+    if o is None:
+        o = torch.empty((N, Tq, H, dv), dtype=q.dtype, device=q.device)
+    rc = _lib.load().kda_decode_multi(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(S_pool),
+                                      S_pool.shape[0], _ptr(slot_in), _ptr(slot_out), N, Tq, H, dk, dv,
+                                      _dtype_code(q.dtype), _ptr(o), _ptr(status), _stream(stream, q.device))
+    if rc != _lib.KDA_OK:
+        raise KdaError(rc, "kda_decode_multi")
+    return o
+
+
 def kda_get_status(workspace, stream=None) -> int:
     buf = workspace.buf if isinstance(workspace, Workspace) else workspace
     return int(_lib.load().kda_get_status(_ptr(buf), _stream(stream, buf.device)))

@@ -120,6 +120,7 @@ const char *kda_status_string(int status) {
         case KDA_ERR_CUDA: return "KDA_ERR_CUDA: a CUDA runtime call failed";
         case KDA_ERR_TIMEOUT: return "KDA_ERR_TIMEOUT: a bounded device wait gave up";
         case KDA_ERR_ALIASING: return "KDA_ERR_ALIASING: an output overlaps an input";
+        case KDA_ERR_BAD_SLOT: return "KDA_ERR_BAD_SLOT: a state-pool slot index is out of range";
         default: return "KDA: unknown status";
     }
 }
@@ -206,6 +207,39 @@ int kda_decode_step(const void *q, const void *k, const void *v, const float *lo
         if (overlaps(ro, r) || overlaps(rs, r)) return KDA_ERR_ALIASING;
     cudaError_t e = kda::launch_decode(q, k, v, log_alpha, beta, S, N, H, dk, dv, dtype, o,
                                        static_cast<cudaStream_t>(stream_));
+    return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+int kda_decode_multi(const void *q, const void *k, const void *v, const float *log_alpha, const float *beta,
+                     float *S_pool, int num_slots, const int32_t *slot_in, const int32_t *slot_out, int N, int Tq,
+                     int H, int dk, int dv, kda_dtype dtype, void *o, int *status, void *stream_) {
+    if (dtype != KDA_F32 && dtype != KDA_BF16) return KDA_ERR_BAD_DTYPE;
+    if (!q || !k || !v || !log_alpha || !beta || !S_pool || !o) return KDA_ERR_NULL_ARG;
+    if (N <= 0 || Tq <= 0 || H <= 0 || dk <= 0 || dv <= 0 || num_slots <= 0) return KDA_ERR_BAD_SHAPE;
+    const int64_t tokens = (int64_t)N * Tq * H, states = (int64_t)num_slots * H;
+    if ((int64_t)N * H > (int64_t)INT32_MAX || tokens * (dk > dv ? dk : dv) > ((int64_t)1 << 40) ||
+        states * dk * dv > ((int64_t)1 << 40))
+        return KDA_ERR_BAD_SHAPE;
+    if ((!slot_in || !slot_out) && N > num_slots) return KDA_ERR_BAD_SHAPE;  // slot n must exist
+    if (!supported_dims(dk, dv)) return KDA_ERR_UNSUPPORTED;
+    const void *ptrs[] = {q, k, v, log_alpha, beta, S_pool, o};
+    for (const void *p : ptrs)
+        if (!aligned16(p)) return KDA_ERR_MISALIGNED;
+    const void *words[] = {slot_in, slot_out, status};
+    for (const void *p : words)
+        if (reinterpret_cast<uintptr_t>(p) % 4 != 0) return KDA_ERR_MISALIGNED;
+    const size_t es = elem_size(dtype);
+    const Range ro = range_of(o, (size_t)tokens * dv * es), rs = range_of(S_pool, (size_t)states * dk * dv * 4),
+                rst = range_of(status, status ? 4 : 0);
+    const Range inputs[] = {range_of(q, (size_t)tokens * dk * es), range_of(k, (size_t)tokens * dk * es),
+                            range_of(v, (size_t)tokens * dv * es), range_of(log_alpha, (size_t)tokens * dk * 4),
+                            range_of(beta, (size_t)tokens * 4), range_of(slot_in, slot_in ? (size_t)N * 4 : 0),
+                            range_of(slot_out, slot_out ? (size_t)N * 4 : 0)};
+    if (overlaps(ro, rs) || overlaps(ro, rst) || overlaps(rs, rst)) return KDA_ERR_ALIASING;
+    for (const Range &r : inputs)
+        if (overlaps(ro, r) || overlaps(rs, r) || overlaps(rst, r)) return KDA_ERR_ALIASING;
+    cudaError_t e = kda::launch_decode_multi(q, k, v, log_alpha, beta, S_pool, num_slots, slot_in, slot_out, N, Tq,
+                                             H, dk, dtype, o, status, static_cast<cudaStream_t>(stream_));
     return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 

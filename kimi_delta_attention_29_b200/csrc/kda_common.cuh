@@ -33,7 +33,8 @@ constexpr int kChunk = 64;
 // Host-side launchers (defined in the .cu files, called by kda_api.cu).
 namespace kda {
 // Kernel ids reported by kda_trace_end.
-enum KernelId { kKernChunkTable = 0, kKernTcPrep = 1, kKernTcState = 2, kKernSimt = 3, kKernDecode = 4 };
+enum KernelId { kKernChunkTable = 0, kKernTcPrep = 1, kKernTcState = 2, kKernSimt = 3, kKernDecode = 4,
+                kKernDecodeMulti = 5 };
 // Diagnostics: bracket one kernel launch with trace events when kda_trace_begin is active.
 void trace_before(int kernel_id, cudaStream_t stream);
 void trace_after(cudaStream_t stream);
@@ -41,6 +42,11 @@ void trace_after(cudaStream_t stream);
 cudaError_t launch_decode(const void *q, const void *k, const void *v, const float *log_alpha,
                           const float *beta, float *S, int N, int H, int dk, int dv, kda_dtype dtype,
                           void *o, cudaStream_t stream);
+
+cudaError_t launch_decode_multi(const void *q, const void *k, const void *v, const float *log_alpha,
+                                const float *beta, float *S_pool, int num_slots, const int32_t *slot_in,
+                                const int32_t *slot_out, int N, int Tq, int H, int dk, kda_dtype dtype, void *o,
+                                int *status, cudaStream_t stream);
 
 // CUDA-core chunkwise forward (any supported dtype, dk = dv in {64, 128}).
 cudaError_t launch_prefill_simt(const void *q, const void *k, const void *v, const float *log_alpha,

@@ -1,4 +1,5 @@
-// Recurrent KDA decode step: one token for each of N*H independent states, in place.
+// Recurrent KDA decode: one token for each of N*H independent states, in place; and several
+// tokens per state over a slot-indexed state pool.
 //
 // Kimi Linear summary page (th.news.hada.io topic 31936), section "Kimi Linear model
 // composition" / "3:1 KDA-MLA hybrid": KDA layers keep a fixed-size per-head state instead of a
@@ -113,6 +114,124 @@ kda_decode_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__r
     }
 }
 
+// Tq tokens per state, the state kept in registers between them: read once from slot_in, written
+// once to slot_out.  Same data layout and reductions per token as kda_decode_kernel, with 16 warps
+// per state (8 state rows per warp) so that the token data of token t + 1 can be fetched into
+// registers while token t is reduced.
+constexpr int kMultiWarps = 16;
+template <int D, typename T>
+__global__ void __launch_bounds__(kMultiWarps * 32, 1)
+kda_decode_multi_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
+                        const float *__restrict__ log_alpha, const float *__restrict__ beta,
+                        float *__restrict__ S_pool, int num_slots, const int32_t *__restrict__ slot_in,
+                        const int32_t *__restrict__ slot_out, int Tq, int H, T *__restrict__ o,
+                        int *__restrict__ status) {
+    constexpr int RPW = D / kMultiWarps;  // rows per warp
+    constexpr int VEC = D / 32;            // columns per lane
+    __shared__ float red_a[kMultiWarps][D];
+    __shared__ float red_b[kMultiWarps][D];
+    __shared__ float s_u[D];
+    __shared__ float s_qk[kMultiWarps];
+
+    const int unit = blockIdx.x;  // n * H + h
+    const int n = unit / H, h = unit % H;
+    const int si = slot_in ? slot_in[n] : n, so = slot_out ? slot_out[n] : n;
+    if (si < 0 || si >= num_slots || so < 0 || so >= num_slots) {
+        if (threadIdx.x == 0 && status) set_status(status, KDA_ERR_BAD_SLOT);
+        return;
+    }
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const float *Sin = S_pool + ((size_t)si * H + h) * D * D;
+    float *Sout = S_pool + ((size_t)so * H + h) * D * D;
+
+    float s[RPW][VEC];
+#pragma unroll
+    for (int m = 0; m < RPW; ++m) VecIO<VEC>::load(Sin + (size_t)(warp + kMultiWarps * m) * D + lane * VEC, s[m]);
+
+    // this thread's rows of k, q, log_alpha for the current token (prefetched one token ahead)
+    auto tok_of = [&](int t) { return ((size_t)n * Tq + t) * H + h; };
+    float kr[RPW], qr[RPW], lr[RPW];
+    auto fetch = [&](int t) {
+        const size_t tk = tok_of(t) * D;
+#pragma unroll
+        for (int m = 0; m < RPW; ++m) {
+            const int i = warp + kMultiWarps * m;
+            kr[m] = Elem<T>::load(k + tk + i);
+            qr[m] = Elem<T>::load(q + tk + i);
+            lr[m] = __ldg(log_alpha + tk + i);
+        }
+    };
+    fetch(0);
+    for (int t = 0; t < Tq; ++t) {
+        float ki[RPW], qi[RPW], ai[RPW];
+#pragma unroll
+        for (int m = 0; m < RPW; ++m) {
+            ki[m] = kr[m];
+            qi[m] = qr[m];
+            ai[m] = expf(lr[m]);
+        }
+        if (t + 1 < Tq) fetch(t + 1);
+        float pa[VEC], pb[VEC];
+#pragma unroll
+        for (int c = 0; c < VEC; ++c) pa[c] = pb[c] = 0.f;
+        float pqk = 0.f;
+#pragma unroll
+        for (int m = 0; m < RPW; ++m) {
+            pqk = fmaf(qi[m], ki[m], pqk);
+#pragma unroll
+            for (int c = 0; c < VEC; ++c) {
+                s[m][c] *= ai[m];
+                pa[c] = fmaf(s[m][c], ki[m], pa[c]);
+                pb[c] = fmaf(s[m][c], qi[m], pb[c]);
+            }
+        }
+#pragma unroll
+        for (int c = 0; c < VEC; ++c) {
+            red_a[warp][lane * VEC + c] = pa[c];
+            red_b[warp][lane * VEC + c] = pb[c];
+        }
+        if (lane == 0) s_qk[warp] = pqk;
+        __syncthreads();
+        if (threadIdx.x < D) {
+            const int j = threadIdx.x;
+            const size_t tk = tok_of(t);
+            float a = 0.f, b = 0.f, qk = 0.f;
+#pragma unroll
+            for (int w = 0; w < kMultiWarps; ++w) {
+                a += red_a[w][j];
+                b += red_b[w][j];
+                qk += s_qk[w];
+            }
+            const float uj = __ldg(beta + tk) * (Elem<T>::load(v + tk * D + j) - a);
+            s_u[j] = uj;
+            Elem<T>::store(o + tk * D + j, fmaf(qk, uj, b));
+        }
+        __syncthreads();
+        float uu[VEC];
+#pragma unroll
+        for (int c = 0; c < VEC; ++c) uu[c] = s_u[lane * VEC + c];
+#pragma unroll
+        for (int m = 0; m < RPW; ++m)
+#pragma unroll
+            for (int c = 0; c < VEC; ++c) s[m][c] = fmaf(ki[m], uu[c], s[m][c]);
+    }
+#pragma unroll
+    for (int m = 0; m < RPW; ++m) VecIO<VEC>::store(Sout + (size_t)(warp + kMultiWarps * m) * D + lane * VEC, s[m]);
+}
+
+template <int D, typename T>
+cudaError_t launch_decode_multi_t(const void *q, const void *k, const void *v, const float *la, const float *beta,
+                                  float *S_pool, int num_slots, const int32_t *slot_in, const int32_t *slot_out,
+                                  int N, int Tq, int H, void *o, int *status, cudaStream_t stream) {
+    const unsigned units = (unsigned)N * (unsigned)H;
+    trace_before(kKernDecodeMulti, stream);
+    kda_decode_multi_kernel<D, T><<<units, kMultiWarps * 32, 0, stream>>>(
+        static_cast<const T *>(q), static_cast<const T *>(k), static_cast<const T *>(v), la, beta, S_pool,
+        num_slots, slot_in, slot_out, Tq, H, static_cast<T *>(o), status);
+    trace_after(stream);
+    return cudaGetLastError();
+}
+
 template <int D, typename T>
 cudaError_t launch_decode_t(const void *q, const void *k, const void *v, const float *la,
                             const float *beta, float *S, int N, int H, void *o, cudaStream_t stream) {
@@ -137,6 +256,18 @@ cudaError_t launch_decode(const void *q, const void *k, const void *v, const flo
     }
     return dtype == KDA_BF16 ? launch_decode_t<64, __nv_bfloat16>(q, k, v, log_alpha, beta, S, N, H, o, stream)
                              : launch_decode_t<64, float>(q, k, v, log_alpha, beta, S, N, H, o, stream);
+}
+
+cudaError_t launch_decode_multi(const void *q, const void *k, const void *v, const float *log_alpha,
+                                const float *beta, float *S_pool, int num_slots, const int32_t *slot_in,
+                                const int32_t *slot_out, int N, int Tq, int H, int dk, kda_dtype dtype, void *o,
+                                int *status, cudaStream_t stream) {
+#define KDA_MULTI(DIM, TYPE)                                                                                  \
+    launch_decode_multi_t<DIM, TYPE>(q, k, v, log_alpha, beta, S_pool, num_slots, slot_in, slot_out, N, Tq, H, o, \
+                                     status, stream)
+    if (dk == 128) return dtype == KDA_BF16 ? KDA_MULTI(128, __nv_bfloat16) : KDA_MULTI(128, float);
+    return dtype == KDA_BF16 ? KDA_MULTI(64, __nv_bfloat16) : KDA_MULTI(64, float);
+#undef KDA_MULTI
 }
 
 }  // namespace kda

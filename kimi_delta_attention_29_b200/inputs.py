@@ -120,3 +120,18 @@ def make_decode_token(N: int, H: int, dk: int, dv: int, dtype=torch.bfloat16, ga
     log_alpha = -F.softplus(torch.randn(N, H, dk, generator=g, **f32) + gate_shift)
     beta = torch.sigmoid(torch.randn(N, H, generator=g, **f32))
     return dict(q=q, k=k, v=v, log_alpha=log_alpha, beta=beta)
+
+
+def make_decode_tokens(N: int, Tq: int, H: int, dk: int, dv: int, dtype=torch.bfloat16, gate_shift=2.0,
+                       seed: int = 2000, device="cpu") -> dict:
+    """Inputs of Tq consecutive decode tokens for N sequences x H heads, token-major [N, Tq, H, ...]
+    (the same distributions as make_decode_token)."""
+    device = torch.device(device)
+    g = torch.Generator(device=device).manual_seed(seed)
+    f32 = dict(device=device, dtype=torch.float32)
+    q = _unit_rows(torch.randn(N, Tq, H, dk, generator=g, **f32)).to(dtype)
+    k = _unit_rows(torch.randn(N, Tq, H, dk, generator=g, **f32)).to(dtype)
+    v = torch.randn(N, Tq, H, dv, generator=g, **f32).to(dtype)
+    log_alpha = -F.softplus(torch.randn(N, Tq, H, dk, generator=g, **f32) + gate_shift)
+    beta = torch.sigmoid(torch.randn(N, Tq, H, generator=g, **f32))
+    return dict(q=q, k=k, v=v, log_alpha=log_alpha, beta=beta)

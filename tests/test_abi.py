@@ -39,7 +39,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 def test_status_strings_and_version(lib):
     assert lib.kda_version() >= 100
-    for code in range(0, -11, -1):
+    for code in range(0, -12, -1):
         s = _lib.status_string(code)
         assert s.startswith("KDA_")
     assert "unknown" in _lib.status_string(-999)
@@ -111,3 +111,29 @@ def test_binding_refuses_noncontiguous():
     x = torch.zeros(4, 8)[:, ::2]
     with pytest.raises(ValueError):
         kda._ptr(x)
+
+
+def _multi(lib, **kw):
+    args = dict(q=A, k=2 * A, v=3 * A, la=4 * A, beta=5 * A, pool=6 * A, P=8, si=None, so=None, N=4, Tq=3, H=2,
+                dk=128, dv=128, dtype=_lib.KDA_BF16, o=7 * A, status=None, stream=None)
+    args.update(kw)
+    c = ctypes.c_void_p
+    return lib.kda_decode_multi(c(args["q"]), c(args["k"]), c(args["v"]), c(args["la"]), c(args["beta"]),
+                                c(args["pool"]), args["P"], c(args["si"]), c(args["so"]), args["N"], args["Tq"],
+                                args["H"], args["dk"], args["dv"], args["dtype"], c(args["o"]), c(args["status"]),
+                                c(args["stream"]))
+
+
+def test_decode_multi_rejects_on_host(lib):
+    assert _multi(lib, dtype=9) == _lib.KDA_ERR_BAD_DTYPE
+    assert _multi(lib, pool=None) == _lib.KDA_ERR_NULL_ARG
+    assert _multi(lib, o=None) == _lib.KDA_ERR_NULL_ARG
+    assert _multi(lib, Tq=0) == _lib.KDA_ERR_BAD_SHAPE
+    assert _multi(lib, P=0) == _lib.KDA_ERR_BAD_SHAPE
+    assert _multi(lib, N=9) == _lib.KDA_ERR_BAD_SHAPE                  # slot n must exist without slot arrays
+    assert _multi(lib, dk=96, dv=96) == _lib.KDA_ERR_UNSUPPORTED
+    assert _multi(lib, q=A + 8) == _lib.KDA_ERR_MISALIGNED
+    assert _multi(lib, si=9 * A + 2) == _lib.KDA_ERR_MISALIGNED         # int32 slot array
+    assert _multi(lib, o=A) == _lib.KDA_ERR_ALIASING                    # o overlaps q
+    assert _multi(lib, pool=5 * A) == _lib.KDA_ERR_ALIASING             # pool overlaps beta
+    assert _multi(lib, status=6 * A) == _lib.KDA_ERR_ALIASING           # status inside the pool
