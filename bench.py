@@ -37,6 +37,7 @@ STATE_BYTES = 128 * 128 * 4                    # one fp32 state (h0 read or h_T 
 REC_WRITE_BYTES = 74240                        # WY record bytes the intra-chunk kernel writes per chunk-head
 REC_READ_BYTES = 32768 + 16384 + 8192 + 512 + 16384  # record bytes the state kernel needs per chunk-head
 DECODE_BYTES_PER_STATE = 2 * STATE_BYTES + 3 * 256 + 512 + 4 + 256  # S read+write, q/k/v, gates, beta, o
+MULTI_TQ = (4, 16)  # tokens per kda_decode_multi call in the decode benchmark
 
 
 def parse_args():
@@ -406,10 +407,52 @@ def decode_bench(args, dev, stream, peaks, barrier, max_over_ranks):
     nbytes = shp.N * shp.H * DECODE_BYTES_PER_STATE
     gbs = nbytes / (ms / 1e3) / 1e9
     traffic = ncu_traffic("kda_decode_kernel", shp.N * shp.H)
-    return {"workload": shp.name, "steps": args.decode_steps, "ms_per_step": ms,
-            "tokens_per_s": shp.N / (ms / 1e3), "hbm_gbs": gbs, "peak_gbs": peaks["hbm_gbs"],
-            "frac": gbs / peaks["hbm_gbs"], "bytes_per_step": nbytes, "traffic": traffic,
-            "note": "inputs cycle through 8 pre-drawn token sets; the 512 MiB state streams from HBM each step"}
+    out = {"workload": shp.name, "steps": args.decode_steps, "ms_per_step": ms,
+           "tokens_per_s": shp.N / (ms / 1e3), "hbm_gbs": gbs, "peak_gbs": peaks["hbm_gbs"],
+           "frac": gbs / peaks["hbm_gbs"], "bytes_per_step": nbytes, "traffic": traffic,
+           "note": "inputs cycle through 8 pre-drawn token sets; the 512 MiB state streams from HBM each step"}
+    out["multi_token"] = [decode_multi_bench(args, dev, stream, peaks, barrier, max_over_ranks, S, tq)
+                          for tq in MULTI_TQ]
+    return out
+
+
+def decode_multi_bench(args, dev, stream, peaks, barrier, max_over_ranks, pool, tq):
+    """The same 256 x 32 states as a slot pool, `tq` tokens per call (kda_decode_multi), slots a fixed
+    permutation, committed in place; decode_steps tokens in all."""
+    import torch
+
+    import kimi_delta_attention_29_b200 as kda
+    from kimi_delta_attention_29_b200 import inputs as gen
+
+    shp = gen.DECODE
+    perm = torch.randperm(shp.N, generator=torch.Generator().manual_seed(3)).to(torch.int32).to(dev)
+    toks = [gen.make_decode_tokens(shp.N, tq, shp.H, shp.dk, shp.dv, dtype=shp.dtype, seed=3000 + s, device=dev)
+            for s in range(4)]
+    o = torch.empty(shp.N, tq, shp.H, shp.dv, dtype=shp.dtype, device=dev)
+    calls = max(1, args.decode_steps // tq)
+
+    def call(s):
+        t = toks[s % len(toks)]
+        kda.kda_decode_multi(t["q"], t["k"], t["v"], t["log_alpha"], t["beta"], pool, slot_in=perm, slot_out=perm,
+                             o=o, stream=stream)
+
+    for s in range(8):
+        call(s)
+    torch.cuda.synchronize(dev)
+    barrier()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for s in range(calls):
+        call(s)
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    ms = max_over_ranks(ev0.elapsed_time(ev1)) / calls
+    states = shp.N * shp.H
+    nbytes = states * (2 * shp.dk * shp.dv * 4 + tq * (DECODE_BYTES_PER_STATE - 2 * shp.dk * shp.dv * 4))
+    gbs = nbytes / (ms / 1e3) / 1e9
+    return {"tq": tq, "calls": calls, "ms_per_call": ms, "tokens_per_s": shp.N * tq / (ms / 1e3),
+            "hbm_gbs": gbs, "frac": gbs / peaks["hbm_gbs"], "bytes_per_call": nbytes}
 
 
 def main():

@@ -115,23 +115,47 @@ kda_decode_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__r
 }
 
 // Tq tokens per state, the state kept in registers between them: read once from slot_in, written
-// once to slot_out.  Same data layout and reductions per token as kda_decode_kernel, with 16 warps
-// per state (8 state rows per warp) so that the token data of token t + 1 can be fetched into
-// registers while token t is reduced.
-constexpr int kMultiWarps = 16;
+// once to slot_out.  Same data layout and reductions per token as kda_decode_kernel.  The token data (q, k, v, log_alpha, beta) is staged in shared
+// memory with cp.async, kTokBatch tokens at a time (half for fp32) and double-buffered, so each
+// token's reductions read it from shared memory while the next batch is in flight; k and q are
+// re-read from there for the update instead of being held in registers, so two CTAs fit per SM.
+constexpr int kMultiWarps = 8;
+constexpr int kTokBatch = 8;
+__device__ __forceinline__ float to_f(float x) { return x; }
+__device__ __forceinline__ float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
+__device__ __forceinline__ void cp_async16(void *dst, const void *src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
+                 "l"(src)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async4(void *dst, const void *src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
+                 "l"(src)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
 template <int D, typename T>
-__global__ void __launch_bounds__(kMultiWarps * 32, 1)
+__global__ void __launch_bounds__(kMultiWarps * 32, 2)
 kda_decode_multi_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
                         const float *__restrict__ log_alpha, const float *__restrict__ beta,
                         float *__restrict__ S_pool, int num_slots, const int32_t *__restrict__ slot_in,
                         const int32_t *__restrict__ slot_out, int Tq, int H, T *__restrict__ o,
                         int *__restrict__ status) {
     constexpr int RPW = D / kMultiWarps;  // rows per warp
-    constexpr int VEC = D / 32;            // columns per lane
+    constexpr int VEC = D / 32;           // columns per lane
+    constexpr int TB = sizeof(T) == 4 ? kTokBatch / 2 : kTokBatch;  // fp32 tokens: half the batch (static shared memory)
     __shared__ float red_a[kMultiWarps][D];
     __shared__ float red_b[kMultiWarps][D];
     __shared__ float s_u[D];
     __shared__ float s_qk[kMultiWarps];
+    __shared__ __align__(16) T sk[2][TB][D];
+    __shared__ __align__(16) T sq[2][TB][D];
+    __shared__ __align__(16) T sv[2][TB][D];
+    __shared__ __align__(16) float sla[2][TB][D];
+    __shared__ float sb[2][TB];
 
     const int unit = blockIdx.x;  // n * H + h
     const int n = unit / H, h = unit % H;
@@ -143,77 +167,97 @@ kda_decode_multi_kernel(const T *__restrict__ q, const T *__restrict__ k, const 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const float *Sin = S_pool + ((size_t)si * H + h) * D * D;
     float *Sout = S_pool + ((size_t)so * H + h) * D * D;
+    auto tok_of = [&](int t) { return ((size_t)n * Tq + t) * H + h; };
 
+    // tokens bi*TB .. bi*TB + TB - 1 (clipped to Tq) into buffer bi % 2, as one cp.async group
+    auto stage = [&](int bi) {
+        const int buf = bi & 1, t0 = bi * TB, nt = min(TB, Tq - t0);
+        constexpr int CPR = D * (int)sizeof(T) / 16;  // 16-byte pieces per q / k / v row
+        constexpr int CPA = D * 4 / 16;               // per log_alpha row
+        constexpr int PER = 3 * CPR + CPA;
+        for (int e = threadIdx.x; e < nt * PER; e += kMultiWarps * 32) {
+            const int tt = e / PER, r = e % PER;
+            const size_t tok = tok_of(t0 + tt);
+            if (r < 3 * CPR) {
+                const int which = r / CPR, pc = r % CPR;
+                const T *src = (which == 0 ? k : which == 1 ? q : v) + tok * D;
+                T *dst = which == 0 ? sk[buf][tt] : which == 1 ? sq[buf][tt] : sv[buf][tt];
+                cp_async16(reinterpret_cast<uint8_t *>(dst) + 16 * pc, reinterpret_cast<const uint8_t *>(src) + 16 * pc);
+            } else {
+                const int pc = r - 3 * CPR;
+                cp_async16(&sla[buf][tt][4 * pc], log_alpha + tok * D + 4 * pc);
+            }
+        }
+        if (threadIdx.x < nt) cp_async4(&sb[buf][threadIdx.x], beta + tok_of(t0 + threadIdx.x));
+        cp_async_commit();
+    };
+
+    stage(0);
     float s[RPW][VEC];
 #pragma unroll
     for (int m = 0; m < RPW; ++m) VecIO<VEC>::load(Sin + (size_t)(warp + kMultiWarps * m) * D + lane * VEC, s[m]);
 
-    // this thread's rows of k, q, log_alpha for the current token (prefetched one token ahead)
-    auto tok_of = [&](int t) { return ((size_t)n * Tq + t) * H + h; };
-    float kr[RPW], qr[RPW], lr[RPW];
-    auto fetch = [&](int t) {
-        const size_t tk = tok_of(t) * D;
-#pragma unroll
-        for (int m = 0; m < RPW; ++m) {
-            const int i = warp + kMultiWarps * m;
-            kr[m] = Elem<T>::load(k + tk + i);
-            qr[m] = Elem<T>::load(q + tk + i);
-            lr[m] = __ldg(log_alpha + tk + i);
+    const int nbatch = (Tq + TB - 1) / TB;
+    for (int bi = 0; bi < nbatch; ++bi) {
+        const int buf = bi & 1, t0 = bi * TB, nt = min(TB, Tq - t0);
+        if (bi + 1 < nbatch) {
+            stage(bi + 1);
+            cp_async_wait<1>();  // this thread's pieces of batch bi have landed
+        } else {
+            cp_async_wait<0>();
         }
-    };
-    fetch(0);
-    for (int t = 0; t < Tq; ++t) {
-        float ki[RPW], qi[RPW], ai[RPW];
+        __syncthreads();  // ... and every other thread's
+        for (int tt = 0; tt < nt; ++tt) {
+            float pa[VEC], pb[VEC];
 #pragma unroll
-        for (int m = 0; m < RPW; ++m) {
-            ki[m] = kr[m];
-            qi[m] = qr[m];
-            ai[m] = expf(lr[m]);
-        }
-        if (t + 1 < Tq) fetch(t + 1);
-        float pa[VEC], pb[VEC];
+            for (int c = 0; c < VEC; ++c) pa[c] = pb[c] = 0.f;
+            float pqk = 0.f;
 #pragma unroll
-        for (int c = 0; c < VEC; ++c) pa[c] = pb[c] = 0.f;
-        float pqk = 0.f;
+            for (int m = 0; m < RPW; ++m) {
+                const int i = warp + kMultiWarps * m;
+                const float ki = to_f(sk[buf][tt][i]);  // shared-memory reads (not the global-memory Elem loads)
+                const float qi = to_f(sq[buf][tt][i]);
+                const float ai = expf(sla[buf][tt][i]);
+                pqk = fmaf(qi, ki, pqk);
 #pragma unroll
-        for (int m = 0; m < RPW; ++m) {
-            pqk = fmaf(qi[m], ki[m], pqk);
+                for (int c = 0; c < VEC; ++c) {
+                    s[m][c] *= ai;
+                    pa[c] = fmaf(s[m][c], ki, pa[c]);
+                    pb[c] = fmaf(s[m][c], qi, pb[c]);
+                }
+            }
 #pragma unroll
             for (int c = 0; c < VEC; ++c) {
-                s[m][c] *= ai[m];
-                pa[c] = fmaf(s[m][c], ki[m], pa[c]);
-                pb[c] = fmaf(s[m][c], qi[m], pb[c]);
+                red_a[warp][lane * VEC + c] = pa[c];
+                red_b[warp][lane * VEC + c] = pb[c];
+            }
+            if (lane == 0) s_qk[warp] = pqk;
+            __syncthreads();
+            if (threadIdx.x < D) {
+                const int j = threadIdx.x;
+                float a = 0.f, b = 0.f, qk = 0.f;
+#pragma unroll
+                for (int w = 0; w < kMultiWarps; ++w) {
+                    a += red_a[w][j];
+                    b += red_b[w][j];
+                    qk += s_qk[w];
+                }
+                const float uj = sb[buf][tt] * (to_f(sv[buf][tt][j]) - a);
+                s_u[j] = uj;
+                Elem<T>::store(o + tok_of(t0 + tt) * D + j, fmaf(qk, uj, b));
+            }
+            __syncthreads();
+            float uu[VEC];
+#pragma unroll
+            for (int c = 0; c < VEC; ++c) uu[c] = s_u[lane * VEC + c];
+#pragma unroll
+            for (int m = 0; m < RPW; ++m) {
+                const float ki = to_f(sk[buf][tt][warp + kMultiWarps * m]);
+#pragma unroll
+                for (int c = 0; c < VEC; ++c) s[m][c] = fmaf(ki, uu[c], s[m][c]);
             }
         }
-#pragma unroll
-        for (int c = 0; c < VEC; ++c) {
-            red_a[warp][lane * VEC + c] = pa[c];
-            red_b[warp][lane * VEC + c] = pb[c];
-        }
-        if (lane == 0) s_qk[warp] = pqk;
-        __syncthreads();
-        if (threadIdx.x < D) {
-            const int j = threadIdx.x;
-            const size_t tk = tok_of(t);
-            float a = 0.f, b = 0.f, qk = 0.f;
-#pragma unroll
-            for (int w = 0; w < kMultiWarps; ++w) {
-                a += red_a[w][j];
-                b += red_b[w][j];
-                qk += s_qk[w];
-            }
-            const float uj = __ldg(beta + tk) * (Elem<T>::load(v + tk * D + j) - a);
-            s_u[j] = uj;
-            Elem<T>::store(o + tk * D + j, fmaf(qk, uj, b));
-        }
-        __syncthreads();
-        float uu[VEC];
-#pragma unroll
-        for (int c = 0; c < VEC; ++c) uu[c] = s_u[lane * VEC + c];
-#pragma unroll
-        for (int m = 0; m < RPW; ++m)
-#pragma unroll
-            for (int c = 0; c < VEC; ++c) s[m][c] = fmaf(ki[m], uu[c], s[m][c]);
+        __syncthreads();  // batch bi's buffer is free before it is staged again
     }
 #pragma unroll
     for (int m = 0; m < RPW; ++m) VecIO<VEC>::store(Sout + (size_t)(warp + kMultiWarps * m) * D + lane * VEC, s[m]);
