@@ -83,6 +83,9 @@ KDA_API size_t kda_chunk_fwd_workspace_size(int B, int T, int H, int dk, int dv,
  *   workspace : device buffer of at least kda_chunk_fwd_workspace_size(...) bytes, 256-byte
  *               aligned; contents on entry are ignored.  Must not be shared by calls that
  *               can run concurrently.
+ * T = 0 (or, with cu_seqlens, sequences of length 0) is allowed: such sequences have no output
+ * rows and their h_T is h0 (zeros without h0).  When B * T = 0 the token tensors (q, k, v,
+ * log_alpha, beta, o) are empty and may be NULL.
  * Supported: dk = dv = 128 with dtype BF16 (tensor-core path) or F32; dk = dv = 64 with F32 or
  * BF16 (CUDA-core path).  Returns KDA_OK once the work is enqueued. */
 KDA_API int kda_chunk_fwd(const void *q, const void *k, const void *v, const float *log_alpha,

@@ -141,10 +141,12 @@ int kda_chunk_fwd(const void *q, const void *k, const void *v, const float *log_
                   int dv, int chunk_size, kda_dtype dtype, void *o, float *h_T, void *workspace,
                   size_t workspace_bytes, void *stream_) {
     if (dtype != KDA_F32 && dtype != KDA_BF16) return KDA_ERR_BAD_DTYPE;
-    if (!q || !k || !v || !log_alpha || !beta || !o || !workspace) return KDA_ERR_NULL_ARG;
+    if (!workspace) return KDA_ERR_NULL_ARG;
     const bool varlen = cu_seqlens != nullptr;
     int rc = check_prefill_shape(B, T, H, dk, dv, num_seqs, varlen, chunk_size);
     if (rc != KDA_OK) return rc;
+    // with no tokens the token tensors are empty (never read) and may be NULL
+    if ((int64_t)B * T > 0 && (!q || !k || !v || !log_alpha || !beta || !o)) return KDA_ERR_NULL_ARG;
     const void *ptrs[] = {q, k, v, log_alpha, beta, h0, cu_seqlens, o, h_T};
     for (const void *p : ptrs)
         if (p && !aligned16(p)) return KDA_ERR_MISALIGNED;

@@ -932,7 +932,7 @@ cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const
     if (e != cudaSuccess) return e;
     // TMA maps of the intra-chunk kernel's input tiles (q, k, V: bf16; log_alpha: fp32)
     const uint64_t tokens = (uint64_t)B * T;
-    CUtensorMap tm_q, tm_k, tm_v, tm_g;
+    CUtensorMap tm_q{}, tm_k{}, tm_v{}, tm_g{};  // left zero (and unused) when there are no tokens
     if (tokens > 0 &&
         ((e = encode_token_map(&tm_q, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, tokens, H, D, CU_TENSOR_MAP_SWIZZLE_NONE)) != cudaSuccess ||
         (e = encode_token_map(&tm_k, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, tokens, H, D, CU_TENSOR_MAP_SWIZZLE_NONE)) != cudaSuccess ||

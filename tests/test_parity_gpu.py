@@ -157,6 +157,20 @@ def test_varlen_small(cuda_device, dtype, d):
 
 
 @pytest.mark.parametrize("dtype,d", [(torch.bfloat16, 128), (torch.float32, 64)])
+def test_empty_inputs_keep_the_state(cuda_device, dtype, d):
+    """No tokens (T = 0; or varlen with every sequence empty): h_T = h0 exactly (zeros without h0)."""
+    x = to_dev(gen.make_prefill(2, 0, 3, d, d, dtype, h0_std=0.3, seed=5), cuda_device)
+    o, hT = run_fwd(x)
+    assert o.numel() == 0 and torch.equal(hT, x["h0"])
+    _, hz = kda.kda_chunk_fwd(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], None, None)
+    assert torch.count_nonzero(hz) == 0
+    cu = torch.zeros(4, dtype=torch.int32)
+    y = to_dev(gen.make_prefill(1, 0, 3, d, d, dtype, h0_std=0.3, seed=6, cu_seqlens=cu), cuda_device)
+    o, hT = run_fwd(y)
+    assert o.numel() == 0 and torch.equal(hT, y["h0"])
+
+
+@pytest.mark.parametrize("dtype,d", [(torch.bfloat16, 128), (torch.float32, 64)])
 def test_zero_values_give_exact_zero(cuda_device, dtype, d):
     x = to_dev(gen.make_prefill(2, 200, 2, d, d, dtype, gate_shift=4.0, seed=1), cuda_device)
     x["v"] = torch.zeros_like(x["v"])
