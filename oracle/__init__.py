@@ -35,6 +35,8 @@ def _bind(path: str):
     lib.kda_oracle_chunkwise.restype = i
     lib.kda_oracle_decode_step.argtypes = [dp, dp, dp, dp, dp, dp, i, i, i, i, dp]
     lib.kda_oracle_decode_step.restype = i
+    lib.kda_oracle_prologue.argtypes = [dp, dp, dp, ctypes.c_int64, i, i, ctypes.c_uint, ctypes.c_double, dp, dp]
+    lib.kda_oracle_prologue.restype = i
     lib.kda_oracle_num_threads.restype = i
     lib.kda_oracle_set_num_threads.argtypes = [i]
     return lib
@@ -113,6 +115,21 @@ class Oracle:
             raise ValueError(f"kda_oracle_decode_step rejected its arguments (rc={rc})")
         return o, S
 
+    def prologue(self, q, k, log_alpha, flags, A_log=None, dt_bias=None, eps=1e-6):
+        """The layer's prologue on token-major q, k, log_alpha [..., H, dk] (float64 copies are
+        returned): flags & 1 L2-normalises q and k rows; flags & 2 turns the gate pre-activation in
+        log_alpha into -exp(A_log[h]) * softplus(g + dt_bias[h, c])."""
+        q, k, la = (np.array(x, dtype=np.float64, copy=True, order="C") for x in (q, k, log_alpha))
+        H, dk = q.shape[-2], q.shape[-1]
+        n_tok = q.size // (H * dk)
+        al = None if A_log is None else _f64(A_log)
+        db = None if dt_bias is None else _f64(dt_bias)
+        rc = self.lib.kda_oracle_prologue(_ptr(q), _ptr(k), _ptr(la), n_tok, H, dk, int(flags), float(eps),
+                                          _ptr(al), _ptr(db))
+        if rc != 0:
+            raise ValueError(f"kda_oracle_prologue rejected its arguments (rc={rc})")
+        return q, k, la
+
     def num_threads(self) -> int:
         return int(self.lib.kda_oracle_num_threads())
 
@@ -136,6 +153,10 @@ def recurrent(*args, **kw):
 
 def chunkwise(*args, **kw):
     return default().chunkwise(*args, **kw)
+
+
+def prologue(*args, **kw):
+    return default().prologue(*args, **kw)
 
 
 def decode_step(*args, **kw):

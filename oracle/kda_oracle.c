@@ -337,6 +337,42 @@ int kda_oracle_chunkwise(const double *q, const double *k, const double *v,
     return KDA_ORACLE_OK;
 }
 
+/* The layer's prologue (page, section "Kimi Linear model composition"): the query and key of every
+ * head are L2-normalised for eigenvalue stability, and the channel-wise decay comes from a low-rank
+ * gate projection through a decay function of the Gated DeltaNet / Mamba kind.  The page names the
+ * kind but not the formula; the form taken here is the one those models use,
+ * log alpha = -exp(A_log) * softplus(g + dt_bias), with A_log per head and dt_bias per channel. */
+static double softplus(double x) { return (x > 0.0 ? x : 0.0) + log1p(exp(-fabs(x))); }
+
+int kda_oracle_prologue(double *q, double *k, double *la, int64_t n_tok, int H, int dk, unsigned flags,
+                        double eps, const double *A_log, const double *dt_bias) {
+    if (n_tok < 0 || H <= 0 || dk <= 0) return KDA_ORACLE_BAD_ARG;
+    if ((flags & 1u) && (!q || !k || !(eps >= 0.0))) return KDA_ORACLE_BAD_ARG;
+    if ((flags & 2u) && (!la || !A_log)) return KDA_ORACLE_BAD_ARG;
+    for (int64_t t = 0; t < n_tok; ++t) {
+        for (int h = 0; h < H; ++h) {
+            const int64_t base = (t * H + h) * (int64_t)dk;
+            if (flags & 1u) {
+                double *rows[2] = {q + base, k + base};
+                for (int r = 0; r < 2; ++r) {
+                    double ss = 0.0;
+                    for (int c = 0; c < dk; ++c) ss += rows[r][c] * rows[r][c];
+                    const double inv = 1.0 / sqrt(ss + eps);
+                    for (int c = 0; c < dk; ++c) rows[r][c] *= inv;
+                }
+            }
+            if (flags & 2u) {
+                const double a = exp(A_log[h]);
+                for (int c = 0; c < dk; ++c) {
+                    const double b = dt_bias ? dt_bias[h * dk + c] : 0.0;
+                    la[base + c] = -a * softplus(la[base + c] + b);
+                }
+            }
+        }
+    }
+    return KDA_ORACLE_OK;
+}
+
 int kda_oracle_num_threads(void) {
 #ifdef _OPENMP
     return omp_get_max_threads();

@@ -33,6 +33,15 @@ int kda_oracle_decode_step(const double *q, const double *k, const double *v,
                            const double *log_alpha, const double *beta, double *S,
                            int N, int H, int dk, int dv, double *o);
 
+/* The KDA layer's prologue, applied in place to n_tok token rows of H heads before the recurrence
+ * (Kimi Linear page, section "Kimi Linear model composition").
+ *   flags & 1: q and k rows are L2-normalised over dk: x / sqrt(sum x^2 + eps).
+ *   flags & 2: la holds the gate pre-activation g and becomes the log decay
+ *              -exp(A_log[h]) * softplus(g + dt_bias[h * dk + c]); dt_bias may be NULL (zero).
+ * q, k, la: [n_tok, H, dk].  A_log: [H] (needed with flags & 2). */
+int kda_oracle_prologue(double *q, double *k, double *la, int64_t n_tok, int H, int dk, unsigned flags,
+                        double eps, const double *A_log, const double *dt_bias);
+
 int kda_oracle_num_threads(void);
 void kda_oracle_set_num_threads(int n);
 

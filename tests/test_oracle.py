@@ -363,3 +363,52 @@ def test_oracle_rejects_bad_seqlens():
         oracle.recurrent(q, k, v, la, beta, None, cu_seqlens=np.array([0, 6, 5, 10]))
     with pytest.raises(ValueError):
         oracle.recurrent(q, k, v, la, beta, None, cu_seqlens=np.array([0, 6, 9]))
+
+
+# ------------------------------------------------------------------------------------- layer prologue
+# Page, section "Kimi Linear model composition": q and k are L2-normalised per head; the channel-wise
+# decay comes from a gate projection through a GDN / Mamba-style decay function, read here as
+# log alpha = -exp(A_log[h]) * softplus(g + dt_bias[h, c]).  These pins fix each part by a property
+# or a closed-form limit, not by re-evaluating the formula.
+def test_prologue_l2_normalisation_pins():
+    rng = np.random.default_rng(31)
+    q, k = rng.normal(size=(5, 3, 8)), rng.normal(size=(5, 3, 8)) * 7.0
+    g = rng.normal(size=(5, 3, 8))
+    qn, kn, la = oracle.prologue(q, k, g, 1, eps=0.0)
+    assert np.allclose(np.linalg.norm(qn, axis=-1), 1.0, atol=1e-14)            # unit rows
+    assert np.allclose(np.linalg.norm(kn, axis=-1), 1.0, atol=1e-14)
+    assert np.allclose(np.sum(qn * q, -1), np.linalg.norm(q, axis=-1), rtol=1e-14)  # same direction
+    q3, k3, _ = oracle.prologue(3.5 * q, 0.25 * k, g, 1, eps=0.0)                 # scale invariance
+    assert np.allclose(q3, qn, rtol=1e-14, atol=0) and np.allclose(k3, kn, rtol=1e-14, atol=0)
+    assert np.array_equal(la, g)                                                  # gate untouched
+    qe, _, _ = oracle.prologue(q, k, g, 1, eps=1e-6)                              # eps inside the root
+    ss = np.sum(q * q, -1, keepdims=True)
+    assert np.allclose(qe * np.sqrt(ss + 1e-6), q, rtol=1e-14)
+
+
+def test_prologue_gate_pins():
+    H, dk = 2, 6
+    A_log = np.array([0.7, -1.3])
+    dt_bias = np.linspace(-0.5, 0.5, H * dk).reshape(H, dk)
+    a = np.exp(A_log)[:, None]
+    z = np.zeros((1, H, dk))
+    # softplus(0) = log 2: g = -dt_bias gives log alpha = -exp(A_log) log 2 on every channel
+    _, _, la0 = oracle.prologue(z, z, -dt_bias[None], 2, A_log=A_log, dt_bias=dt_bias)
+    assert np.allclose(la0[0], -a * np.log(2.0), rtol=1e-15)
+    # large argument: softplus(x) = x + log(1 + e^-x) -> x (linear regime), per head and per channel
+    g = 60.0 + np.arange(H * dk, dtype=np.float64).reshape(1, H, dk)
+    _, _, la1 = oracle.prologue(z, z, g, 2, A_log=A_log, dt_bias=dt_bias)
+    assert np.allclose(la1[0], -a * (g[0] + dt_bias), rtol=1e-15)
+    # very negative argument: softplus(x) -> e^x
+    gn = -40.0 - np.arange(H * dk, dtype=np.float64).reshape(1, H, dk)
+    _, _, la2 = oracle.prologue(z, z, gn, 2, A_log=A_log, dt_bias=dt_bias)
+    assert np.allclose(la2[0], -a * np.exp(gn[0] + dt_bias), rtol=1e-12)
+    # A_log -> -inf: no decay at all (alpha = 1); without dt_bias the bias is zero
+    _, _, la3 = oracle.prologue(z, z, np.ones((1, H, dk)), 2, A_log=np.full(H, -800.0))
+    assert np.all(la3 == 0.0)
+    _, _, la4 = oracle.prologue(z, z, -np.zeros((1, H, dk)), 2, A_log=A_log)
+    assert np.allclose(la4[0], -a * np.log(2.0) * np.ones((H, dk)), rtol=1e-15)
+    # every decay is <= 0 (alpha in (0, 1])
+    _, _, la5 = oracle.prologue(z, z, np.random.default_rng(3).normal(size=(1, H, dk)) * 10, 2, A_log=A_log,
+                                dt_bias=dt_bias)
+    assert np.all(la5 <= 0.0)
