@@ -155,6 +155,34 @@ KDA_API int kda_decode_multi(const void *q, const void *k, const void *v, const 
                              const int32_t *slot_out, int N, int Tq, int H, int dk, int dv, kda_dtype dtype,
                              void *o, int *status, void *stream);
 
+/* The KDA layer's prologue, fused into the kernels (flags of the _ex entry points).  Kimi Linear
+ * summary page (th.news.hada.io topic 31936), section "Kimi Linear model composition": each head's
+ * query and key are L2-normalised for eigenvalue stability, and the channel-wise decay comes from a
+ * low-rank gate projection through a decay function of the Gated DeltaNet / Mamba kind.  The page
+ * does not write the function out; the form used is the one those models use.
+ *   KDA_PROLOGUE_L2NORM_QK : q and k rows become x / sqrt(sum_c x_c^2 + 1e-6) (fp32 arithmetic,
+ *                            per token and head, over dk) before anything else uses them.
+ *   KDA_PROLOGUE_GATE      : log_alpha carries the gate projection output g (any real values); the
+ *                            log decay used is -exp(A_log[h]) * softplus(g + dt_bias[h * dk + c]).
+ *                            A_log: fp32 [H] (required); dt_bias: fp32 [H, dk] or NULL (zero). */
+enum { KDA_PROLOGUE_L2NORM_QK = 1, KDA_PROLOGUE_GATE = 2 };
+
+/* kda_chunk_fwd with the prologue above; flags = 0 is exactly kda_chunk_fwd.  Unknown flag bits
+ * return KDA_ERR_UNSUPPORTED; KDA_PROLOGUE_GATE without A_log returns KDA_ERR_NULL_ARG; A_log and
+ * dt_bias are inputs (16-byte aligned, must not overlap an output). */
+KDA_API int kda_chunk_fwd_ex(const void *q, const void *k, const void *v, const float *log_alpha,
+                             const float *beta, const float *h0, const int32_t *cu_seqlens, int num_seqs,
+                             int B, int T, int H, int dk, int dv, int chunk_size, kda_dtype dtype, void *o,
+                             float *h_T, void *workspace, size_t workspace_bytes, unsigned flags,
+                             const float *A_log, const float *dt_bias, void *stream);
+
+/* kda_decode_multi with the prologue above (a one-token decode with the prologue is Tq = 1). */
+KDA_API int kda_decode_multi_ex(const void *q, const void *k, const void *v, const float *log_alpha,
+                                const float *beta, float *S_pool, int num_slots, const int32_t *slot_in,
+                                const int32_t *slot_out, int N, int Tq, int H, int dk, int dv, kda_dtype dtype,
+                                void *o, int *status, unsigned flags, const float *A_log, const float *dt_bias,
+                                void *stream);
+
 /* Synchronizes `stream`, reads the device status word kept in `workspace` by the last
  * kda_chunk_fwd that used it, clears it, and returns it (KDA_OK, KDA_ERR_BAD_SEQLENS or
  * KDA_ERR_TIMEOUT), or KDA_ERR_CUDA if the synchronization itself failed. */

@@ -98,6 +98,54 @@ def kda_chunk_fwd(q, k, v, log_alpha, beta, h0=None, cu_seqlens=None, chunk_size
     return o, h_T
 
 
+def kda_chunk_fwd_ex(q, k, v, log_alpha, beta, h0=None, cu_seqlens=None, flags: int = 0, A_log=None,
+                     dt_bias=None, chunk_size: int = 64, o=None, h_T=None, output_final_state: bool = True,
+                     workspace=None, stream=None):
+    """kda_chunk_fwd with the layer prologue fused in: flags KDA_PROLOGUE_L2NORM_QK (L2-normalise q and
+    k rows) and / or KDA_PROLOGUE_GATE (log_alpha holds the gate projection g; the decay used is
+    -exp(A_log[h]) * softplus(g + dt_bias[h, c])).  A_log [H] fp32, dt_bias [H, dk] fp32 or None."""
+    torch = _torch()
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    N = B if cu_seqlens is None else cu_seqlens.numel() - 1
+    if o is None:
+        o = torch.empty((B, T, H, dv), dtype=q.dtype, device=q.device)
+    if h_T is None and output_final_state:
+        h_T = torch.empty((N, H, dk, dv), dtype=torch.float32, device=q.device)
+    code = _dtype_code(q.dtype)
+    need = int(_lib.load().kda_chunk_fwd_workspace_size(B, T, H, dk, dv, N, chunk_size, code))
+    if isinstance(workspace, Workspace):
+        ws = workspace.get(need)
+    elif workspace is None:
+        ws = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
+    else:
+        ws = workspace
+    rc = _lib.load().kda_chunk_fwd_ex(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(h0), _ptr(cu_seqlens), N, B, T, H,
+        dk, dv, chunk_size, code, _ptr(o), _ptr(h_T), _ptr(ws), ws.numel() * ws.element_size(), int(flags),
+        _ptr(A_log), _ptr(dt_bias), _stream(stream, q.device))
+    if rc != _lib.KDA_OK:
+        raise KdaError(rc, "kda_chunk_fwd_ex")
+    return o, h_T
+
+
+def kda_decode_multi_ex(q, k, v, log_alpha, beta, S_pool, slot_in=None, slot_out=None, flags: int = 0, A_log=None,
+                        dt_bias=None, o=None, status=None, stream=None):
+    """kda_decode_multi with the layer prologue fused in (see kda_chunk_fwd_ex)."""
+    torch = _torch()
+    N, Tq, H, dk = q.shape
+    dv = v.shape[-1]
+    if o is None:
+        o = torch.empty((N, Tq, H, dv), dtype=q.dtype, device=q.device)
+    rc = _lib.load().kda_decode_multi_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(S_pool),
+                                         S_pool.shape[0], _ptr(slot_in), _ptr(slot_out), N, Tq, H, dk, dv,
+                                         _dtype_code(q.dtype), _ptr(o), _ptr(status), int(flags), _ptr(A_log),
+                                         _ptr(dt_bias), _stream(stream, q.device))
+    if rc != _lib.KDA_OK:
+        raise KdaError(rc, "kda_decode_multi_ex")
+    return o
+
+
 def kda_decode_multi(q, k, v, log_alpha, beta, S_pool, slot_in=None, slot_out=None, o=None, status=None,
                      stream=None):
     """Tq recurrent steps per sequence on a slot-indexed state pool.  q, k [N,Tq,H,dk], v [N,Tq,H,dv]

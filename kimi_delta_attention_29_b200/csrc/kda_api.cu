@@ -136,10 +136,30 @@ size_t kda_chunk_fwd_workspace_size(int B, int T, int H, int dk, int dv, int num
     return kStatusBytes;
 }
 
+// Checks the prologue arguments shared by the _ex entry points (A_log [H], dt_bias [H, dk]).
+static int check_prologue(unsigned flags, const float *A_log, const float *dt_bias, int H, int dk, Range *ra, Range *rb) {
+    if (flags & ~(unsigned)(KDA_PROLOGUE_L2NORM_QK | KDA_PROLOGUE_GATE)) return KDA_ERR_UNSUPPORTED;
+    const bool gate = flags & KDA_PROLOGUE_GATE;
+    if (gate && !A_log) return KDA_ERR_NULL_ARG;
+    if (gate && (!aligned16(A_log) || (dt_bias && !aligned16(dt_bias)))) return KDA_ERR_MISALIGNED;
+    *ra = range_of(A_log, gate ? (size_t)H * 4 : 0);
+    *rb = range_of(dt_bias, gate && dt_bias ? (size_t)H * dk * 4 : 0);
+    return KDA_OK;
+}
+
 int kda_chunk_fwd(const void *q, const void *k, const void *v, const float *log_alpha, const float *beta,
                   const float *h0, const int32_t *cu_seqlens, int num_seqs, int B, int T, int H, int dk,
                   int dv, int chunk_size, kda_dtype dtype, void *o, float *h_T, void *workspace,
-                  size_t workspace_bytes, void *stream_) {
+                  size_t workspace_bytes, void *stream) {
+    return kda_chunk_fwd_ex(q, k, v, log_alpha, beta, h0, cu_seqlens, num_seqs, B, T, H, dk, dv, chunk_size, dtype,
+                            o, h_T, workspace, workspace_bytes, 0u, nullptr, nullptr, stream);
+}
+
+int kda_chunk_fwd_ex(const void *q, const void *k, const void *v, const float *log_alpha, const float *beta,
+                     const float *h0, const int32_t *cu_seqlens, int num_seqs, int B, int T, int H, int dk,
+                     int dv, int chunk_size, kda_dtype dtype, void *o, float *h_T, void *workspace,
+                     size_t workspace_bytes, unsigned flags, const float *A_log, const float *dt_bias,
+                     void *stream_) {
     if (dtype != KDA_F32 && dtype != KDA_BF16) return KDA_ERR_BAD_DTYPE;
     if (!workspace) return KDA_ERR_NULL_ARG;
     const bool varlen = cu_seqlens != nullptr;
@@ -170,6 +190,11 @@ int kda_chunk_fwd(const void *q, const void *k, const void *v, const float *log_
         if (overlaps(rh, inputs[6])) return KDA_ERR_ALIASING;
         if (h0 && h_T != h0 && overlaps(rh, inputs[5])) return KDA_ERR_ALIASING;
     }
+    Range ra, rb;
+    if ((rc = check_prologue(flags, A_log, dt_bias, H, dk, &ra, &rb)) != KDA_OK) return rc;
+    if (overlaps(ro, ra) || overlaps(ro, rb)) return KDA_ERR_ALIASING;
+    if (h_T && (overlaps(range_of(h_T, sbytes), ra) || overlaps(range_of(h_T, sbytes), rb))) return KDA_ERR_ALIASING;
+    const kda::Prologue pro{flags, A_log, dt_bias};
     const size_t need = kda_chunk_fwd_workspace_size(B, T, H, dk, dv, num_seqs, chunk_size, dtype);
     if (need == 0) return KDA_ERR_BAD_SHAPE;
     if (workspace_bytes < need) return KDA_ERR_WORKSPACE_TOO_SMALL;
@@ -179,12 +204,12 @@ int kda_chunk_fwd(const void *q, const void *k, const void *v, const float *log_
     cudaError_t e;
     if (uses_tensor_cores(dk, dv, dtype)) {
         e = kda::launch_prefill_tc(q, k, v, log_alpha, beta, h0, cu_seqlens, num_seqs, B, T, H, o, h_T,
-                                   workspace, workspace_bytes, stream);
+                                   workspace, workspace_bytes, pro, stream);
     } else {
         e = cudaMemsetAsync(workspace, 0, kStatusBytes, stream);
         if (e == cudaSuccess)
             e = kda::launch_prefill_simt(q, k, v, log_alpha, beta, h0, cu_seqlens, num_seqs, B, T, H, dk, dv,
-                                     dtype, o, h_T, status, stream);
+                                     dtype, o, h_T, status, pro, stream);
     }
     return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
@@ -214,7 +239,15 @@ int kda_decode_step(const void *q, const void *k, const void *v, const float *lo
 
 int kda_decode_multi(const void *q, const void *k, const void *v, const float *log_alpha, const float *beta,
                      float *S_pool, int num_slots, const int32_t *slot_in, const int32_t *slot_out, int N, int Tq,
-                     int H, int dk, int dv, kda_dtype dtype, void *o, int *status, void *stream_) {
+                     int H, int dk, int dv, kda_dtype dtype, void *o, int *status, void *stream) {
+    return kda_decode_multi_ex(q, k, v, log_alpha, beta, S_pool, num_slots, slot_in, slot_out, N, Tq, H, dk, dv,
+                               dtype, o, status, 0u, nullptr, nullptr, stream);
+}
+
+int kda_decode_multi_ex(const void *q, const void *k, const void *v, const float *log_alpha, const float *beta,
+                        float *S_pool, int num_slots, const int32_t *slot_in, const int32_t *slot_out, int N,
+                        int Tq, int H, int dk, int dv, kda_dtype dtype, void *o, int *status, unsigned flags,
+                        const float *A_log, const float *dt_bias, void *stream_) {
     if (dtype != KDA_F32 && dtype != KDA_BF16) return KDA_ERR_BAD_DTYPE;
     if (!q || !k || !v || !log_alpha || !beta || !S_pool || !o) return KDA_ERR_NULL_ARG;
     if (N <= 0 || Tq <= 0 || H <= 0 || dk <= 0 || dv <= 0 || num_slots <= 0) return KDA_ERR_BAD_SHAPE;
@@ -240,8 +273,15 @@ int kda_decode_multi(const void *q, const void *k, const void *v, const float *l
     if (overlaps(ro, rs) || overlaps(ro, rst) || overlaps(rs, rst)) return KDA_ERR_ALIASING;
     for (const Range &r : inputs)
         if (overlaps(ro, r) || overlaps(rs, r) || overlaps(rst, r)) return KDA_ERR_ALIASING;
+    Range ra, rb;
+    const int prc = check_prologue(flags, A_log, dt_bias, H, dk, &ra, &rb);
+    if (prc != KDA_OK) return prc;
+    if (overlaps(ro, ra) || overlaps(ro, rb) || overlaps(rs, ra) || overlaps(rs, rb) || overlaps(rst, ra) ||
+        overlaps(rst, rb))
+        return KDA_ERR_ALIASING;
+    const kda::Prologue pro{flags, A_log, dt_bias};
     cudaError_t e = kda::launch_decode_multi(q, k, v, log_alpha, beta, S_pool, num_slots, slot_in, slot_out, N, Tq,
-                                             H, dk, dtype, o, status, static_cast<cudaStream_t>(stream_));
+                                             H, dk, dtype, o, status, pro, static_cast<cudaStream_t>(stream_));
     return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 

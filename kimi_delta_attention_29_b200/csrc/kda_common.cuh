@@ -25,6 +25,20 @@ __device__ __forceinline__ void set_status(int *status, int code) {
     if (status) atomicCAS(status, 0, code);
 }
 
+// The layer's fused prologue (flags of kda_chunk_fwd_ex / kda_decode_multi_ex): q and k rows
+// L2-normalised over the head dim, and the gate pre-activation g turned into the log decay
+// -exp(A_log[h]) * softplus(g + dt_bias[h * dk + c]).
+struct Prologue {
+    unsigned flags;
+    const float *A_log;    // [H]
+    const float *dt_bias;  // [H, dk] or nullptr
+};
+constexpr float kNormEps = 1e-6f;  // inside the square root of the L2 normalisation
+__device__ __forceinline__ float gate_log_decay(float g, float a, float b) {
+    const float x = g + b;
+    return -a * (fmaxf(x, 0.f) + log1pf(expf(-fabsf(x))));  // -a * softplus(x), overflow-free
+}
+
 // Chunk length shared by every kernel.
 constexpr int kChunk = 64;
 
@@ -46,18 +60,18 @@ cudaError_t launch_decode(const void *q, const void *k, const void *v, const flo
 cudaError_t launch_decode_multi(const void *q, const void *k, const void *v, const float *log_alpha,
                                 const float *beta, float *S_pool, int num_slots, const int32_t *slot_in,
                                 const int32_t *slot_out, int N, int Tq, int H, int dk, kda_dtype dtype, void *o,
-                                int *status, cudaStream_t stream);
+                                int *status, const Prologue &pro, cudaStream_t stream);
 
 // CUDA-core chunkwise forward (any supported dtype, dk = dv in {64, 128}).
 cudaError_t launch_prefill_simt(const void *q, const void *k, const void *v, const float *log_alpha,
                                 const float *beta, const float *h0, const int32_t *cu_seqlens,
                                 int num_seqs, int B, int T, int H, int dk, int dv, kda_dtype dtype,
-                                void *o, float *h_T, int *status, cudaStream_t stream);
+                                void *o, float *h_T, int *status, const Prologue &pro, cudaStream_t stream);
 
 // Tensor-core (tcgen05) chunkwise forward: bf16, dk = dv = 128.
 size_t prefill_tc_workspace_bytes(int B, int T, int H, int num_seqs, bool varlen);
 cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const float *log_alpha,
                               const float *beta, const float *h0, const int32_t *cu_seqlens,
                               int num_seqs, int B, int T, int H, void *o, float *h_T, void *workspace,
-                              size_t workspace_bytes, cudaStream_t stream);
+                              size_t workspace_bytes, const Prologue &pro, cudaStream_t stream);
 }  // namespace kda

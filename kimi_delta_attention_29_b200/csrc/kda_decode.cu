@@ -123,6 +123,9 @@ constexpr int kMultiWarps = 8;
 constexpr int kTokBatch = 8;
 __device__ __forceinline__ float to_f(float x) { return x; }
 __device__ __forceinline__ float to_f(__nv_bfloat16 x) { return __bfloat162float(x); }
+template <typename T> __device__ __forceinline__ T from_f(float x);
+template <> __device__ __forceinline__ float from_f<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float x) { return __float2bfloat16_rn(x); }
 __device__ __forceinline__ void cp_async16(void *dst, const void *src) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
                  "l"(src)
@@ -143,7 +146,7 @@ kda_decode_multi_kernel(const T *__restrict__ q, const T *__restrict__ k, const 
                         const float *__restrict__ log_alpha, const float *__restrict__ beta,
                         float *__restrict__ S_pool, int num_slots, const int32_t *__restrict__ slot_in,
                         const int32_t *__restrict__ slot_out, int Tq, int H, T *__restrict__ o,
-                        int *__restrict__ status) {
+                        int *__restrict__ status, const Prologue pro) {
     constexpr int RPW = D / kMultiWarps;  // rows per warp
     constexpr int VEC = D / 32;           // columns per lane
     constexpr int TB = sizeof(T) == 4 ? kTokBatch / 2 : kTokBatch;  // fp32 tokens: half the batch (static shared memory)
@@ -207,6 +210,33 @@ kda_decode_multi_kernel(const T *__restrict__ q, const T *__restrict__ k, const 
             cp_async_wait<0>();
         }
         __syncthreads();  // ... and every other thread's
+        if (pro.flags) {  // the layer prologue on the staged tokens, in shared memory
+            if (pro.flags & KDA_PROLOGUE_L2NORM_QK) {
+                for (int rr = warp; rr < 2 * nt; rr += kMultiWarps) {  // one warp per q or k row
+                    T *row = (rr & 1) ? sk[buf][rr >> 1] : sq[buf][rr >> 1];
+                    float x[VEC], ss = 0.f;
+#pragma unroll
+                    for (int c = 0; c < VEC; ++c) {
+                        x[c] = to_f(row[lane * VEC + c]);
+                        ss = fmaf(x[c], x[c], ss);
+                    }
+#pragma unroll
+                    for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+                    const float inv = rsqrtf(ss + kNormEps);
+#pragma unroll
+                    for (int c = 0; c < VEC; ++c) row[lane * VEC + c] = from_f<T>(x[c] * inv);
+                }
+            }
+            if (pro.flags & KDA_PROLOGUE_GATE) {
+                const float ga = expf(__ldg(pro.A_log + h));
+                for (int e = threadIdx.x; e < nt * D; e += kMultiWarps * 32) {
+                    const int tt = e / D, c = e % D;
+                    const float b = pro.dt_bias ? __ldg(pro.dt_bias + (size_t)h * D + c) : 0.f;
+                    sla[buf][tt][c] = gate_log_decay(sla[buf][tt][c], ga, b);
+                }
+            }
+            __syncthreads();
+        }
         for (int tt = 0; tt < nt; ++tt) {
             float pa[VEC], pb[VEC];
 #pragma unroll
@@ -266,12 +296,12 @@ kda_decode_multi_kernel(const T *__restrict__ q, const T *__restrict__ k, const 
 template <int D, typename T>
 cudaError_t launch_decode_multi_t(const void *q, const void *k, const void *v, const float *la, const float *beta,
                                   float *S_pool, int num_slots, const int32_t *slot_in, const int32_t *slot_out,
-                                  int N, int Tq, int H, void *o, int *status, cudaStream_t stream) {
+                                  int N, int Tq, int H, void *o, int *status, const Prologue &pro, cudaStream_t stream) {
     const unsigned units = (unsigned)N * (unsigned)H;
     trace_before(kKernDecodeMulti, stream);
     kda_decode_multi_kernel<D, T><<<units, kMultiWarps * 32, 0, stream>>>(
         static_cast<const T *>(q), static_cast<const T *>(k), static_cast<const T *>(v), la, beta, S_pool,
-        num_slots, slot_in, slot_out, Tq, H, static_cast<T *>(o), status);
+        num_slots, slot_in, slot_out, Tq, H, static_cast<T *>(o), status, pro);
     trace_after(stream);
     return cudaGetLastError();
 }
@@ -305,10 +335,10 @@ cudaError_t launch_decode(const void *q, const void *k, const void *v, const flo
 cudaError_t launch_decode_multi(const void *q, const void *k, const void *v, const float *log_alpha,
                                 const float *beta, float *S_pool, int num_slots, const int32_t *slot_in,
                                 const int32_t *slot_out, int N, int Tq, int H, int dk, kda_dtype dtype, void *o,
-                                int *status, cudaStream_t stream) {
+                                int *status, const Prologue &pro, cudaStream_t stream) {
 #define KDA_MULTI(DIM, TYPE)                                                                                  \
     launch_decode_multi_t<DIM, TYPE>(q, k, v, log_alpha, beta, S_pool, num_slots, slot_in, slot_out, N, Tq, H, o, \
-                                     status, stream)
+                                     status, pro, stream)
     if (dk == 128) return dtype == KDA_BF16 ? KDA_MULTI(128, __nv_bfloat16) : KDA_MULTI(128, float);
     return dtype == KDA_BF16 ? KDA_MULTI(64, __nv_bfloat16) : KDA_MULTI(64, float);
 #undef KDA_MULTI

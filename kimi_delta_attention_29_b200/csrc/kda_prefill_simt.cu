@@ -54,7 +54,7 @@ kda_prefill_simt_kernel(const T *__restrict__ q, const T *__restrict__ k, const 
                         const float *__restrict__ log_alpha, const float *__restrict__ beta,
                         const float *__restrict__ h0, const int32_t *__restrict__ cu_seqlens,
                         int num_seqs, int T_len, int H, T *__restrict__ o, float *__restrict__ h_T,
-                        int *status) {
+                        int *status, const Prologue pro) {
     constexpr int DV = DK;
     using SM = SimtSmem<DK>;
     constexpr int DKP = SM::DKP, CP = SM::CP;
@@ -100,6 +100,8 @@ kda_prefill_simt_kernel(const T *__restrict__ q, const T *__restrict__ k, const 
         len = T_len;
     }
 
+    const bool gate = pro.flags & KDA_PROLOGUE_GATE, l2 = pro.flags & KDA_PROLOGUE_L2NORM_QK;
+    const float ga = gate ? expf(__ldg(pro.A_log + h)) : 0.f;  // prologue gate: exp(A_log[h])
     const size_t state_off = ((size_t)n * H + h) * DK * DV;
     for (int idx = tid; idx < DK * kNV; idx += kThreads) {
         const int c = idx / kNV, j = idx % kNV;
@@ -118,6 +120,7 @@ kda_prefill_simt_kernel(const T *__restrict__ q, const T *__restrict__ k, const 
                 kv = Elem<T>::load(k + off);
                 qv = Elem<T>::load(q + off);
                 lv = __ldg(log_alpha + off);
+                if (gate) lv = gate_log_decay(lv, ga, pro.dt_bias ? __ldg(pro.dt_bias + (size_t)h * DK + c) : 0.f);
             }
             Xo[r * DKP + c] = kv;
             Xq[r * DKP + c] = qv;
@@ -129,6 +132,16 @@ kda_prefill_simt_kernel(const T *__restrict__ q, const T *__restrict__ k, const 
         }
         if (tid < kC) bt[tid] = tid < L ? __ldg(beta + (size_t)(start + c0 + tid) * H + h) : 0.f;
         __syncthreads();
+        if (l2) {  // prologue: q and k rows L2-normalised (padding rows stay zero)
+            if (tid < 2 * kC) {
+                float *row = (tid < kC ? Xq : Xo) + (tid % kC) * DKP;
+                float ss = 0.f;
+                for (int c = 0; c < DK; ++c) ss = fmaf(row[c], row[c], ss);
+                const float inv = rsqrtf(ss + kNormEps);
+                for (int c = 0; c < DK; ++c) row[c] *= inv;
+            }
+            __syncthreads();
+        }
 
         // 2. per-channel cumulative log-gate and the block-referenced decay factors
         for (int c = tid; c < DK; c += kThreads) {
@@ -238,7 +251,7 @@ kda_prefill_simt_kernel(const T *__restrict__ q, const T *__restrict__ k, const 
 template <int DK, typename T>
 cudaError_t launch_t(const void *q, const void *k, const void *v, const float *la, const float *beta,
                      const float *h0, const int32_t *cu, int num_seqs, int T_len, int H, void *o,
-                     float *h_T, int *status, cudaStream_t stream) {
+                     float *h_T, int *status, const Prologue &pro, cudaStream_t stream) {
     auto kern = kda_prefill_simt_kernel<DK, T>;
     const size_t smem = SimtSmem<DK>::bytes;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -247,7 +260,7 @@ cudaError_t launch_t(const void *q, const void *k, const void *v, const float *l
     trace_before(kKernSimt, stream);
     kern<<<grid, kThreads, smem, stream>>>(static_cast<const T *>(q), static_cast<const T *>(k),
                                            static_cast<const T *>(v), la, beta, h0, cu, num_seqs, T_len,
-                                           H, static_cast<T *>(o), h_T, status);
+                                           H, static_cast<T *>(o), h_T, status, pro);
     trace_after(stream);
     return cudaGetLastError();
 }
@@ -257,16 +270,16 @@ cudaError_t launch_t(const void *q, const void *k, const void *v, const float *l
 cudaError_t launch_prefill_simt(const void *q, const void *k, const void *v, const float *log_alpha,
                                 const float *beta, const float *h0, const int32_t *cu_seqlens,
                                 int num_seqs, int B, int T, int H, int dk, int dv, kda_dtype dtype,
-                                void *o, float *h_T, int *status, cudaStream_t stream) {
+                                void *o, float *h_T, int *status, const Prologue &pro, cudaStream_t stream) {
     (void)B;
     (void)dv;
     if (dk == 128)
         return dtype == KDA_BF16
-                   ? launch_t<128, __nv_bfloat16>(q, k, v, log_alpha, beta, h0, cu_seqlens, num_seqs, T, H, o, h_T, status, stream)
-                   : launch_t<128, float>(q, k, v, log_alpha, beta, h0, cu_seqlens, num_seqs, T, H, o, h_T, status, stream);
+                   ? launch_t<128, __nv_bfloat16>(q, k, v, log_alpha, beta, h0, cu_seqlens, num_seqs, T, H, o, h_T, status, pro, stream)
+                   : launch_t<128, float>(q, k, v, log_alpha, beta, h0, cu_seqlens, num_seqs, T, H, o, h_T, status, pro, stream);
     return dtype == KDA_BF16
-               ? launch_t<64, __nv_bfloat16>(q, k, v, log_alpha, beta, h0, cu_seqlens, num_seqs, T, H, o, h_T, status, stream)
-               : launch_t<64, float>(q, k, v, log_alpha, beta, h0, cu_seqlens, num_seqs, T, H, o, h_T, status, stream);
+               ? launch_t<64, __nv_bfloat16>(q, k, v, log_alpha, beta, h0, cu_seqlens, num_seqs, T, H, o, h_T, status, pro, stream)
+               : launch_t<64, float>(q, k, v, log_alpha, beta, h0, cu_seqlens, num_seqs, T, H, o, h_T, status, pro, stream);
 }
 
 }  // namespace kda

@@ -166,7 +166,7 @@ constexpr uint32_t PREP_R = 32768;         // R^(0..3): K-major sw128, 160 rows 
 constexpr uint32_t PREP_KT = 73728;        // K o 2^G: MN-major 64 k-rows x 128
 constexpr uint32_t PREP_V = 90112;         // V: MN-major 64 k-rows x 128
 constexpr uint32_t PREP_SMALL = 106496;
-constexpr uint32_t PREP_SMEM = PREP_SMALL + (64 + 512 + 512 + 128) * 4 + 48 + 1024;
+constexpr uint32_t PREP_SMEM = PREP_SMALL + (64 + 512 + 512 + 128 + 128) * 4 + 48 + 1024;
 constexpr uint32_t kXAtom = 128 * 128;     // X: bytes per 64-channel atom column
 constexpr uint32_t kRRows = 160;
 constexpr uint32_t kRAtom = kRRows * 128;  // R: bytes per 64-channel atom column
@@ -244,7 +244,7 @@ __device__ __forceinline__ void subst_block_row(float *Asm, float *Mscr, int war
 __global__ void __launch_bounds__(kPrepThreads, 2)
 kda_tc_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
-                   const float *__restrict__ beta, int T_len, int H, int nc, const int *__restrict__ n_chunks,
+                   const Prologue pro, const float *__restrict__ beta, int T_len, int H, int nc, const int *__restrict__ n_chunks,
                    const int4 *__restrict__ table, uint8_t *__restrict__ records, int *status) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = align1024(smem_raw);
@@ -256,7 +256,8 @@ kda_tc_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     float *s_E = s_beta + 64;   // [4][128] block references (base 2)
     float *s_tot = s_E + 512;   // [4][128] per-block gate sums (base 2)
     float *s_gl = s_tot + 512;  // [128]    G_63 (base 2)
-    uint64_t *mbar = reinterpret_cast<uint64_t *>(s_gl + 128);  // [0] W/U, [1] Gram (4 issuers), [2] q k g, [3] V
+    float *s_inv = s_gl + 128;  // [128]    prologue: 1 / |q_r| (rows 0..63), 1 / |k_r| (64..127)
+    uint64_t *mbar = reinterpret_cast<uint64_t *>(s_inv + 128);  // [0] W/U, [1] Gram (4 issuers), [2] q k g, [3] V
     uint32_t *s_tmem = reinterpret_cast<uint32_t *>(mbar + 4);
     // input tiles, landed by TMA where the Gram operands are built later
     const uint8_t *Qin = X;            // q: [64 rows][128] bf16
@@ -311,7 +312,38 @@ kda_tc_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     __syncthreads();  // barriers initialised before anyone waits on them
 
     // ---- k, q (bf16 pairs) and log-gates (fp32 pairs) of this thread's 16 rows, from the landed tiles
+    const bool gate = pro.flags & KDA_PROLOGUE_GATE, l2 = pro.flags & KDA_PROLOGUE_L2NORM_QK;
+    float ga = 0.f, gb0 = 0.f, gb1 = 0.f;  // prologue gate: exp(A_log[h]), dt_bias of this thread's channels
+    if (gate) {
+        ga = expf(__ldg(pro.A_log + h));
+        if (pro.dt_bias) {
+            gb0 = __ldg(pro.dt_bias + (size_t)h * D + c0);
+            gb1 = __ldg(pro.dt_bias + (size_t)h * D + c0 + 1);
+        }
+    }
     const bool in_ok = mbar_wait(mbar + 2, 0);
+    if (l2) {  // inverse L2 norms of the 64 q rows and 64 k rows (fp32 sums of the bf16 values)
+        if (tid < 128) {
+            const uint8_t *rowp = (tid < 64 ? Qin : Kin) + (tid & 63) * (D * 2);
+            float ss = 0.f;
+#pragma unroll
+            for (int x = 0; x < 16; ++x) {
+                const uint4 w = *reinterpret_cast<const uint4 *>(rowp + 16 * ((x + lane) & 15));  // rotated: no bank clash
+                const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 f = unpack_bf16(ws[e]);
+                    ss = fmaf(f.x, f.x, fmaf(f.y, f.y, ss));
+                }
+            }
+            s_inv[tid] = rsqrtf(ss + kNormEps);
+        }
+        __syncthreads();
+    }
+    auto scaled = [](uint32_t u, float sc) {
+        const float2 f = unpack_bf16(u);
+        return pack_bf16(f.x * sc, f.y * sc);
+    };
     float2 g[16];
     uint32_t kk[16], qq[16];
 #pragma unroll
@@ -321,6 +353,11 @@ kda_tc_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             g[m] = *reinterpret_cast<const float2 *>(Gin + (r * D + c0) * 4);
             kk[m] = *reinterpret_cast<const uint32_t *>(Kin + (r * D + c0) * 2);
             qq[m] = *reinterpret_cast<const uint32_t *>(Qin + (r * D + c0) * 2);
+            if (l2) {
+                kk[m] = scaled(kk[m], s_inv[64 + r]);
+                qq[m] = scaled(qq[m], s_inv[r]);
+            }
+            if (gate) g[m] = make_float2(gate_log_decay(g[m].x, ga, gb0), gate_log_decay(g[m].y, ga, gb1));
         } else {
             g[m] = make_float2(0.f, 0.f);
             kk[m] = 0u;
@@ -914,7 +951,7 @@ size_t prefill_tc_workspace_bytes(int B, int T, int H, int num_seqs, bool varlen
 cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const float *log_alpha,
                               const float *beta, const float *h0, const int32_t *cu_seqlens, int num_seqs,
                               int B, int T, int H, void *o, float *h_T, void *workspace, size_t workspace_bytes,
-                              cudaStream_t stream) {
+                              const Prologue &pro, cudaStream_t stream) {
     (void)workspace_bytes;
     const TcLayout lay = tc_layout(B, T, H, num_seqs);
     uint8_t *ws = static_cast<uint8_t *>(workspace);
@@ -948,7 +985,7 @@ cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const
         if (lay.max_chunks > 0) {
             trace_before(kKernTcPrep, stream);
             kda_tc_prep_kernel<<<(unsigned)(lay.max_chunks * H), kPrepThreads, PREP_SMEM, stream>>>(
-                tm_q, tm_k, tm_v, tm_g, beta, T, H, 0, status + 1, table, records, status);
+                tm_q, tm_k, tm_v, tm_g, pro, beta, T, H, 0, status + 1, table, records, status);
             trace_after(stream);
             if ((e = cudaGetLastError()) != cudaSuccess) return e;
         }
@@ -962,7 +999,7 @@ cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const
     if (nc > 0) {
         trace_before(kKernTcPrep, stream);
         kda_tc_prep_kernel<<<(unsigned)((int64_t)B * nc * H), kPrepThreads, PREP_SMEM, stream>>>(
-            tm_q, tm_k, tm_v, tm_g, beta, T, H, nc, nullptr, nullptr, records, status);
+            tm_q, tm_k, tm_v, tm_g, pro, beta, T, H, nc, nullptr, nullptr, records, status);
         trace_after(stream);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }

@@ -137,3 +137,27 @@ def test_decode_multi_rejects_on_host(lib):
     assert _multi(lib, o=A) == _lib.KDA_ERR_ALIASING                    # o overlaps q
     assert _multi(lib, pool=5 * A) == _lib.KDA_ERR_ALIASING             # pool overlaps beta
     assert _multi(lib, status=6 * A) == _lib.KDA_ERR_ALIASING           # status inside the pool
+
+
+def _fwd_ex(lib, flags=0, A_log=None, dt_bias=None, **kw):
+    args = dict(q=A, k=2 * A, v=3 * A, la=4 * A, beta=5 * A, h0=None, cu=None, N=1, B=1, T=128, H=2, dk=128,
+                dv=128, chunk=64, dtype=_lib.KDA_BF16, o=6 * A, hT=7 * A, ws=8 * A, ws_bytes=1 << 40, stream=None)
+    args.update(kw)
+    c = ctypes.c_void_p
+    return lib.kda_chunk_fwd_ex(c(args["q"]), c(args["k"]), c(args["v"]), c(args["la"]), c(args["beta"]),
+                                c(args["h0"]), c(args["cu"]), args["N"], args["B"], args["T"], args["H"], args["dk"],
+                                args["dv"], args["chunk"], args["dtype"], c(args["o"]), c(args["hT"]), c(args["ws"]),
+                                args["ws_bytes"], flags, c(A_log), c(dt_bias), c(args["stream"]))
+
+
+def test_prologue_arguments_rejected_on_host(lib):
+    assert _fwd_ex(lib, flags=4) == _lib.KDA_ERR_UNSUPPORTED                        # unknown flag bit
+    assert _fwd_ex(lib, flags=_lib.KDA_PROLOGUE_GATE) == _lib.KDA_ERR_NULL_ARG       # gate needs A_log
+    assert _fwd_ex(lib, flags=_lib.KDA_PROLOGUE_GATE, A_log=9 * A + 4) == _lib.KDA_ERR_MISALIGNED
+    assert _fwd_ex(lib, flags=_lib.KDA_PROLOGUE_GATE, A_log=9 * A, dt_bias=10 * A + 8) == _lib.KDA_ERR_MISALIGNED
+    assert _fwd_ex(lib, flags=_lib.KDA_PROLOGUE_GATE, A_log=6 * A) == _lib.KDA_ERR_ALIASING     # inside o
+    assert _fwd_ex(lib, flags=3, A_log=9 * A, dt_bias=7 * A) == _lib.KDA_ERR_ALIASING           # inside h_T
+    c = ctypes.c_void_p
+    rc = lib.kda_decode_multi_ex(c(A), c(2 * A), c(3 * A), c(4 * A), c(5 * A), c(6 * A), 8, None, None, 4, 3, 2, 128,
+                                 128, _lib.KDA_BF16, c(7 * A), None, 8, None, None, None)
+    assert rc == _lib.KDA_ERR_UNSUPPORTED
