@@ -87,7 +87,12 @@ KDA_API size_t kda_chunk_fwd_workspace_size(int B, int T, int H, int dk, int dv,
  * rows and their h_T is h0 (zeros without h0).  When B * T = 0 the token tensors (q, k, v,
  * log_alpha, beta, o) are empty and may be NULL.
  * Supported: dk = dv = 128 with dtype BF16 (tensor-core path) or F32; dk = dv = 64 with F32 or
- * BF16 (CUDA-core path).  Returns KDA_OK once the work is enqueued. */
+ * BF16 (CUDA-core path).  Returns KDA_OK once the work is enqueued.
+ * Strong decays: a step's gate below 2^-12 (log_alpha < -8.32) is applied as 2^-12 on the
+ * tensor-core path and below 2^-15 (log_alpha < -10.40) as 2^-15 on the CUDA-core path, so the
+ * chunk's split decay factors stay inside the fp32 exponent range.  Such a step keeps at most
+ * that fraction of the state where the exact recurrence keeps less; any log_alpha <= 0 (down to
+ * -inf) is accepted.  kda_decode_step / kda_decode_multi apply the gate exactly. */
 KDA_API int kda_chunk_fwd(const void *q, const void *k, const void *v, const float *log_alpha,
                   const float *beta, const float *h0, const int32_t *cu_seqlens, int num_seqs,
                   int B, int T, int H, int dk, int dv, int chunk_size, kda_dtype dtype, void *o,

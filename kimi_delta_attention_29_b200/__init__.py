@@ -10,6 +10,7 @@ import ctypes
 
 from . import _lib
 from ._lib import KdaError, status_string  # noqa: F401
+from ._lib import KDA_PROLOGUE_GATE, KDA_PROLOGUE_L2NORM_QK  # noqa: F401
 
 __all__ = ["kda_chunk_fwd", "kda_chunk_fwd_workspace_size", "kda_decode_step", "kda_get_status",
            "kda_status_string", "kda_trace_begin", "kda_trace_end", "KdaError", "Workspace"]

@@ -15,10 +15,11 @@
 //  applies T to V - (K o e^G) S directly, which is the same product taken in the other order.)
 //
 // Decay factors (section "Reduced computation vs general DPLR": fine-grained decay inside a
-// chunk needs log-domain care): e^{G_rc - G_ic} is split at a reference point per 16-row block,
-// E_b = G at row 16b + 7, as  e^{G_r - E_b(r)} * e^{E_b(r) - E_b(i)} * e^{E_b(i) - G_i};
-// each factor stays within e^{+-8 max|log_alpha|} or below 1, so nothing overflows fp32 even when
-// G falls far below -88 within a chunk.
+// chunk needs log-domain care): this path takes every factor as one exponential of a difference
+// that is <= 0 for the pairs it is used on -- 2^{G_r - G_i} per (r, i <= r, channel) in the Gram
+// matrices, 2^{G_r} and 2^{G_last - G_r} per row -- with G in base 2, so no factor can overflow
+// and one that underflows stands for a term below the fp32 range.  Each step's log2 gate is
+// clamped at kMinLog2DecaySimt, which bounds |G| (and with it the rounding of G_r - G_i) over a chunk.
 //
 // One CTA of 256 threads owns (sequence, head, 32 value columns); value columns evolve
 // independently, so the slices need no communication.
@@ -30,17 +31,14 @@ namespace {
 constexpr int kC = kChunk;    // 64 rows per chunk
 constexpr int kNV = 32;       // value columns per CTA
 constexpr int kThreads = 256;
-constexpr int kBlocks = kC / 16;
 
 template <int DK>
 struct SimtSmem {
     static constexpr int DKP = DK + 1;  // padded row stride (bank-conflict free column walks)
     static constexpr int CP = kC + 1;
     static constexpr size_t floats =
-        3 * (size_t)kC * DKP          // Xo (k, then k e^{G-E}), Xq (q e^{G-E}), Y (G, then k e^{E-G})
-        + (size_t)kBlocks * kBlocks * DK  // Cf[b][a][c] = e^{E_b - E_a}
-        + 2 * (size_t)kBlocks * DK        // eb = e^{E_b}, gle = e^{G_last - E_b}
-        + DK                              // egl = e^{G_last}
+        3 * (size_t)kC * DKP          // Xo (k, then k 2^G), Xq (q, then q 2^G), Y (G, then k 2^{G_last - G})
+        + 2 * (size_t)DK                  // gls = G_last, egl = 2^{G_last}
         + 3 * (size_t)kC * kNV            // Vs, X1, Dl
         + (size_t)DK * kNV                // Ss
         + 3 * (size_t)kC * CP             // Am, Pm, Tm
@@ -62,10 +60,8 @@ kda_prefill_simt_kernel(const T *__restrict__ q, const T *__restrict__ k, const 
     float *Xo = smem;
     float *Xq = Xo + kC * DKP;
     float *Y = Xq + kC * DKP;
-    float *Cf = Y + kC * DKP;
-    float *eb = Cf + kBlocks * kBlocks * DK;
-    float *gle = eb + kBlocks * DK;
-    float *egl = gle + kBlocks * DK;
+    float *gls = Y + kC * DKP;
+    float *egl = gls + DK;
     float *Vs = egl + DK;
     float *X1 = Vs + kC * kNV;
     float *Dl = X1 + kC * kNV;
@@ -121,6 +117,7 @@ kda_prefill_simt_kernel(const T *__restrict__ q, const T *__restrict__ k, const 
                 qv = Elem<T>::load(q + off);
                 lv = __ldg(log_alpha + off);
                 if (gate) lv = gate_log_decay(lv, ga, pro.dt_bias ? __ldg(pro.dt_bias + (size_t)h * DK + c) : 0.f);
+                lv = fmaxf(lv * kLog2e, kMinLog2DecaySimt);  // base-2 log gate, clamped
             }
             Xo[r * DKP + c] = kv;
             Xq[r * DKP + c] = qv;
@@ -143,34 +140,15 @@ kda_prefill_simt_kernel(const T *__restrict__ q, const T *__restrict__ k, const 
             __syncthreads();
         }
 
-        // 2. per-channel cumulative log-gate and the block-referenced decay factors
+        // 2. per-channel cumulative base-2 log-gate G (in place in Y)
         for (int c = tid; c < DK; c += kThreads) {
             float acc = 0.f;
             for (int r = 0; r < kC; ++r) {
                 acc += Y[r * DKP + c];
                 Y[r * DKP + c] = acc;
             }
-            float E[kBlocks];
-#pragma unroll
-            for (int b = 0; b < kBlocks; ++b) E[b] = Y[(16 * b + 7) * DKP + c];
-            const float gl = acc;
-#pragma unroll
-            for (int b = 0; b < kBlocks; ++b) {
-#pragma unroll
-                for (int a = 0; a < kBlocks; ++a) Cf[(b * kBlocks + a) * DK + c] = a <= b ? expf(E[b] - E[a]) : 0.f;
-                eb[b * DK + c] = expf(E[b]);
-                gle[b * DK + c] = expf(gl - E[b]);
-            }
-            egl[c] = expf(gl);
-            for (int r = 0; r < kC; ++r) {
-                const float Eb = E[r / 16];
-                const float g = Y[r * DKP + c];
-                const float kk = Xo[r * DKP + c];
-                const float F = expf(g - Eb);
-                Xo[r * DKP + c] = kk * F;
-                Xq[r * DKP + c] *= F;
-                Y[r * DKP + c] = kk * expf(Eb - g);
-            }
+            gls[c] = acc;
+            egl[c] = ex2f(acc);
         }
         __syncthreads();
 
@@ -179,15 +157,25 @@ kda_prefill_simt_kernel(const T *__restrict__ q, const T *__restrict__ k, const 
             const int r = p / kC, i = p % kC;
             float sa = 0.f, sp = 0.f;
             if (i <= r) {
-                const float *cf = Cf + ((r / 16) * kBlocks + i / 16) * DK;
+                const float *gr = Y + r * DKP, *gi = Y + i * DKP;
                 for (int c = 0; c < DK; ++c) {
-                    const float yi = Y[i * DKP + c] * cf[c];
-                    sa = fmaf(Xo[r * DKP + c], yi, sa);
-                    sp = fmaf(Xq[r * DKP + c], yi, sp);
+                    const float kd = Xo[i * DKP + c] * ex2f(gr[c] - gi[c]);
+                    sa = fmaf(Xo[r * DKP + c], kd, sa);
+                    sp = fmaf(Xq[r * DKP + c], kd, sp);
                 }
             }
             Am[r * CP + i] = i < r ? bt[r] * sa : 0.f;
             Pm[r * CP + i] = i <= r ? sp : 0.f;
+        }
+        __syncthreads();
+        // decayed rows for the state terms: K o 2^G, Q o 2^G and K o 2^{G_last - G} (into Y)
+        for (int idx = tid; idx < kC * DK; idx += kThreads) {
+            const int r = idx / DK, c = idx % DK;
+            const float g = Y[r * DKP + c], f = ex2f(g);
+            const float kv = Xo[r * DKP + c];
+            Y[r * DKP + c] = kv * ex2f(gls[c] - g);
+            Xo[r * DKP + c] = kv * f;
+            Xq[r * DKP + c] *= f;
         }
         __syncthreads();
 
@@ -203,12 +191,11 @@ kda_prefill_simt_kernel(const T *__restrict__ q, const T *__restrict__ k, const 
             __syncthreads();
         }
 
-        // 5. X1 = V - (K o e^G) S      (K o e^G)_r = Xo_r * e^{E_b(r)}
+        // 5. X1 = V - (K o 2^G) S
         for (int idx = tid; idx < kC * kNV; idx += kThreads) {
             const int r = idx / kNV, j = idx % kNV;
-            const float *e = eb + (r / 16) * DK;
             float acc = Vs[idx];
-            for (int c = 0; c < DK; ++c) acc = fmaf(-Xo[r * DKP + c] * e[c], Ss[c * kNV + j], acc);
+            for (int c = 0; c < DK; ++c) acc = fmaf(-Xo[r * DKP + c], Ss[c * kNV + j], acc);
             X1[idx] = acc;
         }
         __syncthreads();
@@ -220,22 +207,21 @@ kda_prefill_simt_kernel(const T *__restrict__ q, const T *__restrict__ k, const 
             Dl[idx] = acc;
         }
         __syncthreads();
-        // 7. O = (Q o e^G) S + P Delta
+        // 7. O = (Q o 2^G) S + P Delta
         for (int idx = tid; idx < kC * kNV; idx += kThreads) {
             const int r = idx / kNV, j = idx % kNV;
             if (r >= L) continue;
-            const float *e = eb + (r / 16) * DK;
             float acc = 0.f;
-            for (int c = 0; c < DK; ++c) acc = fmaf(Xq[r * DKP + c] * e[c], Ss[c * kNV + j], acc);
+            for (int c = 0; c < DK; ++c) acc = fmaf(Xq[r * DKP + c], Ss[c * kNV + j], acc);
             for (int i = 0; i <= r; ++i) acc = fmaf(Pm[r * CP + i], Dl[i * kNV + j], acc);
             Elem<T>::store(o + ((size_t)(start + c0 + r) * H + h) * DV + j0 + j, acc);
         }
         __syncthreads();
-        // 8. S <- Diag(e^{G_last}) S + (K o e^{G_last - G})^T Delta;  (K o e^{G_last-G})_i = Y_i e^{G_last - E_b(i)}
+        // 8. S <- Diag(2^{G_last}) S + (K o 2^{G_last - G})^T Delta
         for (int idx = tid; idx < DK * kNV; idx += kThreads) {
             const int c = idx / kNV, j = idx % kNV;
             float acc = egl[c] * Ss[idx];
-            for (int i = 0; i < kC; ++i) acc = fmaf(Y[i * DKP + c] * gle[(i / 16) * DK + c], Dl[i * kNV + j], acc);
+            for (int i = 0; i < kC; ++i) acc = fmaf(Y[i * DKP + c], Dl[i * kNV + j], acc);
             Ss[idx] = acc;
         }
     }

@@ -241,6 +241,9 @@ __device__ __forceinline__ void subst_block_row(float *Asm, float *Mscr, int war
     __syncthreads();
 }
 
+// kFlags: the layer-prologue steps compiled in (KDA_PROLOGUE_* bits; 0 = the plain kernel, which
+// ignores pro).  One instantiation per combination, so each path carries only its own work.
+template <unsigned kFlags>
 __global__ void __launch_bounds__(kPrepThreads, 2)
 kda_tc_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
@@ -286,7 +289,6 @@ kda_tc_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int c0 = 64 * (warp & 1) + 2 * lane;  // this thread's two key channels
     const int qr = warp >> 1;                   // key block: rows 16 qr .. 16 qr + 15
-    constexpr float kLog2e = 1.4426950408889634f;
 
     if (tid == 0) {
         mbar_init(mbar, 1);
@@ -312,9 +314,9 @@ kda_tc_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     __syncthreads();  // barriers initialised before anyone waits on them
 
     // ---- k, q (bf16 pairs) and log-gates (fp32 pairs) of this thread's 16 rows, from the landed tiles
-    const bool gate = pro.flags & KDA_PROLOGUE_GATE, l2 = pro.flags & KDA_PROLOGUE_L2NORM_QK;
+    constexpr bool gate = kFlags & KDA_PROLOGUE_GATE, l2 = kFlags & KDA_PROLOGUE_L2NORM_QK;
     float ga = 0.f, gb0 = 0.f, gb1 = 0.f;  // prologue gate: exp(A_log[h]), dt_bias of this thread's channels
-    if (gate) {
+    if constexpr (gate) {
         ga = expf(__ldg(pro.A_log + h));
         if (pro.dt_bias) {
             gb0 = __ldg(pro.dt_bias + (size_t)h * D + c0);
@@ -322,53 +324,84 @@ kda_tc_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         }
     }
     const bool in_ok = mbar_wait(mbar + 2, 0);
-    if (l2) {  // inverse L2 norms of the 64 q rows and 64 k rows (fp32 sums of the bf16 values)
-        if (tid < 128) {
-            const uint8_t *rowp = (tid < 64 ? Qin : Kin) + (tid & 63) * (D * 2);
-            float ss = 0.f;
+    float2 g[16];
+    uint32_t kk[16], qq[16];
+    if constexpr (!l2) {
 #pragma unroll
-            for (int x = 0; x < 16; ++x) {
-                const uint4 w = *reinterpret_cast<const uint4 *>(rowp + 16 * ((x + lane) & 15));  // rotated: no bank clash
+        for (int m = 0; m < 16; ++m) {
+            const int r = 16 * qr + m;
+            if (r < L) {
+                g[m] = *reinterpret_cast<const float2 *>(Gin + (r * D + c0) * 4);
+                kk[m] = *reinterpret_cast<const uint32_t *>(Kin + (r * D + c0) * 2);
+                qq[m] = *reinterpret_cast<const uint32_t *>(Qin + (r * D + c0) * 2);
+                if constexpr (gate)
+                    g[m] = make_float2(gate_log_decay(g[m].x, ga, gb0), gate_log_decay(g[m].y, ga, gb1));
+            } else {
+                g[m] = make_float2(0.f, 0.f);
+                kk[m] = 0u;
+                qq[m] = 0u;
+            }
+        }
+    } else {
+        // log gates first: their activation is independent of the norms and overlaps the norm loads
+#pragma unroll
+        for (int m = 0; m < 16; ++m) {
+            const int r = 16 * qr + m;
+            g[m] = make_float2(0.f, 0.f);
+            if (r < L) {
+                g[m] = *reinterpret_cast<const float2 *>(Gin + (r * D + c0) * 4);
+                if constexpr (gate)
+                    g[m] = make_float2(gate_log_decay(g[m].x, ga, gb0), gate_log_decay(g[m].y, ga, gb1));
+            }
+        }
+        {  // inverse L2 norms of the 64 q rows and 64 k rows (fp32 sums of the bf16 values)
+            // thread pair (2j, 2j+1) sums the two 128-byte halves of row j (j < 64: q, else k); the
+            // rotation 2j + half puts the 8 lanes of each 128-byte load phase on distinct bank groups
+            const int j = tid >> 1, hf = tid & 1;
+            const uint8_t *rowp = (j < 64 ? Qin : Kin) + (j & 63) * (D * 2) + 128 * hf;
+            float ss[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int x = 0; x < 8; ++x) {
+                const uint4 w = *reinterpret_cast<const uint4 *>(rowp + 16 * ((x + 2 * j + hf) & 7));
                 const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const float2 f = unpack_bf16(ws[e]);
-                    ss = fmaf(f.x, f.x, fmaf(f.y, f.y, ss));
+                    ss[e] = fmaf(f.x, f.x, fmaf(f.y, f.y, ss[e]));
                 }
             }
-            s_inv[tid] = rsqrtf(ss + kNormEps);
+            float tot = (ss[0] + ss[1]) + (ss[2] + ss[3]);
+            tot += __shfl_xor_sync(0xffffffffu, tot, 1);
+            if (!hf) s_inv[j] = rsqrtf(tot + kNormEps);
+            __syncthreads();
         }
-        __syncthreads();
-    }
-    auto scaled = [](uint32_t u, float sc) {
-        const float2 f = unpack_bf16(u);
-        return pack_bf16(f.x * sc, f.y * sc);
-    };
-    float2 g[16];
-    uint32_t kk[16], qq[16];
+        auto scaled = [](uint32_t u, float sc) {
+            const float2 f = unpack_bf16(u);
+            return pack_bf16(f.x * sc, f.y * sc);
+        };
 #pragma unroll
-    for (int m = 0; m < 16; ++m) {
-        const int r = 16 * qr + m;
-        if (r < L) {
-            g[m] = *reinterpret_cast<const float2 *>(Gin + (r * D + c0) * 4);
-            kk[m] = *reinterpret_cast<const uint32_t *>(Kin + (r * D + c0) * 2);
-            qq[m] = *reinterpret_cast<const uint32_t *>(Qin + (r * D + c0) * 2);
-            if (l2) {
+        for (int m = 0; m < 16; ++m) {
+            const int r = 16 * qr + m;
+            kk[m] = 0u;
+            qq[m] = 0u;
+            if (r < L) {
+                kk[m] = *reinterpret_cast<const uint32_t *>(Kin + (r * D + c0) * 2);
+                qq[m] = *reinterpret_cast<const uint32_t *>(Qin + (r * D + c0) * 2);
                 kk[m] = scaled(kk[m], s_inv[64 + r]);
                 qq[m] = scaled(qq[m], s_inv[r]);
             }
-            if (gate) g[m] = make_float2(gate_log_decay(g[m].x, ga, gb0), gate_log_decay(g[m].y, ga, gb1));
-        } else {
-            g[m] = make_float2(0.f, 0.f);
-            kk[m] = 0u;
-            qq[m] = 0u;
         }
     }
 
     // ---- chunk-local cumulative log2-gate G (fp32): block-local prefix, then block offsets
-    g[0] = make_float2(g[0].x * kLog2e, g[0].y * kLog2e);
+    // (each step's log gate clamped at kMinLog2DecayTc, in natural units before the scaling to base
+    // 2 so that the clamp adds one instruction, which bounds the split factors below)
+    constexpr float kMinLog = kMinLog2DecayTc / kLog2e;
+    g[0] = make_float2(fmaxf(g[0].x, kMinLog) * kLog2e, fmaxf(g[0].y, kMinLog) * kLog2e);
 #pragma unroll
-    for (int m = 1; m < 16; ++m) g[m] = make_float2(fmaf(g[m].x, kLog2e, g[m - 1].x), fmaf(g[m].y, kLog2e, g[m - 1].y));
+    for (int m = 1; m < 16; ++m)
+        g[m] = make_float2(fmaf(fmaxf(g[m].x, kMinLog), kLog2e, g[m - 1].x),
+                           fmaf(fmaxf(g[m].y, kMinLog), kLog2e, g[m - 1].y));
     s_tot[qr * D + c0] = g[15].x;
     s_tot[qr * D + c0 + 1] = g[15].y;
     tc_fence_before();
@@ -393,12 +426,19 @@ kda_tc_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     __syncthreads();
 
     const float2 gl = make_float2(s_gl[c0], s_gl[c0 + 1]);
-    // 2^{E_b - E_own} for the later blocks b > own (<= 1), 2^{E_own}, 2^{G_63 - E_own}
+    // Products of a within-block factor 2^{+-(G - E_own)} (exponent in [-96, 96]) with a block- or
+    // chunk-level factor 2^{w} (w <= 0, down to -64 * 12) are taken as 2^{. - 90} * 2^{w + 90}:
+    // each side then stays a normal fp32 number whenever the product can reach 2^-36 of a term,
+    // where 2^{w} alone would flush to zero for w < -126 with 2^{. + w} still significant.
+    // Here: 2^{E_b - E_own + 90} for the later blocks b > own, 2^{E_own + 90}, 2^{G_63 - E_own + 90}.
+    constexpr float kSplitBias = 90.f, kSplitDown = 0x1p-90f;
     float2 Cr[4];
 #pragma unroll
     for (int b = 0; b < 4; ++b)
-        Cr[b] = b > qr ? ex2v(sub2(make_float2(s_E[b * D + c0], s_E[b * D + c0 + 1]), Eown)) : make_float2(1.f, 1.f);
-    const float2 eE = ex2v(Eown), eGL = ex2v(sub2(gl, Eown));
+        Cr[b] = b > qr ? ex2v(make_float2(s_E[b * D + c0] - Eown.x + kSplitBias, s_E[b * D + c0 + 1] - Eown.y + kSplitBias))
+                       : make_float2(0.f, 0.f);
+    const float2 eE = ex2v(make_float2(Eown.x + kSplitBias, Eown.y + kSplitBias));
+    const float2 eGL = ex2v(make_float2(gl.x - Eown.x + kSplitBias, gl.y - Eown.y + kSplitBias));
 
     // ---- operands: X, R^(b) for b >= own block, K o 2^G (smem); Q o 2^G and K o 2^{G63-G} (record).
     // The factors are rounded to bf16 and applied with packed bf16 multiplies on the bf16 inputs.
@@ -407,10 +447,12 @@ kda_tc_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         const int r = 16 * qr + m;
         const float2 F = ex2v(sub2(g[m], Eown));
         const float2 Rf = ex2v(sub2(Eown, g[m]));
+        const float2 Fs = make_float2(F.x * kSplitDown, F.y * kSplitDown);
+        const float2 Rs = make_float2(Rf.x * kSplitDown, Rf.y * kSplitDown);
         const __nv_bfloat162 k2 = as_bf2(kk[m]), q2 = as_bf2(qq[m]);
         const __nv_bfloat162 fx = bf2_of(F);
-        const __nv_bfloat162 fe = bf2_of(make_float2(F.x * eE.x, F.y * eE.y));
-        const __nv_bfloat162 frg = bf2_of(make_float2(Rf.x * eGL.x, Rf.y * eGL.y));
+        const __nv_bfloat162 fe = bf2_of(make_float2(Fs.x * eE.x, Fs.y * eE.y));
+        const __nv_bfloat162 frg = bf2_of(make_float2(Rs.x * eGL.x, Rs.y * eGL.y));
         st_bf2(X + sw128_off(32 * qr + m, c0, 128), __hmul2(k2, fx));
         st_bf2(X + sw128_off(32 * qr + 16 + m, c0, 128), __hmul2(q2, fx));
         st_bf2(KT + sw128_off(r, c0, 64), __hmul2(k2, fe));
@@ -420,7 +462,7 @@ kda_tc_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         for (int b = 0; b < 4; ++b)
             if (b >= qr)
                 st_bf2(Rimg + sw128_off(r_first_row(b) + r, c0, kRRows),
-                       __hmul2(k2, bf2_of(make_float2(Rf.x * Cr[b].x, Rf.y * Cr[b].y))));
+                       __hmul2(k2, bf2_of(b == qr ? Rf : make_float2(Rs.x * Cr[b].x, Rs.y * Cr[b].y))));
     }
     fence_async_smem();
     __syncthreads();
@@ -963,7 +1005,12 @@ cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const
     if (e != cudaSuccess) return e;
 
     // opt in to the large dynamic shared-memory sizes (per device, so on every call)
-    e = cudaFuncSetAttribute(kda_tc_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)PREP_SMEM);
+    constexpr unsigned kL2 = KDA_PROLOGUE_L2NORM_QK, kGate = KDA_PROLOGUE_GATE;
+    auto *prep = pro.flags == (kL2 | kGate) ? kda_tc_prep_kernel<kL2 | kGate>
+               : pro.flags == kL2          ? kda_tc_prep_kernel<kL2>
+               : pro.flags == kGate        ? kda_tc_prep_kernel<kGate>
+                                           : kda_tc_prep_kernel<0>;
+    e = cudaFuncSetAttribute(prep, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)PREP_SMEM);
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(kda_tc_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)STATE_SMEM);
     if (e != cudaSuccess) return e;
@@ -984,7 +1031,7 @@ cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
         if (lay.max_chunks > 0) {
             trace_before(kKernTcPrep, stream);
-            kda_tc_prep_kernel<<<(unsigned)(lay.max_chunks * H), kPrepThreads, PREP_SMEM, stream>>>(
+            prep<<<(unsigned)(lay.max_chunks * H), kPrepThreads, PREP_SMEM, stream>>>(
                 tm_q, tm_k, tm_v, tm_g, pro, beta, T, H, 0, status + 1, table, records, status);
             trace_after(stream);
             if ((e = cudaGetLastError()) != cudaSuccess) return e;
@@ -998,7 +1045,7 @@ cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const
     const int nc = (T + C - 1) / C;
     if (nc > 0) {
         trace_before(kKernTcPrep, stream);
-        kda_tc_prep_kernel<<<(unsigned)((int64_t)B * nc * H), kPrepThreads, PREP_SMEM, stream>>>(
+        prep<<<(unsigned)((int64_t)B * nc * H), kPrepThreads, PREP_SMEM, stream>>>(
             tm_q, tm_k, tm_v, tm_g, pro, beta, T, H, nc, nullptr, nullptr, records, status);
         trace_after(stream);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;

@@ -124,6 +124,27 @@ def test_prefill_bf16_gate_ranges(cuda_device, gate_shift):
     assert rel_err(hT, h_ref) <= 2e-2
 
 
+@pytest.mark.parametrize("dtype,d", [(torch.bfloat16, 128), (torch.float32, 64), (torch.float32, 128)])
+def test_prefill_strong_decay_steps(cuda_device, dtype, d):
+    """Steps whose decay leaves (almost) nothing: 3% of the log-gates at -60, one token with
+    log alpha = -1e4 and one with -inf in every channel.  A block-split decay factor over such a step
+    lies far outside the fp32 range; the chunked kernels apply these steps as a decay of 2^-15, so
+    the result must stay finite and within the usual tolerance of the exact recurrence."""
+    x = gen.make_prefill(2, 300, 2, d, d, dtype, gate_shift=0.0, h0_std=0.5, seed=41)
+    g = torch.Generator().manual_seed(42)
+    la = x["log_alpha"].clone()
+    la[torch.rand(la.shape, generator=g) < 0.03] = -60.0
+    la[0, 100] = -1e4
+    la[1, 37] = float("-inf")
+    x["log_alpha"] = la
+    x = to_dev(x, cuda_device)
+    o, hT = run_fwd(x)
+    o_ref, h_ref = oracle_fwd(x)
+    assert torch.isfinite(o.float()).all() and torch.isfinite(hT).all()
+    assert rel_err(o, o_ref) <= TOL[dtype]
+    assert rel_err(hT, h_ref) <= TOL[dtype]
+
+
 @pytest.mark.parametrize("dtype,d", [(torch.float32, 128), (torch.bfloat16, 64)])
 def test_prefill_cuda_core_path(cuda_device, dtype, d):
     x = to_dev(gen.make_prefill(2, 150, 2, d, d, dtype, gate_shift=1.0, h0_std=0.3, seed=5), cuda_device)

@@ -66,6 +66,24 @@ def test_prefill_prologue_matches_oracle(cuda_device, dtype, d, flags):
     assert rel_err(hT, h_ref) <= TOL[dtype]
 
 
+@pytest.mark.parametrize("dtype,d", [(torch.bfloat16, 128), (torch.float32, 64)])
+def test_prefill_prologue_strong_gates(cuda_device, dtype, d):
+    """Gate activations at the strong end of the layer's range: exp(A_log) up to 16 per head and
+    gate projections ~ 3 N(0,1), so single steps reach log alpha of -100 and beyond."""
+    H, T = 4, 260
+    x = {kk: (vv.to(cuda_device) if isinstance(vv, torch.Tensor) else vv)
+         for kk, vv in gen.make_prefill(1, T, H, d, d, dtype, h0_std=0.3, seed=31).items()}
+    A_log, dt_bias = raw_layer_inputs(x, H, d, cuda_device, seed=7, flags=L2 | GATE)
+    x["log_alpha"] = x["log_alpha"] * 1.5
+    A_log = torch.log(torch.tensor([1.0, 4.0, 9.0, 16.0], device=cuda_device))
+    o, hT = kda.kda_chunk_fwd_ex(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], x["h0"], None, flags=L2 | GATE,
+                                 A_log=A_log, dt_bias=dt_bias)
+    o_ref, h_ref = oracle_with_prologue(x, L2 | GATE, A_log, dt_bias, np64(x["h0"]))
+    assert torch.isfinite(o.float()).all() and torch.isfinite(hT).all()
+    assert rel_err(o, o_ref) <= TOL[dtype]
+    assert rel_err(hT, h_ref) <= TOL[dtype]
+
+
 def test_prefill_prologue_varlen_and_no_bias(cuda_device):
     lens = torch.tensor([70, 0, 130, 5])
     cu = gen.cu_seqlens_from_lengths(lens)
