@@ -354,6 +354,30 @@ def gpu_arm(args):
                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": args.e2e_steps}
     del host, dx, o_h, hT_h
 
+    # the same prefill with the layer prologue fused in (q/k L2 normalisation, gate activation from the
+    # gate projection g; here g = the workload's log_alpha values, A_log = 0, dt_bias = 0)
+    A_log = torch.zeros(H, device=dev)
+    flags = kda.KDA_PROLOGUE_L2NORM_QK | kda.KDA_PROLOGUE_GATE
+
+    def step_pro():
+        kda.kda_chunk_fwd_ex(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], x["h0"], None, flags=flags,
+                             A_log=A_log, o=o, h_T=hT, workspace=ws, stream=stream)
+
+    for _ in range(2):
+        step_pro()
+    torch.cuda.synchronize(dev)
+    barrier()
+    pe0, pe1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    pe0.record(stream)
+    for _ in range(args.steps):
+        step_pro()
+    pe1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    pro_ms = max_over_ranks(pe0.elapsed_time(pe1)) / args.steps
+    prologue = {"ms_per_step": pro_ms, "tokens_per_s": whole_job_rate(tokens_per_step, 1, world, pro_ms),
+                "flags": "l2norm_qk|gate", "vs_plain": ms_per_step / pro_ms}
+
     decode = None
     if not args.no_decode:
         decode = decode_bench(args, dev, stream, peaks, barrier, max_over_ranks)
@@ -366,7 +390,7 @@ def gpu_arm(args):
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config_dict(T),
             "roofline": roofline, "operator_roofline": operator_roofline, "cpu_baseline": cpu_baseline,
-            "e2e": e2e, "gpu_launches": len(traces), "clocks": clk, "decode": decode,
+            "e2e": e2e, "gpu_launches": len(traces), "clocks": clk, "prologue": prologue, "decode": decode,
             "kernels": kst, "peaks": peaks}
     if rank == 0:
         print(json.dumps(line), flush=True)
