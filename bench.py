@@ -214,23 +214,32 @@ def whole_job_rate(units_per_step_per_rank: float, steps: int, world: int, elaps
     return world * units_per_step_per_rank * steps / (elapsed_ms_max / 1e3)
 
 
+def sources_sha256(paths) -> str | None:
+    """sha256 over the concatenated bytes of the repo-relative source files (None if one is missing)."""
+    import hashlib
+    h = hashlib.sha256()
+    for p in paths:
+        full = os.path.join(ROOT, p)
+        if not os.path.exists(full):
+            return None
+        with open(full, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
 def ncu_traffic(kernel: str, units: int):
     """DRAM bytes per launch of `kernel` for `units` work units, scaled from the committed ncu capture
-    in profiles/ncu_traffic.json, or None when the kernel's source changed since that capture."""
-    import hashlib
+    in profiles/ncu_traffic.json, or None when any source the kernel is compiled from (its .cu file
+    and the headers it includes) changed since that capture."""
     path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     if not os.path.exists(path):
         return None
     with open(path) as f:
         rec = json.load(f).get(kernel)
-    if not rec:
+    if not rec or "sources" not in rec:
         return None
-    src = os.path.join(ROOT, rec["source"])
-    if not os.path.exists(src):
+    if sources_sha256(rec["sources"]) != rec["sources_sha256"]:
         return None
-    with open(src, "rb") as f:
-        if hashlib.sha256(f.read()).hexdigest() != rec["source_sha256"]:
-            return None
     return rec["dram_bytes"] / rec["units"] * units
 
 
