@@ -37,6 +37,8 @@ def _bind(path: str):
     lib.kda_oracle_decode_step.restype = i
     lib.kda_oracle_prologue.argtypes = [dp, dp, dp, ctypes.c_int64, i, i, ctypes.c_uint, ctypes.c_double, dp, dp]
     lib.kda_oracle_prologue.restype = i
+    lib.kda_oracle_output_gate_norm.argtypes = [dp, dp, dp, ctypes.c_int64, i, ctypes.c_double, dp]
+    lib.kda_oracle_output_gate_norm.restype = i
     lib.kda_oracle_num_threads.restype = i
     lib.kda_oracle_set_num_threads.argtypes = [i]
     return lib
@@ -130,6 +132,22 @@ class Oracle:
             raise ValueError(f"kda_oracle_prologue rejected its arguments (rc={rc})")
         return q, k, la
 
+    def output_gate_norm(self, o, g, weight=None, eps=1e-6):
+        """The layer's output epilogue on rows of length dv (the last axis of o and g): per-row RMSNorm
+        times weight[dv] times sigmoid(g).  Returns a float64 array shaped like o."""
+        o, g = _f64(o), _f64(g)
+        if o.shape != g.shape or o.ndim < 1:
+            raise ValueError("o and g must have the same shape")
+        dv = o.shape[-1]
+        w = None if weight is None else _f64(weight)
+        if w is not None and w.shape != (dv,):
+            raise ValueError("weight must have shape [dv]")
+        out = np.empty_like(o)
+        rc = self.lib.kda_oracle_output_gate_norm(_ptr(o), _ptr(g), _ptr(w), o.size // dv, dv, float(eps), _ptr(out))
+        if rc != 0:
+            raise ValueError(f"kda_oracle_output_gate_norm rejected its arguments (rc={rc})")
+        return out
+
     def num_threads(self) -> int:
         return int(self.lib.kda_oracle_num_threads())
 
@@ -157,6 +175,10 @@ def chunkwise(*args, **kw):
 
 def prologue(*args, **kw):
     return default().prologue(*args, **kw)
+
+
+def output_gate_norm(*args, **kw):
+    return default().output_gate_norm(*args, **kw)
 
 
 def decode_step(*args, **kw):

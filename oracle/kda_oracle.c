@@ -43,9 +43,9 @@
 
 #include "kda_oracle.h"
 
-/* KDA_ORACLE_MUTANT selects a deliberately wrong variant of the token update.  It
- * exists only so that a test can show that the pins catch plausible mistakes;
- * the library the tests trust is built with the default value 0. */
+/* KDA_ORACLE_MUTANT selects a deliberately wrong variant of the token update (1..5) or
+ * of the output epilogue (6..8).  It exists only so that a test can show that the pins
+ * catch plausible mistakes; the library the tests trust is built with the default value 0. */
 #ifndef KDA_ORACLE_MUTANT
 #define KDA_ORACLE_MUTANT 0
 #endif
@@ -368,6 +368,34 @@ int kda_oracle_prologue(double *q, double *k, double *la, int64_t n_tok, int H, 
                     la[base + c] = -a * softplus(la[base + c] + b);
                 }
             }
+        }
+    }
+    return KDA_ORACLE_OK;
+}
+
+int kda_oracle_output_gate_norm(const double *o, const double *g, const double *weight, int64_t rows, int dv,
+                                double eps, double *out) {
+    if (rows < 0 || dv <= 0 || !(eps >= 0.0)) return KDA_ORACLE_BAD_ARG;
+    if (rows > 0 && (!o || !g || !out)) return KDA_ORACLE_BAD_ARG;
+    for (int64_t r = 0; r < rows; ++r) {
+        const double *x = o + r * dv;
+        double ss = 0.0;
+        for (int j = 0; j < dv; ++j) ss += x[j] * x[j];
+#if KDA_ORACLE_MUTANT == 6
+        const double inv = 1.0 / sqrt(ss + eps);               /* planted: sum instead of mean */
+#elif KDA_ORACLE_MUTANT == 7
+        const double inv = 1.0 / (sqrt(ss / dv) + eps);        /* planted: eps outside the root */
+#else
+        const double inv = 1.0 / sqrt(ss / dv + eps);
+#endif
+        for (int j = 0; j < dv; ++j) {
+            const double w = weight ? weight[j] : 1.0;
+#if KDA_ORACLE_MUTANT == 8
+            const double gate = 1.0 / (1.0 + exp(g[r * dv + j]));  /* planted: sigmoid(-g) */
+#else
+            const double gate = 1.0 / (1.0 + exp(-g[r * dv + j]));
+#endif
+            out[r * dv + j] = x[j] * inv * w * gate;
         }
     }
     return KDA_ORACLE_OK;

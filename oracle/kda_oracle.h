@@ -42,6 +42,14 @@ int kda_oracle_decode_step(const double *q, const double *k, const double *v,
 int kda_oracle_prologue(double *q, double *k, double *la, int64_t n_tok, int H, int dk, unsigned flags,
                         double eps, const double *A_log, const double *dt_bias);
 
+/* The KDA layer's output epilogue (Kimi Linear page, section "Kimi Linear model composition": a
+ * per-head RMSNorm and a data-dependent output gate ahead of the output projection; the gate's
+ * activation is read as the logistic sigmoid), for `rows` rows of length dv:
+ *   out[r, j] = o[r, j] / sqrt(mean_j o[r, j]^2 + eps) * weight[j] * sigmoid(g[r, j]).
+ * weight: [dv] or NULL (ones).  out may be o. */
+int kda_oracle_output_gate_norm(const double *o, const double *g, const double *weight, int64_t rows, int dv,
+                                double eps, double *out);
+
 int kda_oracle_num_threads(void);
 void kda_oracle_set_num_threads(int n);
 

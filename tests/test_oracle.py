@@ -304,6 +304,61 @@ def pin_decode_matches_prefill(orc) -> float:
     return max(err, float(np.abs(S - hT).max()))
 
 
+# ------------------------------------------------------------------------------------- output epilogue
+# out = o / sqrt(mean(o^2) + eps) * weight * sigmoid(g) per row (Kimi Linear page, section "Kimi
+# Linear model composition": per-head RMSNorm and a data-dependent output gate; sigmoid reading).
+def _epi_inputs(rows=5, dv=16, seed=60):
+    rng = np.random.default_rng(seed)
+    return rng.standard_normal((rows, dv)), rng.standard_normal((rows, dv)), 0.5 + rng.random(dv)
+
+
+def pin_epilogue_constant_rows(orc):
+    """Rows of one repeated value c have RMS |c|: with eps = 0 and g = 0 the output is sign(c) w / 2."""
+    rows, dv = 4, 16
+    c = np.array([3.0, -0.25, 1e-3, -7.5])
+    o = np.repeat(c[:, None], dv, axis=1)
+    w = 0.5 + np.arange(dv) / dv
+    out = orc.output_gate_norm(o, np.zeros((rows, dv)), w, eps=0.0)
+    return float(np.abs(out - np.sign(c)[:, None] * w[None] * 0.5).max())
+
+
+def pin_epilogue_unit_rms(orc):
+    """With weight 1, a saturated gate (g = 40: sigmoid = 1 - 4e-18) and eps = 0, every output row has
+    mean square 1, and scaling o by any positive constant changes nothing."""
+    o, _, _ = _epi_inputs()
+    g = np.full_like(o, 40.0)
+    out = orc.output_gate_norm(o, g, None, eps=0.0)
+    out3 = orc.output_gate_norm(3.7 * o, g, None, eps=0.0)
+    return max(float(np.abs((out ** 2).mean(axis=1) - 1.0).max()), float(np.abs(out3 - out).max()))
+
+
+def pin_epilogue_eps_inside_root(orc):
+    """eps equal to a row's mean square halves it under the root: the output shrinks by 1 / sqrt(2)."""
+    o, g, w = _epi_inputs(rows=1)
+    ms = float((o ** 2).mean())
+    a = orc.output_gate_norm(o, g, w, eps=0.0)
+    b = orc.output_gate_norm(o, g, w, eps=ms)
+    return float(np.abs(b - a / np.sqrt(2.0)).max())
+
+
+def pin_epilogue_gate(orc):
+    """sigmoid(ln 3) = 3/4 and sigmoid(-ln 3) = 1/4 against the saturated gate; g = -800 closes it to 0;
+    the gate of channel j scales only channel j."""
+    o, _, w = _epi_inputs(rows=2)
+    ref = orc.output_gate_norm(o, np.full_like(o, 40.0), w, eps=1e-6)
+    up = orc.output_gate_norm(o, np.full_like(o, np.log(3.0)), w, eps=1e-6)
+    dn = orc.output_gate_norm(o, np.full_like(o, -np.log(3.0)), w, eps=1e-6)
+    shut = orc.output_gate_norm(o, np.full_like(o, -800.0), w, eps=1e-6)
+    g1 = np.full_like(o, 40.0)
+    g1[1, 5] = np.log(3.0)
+    one = orc.output_gate_norm(o, g1, w, eps=1e-6)
+    mask = np.ones_like(o, dtype=bool)
+    mask[1, 5] = False
+    return max(float(np.abs(up - 0.75 * ref).max()), float(np.abs(dn - 0.25 * ref).max()),
+               float(np.abs(shut).max()), float(np.abs(one[mask] - ref[mask]).max()),
+               float(abs(one[1, 5] - 0.75 * ref[1, 5])))
+
+
 PINS = {
     "exact_rational": (pin_exact_rational, 1e-13),
     "dense_transition": (pin_dense_transition, 1e-12),
@@ -321,6 +376,10 @@ PINS = {
     "contraction": (pin_contraction, 1e-12),
     "varlen": (pin_varlen, 1e-12),
     "decode_matches_prefill": (pin_decode_matches_prefill, 1e-13),
+    "epilogue_constant_rows": (pin_epilogue_constant_rows, 1e-15),
+    "epilogue_unit_rms": (pin_epilogue_unit_rms, 1e-14),
+    "epilogue_eps_inside_root": (pin_epilogue_eps_inside_root, 1e-15),
+    "epilogue_gate": (pin_epilogue_gate, 1e-15),
 }
 
 
@@ -331,9 +390,10 @@ def test_oracle_pin(name):
     assert err <= tol, f"pin {name}: error {err:.3e} > {tol:.1e}"
 
 
-@pytest.mark.parametrize("mutant", [1, 2, 3, 4, 5])
+@pytest.mark.parametrize("mutant", [1, 2, 3, 4, 5, 6, 7, 8])
 def test_pins_catch_planted_mistakes(mutant, tmp_path):
-    """Every planted mistake in the oracle's token update fails at least one pin."""
+    """Every planted mistake in the oracle's token update (1-5) or output epilogue (6-8) fails at
+    least one pin."""
     orc = oracle.Oracle(oracle_build.build_mutant(mutant, str(tmp_path)))
     failed = []
     for name, (fn, tol) in PINS.items():
