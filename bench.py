@@ -387,6 +387,30 @@ def gpu_arm(args):
     prologue = {"ms_per_step": pro_ms, "tokens_per_s": whole_job_rate(tokens_per_step, 1, world, pro_ms),
                 "flags": "l2norm_qk|gate", "vs_plain": ms_per_step / pro_ms}
 
+    # the layer's output epilogue on this step's output: RMSNorm x weight x sigmoid(g) per (token, head)
+    # row, HBM-bound (reads o and g, writes out: 3 x 2 bytes per element, 3.2 GB at this size)
+    g_out = torch.randn(o.shape, generator=torch.Generator(device=dev).manual_seed(77), device=dev).to(o.dtype)
+    w_out = torch.ones(o.shape[-1], device=dev)
+    out_e = torch.empty_like(o)
+    for _ in range(2):
+        kda.kda_output_gate_norm(o, g_out, w_out, eps=1e-6, out=out_e, stream=stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    ee0, ee1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ee0.record(stream)
+    for _ in range(args.steps):
+        kda.kda_output_gate_norm(o, g_out, w_out, eps=1e-6, out=out_e, stream=stream)
+    ee1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    epi_ms = max_over_ranks(ee0.elapsed_time(ee1)) / args.steps
+    epi_bytes = 3 * o.numel() * o.element_size() + w_out.numel() * 4
+    epilogue = {"kernel": "kda_output_gate_norm_kernel", "ms_per_call": epi_ms,
+                "tokens_per_s": whole_job_rate(tokens_per_step, 1, world, epi_ms),
+                "bytes_per_call": epi_bytes, "hbm_gbs": epi_bytes / (epi_ms * 1e6),
+                "frac": epi_bytes / (epi_ms * 1e6) / peaks["hbm_gbs"]}
+    del g_out, out_e
+
     decode = None
     if not args.no_decode:
         decode = decode_bench(args, dev, stream, peaks, barrier, max_over_ranks)
@@ -399,7 +423,7 @@ def gpu_arm(args):
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config_dict(T),
             "roofline": roofline, "operator_roofline": operator_roofline, "cpu_baseline": cpu_baseline,
-            "e2e": e2e, "gpu_launches": len(traces), "clocks": clk, "prologue": prologue, "decode": decode,
+            "e2e": e2e, "gpu_launches": len(traces), "clocks": clk, "prologue": prologue, "epilogue": epilogue, "decode": decode,
             "kernels": kst, "peaks": peaks}
     if rank == 0:
         print(json.dumps(line), flush=True)

@@ -59,7 +59,8 @@ enum {
     KDA_ERR_CUDA = -8,                /* a CUDA runtime call failed (launch or query) */
     KDA_ERR_TIMEOUT = -9,             /* device-detected: a bounded wait gave up */
     KDA_ERR_ALIASING = -10,           /* o overlaps an input, or h_T partially overlaps h0 */
-    KDA_ERR_BAD_SLOT = -11            /* device-detected: a state-pool slot index is out of range */
+    KDA_ERR_BAD_SLOT = -11,           /* device-detected: a state-pool slot index is out of range */
+    KDA_ERR_BAD_VALUE = -12           /* a scalar argument is out of range (eps < 0 or NaN) */
 };
 
 /* Bytes of device workspace kda_chunk_fwd needs for these sizes (dtype-dependent).  It holds
@@ -187,6 +188,22 @@ KDA_API int kda_decode_multi_ex(const void *q, const void *k, const void *v, con
                                 const int32_t *slot_out, int N, int Tq, int H, int dk, int dv, kda_dtype dtype,
                                 void *o, int *status, unsigned flags, const float *A_log, const float *dt_bias,
                                 void *stream);
+
+/* The KDA layer's output epilogue (Kimi Linear summary page, section "Kimi Linear model
+ * composition": a per-head RMSNorm and a data-dependent output gate ahead of the output
+ * projection; the page does not name the gate's activation, read here as the logistic sigmoid).
+ * For every row r = (token, head) of length dv:
+ *     out[r, j] = o[r, j] / sqrt(mean_j o[r, j]^2 + eps) * weight[j] * sigmoid(g[r, j])
+ *   o, g, out : [n_tok, H, dv] dtype; o is the operator output (kda_chunk_fwd / decode), g the
+ *               output-gate projection of the same tokens.  out == o (exact alias) runs in place;
+ *               any other overlap of out with o, g or weight is rejected.
+ *   weight    : [dv] fp32, shared by all heads, or NULL for ones.
+ *   eps       : >= 0, added to the mean square inside the root (KDA_ERR_BAD_VALUE otherwise).
+ * fp32 arithmetic; the result is rounded to dtype.  Supported: dv in {64, 128}, dtype BF16 or F32.
+ * o, g, out (and weight) 16-byte aligned.  n_tok = 0 enqueues nothing (pointers may be NULL).
+ * Returns KDA_OK once the work is enqueued on `stream`. */
+KDA_API int kda_output_gate_norm(const void *o, const void *g, const float *weight, float eps, int n_tok, int H,
+                                 int dv, kda_dtype dtype, void *out, void *stream);
 
 /* Synchronizes `stream`, reads the device status word kept in `workspace` by the last
  * kda_chunk_fwd that used it, clears it, and returns it (KDA_OK, KDA_ERR_BAD_SEQLENS or

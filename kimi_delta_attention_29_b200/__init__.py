@@ -166,6 +166,22 @@ def kda_decode_multi(q, k, v, log_alpha, beta, S_pool, slot_in=None, slot_out=No
     return o
 
 
+def kda_output_gate_norm(o, g, weight=None, eps: float = 1e-6, out=None, stream=None):
+    """The layer's output epilogue: out = RMSNorm(o) over the head dim (dv) x weight[dv] x sigmoid(g),
+    per (token, head) row.  o, g [..., H, dv] contiguous, bf16 or fp32 (same dtype); weight [dv] fp32 or
+    None; out=o runs in place.  Returns out."""
+    torch = _torch()
+    H, dv = o.shape[-2], o.shape[-1]
+    n_tok = o.numel() // (H * dv) if H * dv else 0
+    if out is None:
+        out = torch.empty_like(o)
+    rc = _lib.load().kda_output_gate_norm(_ptr(o), _ptr(g), _ptr(weight), float(eps), n_tok, H, dv,
+                                          _dtype_code(o.dtype), _ptr(out), _stream(stream, o.device))
+    if rc != _lib.KDA_OK:
+        raise KdaError(rc, "kda_output_gate_norm")
+    return out
+
+
 def kda_get_status(workspace, stream=None) -> int:
     buf = workspace.buf if isinstance(workspace, Workspace) else workspace
     return int(_lib.load().kda_get_status(_ptr(buf), _stream(stream, buf.device)))

@@ -24,6 +24,7 @@ KDA_ERR_CUDA = -8
 KDA_ERR_TIMEOUT = -9
 KDA_ERR_ALIASING = -10
 KDA_ERR_BAD_SLOT = -11
+KDA_ERR_BAD_VALUE = -12
 
 KDA_F32 = 0
 KDA_BF16 = 1
@@ -34,11 +35,12 @@ KDA_PROLOGUE_GATE = 2
 
 # Every entry point include/kda.h declares.
 EXPORTED = ("kda_chunk_fwd_workspace_size", "kda_chunk_fwd", "kda_chunk_fwd_ex", "kda_decode_step",
-            "kda_decode_multi", "kda_decode_multi_ex", "kda_get_status", "kda_status_string", "kda_version",
-            "kda_trace_begin", "kda_trace_end")
+            "kda_decode_multi", "kda_decode_multi_ex", "kda_output_gate_norm", "kda_get_status",
+            "kda_status_string", "kda_version", "kda_trace_begin", "kda_trace_end")
 
 KERNEL_NAMES = {0: "kda_chunk_table_kernel", 1: "kda_tc_prep_kernel", 2: "kda_tc_state_kernel",
-                3: "kda_prefill_simt_kernel", 4: "kda_decode_kernel", 5: "kda_decode_multi_kernel"}
+                3: "kda_prefill_simt_kernel", 4: "kda_decode_kernel", 5: "kda_decode_multi_kernel",
+                6: "kda_output_gate_norm_kernel"}
 
 _lib = None
 
@@ -66,6 +68,8 @@ def load() -> ctypes.CDLL:
     lib.kda_chunk_fwd_ex.restype = i
     lib.kda_decode_multi_ex.argtypes = [vp, vp, vp, fp, fp, fp, i, ip, ip, i, i, i, i, i, i, vp, ip, u, fp, fp, vp]
     lib.kda_decode_multi_ex.restype = i
+    lib.kda_output_gate_norm.argtypes = [vp, vp, fp, ctypes.c_float, i, i, i, i, vp, vp]
+    lib.kda_output_gate_norm.restype = i
     lib.kda_get_status.argtypes = [vp, vp]
     lib.kda_get_status.restype = i
     lib.kda_status_string.argtypes = [i]

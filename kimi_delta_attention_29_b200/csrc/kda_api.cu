@@ -121,6 +121,7 @@ const char *kda_status_string(int status) {
         case KDA_ERR_TIMEOUT: return "KDA_ERR_TIMEOUT: a bounded device wait gave up";
         case KDA_ERR_ALIASING: return "KDA_ERR_ALIASING: an output overlaps an input";
         case KDA_ERR_BAD_SLOT: return "KDA_ERR_BAD_SLOT: a state-pool slot index is out of range";
+        case KDA_ERR_BAD_VALUE: return "KDA_ERR_BAD_VALUE: a scalar argument is out of range";
         default: return "KDA: unknown status";
     }
 }
@@ -282,6 +283,29 @@ int kda_decode_multi_ex(const void *q, const void *k, const void *v, const float
     const kda::Prologue pro{flags, A_log, dt_bias};
     cudaError_t e = kda::launch_decode_multi(q, k, v, log_alpha, beta, S_pool, num_slots, slot_in, slot_out, N, Tq,
                                              H, dk, dtype, o, status, pro, static_cast<cudaStream_t>(stream_));
+    return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+int kda_output_gate_norm(const void *o, const void *g, const float *weight, float eps, int n_tok, int H, int dv,
+                         kda_dtype dtype, void *out, void *stream_) {
+    if (dtype != KDA_F32 && dtype != KDA_BF16) return KDA_ERR_BAD_DTYPE;
+    if (n_tok < 0 || H <= 0 || dv <= 0) return KDA_ERR_BAD_SHAPE;
+    const int64_t rows = (int64_t)n_tok * H;
+    if (rows * dv > ((int64_t)1 << 40)) return KDA_ERR_BAD_SHAPE;
+    if (dv != 64 && dv != 128) return KDA_ERR_UNSUPPORTED;
+    if (!(eps >= 0.f) || eps > 3.0e38f) return KDA_ERR_BAD_VALUE;
+    if (rows == 0) return KDA_OK;
+    if (!o || !g || !out) return KDA_ERR_NULL_ARG;
+    const void *ptrs[] = {o, g, out, weight};
+    for (const void *p : ptrs)
+        if (p && !aligned16(p)) return KDA_ERR_MISALIGNED;
+    const size_t bytes = (size_t)rows * dv * elem_size(dtype);
+    const Range ro = range_of(o, bytes), rg = range_of(g, bytes), rw = range_of(weight, weight ? (size_t)dv * 4 : 0),
+                rout = range_of(out, bytes);
+    if (out != o && overlaps(rout, ro)) return KDA_ERR_ALIASING;
+    if (overlaps(rout, rg) || overlaps(rout, rw)) return KDA_ERR_ALIASING;
+    cudaError_t e = kda::launch_output_gate_norm(o, g, weight, eps, rows, dv, dtype, out,
+                                                 static_cast<cudaStream_t>(stream_));
     return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 

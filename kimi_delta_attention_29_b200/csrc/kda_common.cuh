@@ -34,14 +34,6 @@ struct Prologue {
     const float *dt_bias;  // [H, dk] or nullptr
 };
 constexpr float kNormEps = 1e-6f;  // inside the square root of the L2 normalisation
-__device__ __forceinline__ float gate_log_decay(float g, float a, float b) {
-    const float x = g + b;
-    // -a * softplus(x) in the overflow-free split max(x, 0) + ln(1 + e^{-|x|}).  The second term
-    // lies in (0, ln 2] and its argument 1 + e^{-|x|} in (1, 2], where the documented error
-    // bounds of the __expf / __logf intrinsics keep its absolute error below 1e-6: far under what
-    // the bf16 inputs and the fp32 cumulative gates carry, at a fraction of the libm pair's cost.
-    return -a * (fmaxf(x, 0.f) + __logf(1.f + __expf(-fabsf(x))));
-}
 
 // Strongest per-step decay the chunked prefills apply, as log2(alpha).  A step whose decay is
 // stronger keeps 2^{clamp} of the state instead of less, a change below 2^{clamp} |S| where the
@@ -64,6 +56,24 @@ __device__ __forceinline__ float ex2f(float x) {
     return y;
 }
 
+// log2(x) by the hardware approximation (PTX lg2.approx.ftz.f32: absolute error ~2^-22 on [0.5, 2]).
+__device__ __forceinline__ float lg2f(float x) {
+    float y;
+    asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// The prologue's log decay -a * softplus(g + b), a = exp(A_log[h]), b = dt_bias[h, c], in the
+// overflow-free split softplus(x) = max(x, 0) + ln(1 + e^{-|x|}).  The second term lies in
+// (0, ln 2]: e^{-|x|} by ex2 and ln(1 + t), t in (0, 1], by lg2 on (1, 2], where both hardware
+// approximations keep the absolute error below 1e-6 (far under what the bf16 inputs and the fp32
+// cumulative gates carry).
+__device__ __forceinline__ float gate_log_decay(float g, float a, float b) {
+    const float x = g + b;
+    constexpr float kLn2 = 0.6931471805599453f;
+    return -a * fmaf(lg2f(1.f + ex2f(-fabsf(x) * kLog2e)), kLn2, fmaxf(x, 0.f));
+}
+
 // Chunk length shared by every kernel.
 constexpr int kChunk = 64;
 
@@ -73,7 +83,7 @@ constexpr int kChunk = 64;
 namespace kda {
 // Kernel ids reported by kda_trace_end.
 enum KernelId { kKernChunkTable = 0, kKernTcPrep = 1, kKernTcState = 2, kKernSimt = 3, kKernDecode = 4,
-                kKernDecodeMulti = 5 };
+                kKernDecodeMulti = 5, kKernOutputGateNorm = 6 };
 // Diagnostics: bracket one kernel launch with trace events when kda_trace_begin is active.
 void trace_before(int kernel_id, cudaStream_t stream);
 void trace_after(cudaStream_t stream);
@@ -82,6 +92,8 @@ cudaError_t launch_decode(const void *q, const void *k, const void *v, const flo
                           const float *beta, float *S, int N, int H, int dk, int dv, kda_dtype dtype,
                           void *o, cudaStream_t stream);
 
+cudaError_t launch_output_gate_norm(const void *o, const void *g, const float *weight, float eps, int64_t rows,
+                                    int dv, kda_dtype dtype, void *out, cudaStream_t stream);
 cudaError_t launch_decode_multi(const void *q, const void *k, const void *v, const float *log_alpha,
                                 const float *beta, float *S_pool, int num_slots, const int32_t *slot_in,
                                 const int32_t *slot_out, int N, int Tq, int H, int dk, kda_dtype dtype, void *o,

@@ -39,7 +39,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 def test_status_strings_and_version(lib):
     assert lib.kda_version() >= 100
-    for code in range(0, -12, -1):
+    for code in range(0, -13, -1):
         s = _lib.status_string(code)
         assert s.startswith("KDA_")
     assert "unknown" in _lib.status_string(-999)
@@ -161,3 +161,30 @@ def test_prologue_arguments_rejected_on_host(lib):
     rc = lib.kda_decode_multi_ex(c(A), c(2 * A), c(3 * A), c(4 * A), c(5 * A), c(6 * A), 8, None, None, 4, 3, 2, 128,
                                  128, _lib.KDA_BF16, c(7 * A), None, 8, None, None, None)
     assert rc == _lib.KDA_ERR_UNSUPPORTED
+
+
+def test_output_gate_norm_rejects_on_host(lib):
+    """Every rejection returns before a launch; no call here reaches the kernel."""
+    c, f = ctypes.c_void_p, ctypes.c_float
+    fn = lib.kda_output_gate_norm
+
+    def call(o=A, g=2 * A, w=None, eps=1e-6, n_tok=4, H=2, dv=128, dtype=_lib.KDA_BF16, out=3 * A):
+        return fn(c(o) if o else None, c(g) if g else None, c(w) if w else None, f(eps), n_tok, H, dv, dtype,
+                  c(out) if out else None, None)
+
+    assert call(dtype=7) == _lib.KDA_ERR_BAD_DTYPE
+    assert call(n_tok=-1) == _lib.KDA_ERR_BAD_SHAPE
+    assert call(H=0) == _lib.KDA_ERR_BAD_SHAPE
+    assert call(dv=96) == _lib.KDA_ERR_UNSUPPORTED
+    assert call(eps=-1e-3) == _lib.KDA_ERR_BAD_VALUE
+    assert call(eps=float("nan")) == _lib.KDA_ERR_BAD_VALUE
+    assert call(eps=float("inf")) == _lib.KDA_ERR_BAD_VALUE
+    assert call(n_tok=0, o=None, g=None, out=None) == _lib.KDA_OK           # empty: nothing enqueued
+    assert call(o=None) == _lib.KDA_ERR_NULL_ARG
+    assert call(g=None) == _lib.KDA_ERR_NULL_ARG
+    assert call(out=None) == _lib.KDA_ERR_NULL_ARG
+    assert call(o=A + 8) == _lib.KDA_ERR_MISALIGNED
+    assert call(w=5 * A + 4) == _lib.KDA_ERR_MISALIGNED
+    assert call(out=A + 256) == _lib.KDA_ERR_ALIASING                        # partial overlap with o
+    assert call(out=2 * A) == _lib.KDA_ERR_ALIASING                          # out is g
+    assert call(w=3 * A + 64) == _lib.KDA_ERR_ALIASING                       # weight inside out
