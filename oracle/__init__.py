@@ -37,6 +37,9 @@ def _bind(path: str):
     lib.kda_oracle_decode_step.restype = i
     lib.kda_oracle_prologue.argtypes = [dp, dp, dp, ctypes.c_int64, i, i, ctypes.c_uint, ctypes.c_double, dp, dp]
     lib.kda_oracle_prologue.restype = i
+    lib.kda_oracle_recurrent_bwd.argtypes = [dp, dp, dp, dp, dp, dp, ip, i, i, i, i, i, i, dp, dp, dp, dp, dp, dp,
+                                             dp, dp]
+    lib.kda_oracle_recurrent_bwd.restype = i
     lib.kda_oracle_output_gate_norm.argtypes = [dp, dp, dp, ctypes.c_int64, i, ctypes.c_double, dp]
     lib.kda_oracle_output_gate_norm.restype = i
     lib.kda_oracle_num_threads.restype = i
@@ -88,6 +91,25 @@ class Oracle:
         if rc != 0:
             raise ValueError(f"kda_oracle_recurrent rejected its arguments (rc={rc})")
         return o, hT
+
+    def recurrent_bwd(self, q, k, v, log_alpha, beta, h0=None, cu_seqlens=None, do=None, dhT=None):
+        """Gradients of the token-by-token map for upstream gradients do [B,T,H,dv] (dL/do) and dhT
+        [N,H,dk,dv] (dL/dh_T, None = 0).  Returns a dict of float64 arrays: dq, dk, dv, dlog_alpha,
+        dbeta and dh0 (the gradient for the initial states, zero states when h0 is None)."""
+        q, k, v, la, bt, dout = (_f64(x) for x in (q, k, v, log_alpha, beta, do))
+        B, T, H, dk, dv, N, cu = _shapes(q, v, cu_seqlens)
+        h0a = None if h0 is None else _f64(h0)
+        dhTa = None if dhT is None else _f64(dhT)
+        g = {"dq": np.zeros_like(q), "dk": np.zeros_like(k), "dv": np.zeros_like(v), "dlog_alpha": np.zeros_like(la),
+             "dbeta": np.zeros_like(bt), "dh0": np.zeros((N, H, dk, dv), np.float64)}
+        rc = self.lib.kda_oracle_recurrent_bwd(
+            _ptr(q), _ptr(k), _ptr(v), _ptr(la), _ptr(bt), _ptr(h0a),
+            None if cu is None else cu.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)),
+            N, B, T, H, dk, dv, _ptr(dout), _ptr(dhTa), _ptr(g["dq"]), _ptr(g["dk"]), _ptr(g["dv"]),
+            _ptr(g["dlog_alpha"]), _ptr(g["dbeta"]), _ptr(g["dh0"]))
+        if rc != 0:
+            raise ValueError(f"kda_oracle_recurrent_bwd rejected its arguments (rc={rc})")
+        return g
 
     def chunkwise(self, q, k, v, log_alpha, beta, h0=None, cu_seqlens=None, chunk=64):
         """Chunkwise WY / UT-transform restatement of the same map (float64)."""
@@ -175,6 +197,10 @@ def chunkwise(*args, **kw):
 
 def prologue(*args, **kw):
     return default().prologue(*args, **kw)
+
+
+def recurrent_bwd(*args, **kw):
+    return default().recurrent_bwd(*args, **kw)
 
 
 def output_gate_norm(*args, **kw):

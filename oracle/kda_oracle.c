@@ -43,8 +43,8 @@
 
 #include "kda_oracle.h"
 
-/* KDA_ORACLE_MUTANT selects a deliberately wrong variant of the token update (1..5) or
- * of the output epilogue (6..8).  It exists only so that a test can show that the pins
+/* KDA_ORACLE_MUTANT selects a deliberately wrong variant of the token update (1..5), of the
+ * output epilogue (6..8) or of the backward recurrence (9..11).  It exists only so that a test can show that the pins
  * catch plausible mistakes; the library the tests trust is built with the default value 0. */
 #ifndef KDA_ORACLE_MUTANT
 #define KDA_ORACLE_MUTANT 0
@@ -169,6 +169,112 @@ int kda_oracle_recurrent(const double *q, const double *k, const double *v,
         }
         if (hT) memcpy(hT + soff, S, sizeof(double) * (size_t)dk * dv);
         free(S);
+        free(scratch);
+    }
+    free(starts);
+    free(lens);
+    return KDA_ORACLE_OK;
+}
+
+/* Reverse-mode derivative of kda_oracle_recurrent: the adjoint of the token recurrence taken step
+ * by step backwards in time.  With dS = dL/dS_t (the upstream gradient of the state after token t)
+ * and S' = Diag(alpha) S_{t-1}, a = S'^T k, u = beta (v - a), S_t = S' + k u^T, o_t = S_t^T q:
+ *   dq = S_t do;  dS += q do^T;  du = dS^T k;  dk = dS u + S' da with da = -beta du;
+ *   dv = beta du;  dbeta = du . (v - a);  dS' = dS + k da^T;
+ *   dlog_alpha_i = alpha_i sum_j S_{t-1}[i][j] dS'[i][j];  dS <- Diag(alpha) dS'.
+ * dh0 is dS after the first token.  Every state of a sequence is kept (test sizes only). */
+int kda_oracle_recurrent_bwd(const double *q, const double *k, const double *v, const double *log_alpha,
+                             const double *beta, const double *h0, const int64_t *cu_seqlens, int num_seqs, int B,
+                             int T, int H, int dk, int dv, const double *dout, const double *dhT, double *dq,
+                             double *dk_out, double *dv_out, double *dla, double *dbeta, double *dh0) {
+    if (!q || !k || !v || !log_alpha || !beta || !dout || !dq || !dk_out || !dv_out || !dla || !dbeta)
+        return KDA_ORACLE_BAD_ARG;
+    if (B <= 0 || T < 0 || H <= 0 || dk <= 0 || dv <= 0 || num_seqs <= 0) return KDA_ORACLE_BAD_ARG;
+    int64_t *starts = (int64_t *)malloc(sizeof(int64_t) * (size_t)num_seqs);
+    int64_t *lens = (int64_t *)malloc(sizeof(int64_t) * (size_t)num_seqs);
+    int rc = resolve_sequences(cu_seqlens, num_seqs, B, T, starts, lens);
+    if (rc != KDA_ORACLE_OK) { free(starts); free(lens); return rc; }
+    const size_t sd = (size_t)dk * dv;
+    const int64_t units = (int64_t)num_seqs * H;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t un = 0; un < units; ++un) {
+        const int n = (int)(un / H), h = (int)(un % H);
+        const int64_t t0 = starts[n], len = lens[n];
+        const size_t soff = ((size_t)n * H + h) * sd;
+        double *St = (double *)malloc(sizeof(double) * sd * (size_t)(len + 1));  /* S_0 .. S_len */
+        double *dS = (double *)malloc(sizeof(double) * sd);
+        double *dSp = (double *)malloc(sizeof(double) * sd);
+        double *scratch = (double *)malloc(sizeof(double) * (size_t)dv * 4);
+        double *a = scratch + dv, *du = scratch + 2 * (size_t)dv, *da = scratch + 3 * (size_t)dv;
+        if (h0) memcpy(St, h0 + soff, sizeof(double) * sd);
+        else memset(St, 0, sizeof(double) * sd);
+        for (int64_t s = 0; s < len; ++s) {
+            const int64_t t = t0 + s;
+            memcpy(St + (size_t)(s + 1) * sd, St + (size_t)s * sd, sizeof(double) * sd);
+            kda_token(St + (size_t)(s + 1) * sd, row(q, t, H, h, dk), row(k, t, H, h, dk), row(v, t, H, h, dv),
+                      row(log_alpha, t, H, h, dk), beta[(size_t)t * H + h], dk, dv, NULL, scratch);
+        }
+        if (dhT) memcpy(dS, dhT + soff, sizeof(double) * sd);
+        else memset(dS, 0, sizeof(double) * sd);
+        for (int64_t s = len - 1; s >= 0; --s) {
+            const int64_t t = t0 + s;
+            const double *Sp = St + (size_t)s * sd, *Sn = St + (size_t)(s + 1) * sd;
+            const double *qt = row(q, t, H, h, dk), *kt = row(k, t, H, h, dk), *vt = row(v, t, H, h, dv);
+            const double *lat = row(log_alpha, t, H, h, dk), *dot = row(dout, t, H, h, dv);
+            const double bt = beta[(size_t)t * H + h];
+            double *dqt = dq + ((size_t)t * H + h) * dk, *dkt = dk_out + ((size_t)t * H + h) * dk;
+            double *dvt = dv_out + ((size_t)t * H + h) * dv, *dlat = dla + ((size_t)t * H + h) * dk;
+            for (int i = 0; i < dk; ++i) {                         /* dq = S_t do;  dS += q do^T */
+                double acc = 0.0;
+                for (int j = 0; j < dv; ++j) {
+                    acc += Sn[(size_t)i * dv + j] * dot[j];
+                    dS[(size_t)i * dv + j] += qt[i] * dot[j];
+                }
+                dqt[i] = acc;
+            }
+            for (int j = 0; j < dv; ++j) { a[j] = 0.0; du[j] = 0.0; }
+            for (int i = 0; i < dk; ++i) {                         /* a = S'^T k;  du = dS^T k */
+                const double al = exp(lat[i]);
+                for (int j = 0; j < dv; ++j) {
+                    a[j] += al * Sp[(size_t)i * dv + j] * kt[i];
+                    du[j] += dS[(size_t)i * dv + j] * kt[i];
+                }
+            }
+            double db = 0.0;
+            for (int j = 0; j < dv; ++j) {
+                db += du[j] * (vt[j] - a[j]);
+                dvt[j] = bt * du[j];
+                da[j] = -bt * du[j];
+            }
+#if KDA_ORACLE_MUTANT == 11
+            db = -db;                                              /* planted: sign of dbeta */
+#endif
+            dbeta[(size_t)t * H + h] = db;
+            for (int i = 0; i < dk; ++i) {
+                const double al = exp(lat[i]);
+                double acc = 0.0, accl = 0.0;
+                for (int j = 0; j < dv; ++j) {
+                    const double u = bt * (vt[j] - a[j]);
+                    acc += dS[(size_t)i * dv + j] * u;
+#if KDA_ORACLE_MUTANT != 9
+                    acc += al * Sp[(size_t)i * dv + j] * da[j];    /* dk += S' da */
+#endif
+                    dSp[(size_t)i * dv + j] = dS[(size_t)i * dv + j] + kt[i] * da[j];
+                    accl += Sp[(size_t)i * dv + j] * dSp[(size_t)i * dv + j];
+                }
+                dkt[i] = acc;
+#if KDA_ORACLE_MUTANT == 10
+                dlat[i] = accl;                                    /* planted: alpha factor dropped */
+#else
+                dlat[i] = al * accl;
+#endif
+                for (int j = 0; j < dv; ++j) dS[(size_t)i * dv + j] = al * dSp[(size_t)i * dv + j];
+            }
+        }
+        if (dh0) memcpy(dh0 + soff, dS, sizeof(double) * sd);
+        free(St);
+        free(dS);
+        free(dSp);
         free(scratch);
     }
     free(starts);

@@ -27,6 +27,15 @@ int kda_oracle_chunkwise(const double *q, const double *k, const double *v,
                          const int64_t *cu_seqlens, int num_seqs, int B, int T, int H,
                          int dk, int dv, int chunk, double *o, double *hT);
 
+/* Reverse-mode derivative of kda_oracle_recurrent (the adjoint recurrence, backwards in time).
+ * dout: dL/do [B,T,H,dv]; dhT: dL/dh_T [N,H,dk,dv] or NULL (zero).  Writes dq, dk [B,T,H,dk],
+ * dv [B,T,H,dv], dla [B,T,H,dk], dbeta [B,T,H] and dh0 [N,H,dk,dv] (NULL = not wanted); h0 NULL =
+ * zero initial states. */
+int kda_oracle_recurrent_bwd(const double *q, const double *k, const double *v, const double *log_alpha,
+                             const double *beta, const double *h0, const int64_t *cu_seqlens, int num_seqs, int B,
+                             int T, int H, int dk, int dv, const double *dout, const double *dhT, double *dq,
+                             double *dk_out, double *dv_out, double *dla, double *dbeta, double *dh0);
+
 /* One recurrent step for N*H independent states S [N, H, dk, dv], in place.
  * q, k, log_alpha: [N, H, dk]; v, o: [N, H, dv]; beta: [N, H]. */
 int kda_oracle_decode_step(const double *q, const double *k, const double *v,

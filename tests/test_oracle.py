@@ -359,6 +359,60 @@ def pin_epilogue_gate(orc):
                float(abs(one[1, 5] - 0.75 * ref[1, 5])))
 
 
+# ------------------------------------------------------------------------------------- backward
+def _fd_check(orc, cu_seqlens, use_h0, use_dhT, seed):
+    """Central finite differences of L = <o, W_o> + <h_T, W_h> on a tiny case against the backward
+    oracle's gradients for every input element (step 1e-5: truncation ~1e-10, rounding ~1e-11)."""
+    rng = np.random.default_rng(seed)
+    B, T, H, dk, dv = 1, 7, 2, 3, 4
+    x = {"q": rng.standard_normal((B, T, H, dk)), "k": 0.5 * rng.standard_normal((B, T, H, dk)),
+         "v": rng.standard_normal((B, T, H, dv)), "log_alpha": -rng.random((B, T, H, dk)),
+         "beta": rng.random((B, T, H))}
+    N = 1 if cu_seqlens is None else len(cu_seqlens) - 1
+    if use_h0:
+        x["h0"] = rng.standard_normal((N, H, dk, dv))
+    W_o = rng.standard_normal((B, T, H, dv))
+    W_h = rng.standard_normal((N, H, dk, dv)) if use_dhT else None
+
+    def loss(**kw):
+        o, hT = orc.recurrent(kw["q"], kw["k"], kw["v"], kw["log_alpha"], kw["beta"], kw.get("h0"), cu_seqlens)
+        return float((o * W_o).sum() + (0.0 if W_h is None else (hT * W_h).sum()))
+
+    g = orc.recurrent_bwd(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], x.get("h0"), cu_seqlens, W_o, W_h)
+    names = {"q": "dq", "k": "dk", "v": "dv", "log_alpha": "dlog_alpha", "beta": "dbeta", "h0": "dh0"}
+    err = 0.0
+    for name, a in x.items():
+        fd = np.zeros_like(a)
+        for idx in np.ndindex(a.shape):
+            kw = dict(x)
+            ap, am = a.copy(), a.copy()
+            ap[idx] += 1e-5
+            am[idx] -= 1e-5
+            kw[name] = ap
+            lp = loss(**kw)
+            kw[name] = am
+            fd[idx] = (lp - loss(**kw)) / 2e-5
+        err = max(err, float(np.abs(fd - g[names[name]]).max() / max(np.abs(fd).max(), 1e-300)))
+    if not use_h0:  # dL/dh0 at zero initial states, by differences in h0 around zero
+        h0z = np.zeros((N, H, dk, dv))
+        fd = np.zeros_like(h0z)
+        for idx in np.ndindex(h0z.shape):
+            ap, am = h0z.copy(), h0z.copy()
+            ap[idx] += 1e-5
+            am[idx] -= 1e-5
+            fd[idx] = (loss(**dict(x, h0=ap)) - loss(**dict(x, h0=am))) / 2e-5
+        err = max(err, float(np.abs(fd - g["dh0"]).max() / max(np.abs(fd).max(), 1e-300)))
+    return err
+
+
+def pin_backward_finite_differences(orc):
+    return _fd_check(orc, None, use_h0=True, use_dhT=True, seed=70)
+
+
+def pin_backward_varlen_zero_start(orc):
+    return _fd_check(orc, np.array([0, 3, 3, 7]), use_h0=False, use_dhT=False, seed=71)
+
+
 PINS = {
     "exact_rational": (pin_exact_rational, 1e-13),
     "dense_transition": (pin_dense_transition, 1e-12),
@@ -380,6 +434,8 @@ PINS = {
     "epilogue_unit_rms": (pin_epilogue_unit_rms, 1e-14),
     "epilogue_eps_inside_root": (pin_epilogue_eps_inside_root, 1e-15),
     "epilogue_gate": (pin_epilogue_gate, 1e-15),
+    "backward_finite_differences": (pin_backward_finite_differences, 1e-8),
+    "backward_varlen_zero_start": (pin_backward_varlen_zero_start, 1e-8),
 }
 
 
@@ -390,10 +446,10 @@ def test_oracle_pin(name):
     assert err <= tol, f"pin {name}: error {err:.3e} > {tol:.1e}"
 
 
-@pytest.mark.parametrize("mutant", [1, 2, 3, 4, 5, 6, 7, 8])
+@pytest.mark.parametrize("mutant", [1, 2, 3, 4, 5, 6, 7, 8, 9, 10, 11])
 def test_pins_catch_planted_mistakes(mutant, tmp_path):
-    """Every planted mistake in the oracle's token update (1-5) or output epilogue (6-8) fails at
-    least one pin."""
+    """Every planted mistake in the oracle's token update (1-5), output epilogue (6-8) or backward
+    recurrence (9-11) fails at least one pin."""
     orc = oracle.Oracle(oracle_build.build_mutant(mutant, str(tmp_path)))
     failed = []
     for name, (fn, tol) in PINS.items():
