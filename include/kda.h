@@ -189,6 +189,33 @@ KDA_API int kda_decode_multi_ex(const void *q, const void *k, const void *v, con
                                 void *o, int *status, unsigned flags, const float *A_log, const float *dt_bias,
                                 void *stream);
 
+/* Bytes of device workspace kda_chunk_bwd needs (dk = dv = D): the status block, the varlen chunk
+ * table and, per (chunk, head), the state-pass record (chunk-start state, state gradient and four
+ * 64 x D tiles: 2 D^2 + 256 D floats, 256 KB at D = 128).  Returns 0 for unsupported sizes. */
+KDA_API size_t kda_chunk_bwd_workspace_size(int B, int T, int H, int dk, int dv, int num_seqs, int chunk_size,
+                                            kda_dtype dtype);
+
+/* Chunkwise backward of kda_chunk_fwd (section "Chunkwise parallel algorithm": the same chunks, UT
+ * transform and state passing, differentiated in reverse; the page notes the design's value for
+ * training).  Inputs are kda_chunk_fwd's, with the same shapes, dtype and conventions, plus
+ *   do        : [B, T, H, dv] dtype, dL/do
+ *   dh_T      : [N, H, dk, dv] fp32, dL/dh_T, or NULL (zero)
+ * Outputs (caller-allocated, each must not overlap any input, another output or the workspace):
+ *   dq, dk    : [B, T, H, dk] dtype          dv : [B, T, H, dv] dtype
+ *   dlog_alpha: [B, T, H, dk] fp32           dbeta : [B, T, H] fp32
+ *   dh0       : [N, H, dk, dv] fp32, or NULL (not wanted); with h0 = NULL it is the gradient at
+ *               zero initial states.
+ * fp32 arithmetic on CUDA cores (a state pass per (sequence, head, 16 value columns), then one CTA
+ * per (chunk, head, 32 key channels)); deterministic.  A step whose log gate is below -15 ln 2 is
+ * applied as 2^-15, as in the CUDA-core forward, and its dlog_alpha is 0.  Supported: dk = dv in
+ * {64, 128}, dtype BF16 or F32, chunk_size 64.  Device-detected errors (bad cu_seqlens) go to the
+ * workspace status word (kda_get_status). */
+KDA_API int kda_chunk_bwd(const void *q, const void *k, const void *v, const float *log_alpha, const float *beta,
+                          const float *h0, const int32_t *cu_seqlens, int num_seqs, int B, int T, int H, int dk,
+                          int dv, int chunk_size, kda_dtype dtype, const void *do_, const float *dh_T, void *dq,
+                          void *dk_out, void *dv_out, float *dlog_alpha, float *dbeta, float *dh0, void *workspace,
+                          size_t workspace_bytes, void *stream);
+
 /* The KDA layer's output epilogue (Kimi Linear summary page, section "Kimi Linear model
  * composition": a per-head RMSNorm and a data-dependent output gate ahead of the output
  * projection; the page does not name the gate's activation, read here as the logistic sigmoid).

@@ -166,6 +166,33 @@ def kda_decode_multi(q, k, v, log_alpha, beta, S_pool, slot_in=None, slot_out=No
     return o
 
 
+def kda_chunk_bwd(q, k, v, log_alpha, beta, h0=None, cu_seqlens=None, do=None, dh_T=None, want_dh0: bool = True,
+                  chunk_size: int = 64, workspace=None, stream=None):
+    """Gradients of kda_chunk_fwd for upstream do [B,T,H,dv] (input dtype) and dh_T [N,H,dk,dv] fp32 (None:
+    zero).  Returns a dict: dq, dk [B,T,H,dk] and dv [B,T,H,dv] in the input dtype, dlog_alpha [B,T,H,dk]
+    and dbeta [B,T,H] fp32, dh0 [N,H,dk,dv] fp32 (None unless want_dh0)."""
+    torch = _torch()
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    N = B if cu_seqlens is None else cu_seqlens.numel() - 1
+    code = _dtype_code(q.dtype)
+    lib = _lib.load()
+    need = lib.kda_chunk_bwd_workspace_size(B, T, H, dk, dv, N, chunk_size, code)
+    if need == 0:
+        raise KdaError(_lib.KDA_ERR_UNSUPPORTED, "kda_chunk_bwd_workspace_size")
+    ws = workspace if workspace is not None else torch.empty(need, dtype=torch.uint8, device=q.device)
+    g = {"dq": torch.empty_like(q), "dk": torch.empty_like(k), "dv": torch.empty_like(v),
+         "dlog_alpha": torch.empty_like(log_alpha), "dbeta": torch.empty_like(beta),
+         "dh0": torch.empty((N, H, dk, dv), dtype=torch.float32, device=q.device) if want_dh0 else None}
+    rc = lib.kda_chunk_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(h0), _ptr(cu_seqlens), N, B, T,
+                           H, dk, dv, chunk_size, code, _ptr(do), _ptr(dh_T), _ptr(g["dq"]), _ptr(g["dk"]),
+                           _ptr(g["dv"]), _ptr(g["dlog_alpha"]), _ptr(g["dbeta"]), _ptr(g["dh0"]), _ptr(ws),
+                           ws.numel() * ws.element_size(), _stream(stream, q.device))
+    if rc != _lib.KDA_OK:
+        raise KdaError(rc, "kda_chunk_bwd")
+    return g
+
+
 def kda_output_gate_norm(o, g, weight=None, eps: float = 1e-6, out=None, stream=None):
     """The layer's output epilogue: out = RMSNorm(o) over the head dim (dv) x weight[dv] x sigmoid(g),
     per (token, head) row.  o, g [..., H, dv] contiguous, bf16 or fp32 (same dtype); weight [dv] fp32 or

@@ -286,6 +286,62 @@ int kda_decode_multi_ex(const void *q, const void *k, const void *v, const float
     return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 
+size_t kda_chunk_bwd_workspace_size(int B, int T, int H, int dk, int dv, int num_seqs, int chunk_size,
+                                    kda_dtype dtype) {
+    if (dtype != KDA_F32 && dtype != KDA_BF16) return 0;
+    const bool varlen = (B == 1 && num_seqs > 1);
+    if (check_prefill_shape(B, T, H, dk, dv, num_seqs, varlen, chunk_size) != KDA_OK) return 0;
+    if (dk != dv) return 0;
+    return kda::chunk_bwd_workspace_bytes(B, T, H, dk, num_seqs);
+}
+
+int kda_chunk_bwd(const void *q, const void *k, const void *v, const float *log_alpha, const float *beta,
+                  const float *h0, const int32_t *cu_seqlens, int num_seqs, int B, int T, int H, int dk, int dv,
+                  int chunk_size, kda_dtype dtype, const void *do_, const float *dh_T, void *dq, void *dk_out,
+                  void *dv_out, float *dlog_alpha, float *dbeta, float *dh0, void *workspace, size_t workspace_bytes,
+                  void *stream_) {
+    if (dtype != KDA_F32 && dtype != KDA_BF16) return KDA_ERR_BAD_DTYPE;
+    if (!workspace) return KDA_ERR_NULL_ARG;
+    const int rc = check_prefill_shape(B, T, H, dk, dv, num_seqs, cu_seqlens != nullptr, chunk_size);
+    if (rc != KDA_OK) return rc;
+    if (dk != dv) return KDA_ERR_UNSUPPORTED;
+    const int64_t tokens = (int64_t)B * T;
+    if (tokens > 0 && (!q || !k || !v || !log_alpha || !beta || !do_ || !dq || !dk_out || !dv_out || !dlog_alpha ||
+                       !dbeta))
+        return KDA_ERR_NULL_ARG;
+    const void *ptrs[] = {q, k, v, log_alpha, beta, h0, do_, dh_T, dq, dk_out, dv_out, dlog_alpha, dbeta, dh0};
+    for (const void *p : ptrs)
+        if (p && !aligned16(p)) return KDA_ERR_MISALIGNED;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return KDA_ERR_MISALIGNED;
+    const size_t need = kda::chunk_bwd_workspace_bytes(B, T, H, dk, num_seqs);
+    if (workspace_bytes < need) return KDA_ERR_WORKSPACE_TOO_SMALL;
+    const size_t es = elem_size(dtype), tk = (size_t)tokens * H, sb = (size_t)num_seqs * H * dk * dv * 4;
+    const Range in[] = {range_of(q, tk * dk * es), range_of(k, tk * dk * es), range_of(v, tk * dv * es),
+                        range_of(log_alpha, tk * dk * 4), range_of(beta, tk * 4), range_of(h0, h0 ? sb : 0),
+                        range_of(do_, tk * dv * es), range_of(dh_T, dh_T ? sb : 0),
+                        range_of(cu_seqlens, cu_seqlens ? 4 * (size_t)(num_seqs + 1) : 0)};
+    const Range out[] = {range_of(dq, tk * dk * es), range_of(dk_out, tk * dk * es), range_of(dv_out, tk * dv * es),
+                         range_of(dlog_alpha, tk * dk * 4), range_of(dbeta, tk * 4), range_of(dh0, dh0 ? sb : 0),
+                         range_of(workspace, need)};
+    for (size_t a = 0; a < sizeof(out) / sizeof(out[0]); ++a) {
+        for (const Range &r : in)
+            if (overlaps(out[a], r)) return KDA_ERR_ALIASING;
+        for (size_t b = a + 1; b < sizeof(out) / sizeof(out[0]); ++b)
+            if (overlaps(out[a], out[b])) return KDA_ERR_ALIASING;
+    }
+    if (tokens == 0) {  // nothing to differentiate but the initial states: dh0 = dh_T
+        cudaStream_t st = static_cast<cudaStream_t>(stream_);
+        cudaError_t e = cudaSuccess;
+        if (dh0) e = dh_T ? cudaMemcpyAsync(dh0, dh_T, sb, cudaMemcpyDeviceToDevice, st) : cudaMemsetAsync(dh0, 0, sb, st);
+        if (e == cudaSuccess) e = cudaMemsetAsync(workspace, 0, 256, st);
+        return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+    }
+    cudaError_t e = kda::launch_chunk_bwd(q, k, v, log_alpha, beta, h0, cu_seqlens, num_seqs, B, T, H, dk, dtype, do_,
+                                          dh_T, dq, dk_out, dv_out, dlog_alpha, dbeta, dh0, workspace,
+                                          static_cast<cudaStream_t>(stream_));
+    return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
 int kda_output_gate_norm(const void *o, const void *g, const float *weight, float eps, int n_tok, int H, int dv,
                          kda_dtype dtype, void *out, void *stream_) {
     if (dtype != KDA_F32 && dtype != KDA_BF16) return KDA_ERR_BAD_DTYPE;

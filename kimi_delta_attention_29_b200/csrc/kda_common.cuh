@@ -83,7 +83,7 @@ constexpr int kChunk = 64;
 namespace kda {
 // Kernel ids reported by kda_trace_end.
 enum KernelId { kKernChunkTable = 0, kKernTcPrep = 1, kKernTcState = 2, kKernSimt = 3, kKernDecode = 4,
-                kKernDecodeMulti = 5, kKernOutputGateNorm = 6 };
+                kKernDecodeMulti = 5, kKernOutputGateNorm = 6, kKernBwdState = 7, kKernBwdChunk = 8 };
 // Diagnostics: bracket one kernel launch with trace events when kda_trace_begin is active.
 void trace_before(int kernel_id, cudaStream_t stream);
 void trace_after(cudaStream_t stream);
@@ -104,6 +104,17 @@ cudaError_t launch_prefill_simt(const void *q, const void *k, const void *v, con
                                 const float *beta, const float *h0, const int32_t *cu_seqlens,
                                 int num_seqs, int B, int T, int H, int dk, int dv, kda_dtype dtype,
                                 void *o, float *h_T, int *status, const Prologue &pro, cudaStream_t stream);
+
+// Varlen chunk table from cu_seqlens (validates it; status_blk[0] = status, [1] = chunk count).
+cudaError_t launch_chunk_table(const int32_t *cu_seqlens, int num_seqs, int T, int *status_blk, int *base,
+                               int4 *table, cudaStream_t stream);
+
+// CUDA-core chunkwise backward (dk = dv = D in {64, 128}).
+size_t chunk_bwd_workspace_bytes(int B, int T, int H, int D, int num_seqs);
+cudaError_t launch_chunk_bwd(const void *q, const void *k, const void *v, const float *la, const float *beta,
+                             const float *h0, const int32_t *cu, int num_seqs, int B, int T, int H, int D,
+                             kda_dtype dtype, const void *dout, const float *dhT, void *dq, void *dk, void *dv,
+                             float *dla, float *dbeta, float *dh0, void *workspace, cudaStream_t stream);
 
 // Tensor-core (tcgen05) chunkwise forward: bf16, dk = dv = 128.
 size_t prefill_tc_workspace_bytes(int B, int T, int H, int num_seqs, bool varlen);

@@ -985,6 +985,14 @@ cudaError_t encode_token_map(CUtensorMap *map, const void *base, CUtensorMapData
 
 }  // namespace
 
+cudaError_t launch_chunk_table(const int32_t *cu_seqlens, int num_seqs, int T, int *status_blk, int *base,
+                               int4 *table, cudaStream_t stream) {
+    trace_before(kKernChunkTable, stream);
+    kda_chunk_table_kernel<<<1, 1024, 0, stream>>>(cu_seqlens, num_seqs, T, status_blk, base, table);
+    trace_after(stream);
+    return cudaGetLastError();
+}
+
 size_t prefill_tc_workspace_bytes(int B, int T, int H, int num_seqs, bool varlen) {
     (void)varlen;
     return tc_layout(B, T, H, num_seqs).total;

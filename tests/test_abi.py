@@ -188,3 +188,31 @@ def test_output_gate_norm_rejects_on_host(lib):
     assert call(out=A + 256) == _lib.KDA_ERR_ALIASING                        # partial overlap with o
     assert call(out=2 * A) == _lib.KDA_ERR_ALIASING                          # out is g
     assert call(w=3 * A + 64) == _lib.KDA_ERR_ALIASING                       # weight inside out
+
+
+def test_chunk_bwd_rejects_on_host(lib):
+    """Every rejection returns before a launch; no call here reaches a kernel."""
+    c = ctypes.c_void_p
+    B, T, H, d = 1, 128, 2, 128
+    need = lib.kda_chunk_bwd_workspace_size(B, T, H, d, d, B, 64, _lib.KDA_BF16)
+    assert need > 0
+    assert lib.kda_chunk_bwd_workspace_size(B, T, H, 96, 96, B, 64, _lib.KDA_BF16) == 0
+    assert lib.kda_chunk_bwd_workspace_size(B, T, H, d, d, B, 32, _lib.KDA_BF16) == 0
+
+    def call(dtype=_lib.KDA_BF16, q=A, ws=64 * A, ws_bytes=None, dq=20 * A, chunk=64, dk=d, dv=d, do=7 * A):
+        return lib.kda_chunk_bwd(c(q) if q else None, c(2 * A), c(3 * A), c(4 * A), c(5 * A), None, None, B, B, T, H,
+                                 dk, dv, chunk, dtype, c(do) if do else None, None, c(dq), c(21 * A), c(22 * A),
+                                 c(23 * A), c(24 * A), None, c(ws) if ws else None,
+                                 need if ws_bytes is None else ws_bytes, None)
+
+    assert call(dtype=9) == _lib.KDA_ERR_BAD_DTYPE
+    assert call(ws=0) == _lib.KDA_ERR_NULL_ARG
+    assert call(chunk=32) == _lib.KDA_ERR_UNSUPPORTED
+    assert call(dk=64) == _lib.KDA_ERR_UNSUPPORTED
+    assert call(q=0) == _lib.KDA_ERR_NULL_ARG
+    assert call(do=0) == _lib.KDA_ERR_NULL_ARG
+    assert call(q=A + 4) == _lib.KDA_ERR_MISALIGNED
+    assert call(ws=64 * A + 16) == _lib.KDA_ERR_MISALIGNED
+    assert call(ws_bytes=need - 1) == _lib.KDA_ERR_WORKSPACE_TOO_SMALL
+    assert call(dq=A + 1024) == _lib.KDA_ERR_ALIASING          # dq inside q
+    assert call(dq=21 * A + 256) == _lib.KDA_ERR_ALIASING      # dq overlaps dk
