@@ -49,6 +49,8 @@ def parse_args():
     p.add_argument("--e2e-steps", type=int, default=2)
     p.add_argument("--decode-steps", type=int, default=1024)
     p.add_argument("--no-decode", action="store_true")
+    p.add_argument("--no-backward", action="store_true")
+    p.add_argument("--backward-steps", type=int, default=3)
     p.add_argument("--cpu-seconds", type=float, default=12.0,
                    help="target CPU time of the oracle sample (0 skips the CPU baseline)")
     p.add_argument("--seq-len", type=int, default=131072,
@@ -411,6 +413,10 @@ def gpu_arm(args):
                 "frac": epi_bytes / (epi_ms * 1e6) / peaks["hbm_gbs"]}
     del g_out, out_e
 
+    backward = None
+    if not args.no_backward:
+        backward = backward_bench(args, dev, stream, barrier, max_over_ranks, world)
+
     decode = None
     if not args.no_decode:
         decode = decode_bench(args, dev, stream, peaks, barrier, max_over_ranks)
@@ -423,13 +429,62 @@ def gpu_arm(args):
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config_dict(T),
             "roofline": roofline, "operator_roofline": operator_roofline, "cpu_baseline": cpu_baseline,
-            "e2e": e2e, "gpu_launches": len(traces), "clocks": clk, "prologue": prologue, "epilogue": epilogue, "decode": decode,
+            "e2e": e2e, "gpu_launches": len(traces), "clocks": clk, "prologue": prologue, "epilogue": epilogue, "backward": backward, "decode": decode,
             "kernels": kst, "peaks": peaks}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
     return 0
+
+
+def backward_bench(args, dev, stream, barrier, max_over_ranks, world):
+    """kda_chunk_bwd on the training shape (B=4, H=16, T=4096, d=128, bf16), next to kda_chunk_fwd on the
+    same inputs; kernel split from the library's trace."""
+    import torch
+    import kimi_delta_attention_29_b200 as kda
+    from kimi_delta_attention_29_b200 import inputs as gen
+    shp = gen.TRAIN
+    x = gen.make_prefill_for(shp, seed=0, device=dev)
+    g = torch.Generator(device=dev).manual_seed(11)
+    do = torch.randn(x["v"].shape, generator=g, device=dev).to(x["v"].dtype)
+    N = shp.B
+    ws = torch.empty(kda._lib.load().kda_chunk_bwd_workspace_size(shp.B, shp.T, shp.H, shp.dk, shp.dv, N, 64,
+                                                                  kda._lib.KDA_BF16), dtype=torch.uint8, device=dev)
+    fws = kda.Workspace()
+
+    def bwd():
+        return kda.kda_chunk_bwd(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], x["h0"], None, do=do,
+                                 want_dh0=False, workspace=ws, stream=stream)
+
+    def fwd():
+        return kda.kda_chunk_fwd(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], x["h0"], None, workspace=fws,
+                                 stream=stream)
+
+    def timed(fn, n):
+        fn()
+        torch.cuda.synchronize(dev)
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(n):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier()
+        return max_over_ranks(e0.elapsed_time(e1)) / n
+
+    fwd_ms = timed(fwd, max(args.backward_steps, 3))
+    bwd_ms = timed(bwd, args.backward_steps)
+    kda.kda_trace_begin(64)
+    bwd()
+    per = {}
+    for name, ms in kda.kda_trace_end():
+        per[name] = per.get(name, 0.0) + ms
+    tokens = shp.B * shp.T
+    return {"workload": shp.name, "ms_per_call": bwd_ms, "tokens_per_s": whole_job_rate(tokens, 1, world, bwd_ms),
+            "forward_ms_same_shape": fwd_ms, "bwd_over_fwd": bwd_ms / fwd_ms,
+            "kernels_ms": per, "arith": "fp32 on CUDA cores"}
 
 
 def decode_bench(args, dev, stream, peaks, barrier, max_over_ranks):

@@ -190,8 +190,9 @@ KDA_API int kda_decode_multi_ex(const void *q, const void *k, const void *v, con
                                 void *stream);
 
 /* Bytes of device workspace kda_chunk_bwd needs (dk = dv = D): the status block, the varlen chunk
- * table and, per (chunk, head), the state-pass record (chunk-start state, state gradient and four
- * 64 x D tiles: 2 D^2 + 256 D floats, 256 KB at D = 128).  Returns 0 for unsupported sizes. */
+ * table and, per (chunk, head), the chunk operands (three 64 x 64 and three 64 x D tiles) and the
+ * state-pass record (chunk-start state, state gradient and four 64 x D tiles): 400 KB per
+ * (chunk, head) at D = 128.  Returns 0 for unsupported sizes. */
 KDA_API size_t kda_chunk_bwd_workspace_size(int B, int T, int H, int dk, int dv, int num_seqs, int chunk_size,
                                             kda_dtype dtype);
 
@@ -205,8 +206,8 @@ KDA_API size_t kda_chunk_bwd_workspace_size(int B, int T, int H, int dk, int dv,
  *   dlog_alpha: [B, T, H, dk] fp32           dbeta : [B, T, H] fp32
  *   dh0       : [N, H, dk, dv] fp32, or NULL (not wanted); with h0 = NULL it is the gradient at
  *               zero initial states.
- * fp32 arithmetic on CUDA cores (a state pass per (sequence, head, 16 value columns), then one CTA
- * per (chunk, head, 32 key channels)); deterministic.  A step whose log gate is below -15 ln 2 is
+ * fp32 arithmetic on CUDA cores (chunk operands per (chunk, head), a state pass per (sequence, head,
+ * 16 value columns), then one CTA per (chunk, head, 32 key channels)); deterministic.  A step whose log gate is below -15 ln 2 is
  * applied as 2^-15, as in the CUDA-core forward, and its dlog_alpha is 0.  Supported: dk = dv in
  * {64, 128}, dtype BF16 or F32, chunk_size 64.  Device-detected errors (bad cu_seqlens) go to the
  * workspace status word (kda_get_status). */

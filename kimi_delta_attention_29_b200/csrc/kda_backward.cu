@@ -20,14 +20,18 @@
 // channel, and dlog_alpha is the reverse running sum of dG over the chunk.  (The derivation is
 // checked against the token-by-token adjoint in the tests.)
 //
-// Two kernels, the same split as the forward:
+// Three kernels, the forward's split between chunk-parallel and sequential work:
+//  * kda_bwd_prep_kernel - one CTA per (chunk, head), all chunks in parallel: Abar, P, T and the
+//    decayed rows K o 2^G, Q o 2^G, K o 2^{G_L - G} of the chunk, once.
 //  * kda_bwd_state_kernel - one CTA per (sequence, head, 16 value columns), sequential over chunks:
-//    recomputes the chunk-start states (forward pass), then walks the chunks backwards carrying dS.
-//    Value columns of S and dS evolve independently, so slices need no communication.  Per chunk
-//    it writes dv and a record of S, dS', Z, dDelta, X1 and Delta for the chunk kernel.
+//    recomputes the chunk-start states (forward pass), then walks the chunks backwards carrying dS,
+//    with only its 16-column products per chunk.  Value columns of S and dS evolve independently,
+//    so slices need no communication.  Per chunk it writes dv and a record of S, dS', Z, dDelta,
+//    X1 and Delta for the chunk kernel.
 //  * kda_bwd_chunk_kernel - one CTA per (chunk, head, 32 key channels), all chunks in parallel:
-//    recomputes Abar and T, forms dT, dP, dA from the record, and writes dq, dk, dlog_alpha (and
-//    dbeta from the first channel block).  Every output element has one writer: deterministic.
+//    forms dT, dP, dA from the record and the prep kernel's T and Abar, and writes dq, dk,
+//    dlog_alpha (and dbeta from the first channel block).  Every output element has one writer:
+//    deterministic.
 // Decay factors are single exponentials of differences that are <= 0 where they are used, with
 // each step's base-2 gate clamped at kMinLog2DecaySimt as in the CUDA-core forward (the gradient
 // of a clamped step's log gate is zero).
@@ -37,7 +41,8 @@ namespace kda {
 namespace {
 
 constexpr int kC = kChunk;
-constexpr int kBT = 256;   // threads per CTA, both kernels
+constexpr int kBT = 256;   // threads per CTA of the prep kernel
+constexpr int kBTs = 512;  // threads per CTA of the state pass
 constexpr int kNV = 16;    // value columns per state-pass CTA
 constexpr int kSP = kNV + 1;  // padded row stride of the [D][kNV] state tiles
 constexpr int kCB = 32;    // key channels per chunk-kernel CTA
@@ -125,34 +130,109 @@ __device__ __forceinline__ void ut_inverse(const float *Am, float *Tm) {
     }
 }
 
+// Per chunk-head chunk-level operands (fp32), written once by the prep kernel and read by both
+// other kernels (the state pass re-reads them for every 16-column slice).
+template <int D> struct BwdOps {
+    static constexpr size_t Tm = 0;                          // [C][C]  (I + Diag(beta) Abar)^-1
+    static constexpr size_t Pm = Tm + (size_t)kC * kC;       // [C][C]  decayed q-k Gram, i <= r
+    static constexpr size_t Ab = Pm + (size_t)kC * kC;       // [C][C]  Abar, i < r
+    static constexpr size_t Kt = Ab + (size_t)kC * kC;       // [C][D]  K o 2^G
+    static constexpr size_t Qt = Kt + (size_t)kC * D;        // [C][D]  Q o 2^G
+    static constexpr size_t Kh = Qt + (size_t)kC * D;        // [C][D]  K o 2^{G_L - G}
+    static constexpr size_t eGL = Kh + (size_t)kC * D;       // [D]     2^{G_L}
+    static constexpr size_t floats = eGL + D;
+};
+
+// (chunk, head) of a chunk-parallel CTA: first token and rows; false for an unused table slot.
+__device__ __forceinline__ bool chunk_of(int ci, const int4 *table, const int *n_chunks, int nc, int T_len,
+                                         int64_t &t0, int &L) {
+    if (table) {
+        if (ci >= *n_chunks) return false;
+        const int4 e = table[ci];
+        t0 = e.y;
+        L = e.z;
+    } else {
+        const int n = ci / nc, c = ci % nc;
+        t0 = (int64_t)n * T_len + (int64_t)c * kC;
+        L = min(kC, T_len - c * kC);
+    }
+    return true;
+}
+
+template <int D>
+struct PrepSmem {
+    static constexpr int DKP = D + 1;
+    static constexpr size_t floats = 3 * (size_t)kC * DKP + 3 * (size_t)kC * CP + kC + D;
+    static constexpr size_t bytes = floats * sizeof(float);
+};
+
+// One CTA per (chunk, head): Abar, P, T and the decayed key / query rows of the chunk.
+template <int D, typename T>
+__global__ void __launch_bounds__(kBT, 1)
+kda_bwd_prep_kernel(const T *__restrict__ q, const T *__restrict__ k, const float *__restrict__ la,
+                    const float *__restrict__ beta, const int4 *__restrict__ table, const int *__restrict__ n_chunks,
+                    int nc, int T_len, int H, float *__restrict__ ops) {
+    using SM = PrepSmem<D>;
+    constexpr int DKP = SM::DKP;
+    using O = BwdOps<D>;
+    extern __shared__ float smem[];
+    float *Kc = smem, *Qc = Kc + kC * DKP, *Gc = Qc + kC * DKP;
+    float *Am = Gc + kC * DKP, *Pm = Am + kC * CP, *Xm = Pm + kC * CP, *bt = Xm + kC * CP, *gl = bt + kC;
+    const int h = blockIdx.x % H, ci = blockIdx.x / H, tid = threadIdx.x;
+    int64_t t0;
+    int L;
+    if (!chunk_of(ci, table, n_chunks, nc, T_len, t0, L)) return;
+    float *rec = ops + ((size_t)ci * H + h) * O::floats;
+    load_chunk<D, T>(q, k, la, beta, t0, L, H, h, true, Kc, Qc, Gc, bt, gl);
+    decayed_grams<D>(Kc, Qc, Gc, bt, false, Am, Pm);
+    for (int p = tid; p < kC * kC; p += kBT) {
+        const int r = p / kC, i = p % kC;
+        Xm[r * CP + i] = bt[r] * Am[r * CP + i];  // A = Diag(beta) Abar
+        rec[O::Ab + p] = Am[r * CP + i];
+        rec[O::Pm + p] = Pm[r * CP + i];
+    }
+    __syncthreads();
+    ut_inverse(Xm, Pm);  // T into the P buffer (P is already stored)
+    for (int p = tid; p < kC * kC; p += kBT) rec[O::Tm + p] = Pm[(p / kC) * CP + p % kC];
+    for (int idx = tid; idx < kC * D; idx += kBT) {
+        const int r = idx / D, c = idx % D;
+        const float g = Gc[r * DKP + c], e = ex2f(g);
+        rec[O::Kt + idx] = Kc[r * DKP + c] * e;
+        rec[O::Qt + idx] = Qc[r * DKP + c] * e;
+        rec[O::Kh + idx] = Kc[r * DKP + c] * ex2f(gl[c] - g);
+    }
+    for (int c = tid; c < D; c += kBT) rec[O::eGL + c] = ex2f(gl[c]);
+}
+
 template <int D>
 struct StateSmem {
     static constexpr int DKP = D + 1;
-    static constexpr size_t floats = 3 * (size_t)kC * DKP    // Kc, Qc, Gc
+    static constexpr size_t floats = 2 * (size_t)kC * CP     // sT, sP
+                                     + 3 * (size_t)kC * DKP  // sKt, sKh, sQt
                                      + 6 * (size_t)kC * kNV  // Vs, dOs, X1, Dl, dDl, Zs
                                      + 3 * (size_t)D * kSP   // Ss, dSs, dSn
-                                     + 3 * (size_t)kC * CP   // Am, Pm, Tm
-                                     + kC + 2 * (size_t)D;   // bt, gl, egl
+                                     + kC + (size_t)D;       // bt, egl
     static constexpr size_t bytes = floats * sizeof(float);
 };
 
 template <int D, typename T>
-__global__ void __launch_bounds__(kBT, 1)
-kda_bwd_state_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
-                     const float *__restrict__ la, const float *__restrict__ beta, const float *__restrict__ h0,
+__global__ void __launch_bounds__(kBTs, 1)
+kda_bwd_state_kernel(const T *__restrict__ v, const float *__restrict__ beta, const float *__restrict__ h0,
                      const int32_t *__restrict__ cu_seqlens, const int *__restrict__ chunk_base, int num_seqs,
                      int T_len, int H, const T *__restrict__ dout, const float *__restrict__ dhT,
-                     float *__restrict__ recs, T *__restrict__ dv_out, float *__restrict__ dh0, int *status) {
+                     const float *__restrict__ ops, float *__restrict__ recs, T *__restrict__ dv_out,
+                     float *__restrict__ dh0, int *status) {
     using SM = StateSmem<D>;
     constexpr int DKP = SM::DKP;
     using R = BwdRec<D>;
+    using O = BwdOps<D>;
     extern __shared__ float smem[];
-    float *Kc = smem, *Qc = Kc + kC * DKP, *Gc = Qc + kC * DKP;
-    float *Vs = Gc + kC * DKP, *dOs = Vs + kC * kNV, *X1 = dOs + kC * kNV, *Dl = X1 + kC * kNV;
+    float *sT = smem, *sP = sT + kC * CP;
+    float *sKt = sP + kC * CP, *sKh = sKt + kC * DKP, *sQt = sKh + kC * DKP;
+    float *Vs = sQt + kC * DKP, *dOs = Vs + kC * kNV, *X1 = dOs + kC * kNV, *Dl = X1 + kC * kNV;
     float *dDl = Dl + kC * kNV, *Zs = dDl + kC * kNV;
     float *Ss = Zs + kC * kNV, *dSs = Ss + D * kSP, *dSn = dSs + D * kSP;
-    float *Am = dSn + D * kSP, *Pm = Am + kC * CP, *Tm = Pm + kC * CP;
-    float *bt = Tm + kC * CP, *gl = bt + kC, *egl = gl + D;
+    float *bt = dSn + D * kSP, *egl = bt + kC;
 
     constexpr int slices = D / kNV;
     int bid = blockIdx.x;
@@ -178,37 +258,52 @@ kda_bwd_state_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *
     }
     const int nch = (int)((len + kC - 1) / kC);
     const size_t soff = ((size_t)n * H + h) * D * D;
-    for (int idx = tid; idx < D * kNV; idx += kBT) {
+    for (int idx = tid; idx < D * kNV; idx += kBTs) {
         const int c = idx / kNV, jj = idx % kNV;
         Ss[c * kSP + jj] = h0 ? h0[soff + (size_t)c * D + j0 + jj] : 0.f;
         dSs[c * kSP + jj] = dhT ? dhT[soff + (size_t)c * D + j0 + jj] : 0.f;
     }
-    __syncthreads();
 
-    auto x1_delta = [&]() {  // X1 = V - (K o 2^G) S;  Delta = T Diag(beta) X1
-        for (int idx = tid; idx < kC * kNV; idx += kBT) {
-            const int r = idx / kNV, jj = idx % kNV;
-            float acc = Vs[idx];
-            for (int c = 0; c < D; ++c)
-                acc = fmaf(-Kc[r * DKP + c] * ex2f(Gc[r * DKP + c]), Ss[c * kSP + jj], acc);
-            X1[idx] = acc;
+    // the chunk's operands (from the prep kernel) and V / dO slices; ends with a barrier
+    auto stage = [&](const float *op, int64_t t0, int L, bool bwd) {
+        for (int p = tid; p < kC * kC; p += kBTs) {  // operand tiles by cp.async: all in flight at once
+            const int r = p / kC, i = p % kC;
+            cp_async4(sT + r * CP + i, op + O::Tm + p);
+            if (bwd) cp_async4(sP + r * CP + i, op + O::Pm + p);
         }
-        __syncthreads();
-        for (int idx = tid; idx < kC * kNV; idx += kBT) {
-            const int r = idx / kNV, jj = idx % kNV;
-            float acc = 0.f;
-            for (int i = 0; i <= r; ++i) acc = fmaf(Tm[r * CP + i] * bt[i], X1[i * kNV + jj], acc);
-            Dl[idx] = acc;
+        for (int idx = tid; idx < kC * D; idx += kBTs) {
+            const int r = idx / D, c = idx % D;
+            cp_async4(sKt + r * DKP + c, op + O::Kt + idx);
+            cp_async4(sKh + r * DKP + c, op + O::Kh + idx);
+            if (bwd) cp_async4(sQt + r * DKP + c, op + O::Qt + idx);
         }
-        __syncthreads();
-    };
-    auto load_vs = [&](int64_t t0, int L, bool want_do) {
-        for (int idx = tid; idx < kC * kNV; idx += kBT) {
+        for (int c = tid; c < D; c += kBTs) cp_async4(egl + c, op + O::eGL + c);
+        cp_async_commit();
+        for (int idx = tid; idx < kC * kNV; idx += kBTs) {
             const int r = idx / kNV, jj = idx % kNV;
             const size_t off = ((size_t)(t0 + r) * H + h) * D + j0 + jj;
             Vs[idx] = r < L ? Elem<T>::load(v + off) : 0.f;
-            if (want_do) dOs[idx] = r < L ? Elem<T>::load(dout + off) : 0.f;
+            if (bwd) dOs[idx] = r < L ? Elem<T>::load(dout + off) : 0.f;
         }
+        if (tid < kC) bt[tid] = tid < L ? __ldg(beta + (size_t)(t0 + tid) * H + h) : 0.f;
+        cp_async_wait<0>();
+        __syncthreads();
+    };
+    auto x1_delta = [&]() {  // X1 = V - (K o 2^G) S;  Delta = T Diag(beta) X1
+        for (int idx = tid; idx < kC * kNV; idx += kBTs) {
+            const int r = idx / kNV, jj = idx % kNV;
+            float acc = Vs[idx];
+            for (int c = 0; c < D; ++c) acc = fmaf(-sKt[r * DKP + c], Ss[c * kSP + jj], acc);
+            X1[idx] = acc;
+        }
+        __syncthreads();
+        for (int idx = tid; idx < kC * kNV; idx += kBTs) {
+            const int r = idx / kNV, jj = idx % kNV;
+            float acc = 0.f;
+            for (int i = 0; i <= r; ++i) acc = fmaf(sT[r * CP + i] * bt[i], X1[i * kNV + jj], acc);
+            Dl[idx] = acc;
+        }
+        __syncthreads();
     };
 
     // ---- forward: chunk-start states into the records
@@ -216,28 +311,25 @@ kda_bwd_state_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *
         const int64_t t0 = start + (int64_t)ch * kC;
         const int L = (int)min((int64_t)kC, len - (int64_t)ch * kC);
         float *rec = recs + ((size_t)(cbase + ch) * H + h) * R::floats;
-        for (int idx = tid; idx < kNV * D; idx += kBT) {
+        const float *op = ops + ((size_t)(cbase + ch) * H + h) * O::floats;
+        __syncthreads();  // the previous chunk's reads of the staged tiles are done
+        for (int idx = tid; idx < kNV * D; idx += kBTs) {
             const int jj = idx / D, c = idx % D;
             rec[R::St + (size_t)(j0 + jj) * D + c] = Ss[c * kSP + jj];
         }
-        load_vs(t0, L, false);
-        load_chunk<D, T>(q, k, la, beta, t0, L, H, h, false, Kc, Qc, Gc, bt, gl);
-        decayed_grams<D>(Kc, Qc, Gc, bt, true, Am, nullptr);
-        ut_inverse(Am, Tm);
+        stage(op, t0, L, false);
         x1_delta();
-        for (int idx = tid; idx < D * kNV; idx += kBT) {  // S <- 2^{G_L} S + (K o 2^{G_L - G})^T Delta
+        for (int idx = tid; idx < D * kNV; idx += kBTs) {  // S <- 2^{G_L} S + (K o 2^{G_L - G})^T Delta
             const int c = idx / kNV, jj = idx % kNV;
-            float acc = ex2f(gl[c]) * Ss[c * kSP + jj];
-            for (int r = 0; r < kC; ++r)
-                acc = fmaf(Kc[r * DKP + c] * ex2f(gl[c] - Gc[r * DKP + c]), Dl[r * kNV + jj], acc);
+            float acc = egl[c] * Ss[c * kSP + jj];
+            for (int r = 0; r < kC; ++r) acc = fmaf(sKh[r * DKP + c], Dl[r * kNV + jj], acc);
             dSn[c * kSP + jj] = acc;
         }
         __syncthreads();
-        for (int idx = tid; idx < D * kNV; idx += kBT) {
+        for (int idx = tid; idx < D * kNV; idx += kBTs) {
             const int c = idx / kNV, jj = idx % kNV;
             Ss[c * kSP + jj] = dSn[c * kSP + jj];
         }
-        __syncthreads();
     }
 
     // ---- backward over the chunks, carrying dS (= dL/d state after the chunk)
@@ -245,95 +337,98 @@ kda_bwd_state_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *
         const int64_t t0 = start + (int64_t)ch * kC;
         const int L = (int)min((int64_t)kC, len - (int64_t)ch * kC);
         float *rec = recs + ((size_t)(cbase + ch) * H + h) * R::floats;
-        load_vs(t0, L, true);
-        load_chunk<D, T>(q, k, la, beta, t0, L, H, h, true, Kc, Qc, Gc, bt, gl);
-        for (int c = tid; c < D; c += kBT) egl[c] = ex2f(gl[c]);
-        for (int idx = tid; idx < kNV * D; idx += kBT) {
+        const float *op = ops + ((size_t)(cbase + ch) * H + h) * O::floats;
+        __syncthreads();
+        for (int idx = tid; idx < kNV * D; idx += kBTs) {
             const int jj = idx / D, c = idx % D;
             Ss[c * kSP + jj] = rec[R::St + (size_t)(j0 + jj) * D + c];
             rec[R::dSt + (size_t)(j0 + jj) * D + c] = dSs[c * kSP + jj];
         }
-        decayed_grams<D>(Kc, Qc, Gc, bt, true, Am, Pm);
-        ut_inverse(Am, Tm);
+        stage(op, t0, L, true);
         x1_delta();
         // dDelta = (K o 2^{G_L - G}) dS + P^T dO
-        for (int idx = tid; idx < kC * kNV; idx += kBT) {
+        for (int idx = tid; idx < kC * kNV; idx += kBTs) {
             const int r = idx / kNV, jj = idx % kNV;
             float acc = 0.f;
-            for (int c = 0; c < D; ++c)
-                acc = fmaf(Kc[r * DKP + c] * ex2f(gl[c] - Gc[r * DKP + c]), dSs[c * kSP + jj], acc);
-            for (int i = r; i < kC; ++i) acc = fmaf(Pm[i * CP + r], dOs[i * kNV + jj], acc);
+            for (int c = 0; c < D; ++c) acc = fmaf(sKh[r * DKP + c], dSs[c * kSP + jj], acc);
+            for (int i = r; i < kC; ++i) acc = fmaf(sP[i * CP + r], dOs[i * kNV + jj], acc);
             dDl[idx] = acc;
         }
         __syncthreads();
         // Z = T^T dDelta;  dV = Diag(beta) Z
-        for (int idx = tid; idx < kC * kNV; idx += kBT) {
+        for (int idx = tid; idx < kC * kNV; idx += kBTs) {
             const int r = idx / kNV, jj = idx % kNV;
             float acc = 0.f;
-            for (int i = r; i < kC; ++i) acc = fmaf(Tm[i * CP + r], dDl[i * kNV + jj], acc);
+            for (int i = r; i < kC; ++i) acc = fmaf(sT[i * CP + r], dDl[i * kNV + jj], acc);
             Zs[idx] = acc;
             if (r < L) Elem<T>::store(dv_out + ((size_t)(t0 + r) * H + h) * D + j0 + jj, bt[r] * acc);
         }
         __syncthreads();
-        for (int idx = tid; idx < kC * kNV; idx += kBT) {  // record rows: Z, dDelta ([C][dv])
+        for (int idx = tid; idx < kC * kNV; idx += kBTs) {  // record rows: Z, dDelta ([C][dv])
             const int r = idx / kNV, jj = idx % kNV;
             rec[R::Z + (size_t)r * D + j0 + jj] = Zs[idx];
             rec[R::dD + (size_t)r * D + j0 + jj] = dDl[idx];
         }
-        for (int idx = tid; idx < kNV * kC; idx += kBT) {  // transposed: X1^T, Delta^T ([dv][C])
+        for (int idx = tid; idx < kNV * kC; idx += kBTs) {  // transposed: X1^T, Delta^T ([dv][C])
             const int jj = idx / kC, r = idx % kC;
             rec[R::X1t + (size_t)(j0 + jj) * kC + r] = X1[r * kNV + jj];
             rec[R::Dt + (size_t)(j0 + jj) * kC + r] = Dl[r * kNV + jj];
         }
         // dS <- 2^{G_L} dS + (Q o 2^G)^T dO - (K o 2^G)^T Diag(beta) Z
-        for (int idx = tid; idx < D * kNV; idx += kBT) {
+        for (int idx = tid; idx < D * kNV; idx += kBTs) {
             const int c = idx / kNV, jj = idx % kNV;
             float acc = egl[c] * dSs[c * kSP + jj];
             for (int r = 0; r < kC; ++r) {
-                const float e = ex2f(Gc[r * DKP + c]);
-                acc = fmaf(Qc[r * DKP + c] * e, dOs[r * kNV + jj], acc);
-                acc = fmaf(-Kc[r * DKP + c] * e * bt[r], Zs[r * kNV + jj], acc);
+                acc = fmaf(sQt[r * DKP + c], dOs[r * kNV + jj], acc);
+                acc = fmaf(-sKt[r * DKP + c] * bt[r], Zs[r * kNV + jj], acc);
             }
             dSn[c * kSP + jj] = acc;
         }
         __syncthreads();
-        for (int idx = tid; idx < D * kNV; idx += kBT) {
+        for (int idx = tid; idx < D * kNV; idx += kBTs) {
             const int c = idx / kNV, jj = idx % kNV;
             dSs[c * kSP + jj] = dSn[c * kSP + jj];
         }
-        __syncthreads();
     }
+    __syncthreads();
     if (dh0)
-        for (int idx = tid; idx < D * kNV; idx += kBT) {
+        for (int idx = tid; idx < D * kNV; idx += kBTs) {
             const int c = idx / kNV, jj = idx % kNV;
             dh0[soff + (size_t)c * D + j0 + jj] = dSs[c * kSP + jj];
         }
 }
 
+constexpr int kBT2 = 512;            // chunk kernel: threads per CTA
+constexpr int kCBP = kCB + 1;        // padded row stride of the [C][kCB] channel-block tiles
+constexpr int kRowsPerWarp = kC / (kBT2 / 32);
+
+// Shared memory of the chunk kernel (floats): the channel block's K, Q, G; T, Abar, dT / dA, dP;
+// a staging area for the record tiles (two phases), reused for W and for dG.
 template <int D>
 struct ChunkSmem {
-    static constexpr int DKP = D + 1;
-    static constexpr size_t floats = 3 * (size_t)kC * DKP        // Kc, Qc, Gc
-                                     + 5 * (size_t)kC * CP       // Am (Abar), Tm, Mm (A, dT, dA), Pm (dP), Wm
-                                     + kC + D                    // bt, gl
-                                     + (size_t)kC * (kCB + 1)    // dG of this channel block
-                                     + (size_t)8 * kCB;          // per-warp partial sums of dG_L
+    static constexpr size_t kbq = 3 * (size_t)kC * kCBP;          // Kb, Qb, Gb
+    static constexpr size_t cc = 4 * (size_t)kC * CP;             // Tm, Am, Mm, Pm
+    static constexpr size_t stage = 3 * (size_t)kC * D + (size_t)D * kCB;  // 3 [C][D]-sized tiles + a [D][kCB] block
+    static constexpr size_t floats = kbq + cc + stage + 2 * (size_t)kC + 2 * (size_t)kCB;
     static constexpr size_t bytes = floats * sizeof(float);
 };
 
 template <int D, typename T>
-__global__ void __launch_bounds__(kBT, 1)
+__global__ void __launch_bounds__(kBT2, 1)
 kda_bwd_chunk_kernel(const T *__restrict__ q, const T *__restrict__ k, const float *__restrict__ la,
                      const float *__restrict__ beta, const int4 *__restrict__ table, const int *__restrict__ n_chunks,
-                     int nc, int T_len, int H, const T *__restrict__ dout, const float *__restrict__ recs,
-                     T *__restrict__ dq, T *__restrict__ dk, float *__restrict__ dla, float *__restrict__ dbeta) {
+                     int nc, int T_len, int H, const T *__restrict__ dout, const float *__restrict__ ops,
+                     const float *__restrict__ recs, T *__restrict__ dq, T *__restrict__ dk, float *__restrict__ dla,
+                     float *__restrict__ dbeta) {
     using SM = ChunkSmem<D>;
-    constexpr int DKP = SM::DKP;
     using R = BwdRec<D>;
+    using O = BwdOps<D>;
     extern __shared__ float smem[];
-    float *Kc = smem, *Qc = Kc + kC * DKP, *Gc = Qc + kC * DKP;
-    float *Am = Gc + kC * DKP, *Tm = Am + kC * CP, *Mm = Tm + kC * CP, *Pm = Mm + kC * CP, *Wm = Pm + kC * CP;
-    float *bt = Wm + kC * CP, *gl = bt + kC, *dGs = gl + D, *dGLw = dGs + kC * (kCB + 1);
+    float *Kb = smem, *Qb = Kb + kC * kCBP, *Gb = Qb + kC * kCBP;
+    float *Tm = Gb + kC * kCBP, *Am = Tm + kC * CP, *Mm = Am + kC * CP, *Pm = Mm + kC * CP;
+    float *U = Pm + kC * CP;                                   // staging area
+    float *U0 = U, *U1 = U + kC * D, *U2 = U1 + kC * D, *Ub = U2 + kC * D;  // three [C][D] tiles, one [D][kCB]
+    float *bt = U + SM::stage, *dbs = bt + kC, *glb = dbs + kC, *sds = glb + kCB;
 
     constexpr int blocks = D / kCB;
     int bid = blockIdx.x;
@@ -342,49 +437,117 @@ kda_bwd_chunk_kernel(const T *__restrict__ q, const T *__restrict__ k, const flo
     const int h = bid % H, ci = bid / H;
     int64_t t0;
     int L;
-    if (table) {
-        if (ci >= *n_chunks) return;
-        const int4 e = table[ci];
-        t0 = e.y;
-        L = e.z;
-    } else {
-        const int n = ci / nc, c = ci % nc;
-        t0 = (int64_t)n * T_len + (int64_t)c * kC;
-        L = min(kC, T_len - c * kC);
-    }
+    if (!chunk_of(ci, table, n_chunks, nc, T_len, t0, L)) return;
     const float *rec = recs + ((size_t)ci * H + h) * R::floats;
+    const float *op = ops + ((size_t)ci * H + h) * O::floats;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int c = cb * kCB + lane;  // this lane's channel in the per-(row, channel) phase
 
-    load_chunk<D, T>(q, k, la, beta, t0, L, H, h, true, Kc, Qc, Gc, bt, gl);
-    decayed_grams<D>(Kc, Qc, Gc, bt, false, Am, nullptr);  // Abar
-    for (int p = tid; p < kC * kC; p += kBT) {              // A = Diag(beta) Abar
+    // ---- phase 0: T, Abar (prep kernel); beta; K, Q and the clamped base-2 running gate of this block
+    for (int p = tid; p < kC * kC; p += kBT2) {
         const int r = p / kC, i = p % kC;
-        Mm[r * CP + i] = bt[r] * Am[r * CP + i];
+        cp_async4(Tm + r * CP + i, op + O::Tm + p);
+        cp_async4(Am + r * CP + i, op + O::Ab + p);
     }
-    __syncthreads();
-    ut_inverse(Mm, Tm);
-    // dT[r][i] = beta_i sum_j dDelta[r][j] X1[i][j];  dP[r][i] = sum_j dO[r][j] Delta[i][j] (i <= r)
-    for (int p = tid; p < kC * kC; p += kBT) {
-        const int r = p / kC, i = p % kC;  // a warp spans 32 consecutive i of one row r
-        float st = 0.f, sp = 0.f;
-        const bool live = r < L;
-        const T *dorow = dout + ((size_t)(t0 + (live ? r : 0)) * H + h) * D;
-        for (int j = 0; j < D; ++j) {
-            st = fmaf(rec[R::dD + (size_t)r * D + j], rec[R::X1t + (size_t)j * kC + i], st);
-            if (live && i <= r) sp = fmaf(Elem<T>::load(dorow + j), rec[R::Dt + (size_t)j * kC + i], sp);
+    if (tid < kC) bt[tid] = tid < L ? __ldg(beta + (size_t)(t0 + tid) * H + h) : 0.f;
+    for (int idx = tid; idx < kC * kCB; idx += kBT2) {
+        const int r = idx / kCB, cc = idx % kCB;
+        float kv = 0.f, qv = 0.f, lv = 0.f;
+        if (r < L) {
+            const size_t off = ((size_t)(t0 + r) * H + h) * D + cb * kCB + cc;
+            kv = Elem<T>::load(k + off);
+            qv = Elem<T>::load(q + off);
+            lv = fmaxf(__ldg(la + off) * kLog2e, kMinLog2DecaySimt);
         }
-        Mm[r * CP + i] = bt[i] * st;
-        Pm[r * CP + i] = sp;
+        Kb[r * kCBP + cc] = kv;
+        Qb[r * kCBP + cc] = qv;
+        Gb[r * kCBP + cc] = lv;
+    }
+    // ---- phase 1 staging: dDelta [C][D], X1^T [D][C], Z [C][D], S^T block [D][kCB]
+    for (int idx = tid; idx < kC * D; idx += kBT2) {
+        cp_async4(U0 + idx, rec + R::dD + idx);
+        cp_async4(U1 + idx, rec + R::X1t + idx);
+        cp_async4(U2 + idx, rec + R::Z + idx);
+    }
+    for (int idx = tid; idx < D * kCB; idx += kBT2)
+        cp_async4(Ub + idx, rec + R::St + (size_t)(idx / kCB) * D + cb * kCB + idx % kCB);
+    cp_async_commit();
+    cp_async_wait<0>();
+    __syncthreads();
+    if (tid < kCB) {  // running gate per channel of the block
+        float acc = 0.f;
+        for (int r = 0; r < kC; ++r) {
+            acc += Gb[r * kCBP + tid];
+            Gb[r * kCBP + tid] = acc;
+        }
+        glb[tid] = acc;
+    }
+    // dT[r][i] = beta_i sum_j dDelta[r][j] X1[i][j]
+    for (int p = tid; p < kC * kC; p += kBT2) {
+        const int r = p / kC, i = p % kC;
+        float acc = 0.f;
+        for (int j = 0; j < D; ++j) acc = fmaf(U0[r * D + j], U1[j * kC + i], acc);
+        Mm[r * CP + i] = bt[i] * acc;
+    }
+    if (cb == 0 && tid < kC) {  // dbeta, X1 part: sum_j Z[r][j] X1[r][j]
+        float acc = 0.f;
+        for (int j = 0; j < D; ++j) acc = fmaf(U2[tid * D + j], U1[j * kC + tid], acc);
+        dbs[tid] = acc;
+    }
+    float dKt[kRowsPerWarp], dQt[kRowsPerWarp], dKh[kRowsPerWarp];
+#pragma unroll
+    for (int m = 0; m < kRowsPerWarp; ++m) {  // dK~ = -beta_r (Z S^T)[r][c]
+        const int r = warp + m * (kBT2 / 32);
+        float acc = 0.f;
+        for (int j = 0; j < D; ++j) acc = fmaf(U2[r * D + j], Ub[j * kCB + lane], acc);
+        dKt[m] = -bt[r] * acc;
     }
     __syncthreads();
-    for (int p = tid; p < kC * kC; p += kBT) {  // W = dT T^T  (T lower: m <= i)
+    // ---- phase 2 staging: dO [C][D], Delta^T [D][C], dS'^T block [D][kCB] (S^T block stays)
+    for (int idx = tid; idx < kC * D; idx += kBT2) cp_async4(U1 + idx, rec + R::Dt + idx);
+    for (int idx = tid; idx < D * kCB; idx += kBT2)
+        cp_async4(U2 + idx, rec + R::dSt + (size_t)(idx / kCB) * D + cb * kCB + idx % kCB);
+    cp_async_commit();
+    for (int idx = tid; idx < kC * D; idx += kBT2) {
+        const int r = idx / D, j = idx % D;
+        U0[idx] = r < L ? Elem<T>::load(dout + ((size_t)(t0 + r) * H + h) * D + j) : 0.f;
+    }
+    cp_async_wait<0>();
+    __syncthreads();
+    for (int p = tid; p < kC * kC; p += kBT2) {  // dP[r][i] = sum_j dO[r][j] Delta[i][j]  (i <= r)
+        const int r = p / kC, i = p % kC;
+        float acc = 0.f;
+        if (i <= r)
+            for (int j = 0; j < D; ++j) acc = fmaf(U0[r * D + j], U1[j * kC + i], acc);
+        Pm[r * CP + i] = acc;
+    }
+#pragma unroll
+    for (int m = 0; m < kRowsPerWarp; ++m) {  // dQ~ = (dO S^T)[r][c],  dK^ = (Delta dS'^T)[r][c]
+        const int r = warp + m * (kBT2 / 32);
+        float a = 0.f, b = 0.f;
+        for (int j = 0; j < D; ++j) {
+            a = fmaf(U0[r * D + j], Ub[j * kCB + lane], a);
+            b = fmaf(U1[j * kC + r], U2[j * kCB + lane], b);
+        }
+        dQt[m] = a;
+        dKh[m] = b;
+    }
+    if (warp == 0) {  // sum_j S[c][j] dS'[c][j] for the state-decay term of dG_L
+        float acc = 0.f;
+        for (int j = 0; j < D; ++j) acc = fmaf(Ub[j * kCB + lane], U2[j * kCB + lane], acc);
+        sds[lane] = acc;
+    }
+    __syncthreads();
+    // ---- W = dT T^T (T lower: m <= i) into the staging area, then dA = -strict_lower(T^T W)
+    float *Wm = U;
+    for (int p = tid; p < kC * kC; p += kBT2) {
         const int r = p / kC, i = p % kC;
         float acc = 0.f;
         for (int m = 0; m <= i; ++m) acc = fmaf(Mm[r * CP + m], Tm[i * CP + m], acc);
         Wm[r * CP + i] = acc;
     }
     __syncthreads();
-    for (int p = tid; p < kC * kC; p += kBT) {  // dA = -strict_lower(T^T W)  (T^T upper: m >= r)
+    for (int p = tid; p < kC * kC; p += kBT2) {
         const int r = p / kC, i = p % kC;
         float acc = 0.f;
         if (i < r)
@@ -393,51 +556,41 @@ kda_bwd_chunk_kernel(const T *__restrict__ q, const T *__restrict__ k, const flo
     }
     __syncthreads();
     if (cb == 0) {  // dbeta_r = sum_j Z[r][j] X1[r][j] + sum_{i<r} dA[r][i] Abar[r][i]  (one warp per row)
-        for (int r = warp; r < L; r += kBT / 32) {
+        for (int r = warp; r < L; r += kBT2 / 32) {
             float acc = 0.f;
-            for (int j = lane; j < D; j += 32) acc = fmaf(rec[R::Z + (size_t)r * D + j], rec[R::X1t + (size_t)j * kC + r], acc);
             for (int i = lane; i < r; i += 32) acc = fmaf(Mm[r * CP + i], Am[r * CP + i], acc);
 #pragma unroll
             for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-            if (lane == 0) dbeta[(size_t)(t0 + r) * H + h] = acc;
+            if (lane == 0) dbeta[(size_t)(t0 + r) * H + h] = acc + dbs[r];
         }
     }
 
-    // ---- per (row r, channel c) of this block: lane = channel, warp w takes rows w, w + 8, ...
-    const int c = cb * kCB + lane;
-    const float glc = gl[c];
+    // ---- per (row r, channel c): decayed Gram terms and the factor terms; lane = channel
+    float *dGs = U;  // [C][kCBP]
+    float *dGLw = U + kC * kCBP;  // [warps][kCB]
+    const float glc = glb[lane];
     float dgl = 0.f;
-    for (int r = warp; r < kC; r += kBT / 32) {
-        const float g = Gc[r * DKP + c], kc = Kc[r * DKP + c], qc = Qc[r * DKP + c];
+#pragma unroll
+    for (int m = 0; m < kRowsPerWarp; ++m) {
+        const int r = warp + m * (kBT2 / 32);
+        const float g = Gb[r * kCBP + lane], kc = Kb[r * kCBP + lane], qc = Qb[r * kCBP + lane];
         const float er = ex2f(g), eL = ex2f(glc - g);
-        // state terms: dK~ = -beta_r (Z S^T)_rc, dQ~ = (dO S^T)_rc, dK^ = (Delta dS'^T)_rc
-        float zs = 0.f, os = 0.f, ds = 0.f;
-        if (r < L) {
-            const T *dorow = dout + ((size_t)(t0 + r) * H + h) * D;
-            for (int j = 0; j < D; ++j) {
-                const float sjc = rec[R::St + (size_t)j * D + c];
-                zs = fmaf(rec[R::Z + (size_t)r * D + j], sjc, zs);
-                os = fmaf(Elem<T>::load(dorow + j), sjc, os);
-                ds = fmaf(rec[R::Dt + (size_t)j * kC + r], rec[R::dSt + (size_t)j * D + c], ds);
-            }
-        }
-        const float dKt = -bt[r] * zs, dQt = os, dKh = ds;
-        // decayed Gram terms (this row as the later index r, then as the earlier index)
         float xa = 0.f, yq = 0.f, zk = 0.f;
-        for (int i = 0; i <= r; ++i) {
-            const float kd = Kc[i * DKP + c] * ex2f(g - Gc[i * DKP + c]);
+        for (int i = 0; i <= r; ++i) {  // this row as the later index
+            const float kd = Kb[i * kCBP + lane] * ex2f(g - Gb[i * kCBP + lane]);
             if (i < r) xa = fmaf(Mm[r * CP + i], kd, xa);
             yq = fmaf(Pm[r * CP + i], kd, yq);
         }
-        for (int m = r; m < kC; ++m) {
-            const float e = ex2f(Gc[m * DKP + c] - g);
-            if (m > r) zk = fmaf(bt[m] * Mm[m * CP + r] * Kc[m * DKP + c], e, zk);
-            zk = fmaf(Pm[m * CP + r] * Qc[m * DKP + c], e, zk);
+        for (int mm = r; mm < kC; ++mm) {  // this row as the earlier index
+            const float e = ex2f(Gb[mm * kCBP + lane] - g);
+            if (mm > r) zk = fmaf(bt[mm] * Mm[mm * CP + r] * Kb[mm * kCBP + lane], e, zk);
+            zk = fmaf(Pm[mm * CP + r] * Qb[mm * kCBP + lane], e, zk);
         }
-        const float dkv = dKt * er + dKh * eL + bt[r] * xa + zk;
-        const float dqv = dQt * er + yq;
-        dGs[r * (kCB + 1) + lane] = dKt * kc * er + dQt * qc * er - dKh * kc * eL + bt[r] * kc * xa + qc * yq - kc * zk;
-        dgl = fmaf(dKh * kc, eL, dgl);
+        const float dkv = dKt[m] * er + dKh[m] * eL + bt[r] * xa + zk;
+        const float dqv = dQt[m] * er + yq;
+        dGs[r * kCBP + lane] =
+            dKt[m] * kc * er + dQt[m] * qc * er - dKh[m] * kc * eL + bt[r] * kc * xa + qc * yq - kc * zk;
+        dgl = fmaf(dKh[m] * kc, eL, dgl);
         if (r < L) {
             const size_t off = ((size_t)(t0 + r) * H + h) * D + c;
             Elem<T>::store(dq + off, dqv);
@@ -449,15 +602,13 @@ kda_bwd_chunk_kernel(const T *__restrict__ q, const T *__restrict__ k, const flo
     if (warp == 0 && L > 0) {
         // dG_L: the K^ terms of every row, and the decay of the incoming state 2^{G_L} sum_j S dS'
         float acc = 0.f;
-        for (int w = 0; w < kBT / 32; ++w) acc += dGLw[w * kCB + lane];
-        float sds = 0.f;
-        for (int j = 0; j < D; ++j) sds = fmaf(rec[R::St + (size_t)j * D + c], rec[R::dSt + (size_t)j * D + c], sds);
-        acc = fmaf(ex2f(glc), sds, acc);
-        dGs[(L - 1) * (kCB + 1) + lane] += acc;
+        for (int w = 0; w < kBT2 / 32; ++w) acc += dGLw[w * kCB + lane];
+        acc = fmaf(ex2f(glc), sds[lane], acc);
+        dGs[(L - 1) * kCBP + lane] += acc;
         // dlog_alpha: reverse running sum of dG over the chunk (zero where the step was clamped)
         float run = 0.f;
         for (int r = L - 1; r >= 0; --r) {
-            run += dGs[r * (kCB + 1) + lane];
+            run += dGs[r * kCBP + lane];
             const size_t off = ((size_t)(t0 + r) * H + h) * D + c;
             const bool clamped = __ldg(la + off) * kLog2e < kMinLog2DecaySimt;
             dla[off] = clamped ? 0.f : run;
@@ -469,11 +620,16 @@ template <int D, typename T>
 cudaError_t launch_t(const void *q, const void *k, const void *v, const float *la, const float *beta,
                      const float *h0, const int32_t *cu, int num_seqs, int B, int T_len, int H, const void *dout,
                      const float *dhT, void *dq, void *dk, void *dv, float *dla, float *dbeta, float *dh0,
-                     int *status, int *base, int4 *table, float *recs, int64_t max_chunks, cudaStream_t stream) {
+                     int *status, int *base, int4 *table, float *ops, float *recs, int64_t max_chunks,
+                     cudaStream_t stream) {
+    auto kp = kda_bwd_prep_kernel<D, T>;
     auto ks = kda_bwd_state_kernel<D, T>;
     auto kc = kda_bwd_chunk_kernel<D, T>;
-    cudaError_t e = cudaFuncSetAttribute(ks, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)StateSmem<D>::bytes);
+    cudaError_t e = cudaFuncSetAttribute(kp, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)PrepSmem<D>::bytes);
     if (e != cudaSuccess) return e;
+    if ((e = cudaFuncSetAttribute(ks, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)StateSmem<D>::bytes)) !=
+        cudaSuccess)
+        return e;
     if ((e = cudaFuncSetAttribute(kc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ChunkSmem<D>::bytes)) !=
         cudaSuccess)
         return e;
@@ -483,23 +639,31 @@ cudaError_t launch_t(const void *q, const void *k, const void *v, const float *l
         if ((e = launch_chunk_table(cu, num_seqs, T_len, status, base, table, stream)) != cudaSuccess) return e;
     }
     const int nc = cu ? 0 : (T_len + kC - 1) / kC;
+    const int64_t chunks = cu ? max_chunks : (int64_t)B * nc;
+    const int4 *tab = cu ? table : nullptr;
+    const int *cnt = cu ? status + 1 : nullptr;
+    if (chunks > 0) {
+        trace_before(kKernBwdPrep, stream);
+        kp<<<(unsigned)(chunks * H), kBT, PrepSmem<D>::bytes, stream>>>(qt, kt, la, beta, tab, cnt, nc, T_len, H, ops);
+        trace_after(stream);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
     trace_before(kKernBwdState, stream);
-    ks<<<(unsigned)((int64_t)num_seqs * H * (D / kNV)), kBT, StateSmem<D>::bytes, stream>>>(
-        qt, kt, vt, la, beta, h0, cu, base, num_seqs, T_len, H, dot, dhT, recs, static_cast<T *>(dv), dh0, status);
+    ks<<<(unsigned)((int64_t)num_seqs * H * (D / kNV)), kBTs, StateSmem<D>::bytes, stream>>>(
+        vt, beta, h0, cu, base, num_seqs, T_len, H, dot, dhT, ops, recs, static_cast<T *>(dv), dh0, status);
     trace_after(stream);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    const int64_t chunks = cu ? max_chunks : (int64_t)B * nc;
     if (chunks == 0) return cudaSuccess;
     trace_before(kKernBwdChunk, stream);
-    kc<<<(unsigned)(chunks * H * (D / kCB)), kBT, ChunkSmem<D>::bytes, stream>>>(
-        qt, kt, la, beta, cu ? table : nullptr, cu ? status + 1 : nullptr, nc, T_len, H, dot, recs,
-        static_cast<T *>(dq), static_cast<T *>(dk), dla, dbeta);
+    kc<<<(unsigned)(chunks * H * (D / kCB)), kBT2, ChunkSmem<D>::bytes, stream>>>(
+        qt, kt, la, beta, tab, cnt, nc, T_len, H, dot, ops, recs, static_cast<T *>(dq), static_cast<T *>(dk), dla,
+        dbeta);
     trace_after(stream);
     return cudaGetLastError();
 }
 
 struct BwdLayout {
-    size_t base_off, table_off, rec_off, total;
+    size_t base_off, table_off, ops_off, rec_off, total;
     int64_t max_chunks;
 };
 // One bound for both modes: B ceil(T / C) chunks without cu_seqlens, at most B T / C + N with it.
@@ -509,7 +673,9 @@ BwdLayout bwd_layout(int B, int T, int H, int D, int num_seqs) {
     l.max_chunks = ((int64_t)B * T + kC - 1) / kC + num_seqs;
     l.base_off = 256;
     l.table_off = up(l.base_off + 4 * (size_t)(num_seqs + 1));
-    l.rec_off = up(l.table_off + 16 * (size_t)l.max_chunks);
+    l.ops_off = up(l.table_off + 16 * (size_t)l.max_chunks);
+    const size_t ops_floats = D == 128 ? BwdOps<128>::floats : BwdOps<64>::floats;
+    l.rec_off = up(l.ops_off + (size_t)l.max_chunks * H * ops_floats * sizeof(float));
     const size_t rec_floats = D == 128 ? BwdRec<128>::floats : BwdRec<64>::floats;
     l.total = l.rec_off + (size_t)l.max_chunks * H * rec_floats * sizeof(float);
     return l;
@@ -530,20 +696,21 @@ cudaError_t launch_chunk_bwd(const void *q, const void *k, const void *v, const 
     int *status = reinterpret_cast<int *>(ws);
     int *base = reinterpret_cast<int *>(ws + lay.base_off);
     int4 *table = reinterpret_cast<int4 *>(ws + lay.table_off);
+    float *ops = reinterpret_cast<float *>(ws + lay.ops_off);
     float *recs = reinterpret_cast<float *>(ws + lay.rec_off);
     cudaError_t e = cudaMemsetAsync(ws, 0, 256, stream);
     if (e != cudaSuccess) return e;
     if (dtype == KDA_BF16)
         return D == 128 ? launch_t<128, __nv_bfloat16>(q, k, v, la, beta, h0, cu, num_seqs, B, T, H, dout, dhT, dq, dk,
-                                                       dv, dla, dbeta, dh0, status, base, table, recs,
+                                                       dv, dla, dbeta, dh0, status, base, table, ops, recs,
                                                        lay.max_chunks, stream)
                         : launch_t<64, __nv_bfloat16>(q, k, v, la, beta, h0, cu, num_seqs, B, T, H, dout, dhT, dq, dk,
-                                                      dv, dla, dbeta, dh0, status, base, table, recs, lay.max_chunks,
+                                                      dv, dla, dbeta, dh0, status, base, table, ops, recs, lay.max_chunks,
                                                       stream);
     return D == 128 ? launch_t<128, float>(q, k, v, la, beta, h0, cu, num_seqs, B, T, H, dout, dhT, dq, dk, dv, dla,
-                                           dbeta, dh0, status, base, table, recs, lay.max_chunks, stream)
+                                           dbeta, dh0, status, base, table, ops, recs, lay.max_chunks, stream)
                     : launch_t<64, float>(q, k, v, la, beta, h0, cu, num_seqs, B, T, H, dout, dhT, dq, dk, dv, dla,
-                                          dbeta, dh0, status, base, table, recs, lay.max_chunks, stream);
+                                          dbeta, dh0, status, base, table, ops, recs, lay.max_chunks, stream);
 }
 
 }  // namespace kda

@@ -20,6 +20,22 @@ template <> struct Elem<__nv_bfloat16> {
     static __device__ __forceinline__ void store(__nv_bfloat16 *p, float x) { *p = __float2bfloat16_rn(x); }
 };
 
+// Asynchronous global -> shared copies (cp.async): many in flight per thread without a register
+// round trip; commit a group, then wait for all but the newest N groups.
+__device__ __forceinline__ void cp_async16(void *dst, const void *src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
+                 "l"(src)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async4(void *dst, const void *src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
+                 "l"(src)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
 // Device status word (first int of the prefill workspace).  The first error wins.
 __device__ __forceinline__ void set_status(int *status, int code) {
     if (status) atomicCAS(status, 0, code);
@@ -83,7 +99,8 @@ constexpr int kChunk = 64;
 namespace kda {
 // Kernel ids reported by kda_trace_end.
 enum KernelId { kKernChunkTable = 0, kKernTcPrep = 1, kKernTcState = 2, kKernSimt = 3, kKernDecode = 4,
-                kKernDecodeMulti = 5, kKernOutputGateNorm = 6, kKernBwdState = 7, kKernBwdChunk = 8 };
+                kKernDecodeMulti = 5, kKernOutputGateNorm = 6, kKernBwdState = 7, kKernBwdChunk = 8,
+                kKernBwdPrep = 9 };
 // Diagnostics: bracket one kernel launch with trace events when kda_trace_begin is active.
 void trace_before(int kernel_id, cudaStream_t stream);
 void trace_after(cudaStream_t stream);
