@@ -410,7 +410,8 @@ def gpu_arm(args):
     epilogue = {"kernel": "kda_output_gate_norm_kernel", "ms_per_call": epi_ms,
                 "tokens_per_s": whole_job_rate(tokens_per_step, 1, world, epi_ms),
                 "bytes_per_call": epi_bytes, "hbm_gbs": epi_bytes / (epi_ms * 1e6),
-                "frac": epi_bytes / (epi_ms * 1e6) / peaks["hbm_gbs"]}
+                "frac": epi_bytes / (epi_ms * 1e6) / peaks["hbm_gbs"],
+                "traffic": ncu_traffic("kda_output_gate_norm_kernel", o.numel() // o.shape[-1])}
     del g_out, out_e
 
     backward = None
