@@ -50,6 +50,7 @@ def parse_args():
     p.add_argument("--decode-steps", type=int, default=1024)
     p.add_argument("--no-decode", action="store_true")
     p.add_argument("--no-backward", action="store_true")
+    p.add_argument("--no-cp", action="store_true")
     p.add_argument("--backward-steps", type=int, default=3)
     p.add_argument("--cpu-seconds", type=float, default=12.0,
                    help="target CPU time of the oracle sample (0 skips the CPU baseline)")
@@ -414,6 +415,10 @@ def gpu_arm(args):
                 "traffic": ncu_traffic("kda_output_gate_norm_kernel", o.numel() // o.shape[-1])}
     del g_out, out_e
 
+    cp_line = None
+    if not args.no_cp and world == 1 and args.seq_len == 131072:
+        cp_line = cp_bench(x, dev, stream, ms_per_step)
+
     backward = None
     if not args.no_backward:
         backward = backward_bench(args, dev, stream, barrier, max_over_ranks, world)
@@ -430,7 +435,7 @@ def gpu_arm(args):
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config_dict(T),
             "roofline": roofline, "operator_roofline": operator_roofline, "cpu_baseline": cpu_baseline,
-            "e2e": e2e, "gpu_launches": len(traces), "clocks": clk, "prologue": prologue, "epilogue": epilogue, "backward": backward, "decode": decode,
+            "e2e": e2e, "gpu_launches": len(traces), "clocks": clk, "prologue": prologue, "epilogue": epilogue, "backward": backward, "context_parallel": cp_line, "decode": decode,
             "kernels": kst, "peaks": peaks}
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -486,6 +491,41 @@ def backward_bench(args, dev, stream, barrier, max_over_ranks, world):
     return {"workload": shp.name, "ms_per_call": bwd_ms, "tokens_per_s": whole_job_rate(tokens, 1, world, bwd_ms),
             "forward_ms_same_shape": fwd_ms, "bwd_over_fwd": bwd_ms / fwd_ms,
             "kernels_ms": per, "arith": "fp32 on CUDA cores"}
+
+
+def cp_bench(x, dev, stream, single_ms):
+    """Context parallelism on the long-context sequence: the work ONE rank does for R segments (two
+    passes for its map [M | b], the composition of R maps, one pass from its incoming state), timed on
+    this GPU for the last segment.  The all-gather between GPUs is not part of it."""
+    import torch
+    import kimi_delta_attention_29_b200 as kda
+    from kimi_delta_attention_29_b200 import cp
+    T = x["q"].shape[1]
+    rows = []
+    for R in (2, 4, 8):
+        a, e = T - T // R, T
+        part = [x[n][:, a:e].contiguous() for n in ("q", "k", "v", "log_alpha", "beta")]
+        Mb_all = torch.zeros(R, x["q"].shape[2], 128, 256, device=dev)
+
+        def rank_work():
+            _, Mb = cp.segment_map(*part, stream=stream)
+            Mb_all[R - 1].copy_(Mb)
+            S_in, _ = kda.kda_state_compose(Mb_all, None, stream=stream)
+            return cp.segment_from(*part, S_in[R - 1], stream=stream)
+
+        rank_work()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(3):
+            rank_work()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        ms = e0.elapsed_time(e1) / 3
+        rows.append({"R": R, "segment_tokens": e - a, "rank_ms": ms, "single_gpu_ms": single_ms,
+                     "rank_over_single": ms / single_ms})
+    return {"workload": "long_B1_H32_T131072_d128 split into R segments", "per_rank": rows,
+            "exchange": "all-gather of [M | b] (32 x 128 x 256 fp32 = 4 MiB per rank) not measured: one GPU"}
 
 
 def decode_bench(args, dev, stream, peaks, barrier, max_over_ranks):

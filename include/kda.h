@@ -217,6 +217,22 @@ KDA_API int kda_chunk_bwd(const void *q, const void *k, const void *v, const flo
                           void *dk_out, void *dv_out, float *dlog_alpha, float *dbeta, float *dh0, void *workspace,
                           size_t workspace_bytes, void *stream);
 
+/* Exchange step of context parallelism (one sequence split into R consecutive segments, e.g. one
+ * per GPU).  The recurrence is linear in (state, v) for fixed q, k, alpha, beta (section "From
+ * linear attention to Gated DeltaNet"), so segment r maps its incoming state S_r to
+ * S_{r+1} = M_r S_r + b_r, with b_r the segment's final state from a zero state and M_r its dk x dk
+ * transition (the final state of a pass with v = 0 from S = I, both by kda_chunk_fwd).  Given all
+ * segments' maps this computes S_0 = h0 (zeros if NULL), S_1, ..., S_{R-1} and S_R.
+ *   Mb    : [R, H, dk, dk + dv] fp32, row i of head h of segment r = [M_r[h][i][:], b_r[h][i][:]]
+ *           (the layout of an all-gather of each segment's [M | b])
+ *   h0    : [H, dk, dv] fp32 or NULL
+ *   S_in  : [R, H, dk, dv] fp32 out, the state entering each segment, or NULL
+ *   S_out : [H, dk, dv] fp32 out, the state after the last segment
+ * fp32, one CTA per (head, 32 state columns), the segments applied in order.  Supported: dk in
+ * {64, 128}, dv in {64, 128}, R >= 1.  Outputs must not overlap the inputs or each other. */
+KDA_API int kda_state_compose(const float *Mb, const float *h0, int R, int H, int dk, int dv, float *S_in,
+                              float *S_out, void *stream);
+
 /* The KDA layer's output epilogue (Kimi Linear summary page, section "Kimi Linear model
  * composition": a per-head RMSNorm and a data-dependent output gate ahead of the output
  * projection; the page does not name the gate's activation, read here as the logistic sigmoid).

@@ -193,6 +193,22 @@ def kda_chunk_bwd(q, k, v, log_alpha, beta, h0=None, cu_seqlens=None, do=None, d
     return g
 
 
+def kda_state_compose(Mb, h0=None, want_S_in: bool = True, stream=None):
+    """Composition of R segment maps: Mb [R, H, dk, dk + dv] fp32 (rows [M_r | b_r]), h0 [H, dk, dv] fp32 or
+    None.  Returns (S_in [R, H, dk, dv] or None, S_out [H, dk, dv]): the state entering each segment and
+    the state after the last."""
+    torch = _torch()
+    R, H, dk, w = Mb.shape
+    dv = w - dk
+    S_in = torch.empty((R, H, dk, dv), dtype=torch.float32, device=Mb.device) if want_S_in else None
+    S_out = torch.empty((H, dk, dv), dtype=torch.float32, device=Mb.device)
+    rc = _lib.load().kda_state_compose(_ptr(Mb), _ptr(h0), R, H, dk, dv, _ptr(S_in), _ptr(S_out),
+                                       _stream(stream, Mb.device))
+    if rc != _lib.KDA_OK:
+        raise KdaError(rc, "kda_state_compose")
+    return S_in, S_out
+
+
 def kda_output_gate_norm(o, g, weight=None, eps: float = 1e-6, out=None, stream=None):
     """The layer's output epilogue: out = RMSNorm(o) over the head dim (dv) x weight[dv] x sigmoid(g),
     per (token, head) row.  o, g [..., H, dv] contiguous, bf16 or fp32 (same dtype); weight [dv] fp32 or

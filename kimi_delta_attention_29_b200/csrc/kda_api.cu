@@ -342,6 +342,24 @@ int kda_chunk_bwd(const void *q, const void *k, const void *v, const float *log_
     return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 
+int kda_state_compose(const float *Mb, const float *h0, int R, int H, int dk, int dv, float *S_in, float *S_out,
+                      void *stream_) {
+    if (!Mb || !S_out) return KDA_ERR_NULL_ARG;
+    if (R <= 0 || H <= 0 || dk <= 0 || dv <= 0 || (int64_t)R * H * dk * (dk + dv) > ((int64_t)1 << 40))
+        return KDA_ERR_BAD_SHAPE;
+    if ((dk != 64 && dk != 128) || (dv != 64 && dv != 128)) return KDA_ERR_UNSUPPORTED;
+    const void *ptrs[] = {Mb, h0, S_in, S_out};
+    for (const void *p : ptrs)
+        if (p && !aligned16(p)) return KDA_ERR_MISALIGNED;
+    const size_t sb = (size_t)H * dk * dv * 4;
+    const Range rm = range_of(Mb, (size_t)R * H * dk * (dk + dv) * 4), rh = range_of(h0, h0 ? sb : 0),
+                ri = range_of(S_in, S_in ? (size_t)R * sb : 0), ro = range_of(S_out, sb);
+    if (overlaps(ro, rm) || overlaps(ro, rh) || overlaps(ro, ri) || overlaps(ri, rm) || overlaps(ri, rh))
+        return KDA_ERR_ALIASING;
+    cudaError_t e = kda::launch_state_compose(Mb, h0, R, H, dk, dv, S_in, S_out, static_cast<cudaStream_t>(stream_));
+    return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
 int kda_output_gate_norm(const void *o, const void *g, const float *weight, float eps, int n_tok, int H, int dv,
                          kda_dtype dtype, void *out, void *stream_) {
     if (dtype != KDA_F32 && dtype != KDA_BF16) return KDA_ERR_BAD_DTYPE;

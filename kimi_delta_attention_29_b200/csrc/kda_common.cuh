@@ -100,7 +100,7 @@ namespace kda {
 // Kernel ids reported by kda_trace_end.
 enum KernelId { kKernChunkTable = 0, kKernTcPrep = 1, kKernTcState = 2, kKernSimt = 3, kKernDecode = 4,
                 kKernDecodeMulti = 5, kKernOutputGateNorm = 6, kKernBwdState = 7, kKernBwdChunk = 8,
-                kKernBwdPrep = 9 };
+                kKernBwdPrep = 9, kKernStateCompose = 10 };
 // Diagnostics: bracket one kernel launch with trace events when kda_trace_begin is active.
 void trace_before(int kernel_id, cudaStream_t stream);
 void trace_after(cudaStream_t stream);
@@ -121,6 +121,10 @@ cudaError_t launch_prefill_simt(const void *q, const void *k, const void *v, con
                                 const float *beta, const float *h0, const int32_t *cu_seqlens,
                                 int num_seqs, int B, int T, int H, int dk, int dv, kda_dtype dtype,
                                 void *o, float *h_T, int *status, const Prologue &pro, cudaStream_t stream);
+
+// Composition of per-segment affine state maps (context parallelism); Mb packed [R, H, dk, dk + dv].
+cudaError_t launch_state_compose(const float *Mb, const float *h0, int R, int H, int dk, int dv, float *S_in,
+                                 float *S_out, cudaStream_t stream);
 
 // Varlen chunk table from cu_seqlens (validates it; status_blk[0] = status, [1] = chunk count).
 cudaError_t launch_chunk_table(const int32_t *cu_seqlens, int num_seqs, int T, int *status_blk, int *base,

@@ -216,3 +216,20 @@ def test_chunk_bwd_rejects_on_host(lib):
     assert call(ws_bytes=need - 1) == _lib.KDA_ERR_WORKSPACE_TOO_SMALL
     assert call(dq=A + 1024) == _lib.KDA_ERR_ALIASING          # dq inside q
     assert call(dq=21 * A + 256) == _lib.KDA_ERR_ALIASING      # dq overlaps dk
+
+
+def test_state_compose_rejects_on_host(lib):
+    c = ctypes.c_void_p
+    f = lib.kda_state_compose
+
+    def call(Mb=A, h0=None, R=2, H=2, dk=128, dv=128, S_in=None, S_out=8 * A):
+        return f(c(Mb) if Mb else None, c(h0) if h0 else None, R, H, dk, dv, c(S_in) if S_in else None,
+                 c(S_out) if S_out else None, None)
+
+    assert call(Mb=0) == _lib.KDA_ERR_NULL_ARG
+    assert call(S_out=0) == _lib.KDA_ERR_NULL_ARG
+    assert call(R=0) == _lib.KDA_ERR_BAD_SHAPE
+    assert call(dk=96) == _lib.KDA_ERR_UNSUPPORTED
+    assert call(S_out=8 * A + 4) == _lib.KDA_ERR_MISALIGNED
+    assert call(S_out=A + 4096) == _lib.KDA_ERR_ALIASING                     # output inside Mb
+    assert call(S_in=A + 1024) == _lib.KDA_ERR_ALIASING

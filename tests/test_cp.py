@@ -1,0 +1,137 @@
+"""Context parallelism (kimi_delta_attention_29_b200.cp): one sequence split over the ranks of a
+process group, joined by one all-gather of each segment's affine state map [M | b].
+
+CPU (gloo, 2 and 3 ranks): the host-side flow -- exchange order, each rank's incoming state, empty
+segments, h0 -- with the three per-rank steps (segment map, composition, rerun from the incoming
+state) computed in fp64 by the oracle; the ranks' outputs and final state must equal the oracle's
+single pass over the whole sequence.  The GPU tests run the library's kernels on one GPU, the ranks
+played by token ranges, and check kda_state_compose itself."""
+from __future__ import annotations
+
+import os
+import socket
+import sys
+from datetime import timedelta
+
+import numpy as np
+import pytest
+import torch
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port() -> int:
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _case(seed, T=23, H=2, dk=4, dv=4):
+    rng = np.random.default_rng(seed)
+    unit = lambda x: x / np.linalg.norm(x, axis=-1, keepdims=True)
+    return {"q": unit(rng.standard_normal((1, T, H, dk))), "k": unit(rng.standard_normal((1, T, H, dk))),
+            "v": rng.standard_normal((1, T, H, dv)), "log_alpha": -np.log1p(np.exp(rng.standard_normal((1, T, H, dk)))),
+            "beta": 1 / (1 + np.exp(-rng.standard_normal((1, T, H)))), "h0": 0.5 * rng.standard_normal((1, H, dk, dv))}
+
+
+def _worker(rank, world, port, bounds, use_h0, out):
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=timedelta(seconds=60))
+    import oracle
+    from kimi_delta_attention_29_b200 import cp
+    x = _case(7)
+    a, e = bounds[rank], bounds[rank + 1]
+    t = lambda arr: torch.from_numpy(np.ascontiguousarray(arr))
+    seg = [t(x[n][:, a:e]) for n in ("q", "k", "v", "log_alpha", "beta")]
+    H, dk, dv = x["q"].shape[2], x["q"].shape[3], x["v"].shape[3]
+
+    def segment(q, k, v, la, beta):  # o from zero state, M from v = 0 and S = I, b from zero state
+        o0, b = oracle.recurrent(q.numpy(), k.numpy(), v.numpy(), la.numpy(), beta.numpy(), None)
+        eye = np.broadcast_to(np.eye(dk), (1, H, dk, dk)).copy()
+        _, M = oracle.recurrent(q.numpy(), k.numpy(), np.zeros_like(v.numpy()), la.numpy(), beta.numpy(), eye)
+        return t(o0), t(np.concatenate([M[0], b[0]], axis=2))
+
+    def compose(Mb, s0):  # S_{j+1} = M_j S_j + b_j
+        S = np.zeros((H, dk, dv)) if s0 is None else s0.numpy()
+        S_in = []
+        for j in range(Mb.shape[0]):
+            S_in.append(S)
+            S = np.einsum("hic,hcj->hij", Mb[j, :, :, :dk].numpy(), S) + Mb[j, :, :, dk:].numpy()
+        return t(np.stack(S_in)), t(S)
+
+    def rerun(q, k, v, la, beta, S_in):
+        o, _ = oracle.recurrent(q.numpy(), k.numpy(), v.numpy(), la.numpy(), beta.numpy(), S_in.numpy()[None])
+        return t(o)
+
+    h0 = t(x["h0"]) if use_h0 else None
+    o, hT = cp.kda_chunk_fwd_cp(*seg, h0=h0, segment=segment, compose=compose, rerun=rerun, map_dtype=torch.float64)
+    out.put((rank, o.numpy(), hT.numpy()))
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("bounds,use_h0", [([0, 10, 23], True), ([0, 9, 9, 23], False), ([0, 0, 5, 23], True)])
+def test_cp_ranks_match_single_pass(bounds, use_h0):
+    import oracle
+    world = len(bounds) - 1
+    ctx = mp.get_context("spawn")
+    out = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, world, port, bounds, use_h0, out)) for r in range(world)]
+    for p in procs:
+        p.start()
+    try:
+        res = sorted((out.get(timeout=120) for _ in range(world)), key=lambda r: r[0])
+    finally:
+        for p in procs:
+            p.join(timeout=30)
+            if p.is_alive():
+                p.kill()
+    for p in procs:
+        assert p.exitcode == 0
+    x = _case(7)
+    o_ref, h_ref = oracle.recurrent(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], x["h0"] if use_h0 else None)
+    o = np.concatenate([r[1] for r in res], axis=1)
+    assert o.shape == o_ref.shape
+    assert np.abs(o - o_ref).max() <= 1e-12 * max(1.0, np.abs(o_ref).max())
+    for _, _, hT in res:  # every rank ends with the sequence's final state
+        assert np.abs(hT - h_ref).max() <= 1e-12 * max(1.0, np.abs(h_ref).max())
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("bounds", [[0, 300, 300, 700, 1000], [0, 64, 1000], [0, 1000]])
+def test_cp_segments_on_one_gpu(cuda_device, bounds):
+    import oracle
+    import kimi_delta_attention_29_b200 as kda
+    from kimi_delta_attention_29_b200 import cp
+    from kimi_delta_attention_29_b200 import inputs as gen
+    x = gen.make_prefill(1, 1000, 2, 128, 128, torch.bfloat16, gate_shift=2.0, h0_std=0.1, seed=81, device=cuda_device)
+    o, hT = cp.kda_chunk_fwd_segments(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], bounds, h0=x["h0"])
+    o1, h1 = kda.kda_chunk_fwd(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], x["h0"], None)
+    torch.cuda.synchronize(cuda_device)
+    f = lambda a: a.detach().float().cpu().numpy().astype(np.float64)
+    o_ref, h_ref = oracle.recurrent(f(x["q"]), f(x["k"]), f(x["v"]), f(x["log_alpha"]), f(x["beta"]), f(x["h0"]))
+    rel = lambda a, b: float(np.abs(f(a) - b).max() / np.abs(b).max())
+    assert rel(o, o_ref) <= 2e-2 and rel(hT, h_ref) <= 2e-2
+    assert rel(o, f(o1)) <= 2e-2 and rel(hT, f(h1)) <= 2e-2
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("R,dk,dv", [(1, 128, 128), (5, 128, 128), (3, 64, 64)])
+def test_state_compose_kernel(cuda_device, R, dk, dv):
+    import kimi_delta_attention_29_b200 as kda
+    g = torch.Generator().manual_seed(R)
+    H = 3
+    Mb = (torch.randn(R, H, dk, dk + dv, generator=g) / np.sqrt(dk)).to(cuda_device)
+    h0 = torch.randn(H, dk, dv, generator=g).to(cuda_device)
+    S_in, S_out = kda.kda_state_compose(Mb, h0)
+    torch.cuda.synchronize(cuda_device)
+    M64, S = Mb.double().cpu(), h0.double().cpu()
+    for j in range(R):
+        assert torch.allclose(S_in[j].double().cpu(), S, rtol=1e-4, atol=1e-4 * float(S.abs().max()))
+        S = M64[j, :, :, :dk] @ S + M64[j, :, :, dk:]
+    assert torch.allclose(S_out.double().cpu(), S, rtol=1e-4, atol=1e-4 * float(S.abs().max()))
