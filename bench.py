@@ -455,8 +455,8 @@ def backward_bench(args, dev, stream, barrier, max_over_ranks, world):
     g = torch.Generator(device=dev).manual_seed(11)
     do = torch.randn(x["v"].shape, generator=g, device=dev).to(x["v"].dtype)
     N = shp.B
-    ws = torch.empty(kda._lib.load().kda_chunk_bwd_workspace_size(shp.B, shp.T, shp.H, shp.dk, shp.dv, N, 64,
-                                                                  kda._lib.KDA_BF16), dtype=torch.uint8, device=dev)
+    ws = torch.empty(kda.kda_chunk_bwd_workspace_size(shp.B, shp.T, shp.H, shp.dk, shp.dv, N, 64, shp.dtype),
+                     dtype=torch.uint8, device=dev)
     fws = kda.Workspace()
 
     def bwd():

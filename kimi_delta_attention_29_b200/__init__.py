@@ -55,6 +55,14 @@ def kda_chunk_fwd_workspace_size(B: int, T: int, H: int, dk: int, dv: int, num_s
     return int(_lib.load().kda_chunk_fwd_workspace_size(B, T, H, dk, dv, num_seqs, chunk_size, code))
 
 
+def kda_chunk_bwd_workspace_size(B: int, T: int, H: int, dk: int, dv: int, num_seqs: int,
+                                 chunk_size: int = 64, dtype=None) -> int:
+    """Bytes of device workspace kda_chunk_bwd needs (0 for unsupported sizes)."""
+    torch = _torch()
+    code = _dtype_code(dtype if dtype is not None else torch.bfloat16)
+    return int(_lib.load().kda_chunk_bwd_workspace_size(B, T, H, dk, dv, num_seqs, chunk_size, code))
+
+
 class Workspace:
     """A reusable device workspace for kda_chunk_fwd (grows on demand, never shrinks)."""
 
@@ -177,7 +185,7 @@ def kda_chunk_bwd(q, k, v, log_alpha, beta, h0=None, cu_seqlens=None, do=None, d
     N = B if cu_seqlens is None else cu_seqlens.numel() - 1
     code = _dtype_code(q.dtype)
     lib = _lib.load()
-    need = lib.kda_chunk_bwd_workspace_size(B, T, H, dk, dv, N, chunk_size, code)
+    need = kda_chunk_bwd_workspace_size(B, T, H, dk, dv, N, chunk_size, q.dtype)
     if need == 0:
         raise KdaError(_lib.KDA_ERR_UNSUPPORTED, "kda_chunk_bwd_workspace_size")
     ws = workspace if workspace is not None else torch.empty(need, dtype=torch.uint8, device=q.device)
