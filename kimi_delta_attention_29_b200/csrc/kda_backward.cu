@@ -289,20 +289,28 @@ kda_bwd_state_kernel(const T *__restrict__ v, const float *__restrict__ beta, co
         cp_async_wait<0>();
         __syncthreads();
     };
+    // Register blocking (512 threads): for [C][kNV] tiles a thread owns column jj = tid % 16 of
+    // rows rp = tid / 16 and rp + 32; for [D][kNV] tiles column jj of channels cq + 32 k.
+    const int jj = tid % kNV, rp = tid / kNV;
+    constexpr int kCq = D / 32;
     auto x1_delta = [&]() {  // X1 = V - (K o 2^G) S;  Delta = T Diag(beta) X1
-        for (int idx = tid; idx < kC * kNV; idx += kBTs) {
-            const int r = idx / kNV, jj = idx % kNV;
-            float acc = Vs[idx];
-            for (int c = 0; c < D; ++c) acc = fmaf(-sKt[r * DKP + c], Ss[c * kSP + jj], acc);
-            X1[idx] = acc;
+        float a0 = Vs[rp * kNV + jj], a1 = Vs[(rp + 32) * kNV + jj];
+        for (int c = 0; c < D; ++c) {
+            const float sv = Ss[c * kSP + jj];
+            a0 = fmaf(-sKt[rp * DKP + c], sv, a0);
+            a1 = fmaf(-sKt[(rp + 32) * DKP + c], sv, a1);
         }
+        X1[rp * kNV + jj] = a0;
+        X1[(rp + 32) * kNV + jj] = a1;
         __syncthreads();
-        for (int idx = tid; idx < kC * kNV; idx += kBTs) {
-            const int r = idx / kNV, jj = idx % kNV;
-            float acc = 0.f;
-            for (int i = 0; i <= r; ++i) acc = fmaf(sT[r * CP + i] * bt[i], X1[i * kNV + jj], acc);
-            Dl[idx] = acc;
+        float d0 = 0.f, d1 = 0.f;  // T is zero above its diagonal
+        for (int i = 0; i <= rp + 32; ++i) {
+            const float xb = bt[i] * X1[i * kNV + jj];
+            d0 = fmaf(sT[rp * CP + i], xb, d0);
+            d1 = fmaf(sT[(rp + 32) * CP + i], xb, d1);
         }
+        Dl[rp * kNV + jj] = d0;
+        Dl[(rp + 32) * kNV + jj] = d1;
         __syncthreads();
     };
 
@@ -319,11 +327,17 @@ kda_bwd_state_kernel(const T *__restrict__ v, const float *__restrict__ beta, co
         }
         stage(op, t0, L, false);
         x1_delta();
-        for (int idx = tid; idx < D * kNV; idx += kBTs) {  // S <- 2^{G_L} S + (K o 2^{G_L - G})^T Delta
-            const int c = idx / kNV, jj = idx % kNV;
-            float acc = egl[c] * Ss[c * kSP + jj];
-            for (int r = 0; r < kC; ++r) acc = fmaf(sKh[r * DKP + c], Dl[r * kNV + jj], acc);
-            dSn[c * kSP + jj] = acc;
+        {  // S <- 2^{G_L} S + (K o 2^{G_L - G})^T Delta
+            float acc[kCq];
+#pragma unroll
+            for (int q2 = 0; q2 < kCq; ++q2) acc[q2] = egl[rp + 32 * q2] * Ss[(rp + 32 * q2) * kSP + jj];
+            for (int r = 0; r < kC; ++r) {
+                const float dl = Dl[r * kNV + jj];
+#pragma unroll
+                for (int q2 = 0; q2 < kCq; ++q2) acc[q2] = fmaf(sKh[r * DKP + rp + 32 * q2], dl, acc[q2]);
+            }
+#pragma unroll
+            for (int q2 = 0; q2 < kCq; ++q2) dSn[(rp + 32 * q2) * kSP + jj] = acc[q2];
         }
         __syncthreads();
         for (int idx = tid; idx < D * kNV; idx += kBTs) {
@@ -346,22 +360,33 @@ kda_bwd_state_kernel(const T *__restrict__ v, const float *__restrict__ beta, co
         }
         stage(op, t0, L, true);
         x1_delta();
-        // dDelta = (K o 2^{G_L - G}) dS + P^T dO
-        for (int idx = tid; idx < kC * kNV; idx += kBTs) {
-            const int r = idx / kNV, jj = idx % kNV;
-            float acc = 0.f;
-            for (int c = 0; c < D; ++c) acc = fmaf(sKh[r * DKP + c], dSs[c * kSP + jj], acc);
-            for (int i = r; i < kC; ++i) acc = fmaf(sP[i * CP + r], dOs[i * kNV + jj], acc);
-            dDl[idx] = acc;
+        {  // dDelta = (K o 2^{G_L - G}) dS + P^T dO  (P is zero above its diagonal)
+            float a0 = 0.f, a1 = 0.f;
+            for (int c = 0; c < D; ++c) {
+                const float ds = dSs[c * kSP + jj];
+                a0 = fmaf(sKh[rp * DKP + c], ds, a0);
+                a1 = fmaf(sKh[(rp + 32) * DKP + c], ds, a1);
+            }
+            for (int i = rp; i < kC; ++i) {
+                const float dov = dOs[i * kNV + jj];
+                a0 = fmaf(sP[i * CP + rp], dov, a0);
+                a1 = fmaf(sP[i * CP + rp + 32], dov, a1);
+            }
+            dDl[rp * kNV + jj] = a0;
+            dDl[(rp + 32) * kNV + jj] = a1;
         }
         __syncthreads();
-        // Z = T^T dDelta;  dV = Diag(beta) Z
-        for (int idx = tid; idx < kC * kNV; idx += kBTs) {
-            const int r = idx / kNV, jj = idx % kNV;
-            float acc = 0.f;
-            for (int i = r; i < kC; ++i) acc = fmaf(sT[i * CP + r], dDl[i * kNV + jj], acc);
-            Zs[idx] = acc;
-            if (r < L) Elem<T>::store(dv_out + ((size_t)(t0 + r) * H + h) * D + j0 + jj, bt[r] * acc);
+        {  // Z = T^T dDelta;  dV = Diag(beta) Z  (T[i][r] = 0 for i < r)
+            float z0 = 0.f, z1 = 0.f;
+            for (int i = rp; i < kC; ++i) {
+                const float dd = dDl[i * kNV + jj];
+                z0 = fmaf(sT[i * CP + rp], dd, z0);
+                z1 = fmaf(sT[i * CP + rp + 32], dd, z1);
+            }
+            Zs[rp * kNV + jj] = z0;
+            Zs[(rp + 32) * kNV + jj] = z1;
+            if (rp < L) Elem<T>::store(dv_out + ((size_t)(t0 + rp) * H + h) * D + j0 + jj, bt[rp] * z0);
+            if (rp + 32 < L) Elem<T>::store(dv_out + ((size_t)(t0 + rp + 32) * H + h) * D + j0 + jj, bt[rp + 32] * z1);
         }
         __syncthreads();
         for (int idx = tid; idx < kC * kNV; idx += kBTs) {  // record rows: Z, dDelta ([C][dv])
@@ -374,15 +399,20 @@ kda_bwd_state_kernel(const T *__restrict__ v, const float *__restrict__ beta, co
             rec[R::X1t + (size_t)(j0 + jj) * kC + r] = X1[r * kNV + jj];
             rec[R::Dt + (size_t)(j0 + jj) * kC + r] = Dl[r * kNV + jj];
         }
-        // dS <- 2^{G_L} dS + (Q o 2^G)^T dO - (K o 2^G)^T Diag(beta) Z
-        for (int idx = tid; idx < D * kNV; idx += kBTs) {
-            const int c = idx / kNV, jj = idx % kNV;
-            float acc = egl[c] * dSs[c * kSP + jj];
+        {  // dS <- 2^{G_L} dS + (Q o 2^G)^T dO - (K o 2^G)^T Diag(beta) Z
+            float acc[kCq];
+#pragma unroll
+            for (int q2 = 0; q2 < kCq; ++q2) acc[q2] = egl[rp + 32 * q2] * dSs[(rp + 32 * q2) * kSP + jj];
             for (int r = 0; r < kC; ++r) {
-                acc = fmaf(sQt[r * DKP + c], dOs[r * kNV + jj], acc);
-                acc = fmaf(-sKt[r * DKP + c] * bt[r], Zs[r * kNV + jj], acc);
+                const float dov = dOs[r * kNV + jj], zb = -bt[r] * Zs[r * kNV + jj];
+#pragma unroll
+                for (int q2 = 0; q2 < kCq; ++q2) {
+                    acc[q2] = fmaf(sQt[r * DKP + rp + 32 * q2], dov, acc[q2]);
+                    acc[q2] = fmaf(sKt[r * DKP + rp + 32 * q2], zb, acc[q2]);
+                }
             }
-            dSn[c * kSP + jj] = acc;
+#pragma unroll
+            for (int q2 = 0; q2 < kCq; ++q2) dSn[(rp + 32 * q2) * kSP + jj] = acc[q2];
         }
         __syncthreads();
         for (int idx = tid; idx < D * kNV; idx += kBTs) {
@@ -482,26 +512,43 @@ kda_bwd_chunk_kernel(const T *__restrict__ q, const T *__restrict__ k, const flo
         }
         glb[tid] = acc;
     }
+    // The 64 x 64 products below are register-blocked: thread t owns rows 4 (t / 32) .. + 3 (warp-
+    // uniform, so their operands are broadcast) and columns i0 = t % 32, i0 + 32: six shared loads
+    // feed eight FMAs.
+    const int rb = 4 * warp, i0 = lane;
     // dT[r][i] = beta_i sum_j dDelta[r][j] X1[i][j]
-    for (int p = tid; p < kC * kC; p += kBT2) {
-        const int r = p / kC, i = p % kC;
-        float acc = 0.f;
-        for (int j = 0; j < D; ++j) acc = fmaf(U0[r * D + j], U1[j * kC + i], acc);
-        Mm[r * CP + i] = bt[i] * acc;
+    {
+        float acc[4][2] = {};
+        for (int j = 0; j < D; ++j) {
+            const float x0 = U1[j * kC + i0], x1 = U1[j * kC + i0 + 32];
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+                const float a = U0[(rb + m) * D + j];
+                acc[m][0] = fmaf(a, x0, acc[m][0]);
+                acc[m][1] = fmaf(a, x1, acc[m][1]);
+            }
+        }
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+            Mm[(rb + m) * CP + i0] = bt[i0] * acc[m][0];
+            Mm[(rb + m) * CP + i0 + 32] = bt[i0 + 32] * acc[m][1];
+        }
     }
     if (cb == 0 && tid < kC) {  // dbeta, X1 part: sum_j Z[r][j] X1[r][j]
         float acc = 0.f;
         for (int j = 0; j < D; ++j) acc = fmaf(U2[tid * D + j], U1[j * kC + tid], acc);
         dbs[tid] = acc;
     }
-    float dKt[kRowsPerWarp], dQt[kRowsPerWarp], dKh[kRowsPerWarp];
+    // per-(row, channel) state products: this lane's channel, rows warp + 16 m; each S value is
+    // loaded once for the four rows
+    float dKt[kRowsPerWarp] = {}, dQt[kRowsPerWarp] = {}, dKh[kRowsPerWarp] = {};
+    for (int j = 0; j < D; ++j) {  // dK~ = -beta_r (Z S^T)[r][c]
+        const float sv = Ub[j * kCB + lane];
 #pragma unroll
-    for (int m = 0; m < kRowsPerWarp; ++m) {  // dK~ = -beta_r (Z S^T)[r][c]
-        const int r = warp + m * (kBT2 / 32);
-        float acc = 0.f;
-        for (int j = 0; j < D; ++j) acc = fmaf(U2[r * D + j], Ub[j * kCB + lane], acc);
-        dKt[m] = -bt[r] * acc;
+        for (int m = 0; m < kRowsPerWarp; ++m) dKt[m] = fmaf(U2[(warp + m * (kBT2 / 32)) * D + j], sv, dKt[m]);
     }
+#pragma unroll
+    for (int m = 0; m < kRowsPerWarp; ++m) dKt[m] *= -bt[warp + m * (kBT2 / 32)];
     __syncthreads();
     // ---- phase 2 staging: dO [C][D], Delta^T [D][C], dS'^T block [D][kCB] (S^T block stays)
     for (int idx = tid; idx < kC * D; idx += kBT2) cp_async4(U1 + idx, rec + R::Dt + idx);
@@ -514,23 +561,31 @@ kda_bwd_chunk_kernel(const T *__restrict__ q, const T *__restrict__ k, const flo
     }
     cp_async_wait<0>();
     __syncthreads();
-    for (int p = tid; p < kC * kC; p += kBT2) {  // dP[r][i] = sum_j dO[r][j] Delta[i][j]  (i <= r)
-        const int r = p / kC, i = p % kC;
-        float acc = 0.f;
-        if (i <= r)
-            for (int j = 0; j < D; ++j) acc = fmaf(U0[r * D + j], U1[j * kC + i], acc);
-        Pm[r * CP + i] = acc;
-    }
-#pragma unroll
-    for (int m = 0; m < kRowsPerWarp; ++m) {  // dQ~ = (dO S^T)[r][c],  dK^ = (Delta dS'^T)[r][c]
-        const int r = warp + m * (kBT2 / 32);
-        float a = 0.f, b = 0.f;
+    {  // dP[r][i] = sum_j dO[r][j] Delta[i][j]  (i <= r), register-blocked as dT
+        float acc[4][2] = {};
         for (int j = 0; j < D; ++j) {
-            a = fmaf(U0[r * D + j], Ub[j * kCB + lane], a);
-            b = fmaf(U1[j * kC + r], U2[j * kCB + lane], b);
+            const float x0 = U1[j * kC + i0], x1 = U1[j * kC + i0 + 32];
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+                const float a = U0[(rb + m) * D + j];
+                acc[m][0] = fmaf(a, x0, acc[m][0]);
+                acc[m][1] = fmaf(a, x1, acc[m][1]);
+            }
         }
-        dQt[m] = a;
-        dKh[m] = b;
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+            Pm[(rb + m) * CP + i0] = i0 <= rb + m ? acc[m][0] : 0.f;
+            Pm[(rb + m) * CP + i0 + 32] = i0 + 32 <= rb + m ? acc[m][1] : 0.f;
+        }
+    }
+    for (int j = 0; j < D; ++j) {  // dQ~ = (dO S^T)[r][c],  dK^ = (Delta dS'^T)[r][c]
+        const float sv = Ub[j * kCB + lane], dsv = U2[j * kCB + lane];
+#pragma unroll
+        for (int m = 0; m < kRowsPerWarp; ++m) {
+            const int r = warp + m * (kBT2 / 32);
+            dQt[m] = fmaf(U0[r * D + j], sv, dQt[m]);
+            dKh[m] = fmaf(U1[j * kC + r], dsv, dKh[m]);
+        }
     }
     if (warp == 0) {  // sum_j S[c][j] dS'[c][j] for the state-decay term of dG_L
         float acc = 0.f;
@@ -540,19 +595,40 @@ kda_bwd_chunk_kernel(const T *__restrict__ q, const T *__restrict__ k, const flo
     __syncthreads();
     // ---- W = dT T^T (T lower: m <= i) into the staging area, then dA = -strict_lower(T^T W)
     float *Wm = U;
-    for (int p = tid; p < kC * kC; p += kBT2) {
-        const int r = p / kC, i = p % kC;
-        float acc = 0.f;
-        for (int m = 0; m <= i; ++m) acc = fmaf(Mm[r * CP + m], Tm[i * CP + m], acc);
-        Wm[r * CP + i] = acc;
+    {  // T is stored with zeros above its diagonal, so the sums run over all m
+        float acc[4][2] = {};
+        for (int m = 0; m < kC; ++m) {
+            const float t0v = Tm[i0 * CP + m], t1v = Tm[(i0 + 32) * CP + m];
+#pragma unroll
+            for (int q2 = 0; q2 < 4; ++q2) {
+                const float a = Mm[(rb + q2) * CP + m];
+                acc[q2][0] = fmaf(a, t0v, acc[q2][0]);
+                acc[q2][1] = fmaf(a, t1v, acc[q2][1]);
+            }
+        }
+#pragma unroll
+        for (int q2 = 0; q2 < 4; ++q2) {
+            Wm[(rb + q2) * CP + i0] = acc[q2][0];
+            Wm[(rb + q2) * CP + i0 + 32] = acc[q2][1];
+        }
     }
     __syncthreads();
-    for (int p = tid; p < kC * kC; p += kBT2) {
-        const int r = p / kC, i = p % kC;
-        float acc = 0.f;
-        if (i < r)
-            for (int m = r; m < kC; ++m) acc = fmaf(Tm[m * CP + r], Wm[m * CP + i], acc);
-        Mm[r * CP + i] = -acc;
+    {  // dA[r][i] = -sum_{m >= r} T[m][r] W[m][i] for i < r (T[m][r] = 0 for m < r)
+        float acc[4][2] = {};
+        for (int m = rb; m < kC; ++m) {
+            const float w0 = Wm[m * CP + i0], w1 = Wm[m * CP + i0 + 32];
+#pragma unroll
+            for (int q2 = 0; q2 < 4; ++q2) {
+                const float t = Tm[m * CP + rb + q2];
+                acc[q2][0] = fmaf(t, w0, acc[q2][0]);
+                acc[q2][1] = fmaf(t, w1, acc[q2][1]);
+            }
+        }
+#pragma unroll
+        for (int q2 = 0; q2 < 4; ++q2) {
+            Mm[(rb + q2) * CP + i0] = i0 < rb + q2 ? -acc[q2][0] : 0.f;
+            Mm[(rb + q2) * CP + i0 + 32] = i0 + 32 < rb + q2 ? -acc[q2][1] : 0.f;
+        }
     }
     __syncthreads();
     if (cb == 0) {  // dbeta_r = sum_j Z[r][j] X1[r][j] + sum_{i<r} dA[r][i] Abar[r][i]  (one warp per row)
