@@ -12,8 +12,11 @@ from . import _lib
 from ._lib import KdaError, status_string  # noqa: F401
 from ._lib import KDA_PROLOGUE_GATE, KDA_PROLOGUE_L2NORM_QK  # noqa: F401
 
-__all__ = ["kda_chunk_fwd", "kda_chunk_fwd_workspace_size", "kda_decode_step", "kda_get_status",
-           "kda_status_string", "kda_trace_begin", "kda_trace_end", "KdaError", "Workspace"]
+__all__ = ["kda_chunk_fwd", "kda_chunk_fwd_ex", "kda_chunk_fwd_workspace_size", "kda_chunk_bwd",
+           "kda_chunk_bwd_workspace_size", "kda_decode_step", "kda_decode_multi", "kda_decode_multi_ex",
+           "kda_output_gate_norm", "kda_state_compose", "kda_get_status", "kda_status_string",
+           "kda_trace_begin", "kda_trace_end", "KdaError", "Workspace", "KDA_PROLOGUE_GATE",
+           "KDA_PROLOGUE_L2NORM_QK"]
 
 
 def _torch():
