@@ -234,7 +234,7 @@ kda_decode_multi_kernel(const T *__restrict__ q, const T *__restrict__ k, const 
                 const int i = warp + kMultiWarps * m;
                 const float ki = to_f(sk[buf][tt][i]);  // shared-memory reads (not the global-memory Elem loads)
                 const float qi = to_f(sq[buf][tt][i]);
-                const float ai = expf(sla[buf][tt][i]);
+                const float ai = ex2f(sla[buf][tt][i] * kLog2e);  // alpha_i by the hardware exp2
                 pqk = fmaf(qi, ki, pqk);
 #pragma unroll
                 for (int c = 0; c < VEC; ++c) {
