@@ -528,3 +528,26 @@ def test_prologue_gate_pins():
     _, _, la5 = oracle.prologue(z, z, np.random.default_rng(3).normal(size=(1, H, dk)) * 10, 2, A_log=A_log,
                                 dt_bias=dt_bias)
     assert np.all(la5 <= 0.0)
+
+
+# ----------------------------------------------------------------- chunkwise form of the backward
+def test_chunkwise_backward_matches_the_adjoint():
+    """The chunk-by-chunk reverse pass (the algebra of the GPU backward, oracle/chunkwise_bwd.py)
+    equals the token-by-token adjoint, which the finite-difference pins fix: 3 chunks with a ragged
+    last one, h0 and dh_T, two sequences."""
+    from oracle.chunkwise_bwd import chunkwise_bwd
+    rng = np.random.default_rng(80)
+    B, T, H, dk, dv = 2, 150, 2, 8, 6
+    q = rng.standard_normal((B, T, H, dk))
+    k = rng.standard_normal((B, T, H, dk)) / np.sqrt(dk)
+    v = rng.standard_normal((B, T, H, dv))
+    la = -np.log1p(np.exp(rng.standard_normal((B, T, H, dk)) + 1.0))
+    beta = 1 / (1 + np.exp(-rng.standard_normal((B, T, H))))
+    h0 = 0.3 * rng.standard_normal((B, H, dk, dv))
+    do = rng.standard_normal((B, T, H, dv))
+    dhT = rng.standard_normal((B, H, dk, dv))
+    ref = oracle.recurrent_bwd(q, k, v, la, beta, h0, None, do, dhT)
+    got = chunkwise_bwd(q, k, v, la, beta, h0, do, dhT, chunk=64)
+    for name in ("dq", "dk", "dv", "dlog_alpha", "dbeta", "dh0"):
+        err = np.abs(got[name] - ref[name]).max() / np.abs(ref[name]).max()
+        assert err <= 1e-12, f"{name}: {err:.3e}"
