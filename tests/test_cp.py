@@ -1,7 +1,7 @@
 """Context parallelism (kimi_delta_attention_29_b200.cp): one sequence split over the ranks of a
 process group, joined by one all-gather of each segment's affine state map [M | b].
 
-CPU (gloo, 2 and 3 ranks): the host-side flow -- exchange order, each rank's incoming state, empty
+CPU (gloo, 2 to 4 ranks): the host-side flow -- exchange order, each rank's incoming state, empty
 segments, h0 -- with the three per-rank steps (segment map, composition, rerun from the incoming
 state) computed in fp64 by the oracle; the ranks' outputs and final state must equal the oracle's
 single pass over the whole sequence.  The GPU tests run the library's kernels on one GPU, the ranks
@@ -74,7 +74,8 @@ def _worker(rank, world, port, bounds, use_h0, out):
     dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("bounds,use_h0", [([0, 10, 23], True), ([0, 9, 9, 23], False), ([0, 0, 5, 23], True)])
+@pytest.mark.parametrize("bounds,use_h0", [([0, 10, 23], True), ([0, 9, 9, 23], False), ([0, 0, 5, 23], True),
+                                           ([0, 5, 11, 11, 23], True)])
 def test_cp_ranks_match_single_pass(bounds, use_h0):
     import oracle
     world = len(bounds) - 1
