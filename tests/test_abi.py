@@ -233,3 +233,19 @@ def test_state_compose_rejects_on_host(lib):
     assert call(S_out=8 * A + 4) == _lib.KDA_ERR_MISALIGNED
     assert call(S_out=A + 4096) == _lib.KDA_ERR_ALIASING                     # output inside Mb
     assert call(S_in=A + 1024) == _lib.KDA_ERR_ALIASING
+
+
+def test_binding_constants_match_the_header():
+    """The binding's status codes and prologue flags are the header's, and its trace names cover
+    every kernel id the library reports."""
+    header = open(os.path.join(ROOT, "include", "kda.h")).read()
+    codes = dict((name, int(val)) for name, val in re.findall(r"\b(KDA_(?:OK|ERR_\w+))\s*=\s*(-?\d+)", header))
+    assert codes, "no status codes found in include/kda.h"
+    for name, val in codes.items():
+        assert getattr(_lib, name) == val, name
+    flags = dict((name, int(val)) for name, val in re.findall(r"\b(KDA_PROLOGUE_\w+)\s*=\s*(\d+)", header))
+    assert flags and all(getattr(_lib, n) == v for n, v in flags.items())
+    common = open(os.path.join(ROOT, "kimi_delta_attention_29_b200", "csrc", "kda_common.cuh")).read()
+    enum = re.search(r"enum KernelId \{(.*?)\};", common, re.S).group(1)
+    ids = [int(v) for v in re.findall(r"=\s*(\d+)", enum)]
+    assert sorted(ids) == sorted(_lib.KERNEL_NAMES), (ids, sorted(_lib.KERNEL_NAMES))
