@@ -34,8 +34,6 @@ UNIT = "tokens/s"
 PREFILL_BYTES_PER_TOKEN_HEAD = 768 + 512 + 4 + 256
 PREFILL_FLOP_PER_TOKEN_HEAD = 180224          # five C x d and three d x d products per token at C=64, d=128
 STATE_BYTES = 128 * 128 * 4                    # one fp32 state (h0 read or h_T write)
-REC_WRITE_BYTES = 74240                        # WY record bytes the intra-chunk kernel writes per chunk-head
-REC_READ_BYTES = 32768 + 16384 + 8192 + 512 + 16384  # record bytes the state kernel needs per chunk-head
 DECODE_BYTES_PER_STATE = 2 * STATE_BYTES + 3 * 256 + 512 + 4 + 256  # S read+write, q/k/v, gates, beta, o
 MULTI_TQ = (4, 16)  # tokens per kda_decode_multi call in the decode benchmark
 
@@ -51,6 +49,8 @@ def parse_args():
     p.add_argument("--no-decode", action="store_true")
     p.add_argument("--no-backward", action="store_true")
     p.add_argument("--no-cp", action="store_true")
+    p.add_argument("--no-workloads", action="store_true",
+                   help="skip the training-shape and packed-varlen prefill legs")
     p.add_argument("--backward-steps", type=int, default=3)
     p.add_argument("--cpu-seconds", type=float, default=12.0,
                    help="target CPU time of the oracle sample (0 skips the CPU baseline)")
@@ -246,6 +246,120 @@ def ncu_traffic(kernel: str, units: int):
     return rec["dram_bytes"] / rec["units"] * units
 
 
+def prefill_rooflines(kst, token_heads, chunk_heads, states, ms_per_step, peaks):
+    """Roofline objects of one prefill step on the operator's algorithmic basis: 1,540 B and
+    180,224 FLOP per token-head plus h0 read and h_T written (64 KiB each per (sequence, head)).
+    `roofline` divides those bytes by the dominant kernel's average launch duration (an upper bound
+    on what that kernel alone achieves); `operator_roofline` divides them by the whole step."""
+    dominant = max(kst, key=lambda n: kst[n]["total_ms"])
+    op_bytes = token_heads * PREFILL_BYTES_PER_TOKEN_HEAD + 2 * states * STATE_BYTES
+    op_flop = token_heads * PREFILL_FLOP_PER_TOKEN_HEAD
+    dom_s = kst[dominant]["avg_ms"] / 1e3
+    achieved = op_bytes / dom_s / 1e9
+    traffic = {n: ncu_traffic(n, chunk_heads) for n in kst}
+    traffic_step = None if any(v is None for v in traffic.values()) else sum(traffic.values())
+    roofline = {"kernel": dominant, "bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"], "traffic": traffic[dominant], "peak_source": peaks["source"],
+                "algorithmic_bytes_per_launch": op_bytes, "avg_ms": kst[dominant]["avg_ms"],
+                "tensor_frac_burst": op_flop / dom_s / 1e12 / peaks["bf16_tflops"],
+                "basis": "operator bytes (1,540 B per token-head + h0 + h_T) / the dominant kernel's average "
+                         "launch time; traffic = that kernel's DRAM read+write bytes per launch from "
+                         "profiles/ncu_traffic.json (null if its sources changed since the capture)"}
+    step_s = ms_per_step / 1e3
+    operator_roofline = {"bytes_per_step": op_bytes, "achieved_gbs": op_bytes / step_s / 1e9,
+                         "hbm_frac": op_bytes / step_s / 1e9 / peaks["hbm_gbs"], "flop_per_step": op_flop,
+                         "achieved_tflops": op_flop / step_s / 1e12,
+                         "tensor_frac_burst": op_flop / step_s / 1e12 / peaks["bf16_tflops"],
+                         "tensor_frac_sustained": op_flop / step_s / 1e12 / peaks["bf16_tflops_sustained"],
+                         "dram_bytes_per_step": traffic_step,
+                         "dram_over_algorithmic": None if traffic_step is None else traffic_step / op_bytes,
+                         "note": "whole call (all kernels) against the operator's algorithmic bytes / FLOPs"}
+    return roofline, operator_roofline
+
+
+def workload_bench(shape, args, dev, stream, peaks, barrier, max_over_ranks, world, cpu_seconds):
+    """kda_chunk_fwd on another of the page-shaped workloads (training shape, packed varlen batch):
+    tokens/s, the same roofline objects and an oracle sample on the host cores."""
+    import torch
+    import kimi_delta_attention_29_b200 as kda
+    from kimi_delta_attention_29_b200 import inputs as gen
+    x = gen.make_prefill_for(shape, seed=0, device=dev)
+    B, T, H = x["q"].shape[0], x["q"].shape[1], x["q"].shape[2]
+    cu = x["cu_seqlens"]
+    N = B if cu is None else cu.numel() - 1
+    ws = kda.Workspace(dev)
+
+    def step():
+        kda.kda_chunk_fwd(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], x["h0"], cu, workspace=ws,
+                          stream=stream)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize(dev)
+    assert kda.kda_get_status(ws) == 0, "device status after warm-up"
+    barrier()
+    steps = max(args.steps, 10)
+    kda.kda_trace_begin(16 * steps + 16)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    traces = kda.kda_trace_end()
+    barrier()
+    ms = max_over_ranks(e0.elapsed_time(e1)) / steps
+    kst = kernel_stats(traces)
+    tokens = B * T
+    if cu is None:
+        chunk_heads = B * ((T + 63) // 64) * H
+    else:
+        lens = (cu[1:] - cu[:-1]).cpu()
+        chunk_heads = int(((lens + 63) // 64).sum()) * H
+    roof, op_roof = prefill_rooflines(kst, tokens * H, chunk_heads, N * H, ms, peaks)
+    out = {"workload": shape.name, "tokens": tokens, "sequences": N, "ms_per_step": ms, "steps": steps,
+           "tokens_per_s": whole_job_rate(tokens, 1, world, ms), "roofline": roof, "operator_roofline": op_roof,
+           "kernels": kst, "l2": "inputs larger than the 126 MB L2: no flush"}
+    if cpu_seconds > 0:
+        out["cpu_baseline"] = oracle_sample_shape(x, cpu_seconds)
+    return out
+
+
+def oracle_sample_shape(x, target_s):
+    """The fp64 oracle on the first tokens of every sequence of a workload (all heads), sized to take
+    about target_s seconds; tokens/s over the tokens it covered."""
+    import torch
+    import oracle
+    q, k, v, la, beta = (x[n].cpu() for n in ("q", "k", "v", "log_alpha", "beta"))
+    cu = x["cu_seqlens"]
+    B, T, H = q.shape[:3]
+    starts = [0] * B if cu is None else [int(c) for c in cu[:-1].cpu()]
+    lens = [T] * B if cu is None else [int(b - a) for a, b in zip(cu[:-1].cpu(), cu[1:].cpu())]
+    f = lambda t: t.float().numpy()
+
+    def run(n_tok):
+        rows_q, rows_k, rows_v, rows_la, rows_b, cus = [], [], [], [], [], [0]
+        for i, (a, L) in enumerate(zip(starts, lens)):
+            m = min(L, n_tok)
+            b = i if cu is None else 0
+            rows_q.append(q[b, a:a + m]); rows_k.append(k[b, a:a + m]); rows_v.append(v[b, a:a + m])
+            rows_la.append(la[b, a:a + m]); rows_b.append(beta[b, a:a + m]); cus.append(cus[-1] + m)
+        cat = lambda rs: torch.cat(rs, 0)[None]
+        t0 = time.perf_counter()
+        oracle.recurrent(f(cat(rows_q)).astype("float64"), f(cat(rows_k)).astype("float64"),
+                         f(cat(rows_v)).astype("float64"), f(cat(rows_la)).astype("float64"),
+                         f(cat(rows_b)).astype("float64"), None, cu_seqlens=__import__("numpy").array(cus))
+        return time.perf_counter() - t0, cus[-1]
+
+    dt, tok = run(64)
+    n_tok = int(max(64, min(max(lens), 64 * target_s / max(dt, 1e-3))))
+    dt, tok = run(n_tok)
+    cores = oracle.num_threads()
+    return {"value": tok / dt, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"fp64 recurrent oracle on the first {n_tok} tokens of each of the {len(lens)} sequences "
+                      f"(all {H} heads; {tok} tokens); {dt:.1f} s on {cores} threads"}
+
+
 def gpu_arm(args):
     import torch
     import torch.distributed as dist
@@ -308,29 +422,9 @@ def gpu_arm(args):
 
     # per-kernel timing (live, CUDA events around each library kernel in the timed region)
     kst = kernel_stats(traces)
-    dominant = max(kst, key=lambda n: kst[n]["total_ms"])
     token_heads = B * T * H
     chunk_heads = B * ((T + 63) // 64) * H
-    kbytes = {
-        "kda_tc_prep_kernel": token_heads * (768 + 512 + 4) + chunk_heads * REC_WRITE_BYTES,
-        "kda_tc_state_kernel": chunk_heads * REC_READ_BYTES + token_heads * 256 + 2 * B * H * STATE_BYTES,
-    }
-    peak_bw = peaks["hbm_gbs"]
-    achieved = kbytes.get(dominant, 0) / (kst[dominant]["avg_ms"] / 1e3) / 1e9
-    roofline = {"kernel": dominant, "bound": "hbm", "achieved": achieved, "peak": peak_bw, "unit": "GB/s",
-                "frac": achieved / peak_bw, "traffic": ncu_traffic(dominant, chunk_heads), "peak_source": peaks["source"],
-                "traffic_note": "DRAM read+write bytes per launch from profiles/ncu_traffic.json (a T=8192 capture "
-                                "of the same kernel source, scaled by chunk-heads); null if the source changed",
-                "algorithmic_bytes_per_launch": kbytes.get(dominant, 0), "avg_ms": kst[dominant]["avg_ms"]}
-    op_bytes = token_heads * PREFILL_BYTES_PER_TOKEN_HEAD + 2 * B * H * STATE_BYTES
-    op_flop = token_heads * PREFILL_FLOP_PER_TOKEN_HEAD
-    op_gbs = op_bytes / (ms_per_step / 1e3) / 1e9
-    op_tflops = op_flop / (ms_per_step / 1e3) / 1e12
-    operator_roofline = {"bytes_per_step": op_bytes, "achieved_gbs": op_gbs, "hbm_frac": op_gbs / peak_bw,
-                         "flop_per_step": op_flop, "achieved_tflops": op_tflops,
-                         "tensor_frac": op_tflops / peaks["bf16_tflops_sustained"],
-                         "note": "whole call (all kernels) against the operator's algorithmic bytes / FLOPs; "
-                                 "tensor_frac against the sustained bf16 peak"}
+    roofline, operator_roofline = prefill_rooflines(kst, token_heads, chunk_heads, B * H, ms_per_step, peaks)
 
     # end to end through the public API with host buffers: pinned H2D of the step's inputs, the call,
     # D2H of the results (o and h_T), all inside the timed region
@@ -427,6 +521,12 @@ def gpu_arm(args):
     if not args.no_decode:
         decode = decode_bench(args, dev, stream, peaks, barrier, max_over_ranks)
 
+    workloads = None
+    if not args.no_workloads:
+        workloads = [workload_bench(shp, args, dev, stream, peaks, barrier, max_over_ranks, world,
+                                    args.cpu_seconds / 2 if rank == 0 and world == 1 else 0)
+                     for shp in (gen.TRAIN, gen.VARLEN)]
+
     cpu_baseline = None
     if rank == 0 and world == 1 and args.cpu_seconds > 0:
         cpu_baseline = oracle_sample(args.cpu_seconds)
@@ -436,6 +536,7 @@ def gpu_arm(args):
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config_dict(T),
             "roofline": roofline, "operator_roofline": operator_roofline, "cpu_baseline": cpu_baseline,
             "e2e": e2e, "gpu_launches": len(traces), "clocks": clk, "prologue": prologue, "epilogue": epilogue, "backward": backward, "context_parallel": cp_line, "decode": decode,
+            "workloads": workloads,
             "kernels": kst, "peaks": peaks}
     if rank == 0:
         print(json.dumps(line), flush=True)

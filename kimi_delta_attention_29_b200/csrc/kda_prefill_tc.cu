@@ -39,6 +39,7 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <mutex>
 
 #include "kda_common.cuh"
@@ -51,14 +52,14 @@ using namespace sm100;
 constexpr int D = 128;
 constexpr int C = kChunk;
 
-// Record of one (chunk, head) in the workspace.
-constexpr uint32_t REC_AQ = 0;        // [W; Q o e^G]: K-major sw128, 128 rows x 128 (2 atoms x 16 KiB)
-constexpr uint32_t REC_KH = 32768;    // K o e^{G_63 - G}: MN-major sw128, 64 k-rows x 128 (2 blocks x 8 KiB)
-constexpr uint32_t REC_P = 49152;     // P as an MN-major operand (P^T rows): sw128, 64 k-rows x 64 (8 KiB)
-constexpr uint32_t REC_U = 57344;     // U: bf16, four [64][32] blocks (one per 32-column slice), 64-byte swizzle
-constexpr uint32_t REC_GL = 73728;    // e^{G_63}: fp32 [128]
-constexpr uint32_t REC_BYTES = 74752;
-constexpr uint32_t REC_TX = 32768 + 16384 + 8192 + 4096 + 512;  // bytes one state CTA copies per chunk
+// Record of one (chunk, head) in the workspace: the operand images the state kernel's MMAs read.
+constexpr uint32_t REC_AQ = 0;        // [-W; Q o e^G]: K-major sw128, 128 rows x 128 (2 atoms x 16 KiB)
+constexpr uint32_t REC_P = 32768;     // P^T rows (row i: P[0..63][i]): MN-major sw128, 64 rows x 64 (8 KiB)
+constexpr uint32_t REC_KH = 40960;    // K o e^{G_63 - G}: MN-major sw128, 64 rows x 128 (2 atoms x 8 KiB)
+constexpr uint32_t REC_UT = 57344;    // U^T: fp32 [128 channels][64 rows], 16-byte chunk x of row j at x ^ (j & 7)
+constexpr uint32_t REC_GL = 90112;    // e^{G_63}: fp32 [128]
+constexpr uint32_t REC_TX = 90112 + 512;  // bytes the state kernel copies per chunk
+constexpr uint32_t REC_BYTES = 91136;
 
 struct TcLayout {
     size_t base_off, table_off, rec_off, total;
@@ -89,11 +90,6 @@ __device__ __forceinline__ __nv_bfloat162 as_bf2(uint32_t u) {
 // bf16 -> fp32 is exact: the bf16 bits are the high half of the fp32 word.
 __device__ __forceinline__ float2 unpack_bf16(uint32_t u) {
     return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xFFFF0000u));
-}
-// Byte offset of the 16-byte chunk x (elements 8x..8x+7) of k-row kr of a tile with 64-byte rows stored
-// with the 64-byte swizzle (MN-major sw64 operands, and the U slices of a record).
-__device__ __forceinline__ uint32_t sw64_chunk(uint32_t kr, uint32_t x) {
-    return kr * 64u + ((x ^ ((kr >> 1) & 3u)) << 4);
 }
 __device__ __forceinline__ float2 sub2(float2 a, float2 b) { return make_float2(a.x - b.x, a.y - b.y); }
 
@@ -585,18 +581,21 @@ kda_tc_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     }
     __syncthreads();
 
-    // ---- W = T Diag(beta) (K o e^G), U = T Diag(beta) V  (M=64, N=128, K=64)
+    // ---- W = T Diag(beta) (K o e^G) (M=64, N=128, K=64) and U^T = V^T (T Diag(beta))^T (M=128, N=64, K=64):
+    // U is produced transposed so that each TMEM lane holds one value channel, the row of U^T the
+    // state kernel reads per thread.
     if (ok && tid == 0) ok = mbar_wait(mbar + 3, 0);  // V tile landed
     if (ok && tid == 0) {
         tc_fence_after();
-        const uint32_t id_wu = idesc_bf16_f32(64, 128, 0, 1);
+        const uint32_t id_w = idesc_bf16_f32(64, 128, 0, 1);
+        const uint32_t id_ut = idesc_bf16_f32(128, 64, 1, 0);
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks) {
-            const uint64_t ad = smem_desc_sw128(smem_u32(TB) + ks * 32, 16, 1024);
+            const uint64_t tb = smem_desc_sw128(smem_u32(TB) + ks * 32, 16, 1024);
             const uint64_t bw = smem_desc_sw128(smem_u32(KT) + ks * 2048, 8192, 1024);
-            const uint64_t bu = smem_desc_sw128(smem_u32(Vimg) + ks * 2048, 8192, 1024);
-            mma_bf16_ss(tmem + 0, ad, bw, id_wu, ks > 0);
-            mma_bf16_ss(tmem + 128, ad, bu, id_wu, ks > 0);
+            const uint64_t av = smem_desc_sw128(smem_u32(Vimg) + ks * 2048, 8192, 1024);
+            mma_bf16_ss(tmem + 0, tb, bw, id_w, ks > 0);
+            mma_bf16_ss(tmem + 128, av, tb, id_ut, ks > 0);
         }
         mma_commit(mbar);
     }
@@ -604,27 +603,40 @@ kda_tc_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     ok = __syncthreads_and(ok);
     if (ok) {
         tc_fence_after();
-        // M=64 accumulator layout: row 16 q + l lives in TMEM lane 32 q + l (l < 16).  Warps 0-3 read
-        // W (columns 0..127), warps 4-7 read U (columns 128..255) of their lane quadrant.
-        const int quad = warp & 3, part = warp >> 2;
-        const int r = 16 * quad + lane;
+        const int quad = warp & 3;
         const uint32_t lane_base = (uint32_t)(quad * 32) << 16;
+        if (warp < 4) {
+            // W: M=64 accumulator, row 16 q + l in TMEM lane 32 q + l (l < 16); stored negated (the
+            // state kernel accumulates U^T - S^T W^T onto a U^T preload)
+            const int r = 16 * quad + lane;
 #pragma unroll 1
-        for (int cb = 0; cb < 4; ++cb) {
-            float vals[32];
-            tmem_ld32(tmem + lane_base + 128 * part + 32 * cb, vals);
-            tmem_wait_ld();
-            if (lane < 16) {
+            for (int cb = 0; cb < 4; ++cb) {
+                float vals[32];
+                tmem_ld32(tmem + lane_base + 32 * cb, vals);
+                tmem_wait_ld();
+                if (lane < 16) {
 #pragma unroll
-                for (int x = 0; x < 4; ++x) {
-                    const uint4 w = make_uint4(pack_bf16(vals[8 * x + 0], vals[8 * x + 1]), pack_bf16(vals[8 * x + 2], vals[8 * x + 3]),
-                                               pack_bf16(vals[8 * x + 4], vals[8 * x + 5]), pack_bf16(vals[8 * x + 6], vals[8 * x + 7]));
-                    if (part == 0) {
+                    for (int x = 0; x < 4; ++x) {
+                        const uint4 w = make_uint4(pack_bf16(-vals[8 * x + 0], -vals[8 * x + 1]), pack_bf16(-vals[8 * x + 2], -vals[8 * x + 3]),
+                                                   pack_bf16(-vals[8 * x + 4], -vals[8 * x + 5]), pack_bf16(-vals[8 * x + 6], -vals[8 * x + 7]));
                         *reinterpret_cast<uint4 *>(rec + REC_AQ + sw128_off(r, 32 * cb + 8 * x, 128)) = w;
-                    } else {  // U, one contiguous 64 x 32 block per 32-column slice
-                        *reinterpret_cast<uint4 *>(rec + REC_U + cb * 4096 + sw64_chunk(r, x)) = w;
                     }
                 }
+            }
+        } else {
+            // U^T: M=128 accumulator, channel j = TMEM lane, rows in columns 128..191; kept in fp32 (the
+            // state kernel copies it unchanged into its accumulator)
+            const int j = 32 * quad + lane;
+            uint8_t *urow = rec + REC_UT + j * 256;
+#pragma unroll 1
+            for (int cb = 0; cb < 2; ++cb) {
+                float vals[32];
+                tmem_ld32(tmem + lane_base + 128 + 32 * cb, vals);
+                tmem_wait_ld();
+#pragma unroll
+                for (int x = 0; x < 8; ++x)
+                    *reinterpret_cast<float4 *>(urow + (((8 * cb + x) ^ (j & 7)) << 4)) =
+                        make_float4(vals[4 * x], vals[4 * x + 1], vals[4 * x + 2], vals[4 * x + 3]);
             }
         }
     } else if (tid == 0) {
@@ -636,320 +648,371 @@ kda_tc_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
 }
 
 // ============================================================================ state-passing kernel
-// One CTA per (sequence, head, 32 value columns); the value columns of S evolve independently.
-// Warps 0-3 own the 128 state rows (TMEM lanes) and keep the fp32 master state in registers,
-// warp 4 streams the chunk records into a 2-stage shared-memory ring with bulk copies, warp 5
-// issues every MMA.  Per chunk i:
-//   D_a[i%2]  = [W; Q~] S        (M=128, N=32, K=128)   rows 0..63 -> Delta = U - W S (warps 0-1)
-//   D_b       = K^T Delta        (M=128, N=32, K=64)    -> S <- e^{G_63} S + D_b (warps 0-3)
-//   D_a[i%2] += [0; P] Delta     (M=128, N=32, K=64)    rows 64..127 = output, stored by warps 2-3
-//                                                        while chunk i+1 computes Delta and K^T Delta
-// Only the first two products are on the recurrence's critical path.  Warps 0, 1 and 5 meet at a
-// named barrier when Delta is ready, warps 0-3 and 5 at another when the next state image is.
-constexpr int kNV = 32;            // value columns per CTA
-constexpr int kStages = 2;
-constexpr uint32_t ST_AQ = 0, ST_KH = 32768, ST_AC = 49152, ST_U = 65536, ST_GL = 69632, ST_BYTES = 70656;
-constexpr uint32_t ST_SIMG = kStages * ST_BYTES;  // S (bf16): MN-major sw64, 128 k-rows x 32 (8 KiB)
-constexpr uint32_t ST_DIMG = ST_SIMG + 8192;      // Delta (bf16): MN-major sw64, 64 k-rows x 32 (4 KiB)
-constexpr uint32_t ST_BAR = ST_DIMG + 4096;
+// Persistent CTAs, one (sequence, head) unit at a time: the first unit is blockIdx.x, the next ones
+// come from a work counter in the workspace.  The state is carried transposed, S^T [d_v][d_k], in
+// tensor memory: TMEM lane j is value channel j, so every product has M = 128 (full tensor-core rate)
+// and the state-dependent operand is the A side, read straight from tensor memory.
+//   D2     fp32 master S^T; before each chunk's K^ product it is overwritten with S^T Diag(e^{G_63})
+//   A_S    bf16 copy of S^T (A operand of P1), 2 channels per 32-bit column
+//   A_D    bf16 Delta^T (A operand of P2a, P2b)
+//   D1[2]  per chunk parity: [U^T | .]; P1a adds -S^T W^T to the first half -> Delta^T, P1b writes
+//          (Q~ S)^T into the second half and P2b adds Delta^T P^T -> O^T
+// Per chunk (P1 in two halves so that the Delta^T half, which the recurrence waits for, comes first):
+//   P1a: D1[:, :64] += A_S (-W)^T   (M=128, N=64, K=128)  = Delta^T = U^T - S^T W^T
+//   P1b: D1[:, 64:]  = A_S Q~^T     (M=128, N=64, K=128)  = (Q~ S)^T
+//   P2a: D2 += A_D K^               (M=128, N=128, K=64)  = S_next^T = S^T Diag(e^{G_63}) + Delta^T K^
+//   P2b: D1[:, 64:] += A_D P^T      (M=128, N=64,  K=64)  = O^T = (Q~ S + P Delta)^T
+// Warps:
+//   0-15  the recurrence: Delta^T and the new S^T to bf16 operands (warp w: TMEM lanes 32 (w & 3) ..,
+//         column group w >> 2), then, off the critical path, the decayed state back into D2
+//   16-23 the previous chunk's output (through a shared-memory tile, one TMA tensor store per full
+//         chunk) and the U^T preload of the next chunk's D1 (warp 16 + 4 h + q: TMEM lanes 32 q ..,
+//         half h of the columns)
+//   24    issues the MMAs (one thread); 25 copies the chunk records into a 2-stage ring (one thread)
+constexpr int kChainWarps = 16, kAuxWarps = 8;
+constexpr int kMmaWarp = kChainWarps + kAuxWarps, kCopyWarp = kMmaWarp + 1;
+constexpr int kStateThreads = 32 * (kCopyWarp + 1);
+constexpr int kStStages = 2;
+constexpr uint32_t ST_OUT = kStStages * REC_BYTES;  // [2][64 rows][128] bf16 output staging tiles
+constexpr uint32_t ST_BAR = ST_OUT + 2 * 16384;
 constexpr uint32_t STATE_SMEM = ST_BAR + 256 + 1024;
-constexpr int kStateThreads = 192;        // warps 0-3 state rows, warp 4 copies, warp 5 MMAs
-constexpr uint32_t kStateTmemCols = 128;  // D_a[0] [0,32) | D_a[1] [32,64) | D_b [64,96)
+constexpr uint32_t TM_D1 = 0, TM_D2 = 256, TM_AS = 384, TM_AD = 448;
+constexpr uint32_t kStateTmemCols = 512;
 
-// 64-byte-swizzled operand descriptor (MN-major tiles 32 bf16 wide).
-__device__ __forceinline__ uint64_t smem_desc_sw64(uint32_t start, uint32_t sbo) {
-    uint64_t d = 0;
-    d |= (uint64_t)((start >> 4) & 0x3FFFu);
-    d |= (uint64_t)1 << 16;  // leading byte offset (unused: the tile is one 32-element atom wide)
-    d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
-    d |= (uint64_t)1 << 46;
-    d |= (uint64_t)4 << 61;  // 64-byte swizzle
-    return d;
-}
-// Named barrier over `count` threads that also ANDs a per-thread flag.  Barrier 1: warps 0-3 and 5
-// (160 threads); barrier 2: warps 0, 1 and 5 (96 threads).
-__device__ __forceinline__ bool bar_and(int id, int count, bool pred) {
-    uint32_t r;
-    asm volatile(
-        "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.and.pred q, %2, %3, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
-        : "=r"(r)
-        : "r"((uint32_t)pred), "r"(id), "r"(count)
-        : "memory");
-    return r != 0;
-}
-__device__ __forceinline__ bool bar_and160(bool pred) { return bar_and(1, 160, pred); }
-__device__ __forceinline__ bool bar_and96(bool pred) { return bar_and(2, 96, pred); }
-
-__global__ void __launch_bounds__(kStateThreads, 1)
-kda_tc_state_kernel(const uint8_t *__restrict__ records, const float *__restrict__ h0,
-                    const int *__restrict__ base, const int4 *__restrict__ table, int nc, int T_len, int H,
-                    __nv_bfloat16 *__restrict__ o, float *__restrict__ h_T, int *status) {
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t *sm = align1024(smem_raw);
-    uint8_t *Simg = sm + ST_SIMG;
-    uint8_t *Dimg = sm + ST_DIMG;
-    // Each barrier completes once per chunk (per use of a stage) and cannot complete a second
-    // time before its waiters have seen the first, so the parity waits are unambiguous.
-    uint64_t *full = reinterpret_cast<uint64_t *>(sm + ST_BAR);  // [kStages] record landed
-    uint64_t *empty = full + kStages;   // [kStages] the three products of the stage's chunk are done
-    uint64_t *bar_w = empty + kStages;  // [W; Q~] S done
-    uint64_t *bar_b = bar_w + 1;        // K^T Delta done
-    uint64_t *bar_c = bar_b + 1;        // [0; P] Delta done (and every earlier product)
-    uint32_t *s_tmem = reinterpret_cast<uint32_t *>(bar_c + 1);
-
-    int bid = blockIdx.x;
-    const int slice = bid % (D / kNV);
-    bid /= D / kNV;
-    const int h = bid % H, n = bid / H, j0 = slice * kNV;
-    if (status[0] != 0) return;  // malformed cu_seqlens: nothing to do
-    int c_begin, nchunks;
-    if (table) {
+__device__ __forceinline__ void state_unit(int u, int H, int nc, const int *base, const int *order, int &n,
+                                           int &h, int &c_begin, int &nchunks) {
+    h = u % H;
+    const int r = u / H;
+    if (base) {
+        n = order ? order[r] : r;
         c_begin = base[n];
         nchunks = base[n + 1] - c_begin;
     } else {
+        n = r;
         c_begin = n * nc;
         nchunks = nc;
     }
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+}
 
+__global__ void __launch_bounds__(kStateThreads, 1)
+kda_tc_state_kernel(const __grid_constant__ CUtensorMap tm_o, const uint8_t *__restrict__ records,
+                    const float *__restrict__ h0, const int *__restrict__ base,
+                    const int4 *__restrict__ table, const int *__restrict__ order, int num_units, int nc, int T_len,
+                    int H, __nv_bfloat16 *__restrict__ o, float *__restrict__ h_T, int *status,
+                    int *unit_counter) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = align1024(smem_raw);
+    uint64_t *full = reinterpret_cast<uint64_t *>(sm + ST_BAR);  // [2] record landed in the stage
+    uint64_t *empty = full + 2;   // [2] every MMA reading the stage is done
+    uint64_t *b_p1 = empty + 2;   // P1a done (and every earlier MMA)
+    uint64_t *b_p2a = b_p1 + 1;   // P2a done
+    uint64_t *b_p2b = b_p2a + 1;  // P2b done
+    uint64_t *b_dr = b_p2b + 1;   // Delta^T operand in tensor memory (chain warps)
+    uint64_t *b_sr = b_dr + 1;    // S^T operand in tensor memory (chain warps)
+    uint64_t *b_d2 = b_sr + 1;    // D2 holds the decayed state (chain warps)
+    uint64_t *b_d1 = b_d2 + 1;    // [2] D1 buffer preloaded with U^T (aux warps)
+    uint64_t *b_drain = b_d1 + 2; // final MMA drain
+    uint32_t *s_tmem = reinterpret_cast<uint32_t *>(b_drain + 1);
+    volatile int *s_abort = reinterpret_cast<volatile int *>(s_tmem + 1);
+    volatile int *s_unit = s_abort + 1;
+
+    if (status[0] != 0) return;  // malformed cu_seqlens: nothing to do
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     if (tid == 0) {
-        for (int s = 0; s < kStages; ++s) {
+        for (int s = 0; s < 2; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
+            mbar_init(&b_d1[s], kAuxWarps);
         }
-        mbar_init(bar_w, 1);
-        mbar_init(bar_b, 1);
-        mbar_init(bar_c, 1);
+        mbar_init(b_p1, 1);
+        mbar_init(b_p2a, 1);
+        mbar_init(b_p2b, 1);
+        mbar_init(b_dr, kChainWarps);
+        mbar_init(b_sr, kChainWarps);
+        mbar_init(b_d2, kChainWarps);
+        mbar_init(b_drain, 1);
         mbar_fence_init();
+        *s_abort = 0;
+        *s_unit = blockIdx.x;
     }
     if (warp == 0) {
         tmem_alloc(s_tmem, kStateTmemCols);
         tmem_relinquish();
     }
-    for (int e = tid; e < kStages * 512; e += kStateThreads) {  // zero half of each [0; P] operand
-        const int s = e / 512, x = e % 512;
-        reinterpret_cast<uint4 *>(sm + s * ST_BYTES + ST_AC)[x] = make_uint4(0u, 0u, 0u, 0u);
-    }
-    fence_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *s_tmem;
-    const uint32_t D_A = tmem + 0, D_B = tmem + 64;
+    const int q = warp & 3;                       // TMEM lane quadrant of this warp
+    const int j = 32 * q + lane;                  // value channel = TMEM lane (SIMT warps)
+    const uint32_t lb = (uint32_t)(32 * q) << 16;
+    const int aux_tid0 = 32 * kChainWarps;        // aux thread that issues the TMA output stores
 
-    if (warp == 4) {
-        // ------------------------------------------------ bulk copies (one thread)
-        if (lane == 0) {
-            bool ok = true;
-            auto issue_load = [&](int i) {
-                const int s = i % kStages;
-                uint8_t *st = sm + s * ST_BYTES;
-                const uint8_t *rec = records + ((size_t)(c_begin + i) * H + h) * REC_BYTES;
-                mbar_arrive_expect_tx(&full[s], REC_TX);
-                bulk_g2s(st + ST_AQ, rec + REC_AQ, 32768, &full[s]);
-                bulk_g2s(st + ST_KH, rec + REC_KH, 16384, &full[s]);
-                bulk_g2s(st + ST_AC + 8192, rec + REC_P, 8192, &full[s]);
-                bulk_g2s(st + ST_U, rec + REC_U + slice * 4096, 4096, &full[s]);
-                bulk_g2s(st + ST_GL, rec + REC_GL, 512, &full[s]);
-            };
-            for (int i = 0; i < kStages && i < nchunks; ++i) issue_load(i);
-            for (int i = 0; i + kStages < nchunks && ok; ++i) {
-                ok = mbar_wait(&empty[i % kStages], (i / kStages) & 1);
-                if (ok) issue_load(i + kStages);
-            }
-            if (!ok) set_status(status, KDA_ERR_TIMEOUT);
-        }
-        __syncwarp();
-    } else if (warp == 5) {
-        // ------------------------------------------------ MMA issue (one thread)
-        const uint32_t id_a = idesc_bf16_f32(128, kNV, 0, 1);  // [W; Q~] S
-        const uint32_t id_b = idesc_bf16_f32(128, kNV, 1, 1);  // K^T Delta (K^ stored MN-major), [0; P] Delta
-        const uint64_t d_s = smem_desc_sw64(smem_u32(Simg), 512);
-        const uint64_t d_d = smem_desc_sw64(smem_u32(Dimg), 512);
-        bool ok = bar_and160(true);
-        for (int i = 0; i < nchunks && ok; ++i) {
-            const int s = i % kStages;
-            const uint32_t st = smem_u32(sm + s * ST_BYTES);
-            const uint64_t d_aq = smem_desc_sw128(st + ST_AQ, 16, 1024);
-            const uint64_t d_kh = smem_desc_sw128(st + ST_KH, 8192, 1024);
-            const uint64_t d_ac = smem_desc_sw128(st + ST_AC, 8192, 1024);  // MN-major: zero atom, then P
-            const uint32_t d_a = D_A + 32 * (i & 1);
-            bool w_ok = true;
+    uint32_t gc0 = 0;             // chunks this CTA has processed before the current unit
+    int last_load[2] = {-1, -1};  // copy thread: global chunk index last loaded into each stage
+    for (;;) {
+        const int u = *s_unit;
+        if (u >= num_units) break;
+        int n, h, c_begin, nchunks;
+        state_unit(u, H, nc, base, order, n, h, c_begin, nchunks);
+        const size_t soff = ((size_t)n * H + h) * D * D + j;  // S[k][j] at soff + k * D
+        auto wwait = [&](uint64_t *bar, uint32_t parity) {
+            return __all_sync(0xffffffffu, mbar_wait_or_abort(bar, parity, s_abort));
+        };
+        auto arrive = [&](uint64_t *bar) {
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar);
+        };
+
+        if (warp == kCopyWarp) {
+            // ------------------------------------------------ record copies (one thread)
             if (lane == 0) {
-                w_ok = mbar_wait(&full[s], (i / kStages) & 1);
-                if (w_ok) {
-                    tc_fence_after();
-#pragma unroll
-                    for (int ks = 0; ks < 8; ++ks)  // descriptor start fields advance in 16-byte units
-                        mma_bf16_ss(d_a, d_aq + (uint64_t)(((ks >> 2) * 16384 + (ks & 3) * 32) >> 4),
-                                    d_s + (uint64_t)((ks * 1024) >> 4), id_a, ks > 0);
-                    mma_commit(bar_w);
+                for (int i = 0; i < nchunks; ++i) {
+                    const uint32_t gc = gc0 + i, s = gc & 1;
+                    if (gc >= 2 && !mbar_wait_or_abort(&empty[s], ((gc >> 1) + 1) & 1, s_abort)) {
+                        *s_abort = 1;
+                        break;
+                    }
+                    uint8_t *st = sm + s * REC_BYTES;
+                    const uint8_t *rec = records + ((size_t)(c_begin + i) * H + h) * REC_BYTES;
+                    mbar_arrive_expect_tx(&full[s], REC_TX);
+                    bulk_g2s(st, rec, 32768, &full[s]);
+                    bulk_g2s(st + 32768, rec + 32768, 24576, &full[s]);
+                    bulk_g2s(st + REC_UT, rec + REC_UT, 32768, &full[s]);
+                    bulk_g2s(st + REC_GL, rec + REC_GL, 512, &full[s]);
+                    last_load[s] = (int)gc;
                 }
-            }
-            // Delta is in shared memory (warps 0-1); a failure anywhere is carried to barrier 1
-            const bool d_ok = bar_and96(__shfl_sync(0xffffffffu, w_ok, 0));
-            if (d_ok && lane == 0) {
-                tc_fence_after();
-#pragma unroll
-                for (int ks = 0; ks < 4; ++ks)
-                    mma_bf16_ss(D_B, d_kh + (uint64_t)((ks * 2048) >> 4), d_d + (uint64_t)((ks * 1024) >> 4), id_b,
-                                ks > 0);
-                mma_commit(bar_b);
-#pragma unroll
-                for (int ks = 0; ks < 4; ++ks)
-                    mma_bf16_ss(d_a, d_ac + (uint64_t)((ks * 2048) >> 4), d_d + (uint64_t)((ks * 1024) >> 4), id_b, 1);
-                mma_commit(bar_c);
-                mma_commit(&empty[s]);
             }
             __syncwarp();
-            ok = bar_and160(d_ok);
-        }
-    } else {
-        // ------------------------------------------------ warps 0-3: state row t = tid (TMEM lane)
-        const int t = tid;
-        const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-        const size_t soff = (((size_t)n * H + h) * D + t) * D + j0;
-        float S[kNV];
+        } else if (warp == kMmaWarp) {
+            // ------------------------------------------------ MMA issue (one thread)
+            if (lane == 0) {
+                const uint32_t id_p1 = idesc_bf16_f32(128, 64, 0, 0);
+                const uint32_t id_p2a = idesc_bf16_f32(128, 128, 0, 1);
+                const uint32_t id_p2b = idesc_bf16_f32(128, 64, 0, 1);
+                // operand descriptors of stage 0; stage 1 is REC_BYTES / 16 further in the start field
+                const uint32_t st0 = smem_u32(sm);
+                uint64_t dw[8], dq[8], dk[4], dp[4];
 #pragma unroll
-        for (int x = 0; x < kNV / 4; ++x) {
-            const float4 w = h0 ? *reinterpret_cast<const float4 *>(h0 + soff + 4 * x) : make_float4(0.f, 0.f, 0.f, 0.f);
-            S[4 * x] = w.x; S[4 * x + 1] = w.y; S[4 * x + 2] = w.z; S[4 * x + 3] = w.w;
-        }
-        auto store_S_image = [&]() {
-#pragma unroll
-            for (int x = 0; x < 4; ++x)
-                *reinterpret_cast<uint4 *>(Simg + sw64_chunk(t, x)) =
-                    make_uint4(pack_bf16(S[8 * x], S[8 * x + 1]), pack_bf16(S[8 * x + 2], S[8 * x + 3]),
-                               pack_bf16(S[8 * x + 4], S[8 * x + 5]), pack_bf16(S[8 * x + 6], S[8 * x + 7]));
-        };
-        store_S_image();
-        fence_async_smem();
-        bool ok = bar_and160(true);
-
-        // output rows of chunk i: D_a[i % 2] rows 64..127, read by warps 2 and 3 (row = t - 64)
-        auto write_o = [&](int i) {
-            int64_t t0;
-            int L;
-            if (table) {
-                const int4 e = table[c_begin + i];
-                t0 = e.y;
-                L = e.z;
-            } else {
-                t0 = (int64_t)n * T_len + (int64_t)i * C;
-                L = min(C, T_len - i * C);
-            }
-            float ov[32];
-            tmem_ld32(D_A + 32 * (i & 1) + lane_base, ov);
-            tmem_wait_ld();
-            uint32_t pk[16];  // four 16-byte chunks (4 words each) of this lane's row
-#pragma unroll
-            for (int e = 0; e < 16; ++e) pk[e] = pack_bf16(ov[2 * e], ov[2 * e + 1]);
-            // Lanes l and l ^ 1 (rows 2p and 2p+1 of the chunk) trade 16-byte chunks so that every
-            // store instruction fills whole 32-byte sectors: for chunk pair (2c, 2c+1), the first
-            // store writes both chunks of the even row, the second both chunks of the odd row.
-            const bool odd = lane & 1;
-            const int row = t - 64;
-            const int even_row = row & ~1, odd_row = row | 1;
-#pragma unroll
-            for (int c = 0; c < 2; ++c) {
-                uint4 mine, theirs;
-                uint32_t mv[4], tv[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const uint32_t give = odd ? pk[8 * c + e] : pk[8 * c + 4 + e];  // even gives 2c+1, odd gives 2c
-                    tv[e] = __shfl_xor_sync(0xffffffffu, give, 1);
-                    mv[e] = odd ? pk[8 * c + 4 + e] : pk[8 * c + e];
+                for (int ks = 0; ks < 8; ++ks) {
+                    dw[ks] = smem_desc_sw128(st0 + REC_AQ + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
+                    dq[ks] = smem_desc_sw128(st0 + REC_AQ + 8192 + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
                 }
-                mine = make_uint4(mv[0], mv[1], mv[2], mv[3]);
-                theirs = make_uint4(tv[0], tv[1], tv[2], tv[3]);
-                const int chunk16 = 2 * c + (odd ? 1 : 0);
-                // store 1: the even row (even lane: its own chunk 2c, odd lane: the even row's 2c+1)
-                if (even_row < L)
-                    reinterpret_cast<uint4 *>(o + ((size_t)(t0 + even_row) * H + h) * D + j0)[chunk16] = odd ? theirs : mine;
-                // store 2: the odd row (even lane: the odd row's chunk 2c, odd lane: its own 2c+1)
-                if (odd_row < L)
-                    reinterpret_cast<uint4 *>(o + ((size_t)(t0 + odd_row) * H + h) * D + j0)[chunk16] = odd ? mine : theirs;
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks) {
+                    dk[ks] = smem_desc_sw128(st0 + REC_KH + ks * 2048, 8192, 1024);
+                    dp[ks] = smem_desc_sw128(st0 + REC_P + ks * 2048, 8192, 1024);
+                }
+                for (int i = 0; i < nchunks; ++i) {
+                    const uint32_t gc = gc0 + i, s = gc & 1, b = gc & 1;
+                    const uint64_t so = s ? (uint64_t)(REC_BYTES >> 4) : 0ull;
+                    const uint32_t d1 = tmem + TM_D1 + 128 * b;
+                    bool ok = mbar_wait_or_abort(b_sr, gc & 1, s_abort) &&
+                              mbar_wait_or_abort(&b_d1[b], (gc >> 1) & 1, s_abort) &&
+                              mbar_wait_or_abort(&full[s], (gc >> 1) & 1, s_abort);
+                    if (!ok) { *s_abort = 1; break; }
+                    tc_fence_after();
+#pragma unroll
+                    for (int ks = 0; ks < 8; ++ks)  // -W: rows 0..63 of the [-W; Q~] image
+                        mma_bf16_ts(d1, tmem + TM_AS + 8 * ks, dw[ks] + so, id_p1, 1);
+                    mma_commit(b_p1);
+#pragma unroll
+                    for (int ks = 0; ks < 8; ++ks)  // Q~: rows 64..127
+                        mma_bf16_ts(d1 + 64, tmem + TM_AS + 8 * ks, dq[ks] + so, id_p1, ks > 0);
+                    ok = mbar_wait_or_abort(b_dr, gc & 1, s_abort) && mbar_wait_or_abort(b_d2, gc & 1, s_abort);
+                    if (!ok) { *s_abort = 1; break; }
+                    tc_fence_after();
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks)
+                        mma_bf16_ts(tmem + TM_D2, tmem + TM_AD + 8 * ks, dk[ks] + so, id_p2a, 1);
+                    mma_commit(b_p2a);
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks)
+                        mma_bf16_ts(d1 + 64, tmem + TM_AD + 8 * ks, dp[ks] + so, id_p2b, 1);
+                    mma_commit(b_p2b);
+                    mma_commit(&empty[s]);
+                }
             }
-        };
-
-        for (int i = 0; i < nchunks && ok; ++i) {
-            const int s = i % kStages;
-            const uint8_t *st = sm + s * ST_BYTES;
-            const uint32_t d_a = D_A + 32 * (i & 1);
-            // (1) stage data this thread reads (before the stage can be refilled)
-            bool w_ok = mbar_wait(&full[s], (i / kStages) & 1);
-            const float gl = reinterpret_cast<const float *>(st + ST_GL)[t];
-            // (2) warps 0-1: Delta = U - W S once the previous chunk's [0; P] Delta no longer reads
-            //     the Delta image; warps 2-3: output of the previous chunk
-            if (i > 0) w_ok = w_ok && mbar_wait(bar_c, (i - 1) & 1);
-            w_ok = w_ok && mbar_wait(bar_w, i & 1);
-            if (__all_sync(0xffffffffu, w_ok)) {
-                tc_fence_after();
-                if (warp < 2) {
-                    float ws[32];
-                    tmem_ld32(d_a + lane_base, ws);
-                    uint4 u4s[4];  // all loads first: the Delta stores below could alias them
+            __syncwarp();
+        } else if (warp < kChainWarps) {
+            // ------------------------------------------------ recurrence warps
+            const int g = warp >> 2;  // columns: Delta^T 16 g .., S^T 32 g ..
+            auto store_as = [&](const float (&sv)[32]) {
+                uint32_t w[16];
 #pragma unroll
-                    for (int x = 0; x < 4; ++x) u4s[x] = *reinterpret_cast<const uint4 *>(st + ST_U + sw64_chunk(t, x));
-                    tmem_wait_ld();
+                for (int e = 0; e < 16; ++e) w[e] = pack_bf16(sv[2 * e], sv[2 * e + 1]);
+                tmem_st16(tmem + TM_AS + lb + 16 * g, w);
+                arrive(b_sr);
+            };
+            // D2[:, 32 g ..] <- S^T Diag(e^{G_63}) of chunk gc, for its K^ product
+            auto store_d2 = [&](uint32_t gc, const float (&sv)[32]) -> bool {
+                if (!wwait(&full[gc & 1], (gc >> 1) & 1)) return false;
+                const float *gl = reinterpret_cast<const float *>(sm + (gc & 1) * REC_BYTES + REC_GL) + 32 * g;
+                uint32_t w[32];
 #pragma unroll
-                    for (int x = 0; x < 4; ++x) {
-                        const uint4 u4 = u4s[x];
-                        const uint32_t uw[4] = {u4.x, u4.y, u4.z, u4.w};
-                        uint32_t dw[4];
+                for (int x = 0; x < 8; ++x) {
+                    const float4 e4 = *reinterpret_cast<const float4 *>(gl + 4 * x);
+                    w[4 * x + 0] = __float_as_uint(sv[4 * x + 0] * e4.x);
+                    w[4 * x + 1] = __float_as_uint(sv[4 * x + 1] * e4.y);
+                    w[4 * x + 2] = __float_as_uint(sv[4 * x + 2] * e4.z);
+                    w[4 * x + 3] = __float_as_uint(sv[4 * x + 3] * e4.w);
+                }
+                tmem_st32(tmem + TM_D2 + lb + 32 * g, w);
+                arrive(b_d2);
+                return true;
+            };
+            bool ok = true;
+            float sv[32];
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const float2 uf = unpack_bf16(uw[e]);
-                            dw[e] = pack_bf16(uf.x - ws[8 * x + 2 * e], uf.y - ws[8 * x + 2 * e + 1]);
-                        }
-                        *reinterpret_cast<uint4 *>(Dimg + sw64_chunk(t, x)) = make_uint4(dw[0], dw[1], dw[2], dw[3]);
+            for (int kk = 0; kk < 32; ++kk) sv[kk] = h0 ? __ldg(h0 + soff + (size_t)(32 * g + kk) * D) : 0.f;
+            if (nchunks == 0) {
+                if (h_T) {
+#pragma unroll
+                    for (int kk = 0; kk < 32; ++kk) h_T[soff + (size_t)(32 * g + kk) * D] = sv[kk];
+                }
+            } else {
+                store_as(sv);
+                ok = store_d2(gc0, sv);
+                for (int i = 0; i < nchunks && ok; ++i) {
+                    const uint32_t gc = gc0 + i, b = gc & 1;
+                    // Delta^T -> bf16 operand
+                    if (!wwait(b_p1, gc & 1)) { ok = false; break; }
+                    tc_fence_after();
+                    {
+                        float dv[16];
+                        tmem_ld16(tmem + TM_D1 + 128 * b + lb + 16 * g, dv);
+                        tmem_wait_ld();
+                        uint32_t w[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) w[e] = pack_bf16(dv[2 * e], dv[2 * e + 1]);
+                        tmem_st8(tmem + TM_AD + lb + 8 * g, w);
+                        arrive(b_dr);
                     }
-                } else if (i > 0) {
-                    write_o(i - 1);
+                    // new state -> bf16 operand, or h_T after the last chunk
+                    if (!wwait(b_p2a, gc & 1)) { ok = false; break; }
+                    tc_fence_after();
+                    float nv[32];
+                    tmem_ld32(tmem + TM_D2 + lb + 32 * g, nv);
+                    tmem_wait_ld();
+                    if (i + 1 < nchunks) {
+                        store_as(nv);
+                        if (!store_d2(gc + 1, nv)) { ok = false; break; }
+                    } else if (h_T) {
+#pragma unroll
+                        for (int kk = 0; kk < 32; ++kk) h_T[soff + (size_t)(32 * g + kk) * D] = nv[kk];
+                    }
                 }
-            } else {
-                w_ok = false;
             }
-            tc_fence_before();
-            if (warp < 2) {  // hand Delta to the MMA warp; warps 2-3 go on (their output stores overlap K^T Delta)
-                fence_async_smem();
-                w_ok = bar_and96(w_ok);
-            }
-            // (3) S <- e^{G_63} S + K^T Delta and its bf16 operand image
-            w_ok = w_ok && mbar_wait(bar_b, i & 1);
-            if (__all_sync(0xffffffffu, w_ok)) {
-                tc_fence_after();
-                float upd[32];
-                tmem_ld32(D_B + lane_base, upd);
+            if (!ok) *s_abort = 1;
+        } else {
+            // ------------------------------------------------ aux warps
+            const int hf = (warp - kChainWarps) >> 2;  // column half
+            const int atid = tid - aux_tid0;          // 0..255
+            auto chunk_rows = [&](int i, int64_t &t0, int &L) {
+                if (table) {
+                    const int4 e = table[c_begin + i];
+                    t0 = e.y;
+                    L = e.z;
+                } else {
+                    t0 = (int64_t)n * T_len + (int64_t)i * C;
+                    L = min(C, T_len - i * C);
+                }
+            };
+            // D1[b][:, 32 hf .. +32] <- U^T of chunk gc (its record is in stage gc & 1)
+            auto preload_d1 = [&](uint32_t gc) -> bool {
+                const uint32_t s = gc & 1, b = gc & 1;
+                if (!wwait(&full[s], (gc >> 1) & 1)) return false;
+                const uint8_t *urow = sm + s * REC_BYTES + REC_UT + j * 256;
+                uint32_t uf[32];
+#pragma unroll
+                for (int x = 0; x < 8; ++x) {
+                    const uint4 w = *reinterpret_cast<const uint4 *>(urow + (((8 * hf + x) ^ (j & 7)) << 4));
+                    uf[4 * x] = w.x; uf[4 * x + 1] = w.y; uf[4 * x + 2] = w.z; uf[4 * x + 3] = w.w;
+                }
+                tmem_st32(tmem + TM_D1 + 128 * b + lb + 32 * hf, uf);
+                arrive(&b_d1[b]);
+                return true;
+            };
+            // output of chunk i (O^T in D1[b] columns 64..127; this thread: channel j, rows 32 hf ..
+            // 32 hf + 31) -> staging tile [64][128] bf16 -> global.  The tile of parity b is written
+            // again two chunks later; aux_tid0 waits for every earlier TMA store to finish reading
+            // before it passes the barrier that precedes those writes.
+            auto store_out = [&](int i, uint32_t gc) {
+                float ov[32];
+                tmem_ld32(tmem + TM_D1 + 128 * (gc & 1) + lb + 64 + 32 * hf, ov);
                 tmem_wait_ld();
+                uint16_t *tile = reinterpret_cast<uint16_t *>(sm + ST_OUT + (gc & 1) * 16384);
 #pragma unroll
-                for (int j = 0; j < kNV; ++j) S[j] = fmaf(gl, S[j], upd[j]);
-                store_S_image();
-            } else {
-                w_ok = false;
-            }
-            tc_fence_before();
-            fence_async_smem();
-            ok = bar_and160(w_ok);
-        }
-        if (ok && nchunks > 0) {  // output of the last chunk
-            bool w_ok = mbar_wait(bar_c, (nchunks - 1) & 1);
-            if (__all_sync(0xffffffffu, w_ok)) {
-                tc_fence_after();
-                if (warp >= 2) write_o(nchunks - 1);
-            } else {
-                ok = false;
-            }
-        }
-        if (!ok) {
-            if (lane == 0) set_status(status, KDA_ERR_TIMEOUT);
-        } else if (h_T) {
-            float *hrow = h_T + soff;
+                for (int rr = 0; rr < 32; rr += 2) {
+                    const uint32_t w = pack_bf16(ov[rr], ov[rr + 1]);
+                    tile[(32 * hf + rr) * D + j] = (uint16_t)(w & 0xFFFFu);
+                    tile[(32 * hf + rr + 1) * D + j] = (uint16_t)(w >> 16);
+                }
+                int64_t t0;
+                int L;
+                chunk_rows(i, t0, L);
+                fence_async_smem();
+                if (tid == aux_tid0) bulk_wait_group_read<0>();
+                asm volatile("bar.sync 1, %0;" ::"n"(32 * kAuxWarps) : "memory");
+                if (L == C) {
+                    if (tid == aux_tid0) {
+                        tma_store_3d(&tm_o, tile, 0, h, (int)t0);
+                        bulk_commit_group();
+                    }
+                } else {
 #pragma unroll
-            for (int x = 0; x < kNV / 4; ++x)
-                reinterpret_cast<float4 *>(hrow)[x] = make_float4(S[4 * x], S[4 * x + 1], S[4 * x + 2], S[4 * x + 3]);
+                    for (int e = 0; e < 4; ++e) {
+                        const int c16 = atid + 32 * kAuxWarps * e, r = c16 >> 4;
+                        if (r < L)
+                            reinterpret_cast<uint4 *>(o + ((size_t)(t0 + r) * H + h) * D)[c16 & 15] =
+                                reinterpret_cast<const uint4 *>(tile)[c16];
+                    }
+                }
+            };
+
+            bool ok = true;
+            if (nchunks > 0) {
+                ok = preload_d1(gc0);
+                for (int i = 0; i < nchunks && ok; ++i) {
+                    const uint32_t gc = gc0 + i;
+                    const bool more = i + 1 < nchunks;
+                    // P1a of this chunk done => P2b of the previous one done: its output is final.
+                    // Waited for every chunk: a parity wait is only unambiguous when the phase before
+                    // the awaited one is known to be complete.
+                    if (!wwait(b_p1, gc & 1)) { ok = false; break; }
+                    if (i > 0) {
+                        tc_fence_after();
+                        store_out(i - 1, gc - 1);
+                    }
+                    if (more && !preload_d1(gc + 1)) { ok = false; break; }
+                }
+                if (ok) ok = wwait(b_p2b, (gc0 + nchunks - 1) & 1);
+                if (ok) {
+                    tc_fence_after();
+                    store_out(nchunks - 1, gc0 + nchunks - 1);
+                }
+            }
+            if (!ok) *s_abort = 1;
         }
+        gc0 += nchunks;
+        __syncthreads();
+        if (tid == 0) *s_unit = *s_abort ? num_units : atomicAdd(unit_counter, 1) + (int)gridDim.x;
+        __syncthreads();
     }
+    // teardown: no tensor-core op or bulk copy of this CTA may still be in flight when its tensor
+    // and shared memory are released
+    if (warp == kMmaWarp && lane == 0) {
+        mma_commit(b_drain);
+        mbar_wait(b_drain, 0, 200000000ull);
+    }
+    if (warp == kCopyWarp && lane == 0) {
+        for (int s = 0; s < 2; ++s)
+            if (last_load[s] >= 0) mbar_wait(&full[s], ((uint32_t)last_load[s] >> 1) & 1, 200000000ull);
+    }
+    if (tid == aux_tid0) bulk_wait_group<0>();
+    if (*s_abort && tid == 0) set_status(status, KDA_ERR_TIMEOUT);
     tc_fence_before();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tmem, kStateTmemCols);
@@ -981,6 +1044,18 @@ cudaError_t encode_token_map(CUtensorMap *map, const void *base, CUtensorMapData
     const CUresult r = enc(map, dt, 3, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                            swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+// Streaming multiprocessors of the current device (cached per device).
+int sm_count() {
+    static int cached[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    if (cached[dev] == 0) {
+        int n = 0;
+        cached[dev] = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && n > 0 ? n : 148;
+    }
+    return cached[dev];
 }
 
 }  // namespace
@@ -1031,7 +1106,13 @@ cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const
         (e = encode_token_map(&tm_v, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, tokens, H, 64, CU_TENSOR_MAP_SWIZZLE_128B)) != cudaSuccess ||
         (e = encode_token_map(&tm_g, log_alpha, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, tokens, H, D, CU_TENSOR_MAP_SWIZZLE_NONE)) != cudaSuccess))
         return e;
+    CUtensorMap tm_o{};  // output rows [tokens][H][128] bf16, box 128 x 1 x 64
+    if (tokens > 0 &&
+        (e = encode_token_map(&tm_o, o, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, tokens, H, D, CU_TENSOR_MAP_SWIZZLE_NONE)) != cudaSuccess)
+        return e;
     auto *ob = static_cast<__nv_bfloat16 *>(o);
+    const int num_units = (cu_seqlens ? num_seqs : B) * H;
+    const int state_grid = std::max(1, std::min(num_units, sm_count()));
     if (cu_seqlens) {
         trace_before(kKernChunkTable, stream);
         kda_chunk_table_kernel<<<1, 1024, 0, stream>>>(cu_seqlens, num_seqs, T, status, base, table);
@@ -1044,9 +1125,10 @@ cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const
             trace_after(stream);
             if ((e = cudaGetLastError()) != cudaSuccess) return e;
         }
+        if (num_units == 0) return cudaSuccess;
         trace_before(kKernTcState, stream);
-        kda_tc_state_kernel<<<(unsigned)num_seqs * H * (D / kNV), kStateThreads, STATE_SMEM, stream>>>(
-            records, h0, base, table, 0, T, H, ob, h_T, status);
+        kda_tc_state_kernel<<<(unsigned)state_grid, kStateThreads, STATE_SMEM, stream>>>(
+            tm_o, records, h0, base, table, nullptr, num_units, 0, T, H, ob, h_T, status, status + 2);
         trace_after(stream);
         return cudaGetLastError();
     }
@@ -1058,9 +1140,10 @@ cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const
         trace_after(stream);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
+    if (num_units == 0) return cudaSuccess;
     trace_before(kKernTcState, stream);
-    kda_tc_state_kernel<<<(unsigned)B * H * (D / kNV), kStateThreads, STATE_SMEM, stream>>>(
-        records, h0, nullptr, nullptr, nc, T, H, ob, h_T, status);
+    kda_tc_state_kernel<<<(unsigned)state_grid, kStateThreads, STATE_SMEM, stream>>>(
+        tm_o, records, h0, nullptr, nullptr, nullptr, num_units, nc, T, H, ob, h_T, status, status + 2);
     trace_after(stream);
     return cudaGetLastError();
 }

@@ -19,3 +19,22 @@ def cuda_device():
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     return torch.device("cuda:0")
+
+
+# Achieved parity errors of the full-size workloads, printed in the terminal summary of every run (a
+# passing test shows no output otherwise), so the margin under the tolerance is on record.
+PARITY_RECORDS: list[tuple[str, float, float, float]] = []
+
+
+@pytest.fixture(scope="session")
+def parity_log():
+    """Tests call parity_log(label, err_o, err_h, tol) to put an achieved error on record."""
+    return lambda label, eo, eh, tol: PARITY_RECORDS.append((label, eo, eh, tol))
+
+
+def pytest_terminal_summary(terminalreporter, exitstatus, config):
+    if not PARITY_RECORDS:
+        return
+    terminalreporter.section("achieved parity (max |gpu - oracle| / max |oracle|)")
+    for label, eo, eh, tol in PARITY_RECORDS:
+        terminalreporter.write_line(f"{label}: o {eo:.3e}  h_T {eh:.3e}  (tolerance {tol:.0e})")
