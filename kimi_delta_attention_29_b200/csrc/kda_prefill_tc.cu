@@ -56,13 +56,13 @@ constexpr int C = kChunk;
 constexpr uint32_t REC_AQ = 0;        // [-W; Q o e^G]: K-major sw128, 128 rows x 128 (2 atoms x 16 KiB)
 constexpr uint32_t REC_P = 32768;     // P^T rows (row i: P[0..63][i]): MN-major sw128, 64 rows x 64 (8 KiB)
 constexpr uint32_t REC_KH = 40960;    // K o e^{G_63 - G}: MN-major sw128, 64 rows x 128 (2 atoms x 8 KiB)
-constexpr uint32_t REC_UT = 57344;    // U^T: fp32 [128 channels][64 rows], 16-byte chunk x of row j at x ^ (j & 7)
-constexpr uint32_t REC_GL = 90112;    // e^{G_63}: fp32 [128]
-constexpr uint32_t REC_TX = 90112 + 512;  // bytes the state kernel copies per chunk
-constexpr uint32_t REC_BYTES = 91136;
+constexpr uint32_t REC_UT = 57344;    // U^T: bf16 [128 channels][64 rows], 16-byte chunk x of row j at x ^ (j & 7)
+constexpr uint32_t REC_GL = 73728;    // e^{G_63}: fp32 [128]
+constexpr uint32_t REC_TX = 73728 + 512;  // bytes the state kernel copies per chunk
+constexpr uint32_t REC_BYTES = 74752;
 
 struct TcLayout {
-    size_t base_off, table_off, rec_off, total;
+    size_t base_off, table_off, flags_off, rec_off, total;
     int64_t max_chunks;
 };
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -71,9 +71,32 @@ TcLayout tc_layout(int B, int T, int H, int num_seqs) {
     l.max_chunks = ((int64_t)B * T + C - 1) / C + num_seqs;
     l.base_off = 256;  // after the status block: [0] status, [1] chunk count
     l.table_off = align_up(l.base_off + 4 * (size_t)(num_seqs + 1), 1024);
-    l.rec_off = align_up(l.table_off + 16 * (size_t)l.max_chunks, 1024);
+    l.flags_off = align_up(l.table_off + 16 * (size_t)l.max_chunks, 1024);  // one ready word per record
+    l.rec_off = align_up(l.flags_off + 4 * (size_t)l.max_chunks * H, 1024);
     l.total = l.rec_off + (size_t)l.max_chunks * H * REC_BYTES;
     return l;
+}
+
+// Record hand-off between the two kernels, which run concurrently: the intra-chunk kernel publishes
+// each finished record with a release store of its ready word, the state kernel acquires it before
+// the bulk copy (and orders that copy, an async-proxy read, after the acquire).
+__device__ __forceinline__ void publish_flag(int *flag) {
+    asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(flag), "r"(1) : "memory");
+}
+__device__ __forceinline__ bool wait_flag(const int *flag, const volatile int *abort, uint64_t limit_ns = 2000000000ull) {
+    uint32_t v;
+    uint64_t t0 = 0;
+    for (int it = 0;; ++it) {
+        asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(flag) : "memory");
+        if (v != 0) break;
+        if (it == 0) t0 = sm100::global_ns();
+        if ((it & 15) == 15) {
+            if (*abort || sm100::global_ns() - t0 > limit_ns) return false;
+        }
+        __nanosleep(64);
+    }
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+    return true;
 }
 
 __device__ __forceinline__ uint8_t *align1024(uint8_t *p) {
@@ -244,7 +267,7 @@ __global__ void __launch_bounds__(kPrepThreads, 2)
 kda_tc_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
                    const Prologue pro, const float *__restrict__ beta, int T_len, int H, int nc, const int *__restrict__ n_chunks,
-                   const int4 *__restrict__ table, uint8_t *__restrict__ records, int *status) {
+                   const int4 *__restrict__ table, uint8_t *__restrict__ records, int *flags, int *status) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = align1024(smem_raw);
     uint8_t *X = sm + PREP_X;     // [K; Q] o 2^{G - E_b}, per block b: 16 k-rows then 16 q-rows
@@ -624,26 +647,31 @@ kda_tc_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                 }
             }
         } else {
-            // U^T: M=128 accumulator, channel j = TMEM lane, rows in columns 128..191; kept in fp32 (the
-            // state kernel copies it unchanged into its accumulator)
+            // U^T: M=128 accumulator, channel j = TMEM lane, rows in columns 128..191
             const int j = 32 * quad + lane;
-            uint8_t *urow = rec + REC_UT + j * 256;
+            uint8_t *urow = rec + REC_UT + j * 128;
 #pragma unroll 1
             for (int cb = 0; cb < 2; ++cb) {
                 float vals[32];
                 tmem_ld32(tmem + lane_base + 128 + 32 * cb, vals);
                 tmem_wait_ld();
 #pragma unroll
-                for (int x = 0; x < 8; ++x)
-                    *reinterpret_cast<float4 *>(urow + (((8 * cb + x) ^ (j & 7)) << 4)) =
-                        make_float4(vals[4 * x], vals[4 * x + 1], vals[4 * x + 2], vals[4 * x + 3]);
+                for (int x = 0; x < 4; ++x) {
+                    const uint4 w = make_uint4(pack_bf16(vals[8 * x + 0], vals[8 * x + 1]), pack_bf16(vals[8 * x + 2], vals[8 * x + 3]),
+                                               pack_bf16(vals[8 * x + 4], vals[8 * x + 5]), pack_bf16(vals[8 * x + 6], vals[8 * x + 7]));
+                    *reinterpret_cast<uint4 *>(urow + (((4 * cb + x) ^ (j & 7)) << 4)) = w;
+                }
             }
         }
     } else if (tid == 0) {
         set_status(status, KDA_ERR_TIMEOUT);
     }
+    // every record store of this CTA is performed before the ready word is published (after a
+    // timeout too: the status word carries the error and the consumer must not wait in vain)
+    __threadfence();
     tc_fence_before();
     __syncthreads();
+    if (tid == 0) publish_flag(flags + (size_t)chunk * H + h);
     if (warp == 0) tmem_dealloc(tmem, kPrepTmemCols);
 }
 
@@ -696,7 +724,7 @@ __device__ __forceinline__ void state_unit(int u, int H, int nc, const int *base
 
 __global__ void __launch_bounds__(kStateThreads, 1)
 kda_tc_state_kernel(const __grid_constant__ CUtensorMap tm_o, const uint8_t *__restrict__ records,
-                    const float *__restrict__ h0, const int *__restrict__ base,
+                    const int *__restrict__ flags, const float *__restrict__ h0, const int *__restrict__ base,
                     const int4 *__restrict__ table, const int *__restrict__ order, int num_units, int nc, int T_len,
                     int H, __nv_bfloat16 *__restrict__ o, float *__restrict__ h_T, int *status,
                     int *unit_counter) {
@@ -776,11 +804,16 @@ kda_tc_state_kernel(const __grid_constant__ CUtensorMap tm_o, const uint8_t *__r
                         break;
                     }
                     uint8_t *st = sm + s * REC_BYTES;
-                    const uint8_t *rec = records + ((size_t)(c_begin + i) * H + h) * REC_BYTES;
+                    const size_t ri = (size_t)(c_begin + i) * H + h;
+                    const uint8_t *rec = records + ri * REC_BYTES;
+                    if (!wait_flag(flags + ri, s_abort)) {
+                        *s_abort = 1;
+                        break;
+                    }
                     mbar_arrive_expect_tx(&full[s], REC_TX);
                     bulk_g2s(st, rec, 32768, &full[s]);
                     bulk_g2s(st + 32768, rec + 32768, 24576, &full[s]);
-                    bulk_g2s(st + REC_UT, rec + REC_UT, 32768, &full[s]);
+                    bulk_g2s(st + REC_UT, rec + REC_UT, 16384, &full[s]);
                     bulk_g2s(st + REC_GL, rec + REC_GL, 512, &full[s]);
                     last_load[s] = (int)gc;
                 }
@@ -924,12 +957,22 @@ kda_tc_state_kernel(const __grid_constant__ CUtensorMap tm_o, const uint8_t *__r
             auto preload_d1 = [&](uint32_t gc) -> bool {
                 const uint32_t s = gc & 1, b = gc & 1;
                 if (!wwait(&full[s], (gc >> 1) & 1)) return false;
-                const uint8_t *urow = sm + s * REC_BYTES + REC_UT + j * 256;
-                uint32_t uf[32];
+                {   // the record is in shared memory: drop its L2 lines without writing them back
+                    const uint8_t *rec = records + ((size_t)(c_begin + (int)(gc - gc0)) * H + h) * REC_BYTES;
+                    for (int l = atid; l < (int)(REC_TX / 128); l += 32 * kAuxWarps)
+                        asm volatile("discard.global.L2 [%0], 128;" ::"l"(rec + 128 * l) : "memory");
+                }
+                const uint8_t *urow = sm + s * REC_BYTES + REC_UT + j * 128;
+                uint32_t uf[32];  // bf16 -> fp32 is exact: the bf16 bits are the high half of the word
 #pragma unroll
-                for (int x = 0; x < 8; ++x) {
-                    const uint4 w = *reinterpret_cast<const uint4 *>(urow + (((8 * hf + x) ^ (j & 7)) << 4));
-                    uf[4 * x] = w.x; uf[4 * x + 1] = w.y; uf[4 * x + 2] = w.z; uf[4 * x + 3] = w.w;
+                for (int x = 0; x < 4; ++x) {
+                    const uint4 w = *reinterpret_cast<const uint4 *>(urow + (((4 * hf + x) ^ (j & 7)) << 4));
+                    const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        uf[8 * x + 2 * e] = wv[e] << 16;
+                        uf[8 * x + 2 * e + 1] = wv[e] & 0xFFFF0000u;
+                    }
                 }
                 tmem_st32(tmem + TM_D1 + 128 * b + lb + 32 * hf, uf);
                 arrive(&b_d1[b]);
@@ -1046,6 +1089,31 @@ cudaError_t encode_token_map(CUtensorMap *map, const void *base, CUtensorMapData
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
+// High-priority side stream of the current device for the state kernel, with the fork / join events
+// (created on first use and kept for the life of the process; the mutex serialises the fork, the
+// launches and the join of concurrent host callers).
+struct SideStream {
+    cudaStream_t stream = nullptr;
+    cudaEvent_t fork = nullptr, join = nullptr;
+    std::mutex mu;
+};
+SideStream *side_stream() {
+    static SideStream per_dev[64];
+    static std::once_flag once[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    SideStream *s = &per_dev[dev];
+    std::call_once(once[dev], [s] {
+        int lo = 0, hi = 0;
+        cudaDeviceGetStreamPriorityRange(&lo, &hi);
+        if (cudaStreamCreateWithPriority(&s->stream, cudaStreamNonBlocking, hi) != cudaSuccess ||
+            cudaEventCreateWithFlags(&s->fork, cudaEventDisableTiming) != cudaSuccess ||
+            cudaEventCreateWithFlags(&s->join, cudaEventDisableTiming) != cudaSuccess)
+            s->stream = nullptr;
+    });
+    return s->stream ? s : nullptr;
+}
+
 // Streaming multiprocessors of the current device (cached per device).
 int sm_count() {
     static int cached[64] = {0};
@@ -1083,8 +1151,10 @@ cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const
     int *status = reinterpret_cast<int *>(ws);
     int *base = reinterpret_cast<int *>(ws + lay.base_off);
     int4 *table = reinterpret_cast<int4 *>(ws + lay.table_off);
+    int *flags = reinterpret_cast<int *>(ws + lay.flags_off);
     uint8_t *records = ws + lay.rec_off;
-    cudaError_t e = cudaMemsetAsync(ws, 0, 256, stream);
+    // status block, chunk table and record ready words start at zero
+    cudaError_t e = cudaMemsetAsync(ws, 0, lay.rec_off, stream);
     if (e != cudaSuccess) return e;
 
     // opt in to the large dynamic shared-memory sizes (per device, so on every call)
@@ -1097,55 +1167,62 @@ cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(kda_tc_state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)STATE_SMEM);
     if (e != cudaSuccess) return e;
-    // TMA maps of the intra-chunk kernel's input tiles (q, k, V: bf16; log_alpha: fp32)
+    // TMA maps of the intra-chunk kernel's input tiles (q, k, V: bf16; log_alpha: fp32) and of the
+    // state kernel's output rows
     const uint64_t tokens = (uint64_t)B * T;
-    CUtensorMap tm_q{}, tm_k{}, tm_v{}, tm_g{};  // left zero (and unused) when there are no tokens
+    CUtensorMap tm_q{}, tm_k{}, tm_v{}, tm_g{}, tm_o{};  // left zero (and unused) when there are no tokens
     if (tokens > 0 &&
         ((e = encode_token_map(&tm_q, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, tokens, H, D, CU_TENSOR_MAP_SWIZZLE_NONE)) != cudaSuccess ||
         (e = encode_token_map(&tm_k, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, tokens, H, D, CU_TENSOR_MAP_SWIZZLE_NONE)) != cudaSuccess ||
         (e = encode_token_map(&tm_v, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, tokens, H, 64, CU_TENSOR_MAP_SWIZZLE_128B)) != cudaSuccess ||
-        (e = encode_token_map(&tm_g, log_alpha, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, tokens, H, D, CU_TENSOR_MAP_SWIZZLE_NONE)) != cudaSuccess))
-        return e;
-    CUtensorMap tm_o{};  // output rows [tokens][H][128] bf16, box 128 x 1 x 64
-    if (tokens > 0 &&
-        (e = encode_token_map(&tm_o, o, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, tokens, H, D, CU_TENSOR_MAP_SWIZZLE_NONE)) != cudaSuccess)
+        (e = encode_token_map(&tm_g, log_alpha, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, tokens, H, D, CU_TENSOR_MAP_SWIZZLE_NONE)) != cudaSuccess ||
+        (e = encode_token_map(&tm_o, o, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, tokens, H, D, CU_TENSOR_MAP_SWIZZLE_NONE)) != cudaSuccess))
         return e;
     auto *ob = static_cast<__nv_bfloat16 *>(o);
-    const int num_units = (cu_seqlens ? num_seqs : B) * H;
-    const int state_grid = std::max(1, std::min(num_units, sm_count()));
-    if (cu_seqlens) {
+    const bool varlen = cu_seqlens != nullptr;
+    const int num_units = (varlen ? num_seqs : B) * H;
+    const int nc = varlen ? 0 : (T + C - 1) / C;
+    const int64_t prep_ctas = varlen ? lay.max_chunks * H : (int64_t)B * nc * H;
+    if (varlen) {
         trace_before(kKernChunkTable, stream);
         kda_chunk_table_kernel<<<1, 1024, 0, stream>>>(cu_seqlens, num_seqs, T, status, base, table);
         trace_after(stream);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
-        if (lay.max_chunks > 0) {
-            trace_before(kKernTcPrep, stream);
-            prep<<<(unsigned)(lay.max_chunks * H), kPrepThreads, PREP_SMEM, stream>>>(
-                tm_q, tm_k, tm_v, tm_g, pro, beta, T, H, 0, status + 1, table, records, status);
-            trace_after(stream);
-            if ((e = cudaGetLastError()) != cudaSuccess) return e;
-        }
-        if (num_units == 0) return cudaSuccess;
+    }
+    if (num_units == 0) return cudaSuccess;
+    const int4 *tbl = varlen ? table : nullptr;
+    const int *bas = varlen ? base : nullptr;
+    // A quarter of the SMs at most pass the state (one CTA per SM, a (sequence, head) unit at a
+    // time); the intra-chunk kernel fills the rest and runs at the same time.
+    const int state_grid = std::max(1, std::min(num_units, std::max(1, sm_count() / 4)));
+    if (prep_ctas == 0) {  // no tokens: the state kernel alone writes h_T
         trace_before(kKernTcState, stream);
         kda_tc_state_kernel<<<(unsigned)state_grid, kStateThreads, STATE_SMEM, stream>>>(
-            tm_o, records, h0, base, table, nullptr, num_units, 0, T, H, ob, h_T, status, status + 2);
+            tm_o, records, flags, h0, bas, tbl, nullptr, num_units, nc, T, H, ob, h_T, status, status + 2);
         trace_after(stream);
         return cudaGetLastError();
     }
-    const int nc = (T + C - 1) / C;
-    if (nc > 0) {
-        trace_before(kKernTcPrep, stream);
-        prep<<<(unsigned)((int64_t)B * nc * H), kPrepThreads, PREP_SMEM, stream>>>(
-            tm_q, tm_k, tm_v, tm_g, pro, beta, T, H, nc, nullptr, nullptr, records, status);
-        trace_after(stream);
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    }
-    if (num_units == 0) return cudaSuccess;
-    trace_before(kKernTcState, stream);
-    kda_tc_state_kernel<<<(unsigned)state_grid, kStateThreads, STATE_SMEM, stream>>>(
-        tm_o, records, h0, nullptr, nullptr, nullptr, num_units, nc, T, H, ob, h_T, status, status + 2);
+    // The two kernels run concurrently: the state kernel on a high-priority side stream forked from
+    // `stream` (launched first, so its CTAs are resident before the intra-chunk grid fills the GPU),
+    // the intra-chunk kernel on `stream`, which then joins the side stream.  The intra-chunk kernel
+    // never waits for the state kernel, so the result does not depend on the two overlapping.
+    SideStream *side = side_stream();
+    if (!side) return cudaErrorInitializationError;
+    std::lock_guard<std::mutex> lock(side->mu);
+    trace_before(kKernTcPrefill, stream);
+    if ((e = cudaEventRecord(side->fork, stream)) != cudaSuccess) return e;
+    if ((e = cudaStreamWaitEvent(side->stream, side->fork, 0)) != cudaSuccess) return e;
+    kda_tc_state_kernel<<<(unsigned)state_grid, kStateThreads, STATE_SMEM, side->stream>>>(
+        tm_o, records, flags, h0, bas, tbl, nullptr, num_units, nc, T, H, ob, h_T, status, status + 2);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if ((e = cudaEventRecord(side->join, side->stream)) != cudaSuccess) return e;
+    prep<<<(unsigned)prep_ctas, kPrepThreads, PREP_SMEM, stream>>>(tm_q, tm_k, tm_v, tm_g, pro, beta, T, H, nc,
+                                                                    varlen ? status + 1 : nullptr, tbl, records,
+                                                                    flags, status);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if ((e = cudaStreamWaitEvent(stream, side->join, 0)) != cudaSuccess) return e;
     trace_after(stream);
-    return cudaGetLastError();
+    return cudaSuccess;
 }
 
 }  // namespace kda
