@@ -683,11 +683,10 @@ kda_tc_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
 //   D2     fp32 master S^T; before each chunk's K^ product it is overwritten with S^T Diag(e^{G_63})
 //   A_S    bf16 copy of S^T (A operand of P1), 2 channels per 32-bit column
 //   A_D    bf16 Delta^T (A operand of P2a, P2b)
-//   D1[2]  per chunk parity: [U^T | .]; P1a adds -S^T W^T to the first half -> Delta^T, P1b writes
-//          (Q~ S)^T into the second half and P2b adds Delta^T P^T -> O^T
-// Per chunk (P1 in two halves so that the Delta^T half, which the recurrence waits for, comes first):
-//   P1a: D1[:, :64] += A_S (-W)^T   (M=128, N=64, K=128)  = Delta^T = U^T - S^T W^T
-//   P1b: D1[:, 64:]  = A_S Q~^T     (M=128, N=64, K=128)  = (Q~ S)^T
+//   D1[2]  per chunk parity: preloaded with [U^T | 0]; P1 adds S^T [-W; Q~]^T -> [Delta^T | (Q~ S)^T]
+//          and P2b adds Delta^T P^T to the second half -> O^T
+// Per chunk:
+//   P1:  D1 += A_S [-W; Q~]^T       (M=128, N=128, K=128) onto [U^T | 0] = [Delta^T | (Q~ S)^T]
 //   P2a: D2 += A_D K^               (M=128, N=128, K=64)  = S_next^T = S^T Diag(e^{G_63}) + Delta^T K^
 //   P2b: D1[:, 64:] += A_D P^T      (M=128, N=64,  K=64)  = O^T = (Q~ S + P Delta)^T
 // Warps:
@@ -732,7 +731,7 @@ kda_tc_state_kernel(const __grid_constant__ CUtensorMap tm_o, const uint8_t *__r
     uint8_t *sm = align1024(smem_raw);
     uint64_t *full = reinterpret_cast<uint64_t *>(sm + ST_BAR);  // [2] record landed in the stage
     uint64_t *empty = full + 2;   // [2] every MMA reading the stage is done
-    uint64_t *b_p1 = empty + 2;   // P1a done (and every earlier MMA)
+    uint64_t *b_p1 = empty + 2;   // P1 done (and every earlier MMA)
     uint64_t *b_p2a = b_p1 + 1;   // P2a done
     uint64_t *b_p2b = b_p2a + 1;  // P2b done
     uint64_t *b_dr = b_p2b + 1;   // Delta^T operand in tensor memory (chain warps)
@@ -822,17 +821,15 @@ kda_tc_state_kernel(const __grid_constant__ CUtensorMap tm_o, const uint8_t *__r
         } else if (warp == kMmaWarp) {
             // ------------------------------------------------ MMA issue (one thread)
             if (lane == 0) {
-                const uint32_t id_p1 = idesc_bf16_f32(128, 64, 0, 0);
+                const uint32_t id_p1 = idesc_bf16_f32(128, 128, 0, 0);
                 const uint32_t id_p2a = idesc_bf16_f32(128, 128, 0, 1);
                 const uint32_t id_p2b = idesc_bf16_f32(128, 64, 0, 1);
                 // operand descriptors of stage 0; stage 1 is REC_BYTES / 16 further in the start field
                 const uint32_t st0 = smem_u32(sm);
-                uint64_t dw[8], dq[8], dk[4], dp[4];
+                uint64_t dw[8], dk[4], dp[4];
 #pragma unroll
-                for (int ks = 0; ks < 8; ++ks) {
+                for (int ks = 0; ks < 8; ++ks)
                     dw[ks] = smem_desc_sw128(st0 + REC_AQ + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
-                    dq[ks] = smem_desc_sw128(st0 + REC_AQ + 8192 + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
-                }
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks) {
                     dk[ks] = smem_desc_sw128(st0 + REC_KH + ks * 2048, 8192, 1024);
@@ -848,12 +845,9 @@ kda_tc_state_kernel(const __grid_constant__ CUtensorMap tm_o, const uint8_t *__r
                     if (!ok) { *s_abort = 1; break; }
                     tc_fence_after();
 #pragma unroll
-                    for (int ks = 0; ks < 8; ++ks)  // -W: rows 0..63 of the [-W; Q~] image
+                    for (int ks = 0; ks < 8; ++ks)  // [-W; Q~] as one N=128 product onto [U^T | 0]
                         mma_bf16_ts(d1, tmem + TM_AS + 8 * ks, dw[ks] + so, id_p1, 1);
                     mma_commit(b_p1);
-#pragma unroll
-                    for (int ks = 0; ks < 8; ++ks)  // Q~: rows 64..127
-                        mma_bf16_ts(d1 + 64, tmem + TM_AS + 8 * ks, dq[ks] + so, id_p1, ks > 0);
                     ok = mbar_wait_or_abort(b_dr, gc & 1, s_abort) && mbar_wait_or_abort(b_d2, gc & 1, s_abort);
                     if (!ok) { *s_abort = 1; break; }
                     tc_fence_after();
@@ -975,6 +969,9 @@ kda_tc_state_kernel(const __grid_constant__ CUtensorMap tm_o, const uint8_t *__r
                     }
                 }
                 tmem_st32(tmem + TM_D1 + 128 * b + lb + 32 * hf, uf);
+#pragma unroll
+                for (int e = 0; e < 32; ++e) uf[e] = 0u;  // the output half starts from zero
+                tmem_st32(tmem + TM_D1 + 128 * b + lb + 64 + 32 * hf, uf);
                 arrive(&b_d1[b]);
                 return true;
             };
@@ -1021,7 +1018,7 @@ kda_tc_state_kernel(const __grid_constant__ CUtensorMap tm_o, const uint8_t *__r
                 for (int i = 0; i < nchunks && ok; ++i) {
                     const uint32_t gc = gc0 + i;
                     const bool more = i + 1 < nchunks;
-                    // P1a of this chunk done => P2b of the previous one done: its output is final.
+                    // P1 of this chunk done => P2b of the previous one done: its output is final.
                     // Waited for every chunk: a parity wait is only unambiguous when the phase before
                     // the awaited one is known to be complete.
                     if (!wwait(b_p1, gc & 1)) { ok = false; break; }
