@@ -62,7 +62,7 @@ constexpr uint32_t REC_TX = 73728 + 512;  // bytes the state kernel copies per c
 constexpr uint32_t REC_BYTES = 74752;
 
 struct TcLayout {
-    size_t base_off, table_off, flags_off, rec_off, total;
+    size_t base_off, order_off, table_off, flags_off, rec_off, total;
     int64_t max_chunks;
 };
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -70,7 +70,8 @@ TcLayout tc_layout(int B, int T, int H, int num_seqs) {
     TcLayout l;
     l.max_chunks = ((int64_t)B * T + C - 1) / C + num_seqs;
     l.base_off = 256;  // after the status block: [0] status, [1] chunk count
-    l.table_off = align_up(l.base_off + 4 * (size_t)(num_seqs + 1), 1024);
+    l.order_off = align_up(l.base_off + 4 * (size_t)(num_seqs + 1), 256);  // state units, longest first
+    l.table_off = align_up(l.order_off + 4 * (size_t)num_seqs, 1024);
     l.flags_off = align_up(l.table_off + 16 * (size_t)l.max_chunks, 1024);  // one ready word per record
     l.rec_off = align_up(l.flags_off + 4 * (size_t)l.max_chunks * H, 1024);
     l.total = l.rec_off + (size_t)l.max_chunks * H * REC_BYTES;
@@ -117,15 +118,25 @@ __device__ __forceinline__ float2 unpack_bf16(uint32_t u) {
 __device__ __forceinline__ float2 sub2(float2 a, float2 b) { return make_float2(a.x - b.x, a.y - b.y); }
 
 // ============================================================================ chunk table (varlen)
-// One CTA: validates cu_seqlens (0 = cu[0] <= cu[1] <= ... <= cu[N] = T), then writes the chunk
-// count per sequence as exclusive offsets base[0..N] and one (sequence, first token, rows) entry per
-// chunk.  On malformed input it records KDA_ERR_BAD_SEQLENS and publishes zero chunks.
+// One CTA: validates cu_seqlens (0 = cu[0] <= cu[1] <= ... <= cu[N] = T), then lays the chunks out
+// sequence after sequence: base[p] is the first chunk of the p-th sequence laid out (base[N] = the
+// chunk count) and each chunk gets one (sequence, first token, rows) entry.  On malformed input it
+// records KDA_ERR_BAD_SEQLENS and publishes zero chunks.
+// Without `order` the sequences are laid out in index order.  With it (N <= kOrderMax) they are laid
+// out longest first (ties by index) and order[p] names the p-th one: the intra-chunk kernel walks the
+// chunks and the state pass its (sequence, head) units in that order, so the longest sequences, whose
+// state chains run longest, are neither produced nor started last.
+constexpr int kOrderMax = 4096;
 __global__ void __launch_bounds__(1024) kda_chunk_table_kernel(const int32_t *__restrict__ cu, int N, int T,
                                                                int *__restrict__ status_blk,
-                                                               int *__restrict__ base, int4 *__restrict__ table) {
+                                                               int *__restrict__ base, int4 *__restrict__ table,
+                                                               int *__restrict__ order) {
     __shared__ int s_bad;
     __shared__ int s_scan[2][1024];
+    __shared__ int s_cnt[kOrderMax];
+    __shared__ int s_seq[kOrderMax];
     const int tid = threadIdx.x;
+    const bool sorted = order != nullptr && N <= kOrderMax;
     if (tid == 0) s_bad = (cu[0] != 0 || cu[N] != T) ? 1 : 0;
     __syncthreads();
     for (int i = tid; i < N; i += 1024)
@@ -137,12 +148,33 @@ __global__ void __launch_bounds__(1024) kda_chunk_table_kernel(const int32_t *__
             status_blk[1] = 0;
         }
         for (int i = tid; i <= N; i += 1024) base[i] = 0;
+        if (sorted)
+            for (int i = tid; i < N; i += 1024) order[i] = i;
         return;
     }
+    if (sorted) {
+        for (int n = tid; n < N; n += 1024) s_cnt[n] = (cu[n + 1] - cu[n] + C - 1) / C;
+        __syncthreads();
+        for (int n = tid; n < N; n += 1024) {
+            const int cn = s_cnt[n];
+            int rank = 0;
+            for (int m = 0; m < N; ++m) {
+                const int cm = s_cnt[m];
+                rank += cm > cn || (cm == cn && m < n);
+            }
+            s_seq[rank] = n;
+            order[rank] = n;
+        }
+        __syncthreads();
+    }
+    auto seq_at = [&](int p) { return sorted ? s_seq[p] : p; };
     const int per = (N + 1023) / 1024;
     const int lo = min(N, tid * per), hi = min(N, lo + per);
     int sum = 0;
-    for (int n = lo; n < hi; ++n) sum += (cu[n + 1] - cu[n] + C - 1) / C;
+    for (int p = lo; p < hi; ++p) {
+        const int n = seq_at(p);
+        sum += (cu[n + 1] - cu[n] + C - 1) / C;
+    }
     s_scan[0][tid] = sum;
     __syncthreads();
     int src = 0;
@@ -153,8 +185,9 @@ __global__ void __launch_bounds__(1024) kda_chunk_table_kernel(const int32_t *__
         __syncthreads();
     }
     int acc = s_scan[src][tid] - sum;  // exclusive prefix of this thread's segment
-    for (int n = lo; n < hi; ++n) {
-        base[n] = acc;
+    for (int p = lo; p < hi; ++p) {
+        const int n = seq_at(p);
+        base[p] = acc;
         const int len = cu[n + 1] - cu[n];
         for (int c = 0; c * C < len; ++c) table[acc + c] = make_int4(n, cu[n] + c * C, min(C, len - c * C), 0);
         acc += (len + C - 1) / C;
@@ -710,10 +743,10 @@ __device__ __forceinline__ void state_unit(int u, int H, int nc, const int *base
                                            int &h, int &c_begin, int &nchunks) {
     h = u % H;
     const int r = u / H;
-    if (base) {
+    if (base) {  // base is in layout order: the r-th sequence laid out is order[r] (r without order)
         n = order ? order[r] : r;
-        c_begin = base[n];
-        nchunks = base[n + 1] - c_begin;
+        c_begin = base[r];
+        nchunks = base[r + 1] - c_begin;
     } else {
         n = r;
         c_begin = n * nc;
@@ -1128,7 +1161,7 @@ int sm_count() {
 cudaError_t launch_chunk_table(const int32_t *cu_seqlens, int num_seqs, int T, int *status_blk, int *base,
                                int4 *table, cudaStream_t stream) {
     trace_before(kKernChunkTable, stream);
-    kda_chunk_table_kernel<<<1, 1024, 0, stream>>>(cu_seqlens, num_seqs, T, status_blk, base, table);
+    kda_chunk_table_kernel<<<1, 1024, 0, stream>>>(cu_seqlens, num_seqs, T, status_blk, base, table, nullptr);
     trace_after(stream);
     return cudaGetLastError();
 }
@@ -1148,6 +1181,7 @@ cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const
     int *status = reinterpret_cast<int *>(ws);
     int *base = reinterpret_cast<int *>(ws + lay.base_off);
     int4 *table = reinterpret_cast<int4 *>(ws + lay.table_off);
+    int *order = reinterpret_cast<int *>(ws + lay.order_off);
     int *flags = reinterpret_cast<int *>(ws + lay.flags_off);
     uint8_t *records = ws + lay.rec_off;
     // status block, chunk table and record ready words start at zero
@@ -1182,20 +1216,21 @@ cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const
     const int64_t prep_ctas = varlen ? lay.max_chunks * H : (int64_t)B * nc * H;
     if (varlen) {
         trace_before(kKernChunkTable, stream);
-        kda_chunk_table_kernel<<<1, 1024, 0, stream>>>(cu_seqlens, num_seqs, T, status, base, table);
+        kda_chunk_table_kernel<<<1, 1024, 0, stream>>>(cu_seqlens, num_seqs, T, status, base, table, order);
         trace_after(stream);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     if (num_units == 0) return cudaSuccess;
     const int4 *tbl = varlen ? table : nullptr;
     const int *bas = varlen ? base : nullptr;
+    const int *ord = varlen && num_seqs <= kOrderMax ? order : nullptr;
     // A quarter of the SMs at most pass the state (one CTA per SM, a (sequence, head) unit at a
     // time); the intra-chunk kernel fills the rest and runs at the same time.
     const int state_grid = std::max(1, std::min(num_units, std::max(1, sm_count() / 4)));
     if (prep_ctas == 0) {  // no tokens: the state kernel alone writes h_T
         trace_before(kKernTcState, stream);
         kda_tc_state_kernel<<<(unsigned)state_grid, kStateThreads, STATE_SMEM, stream>>>(
-            tm_o, records, flags, h0, bas, tbl, nullptr, num_units, nc, T, H, ob, h_T, status, status + 2);
+            tm_o, records, flags, h0, bas, tbl, ord, num_units, nc, T, H, ob, h_T, status, status + 2);
         trace_after(stream);
         return cudaGetLastError();
     }
@@ -1210,7 +1245,7 @@ cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const
     if ((e = cudaEventRecord(side->fork, stream)) != cudaSuccess) return e;
     if ((e = cudaStreamWaitEvent(side->stream, side->fork, 0)) != cudaSuccess) return e;
     kda_tc_state_kernel<<<(unsigned)state_grid, kStateThreads, STATE_SMEM, side->stream>>>(
-        tm_o, records, flags, h0, bas, tbl, nullptr, num_units, nc, T, H, ob, h_T, status, status + 2);
+        tm_o, records, flags, h0, bas, tbl, ord, num_units, nc, T, H, ob, h_T, status, status + 2);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if ((e = cudaEventRecord(side->join, side->stream)) != cudaSuccess) return e;
     prep<<<(unsigned)prep_ctas, kPrepThreads, PREP_SMEM, stream>>>(tm_q, tm_k, tm_v, tm_g, pro, beta, T, H, nc,
