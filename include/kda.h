@@ -110,8 +110,14 @@ KDA_API int kda_chunk_fwd(const void *q, const void *k, const void *v, const flo
  *     KDA_ERR_WORKSPACE_TOO_SMALL before anything is launched.  For the tensor-core path
  *     (bf16, d = 128) that is roughly num_chunks * H <= 896, where num_chunks = ceil(B*T/64) + N;
  *     e.g. H = 32 heads up to T = 1728 tokens for one sequence.
- *   - The first call on a device looks up the scratch's device address for that device (with
- *     that device current) and caches it; make that first call before any stream capture.
+ *   - Make the first call on each device before reserving device memory for a pool of your own,
+ *     and before any stream capture.  That first call needs free device memory: the CUDA runtime
+ *     loads the library's device code, and the scratch with it, into a device's memory on first
+ *     use (lazy module loading), and the call also looks up the scratch's device address and
+ *     creates the side stream the prefill uses.  Later calls need no device memory.
+ *   - The looked-up address and side stream belong to the CUDA context current at that first
+ *     call.  After a device reset (cudaDeviceReset) the next call on that device finds a new
+ *     context, looks both up again and is a first call in the sense above.
  *   - All calls share the one scratch array, which keeps the last call's contents (the status
  *     word is cleared at the start of every call).  Calls that overlap on the GPU (on different
  *     streams, or from different host threads) race on it and must be serialized by the caller.
@@ -232,6 +238,25 @@ KDA_API int kda_chunk_bwd(const void *q, const void *k, const void *v, const flo
  * {64, 128}, dv in {64, 128}, R >= 1.  Outputs must not overlap the inputs or each other. */
 KDA_API int kda_state_compose(const float *Mb, const float *h0, int R, int H, int dk, int dv, float *S_in,
                               float *S_out, void *stream);
+
+/* One segment's map [M | b] for kda_state_compose in a single pass (and, optionally, its outputs from
+ * a zero incoming state).  Same definitions as above: b is the final state of the segment run from a
+ * zero state, M the final state of a run with v = 0 from S = I; here both share one pass of the
+ * intra-chunk work (section "Chunkwise parallel algorithm": the per-chunk quantities do not depend on
+ * the state), followed by two state passes per head, one from 0 with v and one from I with v = 0.
+ *   q, k      : [1, T, H, dk] dtype     v : [1, T, H, dv] dtype
+ *   log_alpha : [1, T, H, dk] fp32      beta : [1, T, H] fp32
+ *   o0        : [1, T, H, dv] dtype out, the outputs from a zero incoming state, or NULL (not wanted)
+ *   Mb        : [H, dk, dk + dv] fp32 out, row i of head h = [M[h][i][:], b[h][i][:]]
+ *   workspace : kda_chunk_fwd_workspace_size(1, T, H, dk, dv, 1, chunk_size, dtype) bytes, 256-byte
+ *               aligned, owned by the caller; not in use by another call until this one completes.
+ * Supported: dtype BF16, dk = dv = 128, chunk_size 64 (the tensor-core path); other sizes return
+ * KDA_ERR_UNSUPPORTED (run kda_chunk_fwd twice for them).  T = 0 gives [I | 0].  Outputs must not
+ * overlap the inputs, each other or the workspace.  Asynchronous on `stream`; device-detected errors
+ * (timeouts) go to the workspace status word (kda_get_status). */
+KDA_API int kda_segment_map(const void *q, const void *k, const void *v, const float *log_alpha, const float *beta,
+                            int T, int H, int dk, int dv, int chunk_size, kda_dtype dtype, void *o0, float *Mb,
+                            void *workspace, size_t workspace_bytes, void *stream);
 
 /* The KDA layer's output epilogue (Kimi Linear summary page, section "Kimi Linear model
  * composition": a per-head RMSNorm and a data-dependent output gate ahead of the output

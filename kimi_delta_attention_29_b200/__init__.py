@@ -14,7 +14,7 @@ from ._lib import KDA_PROLOGUE_GATE, KDA_PROLOGUE_L2NORM_QK  # noqa: F401
 
 __all__ = ["kda_chunk_fwd", "kda_chunk_fwd_ex", "kda_chunk_fwd_workspace_size", "kda_chunk_bwd",
            "kda_chunk_bwd_workspace_size", "kda_decode_step", "kda_decode_multi", "kda_decode_multi_ex",
-           "kda_output_gate_norm", "kda_state_compose", "kda_get_status", "kda_status_string",
+           "kda_output_gate_norm", "kda_state_compose", "kda_segment_map", "kda_get_status", "kda_status_string",
            "kda_trace_begin", "kda_trace_end", "KdaError", "Workspace", "KDA_PROLOGUE_GATE",
            "KDA_PROLOGUE_L2NORM_QK"]
 
@@ -218,6 +218,32 @@ def kda_state_compose(Mb, h0=None, want_S_in: bool = True, stream=None):
     if rc != _lib.KDA_OK:
         raise KdaError(rc, "kda_state_compose")
     return S_in, S_out
+
+
+def kda_segment_map(q, k, v, log_alpha, beta, want_o: bool = True, chunk_size: int = 64, workspace=None,
+                    stream=None):
+    """One segment's map for kda_state_compose in one pass: q, k [1,T,H,dk], v [1,T,H,dv] bf16 with
+    dk = dv = 128, log_alpha [1,T,H,dk] fp32, beta [1,T,H] fp32.  Returns (o0 [1,T,H,dv] or None, Mb
+    [H, dk, dk + dv] fp32): the outputs from a zero incoming state and the rows [M | b]."""
+    torch = _torch()
+    _, T, H, dk = q.shape
+    dv = v.shape[-1]
+    o0 = torch.empty((1, T, H, dv), dtype=q.dtype, device=q.device) if want_o else None
+    Mb = torch.empty((H, dk, dk + dv), dtype=torch.float32, device=q.device)
+    code = _dtype_code(q.dtype)
+    need = int(_lib.load().kda_chunk_fwd_workspace_size(1, T, H, dk, dv, 1, chunk_size, code))
+    if isinstance(workspace, Workspace):
+        ws = workspace.get(need)
+    elif workspace is None:
+        ws = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
+    else:
+        ws = workspace
+    rc = _lib.load().kda_segment_map(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), T, H, dk, dv,
+                                     chunk_size, code, _ptr(o0), _ptr(Mb), _ptr(ws), ws.numel() * ws.element_size(),
+                                     _stream(stream, q.device))
+    if rc != _lib.KDA_OK:
+        raise KdaError(rc, "kda_segment_map")
+    return o0, Mb
 
 
 def kda_output_gate_norm(o, g, weight=None, eps: float = 1e-6, out=None, stream=None):

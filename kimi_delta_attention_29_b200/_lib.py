@@ -36,7 +36,7 @@ KDA_PROLOGUE_GATE = 2
 # Every entry point include/kda.h declares.
 EXPORTED = ("kda_chunk_fwd_workspace_size", "kda_chunk_fwd", "kda_chunk_fwd_ex", "kda_decode_step",
             "kda_decode_multi", "kda_decode_multi_ex", "kda_output_gate_norm", "kda_chunk_bwd_workspace_size",
-            "kda_chunk_bwd", "kda_state_compose", "kda_get_status",
+            "kda_chunk_bwd", "kda_state_compose", "kda_segment_map", "kda_get_status",
             "kda_status_string", "kda_version", "kda_trace_begin", "kda_trace_end")
 
 KERNEL_NAMES = {0: "kda_chunk_table_kernel", 1: "kda_tc_prep_kernel", 2: "kda_tc_state_kernel",
@@ -78,6 +78,8 @@ def load() -> ctypes.CDLL:
     lib.kda_chunk_bwd.restype = i
     lib.kda_state_compose.argtypes = [fp, fp, i, i, i, i, fp, fp, vp]
     lib.kda_state_compose.restype = i
+    lib.kda_segment_map.argtypes = [vp, vp, vp, fp, fp, i, i, i, i, i, i, vp, fp, vp, sz, vp]
+    lib.kda_segment_map.restype = i
     lib.kda_output_gate_norm.argtypes = [vp, vp, fp, ctypes.c_float, i, i, i, i, vp, vp]
     lib.kda_output_gate_norm.restype = i
     lib.kda_get_status.argtypes = [vp, vp]

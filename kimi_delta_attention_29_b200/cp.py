@@ -9,26 +9,32 @@ d_k x d_k transition, the final state of a pass with v = 0 from S_in = I.  One e
 the segments (section "Chunkwise parallel algorithm": each chunk's final state seeds the next; here
 each segment's does): every rank all-gathers the [M | b] of all segments, the library composes them
 into each segment's incoming state (kda_state_compose), and each rank runs its segment again from
-that state for its outputs.  Per rank: three chunkwise prefills of its segment and one all-gather of
-d_k (d_k + d_v) floats per head; the composition is R small products per head.
+that state for its outputs.  Per rank: one map pass of its segment (the intra-chunk work once, two
+state passes per head: kda_segment_map), one all-gather of d_k (d_k + d_v) floats per head, the
+composition (R small products per head) and one chunkwise prefill from the incoming state; rank 0
+without h0 keeps the map pass's outputs.
 """
 from __future__ import annotations
 
 from typing import Callable, Sequence
 
 
-def segment_map(q, k, v, log_alpha, beta, stream=None, workspace=None):
-    """One segment's outputs from a zero state and its map [M | b] [H, dk, dk + dv] (fp32).
-    q, k [1, T, H, dk], v [1, T, H, dv] with dv = dk; log_alpha [1, T, H, dk]; beta [1, T, H]."""
+def segment_map(q, k, v, log_alpha, beta, stream=None, workspace=None, want_o: bool = True):
+    """One segment's outputs from a zero state (None unless want_o) and its map [M | b] [H, dk, dk + dv]
+    (fp32).  q, k [1, T, H, dk], v [1, T, H, dv] with dv = dk; log_alpha [1, T, H, dk]; beta [1, T, H].
+    On the tensor-core path (bf16, dk = dv = 128) one pass: kda_segment_map; otherwise two prefills, one
+    from zero and one with v = 0 from the identity."""
     import torch
-    from . import kda_chunk_fwd
+    from . import kda_chunk_fwd, kda_segment_map
     H, dk, dv = q.shape[2], q.shape[3], v.shape[3]
     if dk != dv:
         raise ValueError("the segment transition is formed as a state with dv = dk columns")
+    if q.dtype == torch.bfloat16 and dk == 128:
+        return kda_segment_map(q, k, v, log_alpha, beta, want_o=want_o, workspace=workspace, stream=stream)
     o0, b = kda_chunk_fwd(q, k, v, log_alpha, beta, None, None, workspace=workspace, stream=stream)
     eye = torch.eye(dk, dtype=torch.float32, device=q.device).expand(1, H, dk, dk).contiguous()
     _, M = kda_chunk_fwd(q, k, torch.zeros_like(v), log_alpha, beta, eye, None, workspace=workspace, stream=stream)
-    return o0, torch.cat([M[0], b[0]], dim=2).contiguous()
+    return (o0 if want_o else None), torch.cat([M[0], b[0]], dim=2).contiguous()
 
 
 def identity_map(H, dk, dv, device, dtype=None):
@@ -63,10 +69,11 @@ def kda_chunk_fwd_cp(q, k, v, log_alpha, beta, h0=None, group=None, stream=None,
     import torch
     import torch.distributed as dist
     from . import kda_state_compose
-    seg = segment or (lambda *a: segment_map(*a, stream=stream, workspace=workspace))
+    world, rank = dist.get_world_size(group), dist.get_rank(group)
+    keep_o = rank == 0 and h0 is None  # the only rank whose map-pass outputs are final
+    seg = segment or (lambda *a: segment_map(*a, stream=stream, workspace=workspace, want_o=keep_o))
     comp = compose or (lambda Mb, s0: kda_state_compose(Mb, s0, stream=stream))
     run = rerun or (lambda *a: segment_from(*a, stream=stream, workspace=workspace))
-    world, rank = dist.get_world_size(group), dist.get_rank(group)
     map_dtype = map_dtype or torch.float32
     H, dk, dv = q.shape[2], q.shape[3], v.shape[3]
     o = None
@@ -96,7 +103,7 @@ def kda_chunk_fwd_segments(q, k, v, log_alpha, beta, bounds: Sequence[int], h0=N
         part = [x[:, a:e].contiguous() for x in (q, k, v, log_alpha, beta)]
         parts.append(part)
         if e > a:
-            o0, Mb = segment_map(*part, stream=stream, workspace=workspace)
+            o0, Mb = segment_map(*part, stream=stream, workspace=workspace, want_o=(a == 0 and h0 is None))
         else:
             o0, Mb = torch.empty_like(part[2]), identity_map(q.shape[2], q.shape[3], v.shape[3], q.device)
         outs.append(o0)

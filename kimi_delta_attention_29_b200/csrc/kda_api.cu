@@ -360,6 +360,36 @@ int kda_state_compose(const float *Mb, const float *h0, int R, int H, int dk, in
     return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 
+int kda_segment_map(const void *q, const void *k, const void *v, const float *log_alpha, const float *beta, int T,
+                    int H, int dk, int dv, int chunk_size, kda_dtype dtype, void *o0, float *Mb, void *workspace,
+                    size_t workspace_bytes, void *stream_) {
+    if (dtype != KDA_F32 && dtype != KDA_BF16) return KDA_ERR_BAD_DTYPE;
+    if (!workspace || !Mb) return KDA_ERR_NULL_ARG;
+    int rc = check_prefill_shape(1, T, H, dk, dv, 1, false, chunk_size);
+    if (rc != KDA_OK) return rc;
+    if (!uses_tensor_cores(dk, dv, dtype)) return KDA_ERR_UNSUPPORTED;
+    if (T > 0 && (!q || !k || !v || !log_alpha || !beta)) return KDA_ERR_NULL_ARG;
+    const void *ptrs[] = {q, k, v, log_alpha, beta, o0, Mb};
+    for (const void *p : ptrs)
+        if (p && !aligned16(p)) return KDA_ERR_MISALIGNED;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return KDA_ERR_MISALIGNED;
+    const size_t es = elem_size(dtype), tok = (size_t)T * H;
+    const size_t need = kda_chunk_fwd_workspace_size(1, T, H, dk, dv, 1, chunk_size, dtype);
+    if (need == 0) return KDA_ERR_BAD_SHAPE;
+    if (workspace_bytes < need) return KDA_ERR_WORKSPACE_TOO_SMALL;
+    const Range rm = range_of(Mb, (size_t)H * dk * (dk + dv) * 4), ro = range_of(o0, o0 ? tok * dv * es : 0),
+                rw = range_of(workspace, need);
+    const Range inputs[] = {range_of(q, tok * dk * es), range_of(k, tok * dk * es), range_of(v, tok * dv * es),
+                            range_of(log_alpha, tok * dk * 4), range_of(beta, tok * 4)};
+    if (overlaps(rm, ro) || overlaps(rm, rw) || overlaps(ro, rw)) return KDA_ERR_ALIASING;
+    for (const Range &r : inputs)
+        if (overlaps(rm, r) || overlaps(ro, r)) return KDA_ERR_ALIASING;
+    const kda::Prologue pro{0u, nullptr, nullptr};
+    cudaError_t e = kda::launch_prefill_tc(q, k, v, log_alpha, beta, nullptr, nullptr, 1, 1, T, H, o0, nullptr,
+                                           workspace, workspace_bytes, pro, static_cast<cudaStream_t>(stream_), Mb);
+    return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
 int kda_output_gate_norm(const void *o, const void *g, const float *weight, float eps, int n_tok, int H, int dv,
                          kda_dtype dtype, void *out, void *stream_) {
     if (dtype != KDA_F32 && dtype != KDA_BF16) return KDA_ERR_BAD_DTYPE;

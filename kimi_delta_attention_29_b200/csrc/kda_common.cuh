@@ -137,10 +137,16 @@ cudaError_t launch_chunk_bwd(const void *q, const void *k, const void *v, const 
                              kda_dtype dtype, const void *dout, const float *dhT, void *dq, void *dk, void *dv,
                              float *dla, float *dbeta, float *dh0, void *workspace, cudaStream_t stream);
 
-// Tensor-core (tcgen05) chunkwise forward: bf16, dk = dv = 128.
+// Unique id of the CUDA context current on the calling thread (0 when none is current yet).  Caches of
+// per-device handles compare it so that they are rebuilt after a device reset.
+unsigned long long current_context_id();
+// Tensor-core (tcgen05) chunkwise forward: bf16, dk = dv = 128.  With map_out [H, 128, 256] (one
+// sequence, h0 and h_T NULL, o optional) it writes the sequence's affine state map [M | b] instead:
+// b = final state from zero (outputs to o when given), M = final state with v = 0 from the identity.
 size_t prefill_tc_workspace_bytes(int B, int T, int H, int num_seqs, bool varlen);
 cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const float *log_alpha,
                               const float *beta, const float *h0, const int32_t *cu_seqlens,
                               int num_seqs, int B, int T, int H, void *o, float *h_T, void *workspace,
-                              size_t workspace_bytes, const Prologue &pro, cudaStream_t stream);
+                              size_t workspace_bytes, const Prologue &pro, cudaStream_t stream,
+                              float *map_out = nullptr);
 }  // namespace kda

@@ -115,10 +115,13 @@ kda_decode_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__r
 }
 
 // Tq tokens per state, the state kept in registers between them: read once from slot_in, written
-// once to slot_out.  Same data layout and reductions per token as kda_decode_kernel.  The token data (q, k, v, log_alpha, beta) is staged in shared
-// memory with cp.async, kTokBatch tokens at a time (half for fp32) and double-buffered, so each
-// token's reductions read it from shared memory while the next batch is in flight; k and q are
-// re-read from there for the update instead of being held in registers, so two CTAs fit per SM.
+// once to slot_out.  The columns of S evolve independently (each column j only meets u_j and the
+// sums over the rows of column j), so warp w owns columns 16 w .. 16 w + 15 for every token and
+// never waits for another warp: lane (rg, cg) = (lane >> 2, lane & 3) holds rows rg + 8 r (r < D/8)
+// of columns 16 w + 4 cg .. + 3, the row sums S^T k and S^T q of a token are warp shuffles over the
+// 8 row groups, and u is handed back to the row groups by shuffles too.  The token data (q, k, v,
+// log_alpha, beta) is staged in shared memory with cp.async, kTokBatch tokens at a time (half for
+// fp32) and double-buffered; the CTA meets at a barrier once per batch, not per token.
 constexpr int kMultiWarps = 8;
 constexpr int kTokBatch = 8;
 __device__ __forceinline__ float to_f(float x) { return x; }
@@ -134,13 +137,11 @@ kda_decode_multi_kernel(const T *__restrict__ q, const T *__restrict__ k, const 
                         float *__restrict__ S_pool, int num_slots, const int32_t *__restrict__ slot_in,
                         const int32_t *__restrict__ slot_out, int Tq, int H, T *__restrict__ o,
                         int *__restrict__ status, const Prologue pro) {
-    constexpr int RPW = D / kMultiWarps;  // rows per warp
-    constexpr int VEC = D / 32;           // columns per lane
+    constexpr int RPL = D / 8;                   // rows per lane: rg + 8 r
+    constexpr int CPW = D / kMultiWarps;         // columns per warp
+    constexpr int CPL = CPW / 4;                 // columns per lane (4 for D = 128, 2 for D = 64)
+    constexpr int VEC = D / 32;                  // prologue: elements of a q / k row per lane
     constexpr int TB = sizeof(T) == 4 ? kTokBatch / 2 : kTokBatch;  // fp32 tokens: half the batch (static shared memory)
-    __shared__ float red_a[kMultiWarps][D];
-    __shared__ float red_b[kMultiWarps][D];
-    __shared__ float s_u[D];
-    __shared__ float s_qk[kMultiWarps];
     __shared__ __align__(16) T sk[2][TB][D];
     __shared__ __align__(16) T sq[2][TB][D];
     __shared__ __align__(16) T sv[2][TB][D];
@@ -183,9 +184,17 @@ kda_decode_multi_kernel(const T *__restrict__ q, const T *__restrict__ k, const 
     };
 
     stage(0);
-    float s[RPW][VEC];
+    const int rg = lane >> 2, cg = lane & 3;
+    const int col0 = CPW * warp + CPL * cg;  // this lane's first column
+    constexpr int CP2 = CPL / 2;  // column pairs per lane: the state math runs on packed fp32 pairs
+    float2 s[RPL][CP2];
 #pragma unroll
-    for (int m = 0; m < RPW; ++m) VecIO<VEC>::load(Sin + (size_t)(warp + kMultiWarps * m) * D + lane * VEC, s[m]);
+    for (int r = 0; r < RPL; ++r) {
+        float x[CPL];
+        VecIO<CPL>::load(Sin + (size_t)(rg + 8 * r) * D + col0, x);
+#pragma unroll
+        for (int c = 0; c < CP2; ++c) s[r][c] = make_float2(x[2 * c], x[2 * c + 1]);
+    }
 
     const int nbatch = (Tq + TB - 1) / TB;
     for (int bi = 0; bi < nbatch; ++bi) {
@@ -225,59 +234,73 @@ kda_decode_multi_kernel(const T *__restrict__ q, const T *__restrict__ k, const 
             __syncthreads();
         }
         for (int tt = 0; tt < nt; ++tt) {
-            float pa[VEC], pb[VEC];
+            // decay, then this lane's partial row sums of S^T k, S^T q (its CPL columns) and k . q
+            float2 pa[CP2], pb[CP2];
+            float kr[RPL];
 #pragma unroll
-            for (int c = 0; c < VEC; ++c) pa[c] = pb[c] = 0.f;
+            for (int c = 0; c < CP2; ++c) pa[c] = pb[c] = make_float2(0.f, 0.f);
             float pqk = 0.f;
 #pragma unroll
-            for (int m = 0; m < RPW; ++m) {
-                const int i = warp + kMultiWarps * m;
-                const float ki = to_f(sk[buf][tt][i]);  // shared-memory reads (not the global-memory Elem loads)
+            for (int r = 0; r < RPL; ++r) {
+                const int i = rg + 8 * r;
+                const float ki = to_f(sk[buf][tt][i]);
                 const float qi = to_f(sq[buf][tt][i]);
                 const float ai = ex2f(sla[buf][tt][i] * kLog2e);  // alpha_i by the hardware exp2
+                kr[r] = ki;
                 pqk = fmaf(qi, ki, pqk);
+                const float2 a2 = make_float2(ai, ai), k2 = make_float2(ki, ki), q2 = make_float2(qi, qi);
 #pragma unroll
-                for (int c = 0; c < VEC; ++c) {
-                    s[m][c] *= ai;
-                    pa[c] = fmaf(s[m][c], ki, pa[c]);
-                    pb[c] = fmaf(s[m][c], qi, pb[c]);
+                for (int c = 0; c < CP2; ++c) {
+                    s[r][c] = __fmul2_rn(s[r][c], a2);
+                    pa[c] = __ffma2_rn(s[r][c], k2, pa[c]);
+                    pb[c] = __ffma2_rn(s[r][c], q2, pb[c]);
+                }
+            }
+            // sums over the 8 row groups (lane bits 2..4): each lane ends with the totals of every
+            // one of its columns
+#pragma unroll
+            for (int off = 4; off < 32; off <<= 1) {
+#pragma unroll
+                for (int c = 0; c < CP2; ++c) {
+                    pa[c].x += __shfl_xor_sync(0xffffffffu, pa[c].x, off);
+                    pa[c].y += __shfl_xor_sync(0xffffffffu, pa[c].y, off);
+                    pb[c].x += __shfl_xor_sync(0xffffffffu, pb[c].x, off);
+                    pb[c].y += __shfl_xor_sync(0xffffffffu, pb[c].y, off);
+                }
+                pqk += __shfl_xor_sync(0xffffffffu, pqk, off);
+            }
+            // u_j = beta (v_j - (S'^T k)_j); o_j = (S'^T q)_j + (k . q) u_j, with S' the decayed state
+            const float bt = sb[buf][tt];
+            float2 uu[CP2];
+#pragma unroll
+            for (int c = 0; c < CP2; ++c) {
+                uu[c] = make_float2(bt * (to_f(sv[buf][tt][col0 + 2 * c]) - pa[c].x),
+                                    bt * (to_f(sv[buf][tt][col0 + 2 * c + 1]) - pa[c].y));
+                if (rg == 0) {  // row group 0 writes the warp's columns of o
+                    T *orow = o + tok_of(t0 + tt) * D + col0 + 2 * c;
+                    Elem<T>::store(orow, fmaf(pqk, uu[c].x, pb[c].x));
+                    Elem<T>::store(orow + 1, fmaf(pqk, uu[c].y, pb[c].y));
                 }
             }
 #pragma unroll
-            for (int c = 0; c < VEC; ++c) {
-                red_a[warp][lane * VEC + c] = pa[c];
-                red_b[warp][lane * VEC + c] = pb[c];
-            }
-            if (lane == 0) s_qk[warp] = pqk;
-            __syncthreads();
-            if (threadIdx.x < D) {
-                const int j = threadIdx.x;
-                float a = 0.f, b = 0.f, qk = 0.f;
+            for (int r = 0; r < RPL; ++r) {
+                const float2 k2 = make_float2(kr[r], kr[r]);
 #pragma unroll
-                for (int w = 0; w < kMultiWarps; ++w) {
-                    a += red_a[w][j];
-                    b += red_b[w][j];
-                    qk += s_qk[w];
-                }
-                const float uj = sb[buf][tt] * (to_f(sv[buf][tt][j]) - a);
-                s_u[j] = uj;
-                Elem<T>::store(o + tok_of(t0 + tt) * D + j, fmaf(qk, uj, b));
-            }
-            __syncthreads();
-            float uu[VEC];
-#pragma unroll
-            for (int c = 0; c < VEC; ++c) uu[c] = s_u[lane * VEC + c];
-#pragma unroll
-            for (int m = 0; m < RPW; ++m) {
-                const float ki = to_f(sk[buf][tt][warp + kMultiWarps * m]);
-#pragma unroll
-                for (int c = 0; c < VEC; ++c) s[m][c] = fmaf(ki, uu[c], s[m][c]);
+                for (int c = 0; c < CP2; ++c) s[r][c] = __ffma2_rn(k2, uu[c], s[r][c]);
             }
         }
         __syncthreads();  // batch bi's buffer is free before it is staged again
     }
 #pragma unroll
-    for (int m = 0; m < RPW; ++m) VecIO<VEC>::store(Sout + (size_t)(warp + kMultiWarps * m) * D + lane * VEC, s[m]);
+    for (int r = 0; r < RPL; ++r) {
+        float x[CPL];
+#pragma unroll
+        for (int c = 0; c < CP2; ++c) {
+            x[2 * c] = s[r][c].x;
+            x[2 * c + 1] = s[r][c].y;
+        }
+        VecIO<CPL>::store(Sout + (size_t)(rg + 8 * r) * D + col0, x);
+    }
 }
 
 template <int D, typename T>

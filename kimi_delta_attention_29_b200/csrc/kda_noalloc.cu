@@ -4,12 +4,13 @@
 // its input and output buffers, or an engine that has already reserved all free device memory
 // for its own pool.  They cannot supply the workspace kda_chunk_fwd needs, so this entry point
 // runs the same kernels with a fixed scratch area that the library owns: a file-scope
-// __device__ array, created when the module is loaded and kept by every GPU that loads the
-// library until the process exits.  Nothing here allocates.
+// __device__ array, created when the module is loaded on a device and kept there until the
+// process exits or the device is reset.  Nothing here allocates.
 //
 // In host code the array's name is only a host-side stand-in, so the device address is looked
-// up with cudaGetSymbolAddress once per device (the first call on that device, with it current)
-// and cached.
+// up with cudaGetSymbolAddress on the first call on each device (with it current) and cached with
+// the id of the CUDA context it belongs to: after a device reset the module, and with it the array,
+// is loaded again in a new context, and the next call looks the address up again.
 #include <mutex>
 
 #include "kda_common.cuh"
@@ -23,19 +24,22 @@ static __device__ __align__(256) unsigned char g_kda_noalloc_scratch[kNoallocScr
 
 std::mutex g_mu;
 void *g_scratch_ptr[kMaxDevices] = {};
+unsigned long long g_scratch_ctx[kMaxDevices] = {};
 
-// Device address of the static scratch on the current device (looked up once per device).
+// Device address of the static scratch on the current device, in the current context.
 cudaError_t scratch_for_current_device(void **out) {
     int dev = -1;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
     std::lock_guard<std::mutex> lock(g_mu);
-    if (!g_scratch_ptr[dev]) {
+    const unsigned long long ctx = kda::current_context_id();
+    if (!g_scratch_ptr[dev] || ctx == 0 || g_scratch_ctx[dev] != ctx) {
         void *p = nullptr;
         e = cudaGetSymbolAddress(&p, g_kda_noalloc_scratch);
         if (e != cudaSuccess) return e;
         g_scratch_ptr[dev] = p;
+        g_scratch_ctx[dev] = kda::current_context_id();  // the lookup has made a context current
     }
     *out = g_scratch_ptr[dev];
     return cudaSuccess;

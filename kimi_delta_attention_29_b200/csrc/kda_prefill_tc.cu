@@ -20,15 +20,16 @@
 //     depend on the state: log-gate cumsum, decay factors, the two Gram matrices (tcgen05, formed
 //     transposed: one M=64, N=32 product per 16-row block with k-rows and q-rows side by side, so
 //     each block can use its own decay reference), the UT transform in fp32 on CUDA cores (blocked
-//     forward substitution), and W, U (tcgen05, M=64, N=128).  It writes [W; Q o e^G],
-//     K o e^{G_63-G}, P, U and e^{G_63} for the chunk as ready-to-use swizzled operand images
-//     ("records") in the workspace.  Its q, k, log-gate and V tiles arrive by TMA (tensor maps
-//     encoded per call), V directly in the swizzled layout the W/U product reads.
-//  2. kda_tc_state_kernel - one CTA per (sequence, head, 32 value columns); the value columns of S
-//     evolve independently.  It walks the sequence's chunks in order, bulk-copying each record into
-//     a 2-stage shared-memory ring, and runs per chunk: D_a = [W; Q~] S (M=128, N=32, K=128),
-//     Delta = U - D_a[0:64], D_b = K^T Delta (M=128, K=64), D_a[64:128] += P Delta, then
-//     S <- e^{G_63} S + D_b with the fp32 master state in registers and a bf16 copy as MMA operand.
+//     forward substitution), and W, U^T (tcgen05).  It writes [-W; Q o e^G], K o e^{G_63-G}, P,
+//     U^T and e^{G_63} for the chunk as ready-to-use swizzled operand images ("records") in the
+//     workspace and then publishes the record's ready word.  Its q, k, log-gate and V tiles arrive
+//     by TMA (tensor maps encoded per call), V directly in the swizzled layout the U^T product reads.
+//  2. kda_tc_state_kernel - persistent, one (sequence, head) unit per CTA at a time, the state
+//     carried transposed in tensor memory so every product runs at M = 128.  It waits for each
+//     record's ready word, bulk-copies the record into a 2-stage shared-memory ring and runs the
+//     chunk's three products (see the kernel's own comment).  It runs concurrently with kernel 1 on
+//     a high-priority side stream, a quarter of the SMs at most, so the records of a chunk are
+//     usually consumed while still in L2 (and then dropped from it without a write-back).
 //
 // Decay references (secondary chunking): block b (rows 16b..16b+15) uses E_b = G at row 16b+7.
 // For a row r of block b and a key row i <= r, e^{G_r - G_i} = e^{G_r - E_b} e^{E_b - G_i}: the first
@@ -40,6 +41,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <cstdlib>
 #include <mutex>
 
 #include "kda_common.cuh"
@@ -362,7 +364,9 @@ kda_tc_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         tmem_alloc(s_tmem, kPrepTmemCols);
         tmem_relinquish();
     }
-    if (tid < 64) s_beta[tid] = tid < L ? __ldg(beta + ((size_t)t0 + tid) * H + h) : 0.f;
+    // beta of the chunk's rows: held in a register until the gate scan is done, so the global load's
+    // latency overlaps the input tiles' arrival and the scan
+    const float beta_r = tid < 64 && tid < L ? __ldg(beta + ((size_t)t0 + tid) * H + h) : 0.f;
     __syncthreads();  // barriers initialised before anyone waits on them
 
     // ---- k, q (bf16 pairs) and log-gates (fp32 pairs) of this thread's 16 rows, from the landed tiles
@@ -475,6 +479,7 @@ kda_tc_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         s_gl[c0] = g[15].x;
         s_gl[c0 + 1] = g[15].y;
     }
+    if (tid < 64) s_beta[tid] = beta_r;
     __syncthreads();
 
     const float2 gl = make_float2(s_gl[c0], s_gl[c0 + 1]);
@@ -641,7 +646,9 @@ kda_tc_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     // U is produced transposed so that each TMEM lane holds one value channel, the row of U^T the
     // state kernel reads per thread.
     if (ok && tid == 0) ok = mbar_wait(mbar + 3, 0);  // V tile landed
+    bool wu_issued = false;
     if (ok && tid == 0) {
+        wu_issued = true;
         tc_fence_after();
         const uint32_t id_w = idesc_bf16_f32(64, 128, 0, 1);
         const uint32_t id_ut = idesc_bf16_f32(128, 64, 1, 0);
@@ -699,12 +706,23 @@ kda_tc_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     } else if (tid == 0) {
         set_status(status, KDA_ERR_TIMEOUT);
     }
+    if (!ok && tid == 0) {
+        // a wait gave up: let every copy and product this CTA started land before its shared and
+        // tensor memory are released (each of these waits is bounded too)
+        mbar_wait(mbar + 2, 0);
+        mbar_wait(mbar + 3, 0);
+        mbar_wait(mbar + 1, 0);
+        if (wu_issued) mbar_wait(mbar, 0);
+    }
     // every record store of this CTA is performed before the ready word is published (after a
-    // timeout too: the status word carries the error and the consumer must not wait in vain)
-    __threadfence();
+    // timeout too: the status word carries the error and the consumer must not wait in vain): the
+    // CTA barrier orders all threads' stores before thread 0's gpu-scope fence and release store
     tc_fence_before();
     __syncthreads();
-    if (tid == 0) publish_flag(flags + (size_t)chunk * H + h);
+    if (tid == 0) {
+        __threadfence();
+        publish_flag(flags + (size_t)chunk * H + h);
+    }
     if (warp == 0) tmem_dealloc(tmem, kPrepTmemCols);
 }
 
@@ -758,8 +776,8 @@ __global__ void __launch_bounds__(kStateThreads, 1)
 kda_tc_state_kernel(const __grid_constant__ CUtensorMap tm_o, const uint8_t *__restrict__ records,
                     const int *__restrict__ flags, const float *__restrict__ h0, const int *__restrict__ base,
                     const int4 *__restrict__ table, const int *__restrict__ order, int num_units, int nc, int T_len,
-                    int H, __nv_bfloat16 *__restrict__ o, float *__restrict__ h_T, int *status,
-                    int *unit_counter) {
+                    int H, __nv_bfloat16 *__restrict__ o, float *__restrict__ h_T, float *__restrict__ Mb,
+                    int *status, int *unit_counter) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = align1024(smem_raw);
     uint64_t *full = reinterpret_cast<uint64_t *>(sm + ST_BAR);  // [2] record landed in the stage
@@ -813,9 +831,19 @@ kda_tc_state_kernel(const __grid_constant__ CUtensorMap tm_o, const uint8_t *__r
     for (;;) {
         const int u = *s_unit;
         if (u >= num_units) break;
+        // Map mode (Mb set; one sequence, no h0, no h_T): units 0 .. H-1 run head h = u from the zero
+        // state (the map's b, outputs to o when given), units H .. 2H-1 run head h = u - H with v = 0
+        // from the identity (the map's M, no outputs).  Their final states go to Mb [H, D, 2D]:
+        // M in columns 0 .. D-1, b in columns D .. 2D-1.
+        const bool map_mode = Mb != nullptr;
+        const bool m_unit = map_mode && u >= H;
         int n, h, c_begin, nchunks;
-        state_unit(u, H, nc, base, order, n, h, c_begin, nchunks);
+        state_unit(map_mode ? u % H : u, H, nc, base, order, n, h, c_begin, nchunks);
         const size_t soff = ((size_t)n * H + h) * D * D + j;  // S[k][j] at soff + k * D
+        float *const hT_col = map_mode ? Mb + (size_t)h * D * (2 * D) + (m_unit ? 0 : D) + j
+                                       : (h_T ? h_T + soff : nullptr);  // S[k][j] at hT_col + k * hT_ld
+        const size_t hT_ld = map_mode ? 2 * D : D;
+        const bool write_o = o != nullptr && !m_unit;
         auto wwait = [&](uint64_t *bar, uint32_t parity) {
             return __all_sync(0xffffffffu, mbar_wait_or_abort(bar, parity, s_abort));
         };
@@ -926,11 +954,12 @@ kda_tc_state_kernel(const __grid_constant__ CUtensorMap tm_o, const uint8_t *__r
             bool ok = true;
             float sv[32];
 #pragma unroll
-            for (int kk = 0; kk < 32; ++kk) sv[kk] = h0 ? __ldg(h0 + soff + (size_t)(32 * g + kk) * D) : 0.f;
+            for (int kk = 0; kk < 32; ++kk)
+                sv[kk] = m_unit ? (32 * g + kk == j ? 1.f : 0.f) : h0 ? __ldg(h0 + soff + (size_t)(32 * g + kk) * D) : 0.f;
             if (nchunks == 0) {
-                if (h_T) {
+                if (hT_col) {
 #pragma unroll
-                    for (int kk = 0; kk < 32; ++kk) h_T[soff + (size_t)(32 * g + kk) * D] = sv[kk];
+                    for (int kk = 0; kk < 32; ++kk) hT_col[(size_t)(32 * g + kk) * hT_ld] = sv[kk];
                 }
             } else {
                 store_as(sv);
@@ -959,9 +988,9 @@ kda_tc_state_kernel(const __grid_constant__ CUtensorMap tm_o, const uint8_t *__r
                     if (i + 1 < nchunks) {
                         store_as(nv);
                         if (!store_d2(gc + 1, nv)) { ok = false; break; }
-                    } else if (h_T) {
+                    } else if (hT_col) {
 #pragma unroll
-                        for (int kk = 0; kk < 32; ++kk) h_T[soff + (size_t)(32 * g + kk) * D] = nv[kk];
+                        for (int kk = 0; kk < 32; ++kk) hT_col[(size_t)(32 * g + kk) * hT_ld] = nv[kk];
                     }
                 }
             }
@@ -984,7 +1013,8 @@ kda_tc_state_kernel(const __grid_constant__ CUtensorMap tm_o, const uint8_t *__r
             auto preload_d1 = [&](uint32_t gc) -> bool {
                 const uint32_t s = gc & 1, b = gc & 1;
                 if (!wwait(&full[s], (gc >> 1) & 1)) return false;
-                {   // the record is in shared memory: drop its L2 lines without writing them back
+                if (!map_mode) {  // the record is in shared memory: drop its L2 lines without writing them back
+                    // (a map launch reads every record twice, so there it stays)
                     const uint8_t *rec = records + ((size_t)(c_begin + (int)(gc - gc0)) * H + h) * REC_BYTES;
                     for (int l = atid; l < (int)(REC_TX / 128); l += 32 * kAuxWarps)
                         asm volatile("discard.global.L2 [%0], 128;" ::"l"(rec + 128 * l) : "memory");
@@ -993,6 +1023,11 @@ kda_tc_state_kernel(const __grid_constant__ CUtensorMap tm_o, const uint8_t *__r
                 uint32_t uf[32];  // bf16 -> fp32 is exact: the bf16 bits are the high half of the word
 #pragma unroll
                 for (int x = 0; x < 4; ++x) {
+                    if (m_unit) {  // v = 0: U = 0
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) uf[8 * x + e] = 0u;
+                        continue;
+                    }
                     const uint4 w = *reinterpret_cast<const uint4 *>(urow + (((4 * hf + x) ^ (j & 7)) << 4));
                     const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
@@ -1013,6 +1048,7 @@ kda_tc_state_kernel(const __grid_constant__ CUtensorMap tm_o, const uint8_t *__r
             // again two chunks later; aux_tid0 waits for every earlier TMA store to finish reading
             // before it passes the barrier that precedes those writes.
             auto store_out = [&](int i, uint32_t gc) {
+                if (!write_o) return;
                 float ov[32];
                 tmem_ld32(tmem + TM_D1 + 128 * (gc & 1) + lb + 64 + 32 * hf, ov);
                 tmem_wait_ld();
@@ -1120,28 +1156,36 @@ cudaError_t encode_token_map(CUtensorMap *map, const void *base, CUtensorMapData
 }
 
 // High-priority side stream of the current device for the state kernel, with the fork / join events
-// (created on first use and kept for the life of the process; the mutex serialises the fork, the
-// launches and the join of concurrent host callers).
+// (created on first use in each CUDA context of the device and kept while that context lives: a
+// device reset destroys them with the context, and the next call creates new ones).  The mutex
+// serialises the fork, the launches and the join of concurrent host callers.
 struct SideStream {
     cudaStream_t stream = nullptr;
     cudaEvent_t fork = nullptr, join = nullptr;
+    unsigned long long ctx = 0;  // context the handles belong to
     std::mutex mu;
 };
 SideStream *side_stream() {
     static SideStream per_dev[64];
-    static std::once_flag once[64];
+    static std::mutex create_mu;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
     SideStream *s = &per_dev[dev];
-    std::call_once(once[dev], [s] {
-        int lo = 0, hi = 0;
-        cudaDeviceGetStreamPriorityRange(&lo, &hi);
-        if (cudaStreamCreateWithPriority(&s->stream, cudaStreamNonBlocking, hi) != cudaSuccess ||
-            cudaEventCreateWithFlags(&s->fork, cudaEventDisableTiming) != cudaSuccess ||
-            cudaEventCreateWithFlags(&s->join, cudaEventDisableTiming) != cudaSuccess)
-            s->stream = nullptr;
-    });
-    return s->stream ? s : nullptr;
+    std::lock_guard<std::mutex> lock(create_mu);
+    const unsigned long long ctx = current_context_id();
+    if (s->stream && ctx != 0 && s->ctx == ctx) return s;
+    // first use in this context (the handles of an earlier, reset context are gone with it)
+    int lo = 0, hi = 0;
+    cudaDeviceGetStreamPriorityRange(&lo, &hi);
+    s->stream = nullptr;
+    if (cudaStreamCreateWithPriority(&s->stream, cudaStreamNonBlocking, hi) != cudaSuccess ||
+        cudaEventCreateWithFlags(&s->fork, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&s->join, cudaEventDisableTiming) != cudaSuccess) {
+        s->stream = nullptr;
+        return nullptr;
+    }
+    s->ctx = current_context_id();
+    return s;
 }
 
 // Streaming multiprocessors of the current device (cached per device).
@@ -1157,6 +1201,27 @@ int sm_count() {
 }
 
 }  // namespace
+
+unsigned long long current_context_id() {
+    static PFN_cuCtxGetCurrent_v4000 get_current = nullptr;
+    static PFN_cuCtxGetId_v12000 get_id = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult qr;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &qr) == cudaSuccess &&
+            qr == cudaDriverEntryPointSuccess)
+            get_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
+        p = nullptr;
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &qr) == cudaSuccess &&
+            qr == cudaDriverEntryPointSuccess)
+            get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(p);
+    });
+    CUcontext c = nullptr;
+    unsigned long long id = 0;
+    if (!get_current || !get_id || get_current(&c) != CUDA_SUCCESS || !c || get_id(c, &id) != CUDA_SUCCESS) return 0;
+    return id;
+}
 
 cudaError_t launch_chunk_table(const int32_t *cu_seqlens, int num_seqs, int T, int *status_blk, int *base,
                                int4 *table, cudaStream_t stream) {
@@ -1174,7 +1239,7 @@ size_t prefill_tc_workspace_bytes(int B, int T, int H, int num_seqs, bool varlen
 cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const float *log_alpha,
                               const float *beta, const float *h0, const int32_t *cu_seqlens, int num_seqs,
                               int B, int T, int H, void *o, float *h_T, void *workspace, size_t workspace_bytes,
-                              const Prologue &pro, cudaStream_t stream) {
+                              const Prologue &pro, cudaStream_t stream, float *map_out) {
     (void)workspace_bytes;
     const TcLayout lay = tc_layout(B, T, H, num_seqs);
     uint8_t *ws = static_cast<uint8_t *>(workspace);
@@ -1207,11 +1272,12 @@ cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const
         (e = encode_token_map(&tm_k, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, tokens, H, D, CU_TENSOR_MAP_SWIZZLE_NONE)) != cudaSuccess ||
         (e = encode_token_map(&tm_v, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, tokens, H, 64, CU_TENSOR_MAP_SWIZZLE_128B)) != cudaSuccess ||
         (e = encode_token_map(&tm_g, log_alpha, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, tokens, H, D, CU_TENSOR_MAP_SWIZZLE_NONE)) != cudaSuccess ||
-        (e = encode_token_map(&tm_o, o, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, tokens, H, D, CU_TENSOR_MAP_SWIZZLE_NONE)) != cudaSuccess))
+        (o && (e = encode_token_map(&tm_o, o, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, tokens, H, D, CU_TENSOR_MAP_SWIZZLE_NONE)) != cudaSuccess)))
         return e;
     auto *ob = static_cast<__nv_bfloat16 *>(o);
     const bool varlen = cu_seqlens != nullptr;
-    const int num_units = (varlen ? num_seqs : B) * H;
+    // map mode (one sequence): a zero-start unit and an identity-start unit per head
+    const int num_units = map_out ? 2 * H : (varlen ? num_seqs : B) * H;
     const int nc = varlen ? 0 : (T + C - 1) / C;
     const int64_t prep_ctas = varlen ? lay.max_chunks * H : (int64_t)B * nc * H;
     if (varlen) {
@@ -1226,11 +1292,33 @@ cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const
     const int *ord = varlen && num_seqs <= kOrderMax ? order : nullptr;
     // A quarter of the SMs at most pass the state (one CTA per SM, a (sequence, head) unit at a
     // time); the intra-chunk kernel fills the rest and runs at the same time.
-    const int state_grid = std::max(1, std::min(num_units, std::max(1, sm_count() / 4)));
+    // A map launch has twice the state work for the same intra-chunk work: half of the SMs.
+    const int state_grid = std::max(1, std::min(num_units, std::max(1, sm_count() / (map_out ? 2 : 4))));
     if (prep_ctas == 0) {  // no tokens: the state kernel alone writes h_T
         trace_before(kKernTcState, stream);
         kda_tc_state_kernel<<<(unsigned)state_grid, kStateThreads, STATE_SMEM, stream>>>(
-            tm_o, records, flags, h0, bas, tbl, ord, num_units, nc, T, H, ob, h_T, status, status + 2);
+            tm_o, records, flags, h0, bas, tbl, ord, num_units, nc, T, H, ob, h_T, map_out, status, status + 2);
+        trace_after(stream);
+        return cudaGetLastError();
+    }
+    // KDA_PREFILL_SERIAL=1 in the environment (read once per process) runs the intra-chunk kernel to
+    // completion before the state kernel, both on `stream`: same results, no overlap.  Profilers that
+    // serialise kernel launches need it, since the state kernel, launched first in the concurrent
+    // order, would wait for records that no kernel produces until it has finished.
+    static const bool serial = [] {
+        const char *v = std::getenv("KDA_PREFILL_SERIAL");
+        return v != nullptr && v[0] == '1';
+    }();
+    if (serial) {
+        trace_before(kKernTcPrep, stream);
+        prep<<<(unsigned)prep_ctas, kPrepThreads, PREP_SMEM, stream>>>(tm_q, tm_k, tm_v, tm_g, pro, beta, T, H, nc,
+                                                                        varlen ? status + 1 : nullptr, tbl, records,
+                                                                        flags, status);
+        trace_after(stream);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        trace_before(kKernTcState, stream);
+        kda_tc_state_kernel<<<(unsigned)state_grid, kStateThreads, STATE_SMEM, stream>>>(
+            tm_o, records, flags, h0, bas, tbl, ord, num_units, nc, T, H, ob, h_T, map_out, status, status + 2);
         trace_after(stream);
         return cudaGetLastError();
     }
@@ -1245,7 +1333,7 @@ cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const
     if ((e = cudaEventRecord(side->fork, stream)) != cudaSuccess) return e;
     if ((e = cudaStreamWaitEvent(side->stream, side->fork, 0)) != cudaSuccess) return e;
     kda_tc_state_kernel<<<(unsigned)state_grid, kStateThreads, STATE_SMEM, side->stream>>>(
-        tm_o, records, flags, h0, bas, tbl, ord, num_units, nc, T, H, ob, h_T, status, status + 2);
+        tm_o, records, flags, h0, bas, tbl, ord, num_units, nc, T, H, ob, h_T, map_out, status, status + 2);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if ((e = cudaEventRecord(side->join, side->stream)) != cudaSuccess) return e;
     prep<<<(unsigned)prep_ctas, kPrepThreads, PREP_SMEM, stream>>>(tm_q, tm_k, tm_v, tm_g, pro, beta, T, H, nc,

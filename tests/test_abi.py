@@ -235,6 +235,31 @@ def test_state_compose_rejects_on_host(lib):
     assert call(S_in=A + 1024) == _lib.KDA_ERR_ALIASING
 
 
+def test_segment_map_rejects_on_host(lib):
+    c = ctypes.c_void_p
+    f = lib.kda_segment_map
+    W = 1 << 30  # a workspace address no argument below reaches
+
+    def call(T=100, H=2, dk=128, dv=128, dtype=_lib.KDA_BF16, o0=None, Mb=8 * A, ws=W, ws_bytes=1 << 30, x=A):
+        ptr = lambda p: c(p) if p else None
+        return f(ptr(x), ptr(x + A // 4), ptr(x + A // 2), ptr(x + 3 * A // 4), ptr(x + A - 4096), T, H, dk, dv, 64,
+                 dtype, ptr(o0), ptr(Mb), ptr(ws), ws_bytes, None)
+
+    assert call(Mb=0) == _lib.KDA_ERR_NULL_ARG
+    assert call(ws=0) == _lib.KDA_ERR_NULL_ARG
+    assert call(x=0) == _lib.KDA_ERR_NULL_ARG
+    assert call(dtype=7) == _lib.KDA_ERR_BAD_DTYPE
+    assert call(T=-1) == _lib.KDA_ERR_BAD_SHAPE
+    assert call(dk=64, dv=64) == _lib.KDA_ERR_UNSUPPORTED          # CUDA-core sizes: two prefills instead
+    assert call(dtype=_lib.KDA_F32) == _lib.KDA_ERR_UNSUPPORTED
+    assert call(Mb=8 * A + 4) == _lib.KDA_ERR_MISALIGNED
+    assert call(ws=W + 16) == _lib.KDA_ERR_MISALIGNED
+    assert call(ws_bytes=1024) == _lib.KDA_ERR_WORKSPACE_TOO_SMALL
+    assert call(Mb=A + 4096) == _lib.KDA_ERR_ALIASING                 # map inside q
+    assert call(o0=8 * A + 4096) == _lib.KDA_ERR_ALIASING             # outputs inside the map
+    assert call(Mb=W + 4096) == _lib.KDA_ERR_ALIASING                 # map inside the workspace
+
+
 def test_binding_constants_match_the_header():
     """The binding's status codes and prologue flags are the header's, and its trace names cover
     every kernel id the library reports."""

@@ -136,3 +136,45 @@ def test_state_compose_kernel(cuda_device, R, dk, dv):
         assert torch.allclose(S_in[j].double().cpu(), S, rtol=1e-4, atol=1e-4 * float(S.abs().max()))
         S = M64[j, :, :, :dk] @ S + M64[j, :, :, dk:]
     assert torch.allclose(S_out.double().cpu(), S, rtol=1e-4, atol=1e-4 * float(S.abs().max()))
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("T,want_o,gate_shift", [(1000, True, -6.0), (64, True, 1.5), (777, False, -6.0),
+                                                  (200, True, -6.0), (0, True, 2.0)])
+def test_segment_map_one_pass(cuda_device, T, want_o, gate_shift):
+    """kda_segment_map against the oracle: b = final state from zero (with outputs o0), M = final state
+    of a v = 0 pass from the identity (the definitions of the map in include/kda.h).  log alpha =
+    -softplus(N(0,1) + gate_shift): at -6 (alpha near 0.9975) M stays measurable over ~1000 tokens
+    (max |M| ~ 1e-3, the delta rule's own contraction); at 1.5 it is below 1e-38 after 64 tokens and
+    only b and the outputs are compared."""
+    import oracle
+    import kimi_delta_attention_29_b200 as kda
+    from kimi_delta_attention_29_b200 import inputs as gen
+    H, d = 3, 128
+    x = gen.make_prefill(1, T, H, d, d, torch.bfloat16, gate_shift=gate_shift, seed=90 + T, device=cuda_device)
+    o0, Mb = kda.kda_segment_map(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], want_o=want_o)
+    torch.cuda.synchronize(cuda_device)
+    assert Mb.shape == (H, d, 2 * d) and (o0 is not None) == want_o
+    f = lambda a: a.detach().float().cpu().numpy().astype(np.float64)
+    eye = np.broadcast_to(np.eye(d), (1, H, d, d)).copy()
+    if T == 0:
+        assert np.array_equal(f(Mb[:, :, :d]), eye[0]) and not f(Mb[:, :, d:]).any()
+        return
+    o_ref, b_ref = oracle.recurrent(f(x["q"]), f(x["k"]), f(x["v"]), f(x["log_alpha"]), f(x["beta"]), None)
+    _, M_ref = oracle.recurrent(f(x["q"]), f(x["k"]), np.zeros_like(f(x["v"])), f(x["log_alpha"]), f(x["beta"]), eye)
+    rel = lambda a, b: float(np.abs(a - b).max() / np.abs(b).max())
+    check_m = gate_shift < 0
+    assert not check_m or np.abs(M_ref).max() > 1e-4  # the case exercises M
+    assert rel(f(Mb[:, :, d:]), b_ref[0]) <= 2e-2
+    if check_m:
+        assert rel(f(Mb[:, :, :d]), M_ref[0]) <= 2e-2
+    if want_o:
+        assert rel(f(o0), o_ref) <= 2e-2
+    # the same map from two separate prefills
+    _, b2 = kda.kda_chunk_fwd(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], None, None)
+    _, M2 = kda.kda_chunk_fwd(x["q"], x["k"], torch.zeros_like(x["v"]), x["log_alpha"], x["beta"],
+                              torch.from_numpy(eye).float().to(cuda_device), None)
+    torch.cuda.synchronize(cuda_device)
+    assert rel(f(Mb[:, :, d:]), f(b2[0])) <= 2e-2
+    if check_m:
+        assert rel(f(Mb[:, :, :d]), f(M2[0])) <= 2e-2

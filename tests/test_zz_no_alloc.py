@@ -76,3 +76,23 @@ def test_noalloc_rejects_sizes_beyond_its_scratch(cuda_device):
     o = torch.empty_like(x["v"])
     hT = torch.empty(1, 32, 128, 128, device=cuda_device)
     assert _call_noalloc(fn, x, o, hT, stream) == _lib.KDA_ERR_WORKSPACE_TOO_SMALL
+
+
+def test_noalloc_varlen_matches_workspace_entry_point(cuda_device):
+    """Packed sequences (cu_seqlens) through the no-alloc entry point: the chunk table, the
+    longest-first layout and the ready words all live in the shared scratch."""
+    fn = _noalloc_fn()
+    stream = torch.cuda.current_stream(cuda_device)
+    lengths = torch.tensor([64, 1, 300, 127, 65, 129], dtype=torch.int64)  # full, ragged and 1-token chunks
+    cu = gen.cu_seqlens_from_lengths(lengths)
+    x = gen.make_prefill(1, int(cu[-1]), 8, 128, 128, torch.bfloat16, gate_shift=1.5, h0_std=0.2, seed=24,
+                         device=cuda_device, cu_seqlens=cu)
+    assert kda.kda_chunk_fwd_workspace_size(1, int(cu[-1]), 8, 128, 128, x["num_seqs"]) <= 64 << 20
+    o_ref, h_ref = kda.kda_chunk_fwd(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], x["h0"], x["cu_seqlens"])
+    o = torch.full_like(o_ref, float("nan"))
+    hT = torch.full_like(h_ref, float("nan"))
+    assert _call_noalloc(fn, x, o, hT, stream) == _lib.KDA_OK
+    torch.cuda.synchronize(cuda_device)
+    assert torch.isfinite(o.float()).all() and torch.isfinite(hT).all()
+    assert _rel(o, o_ref) <= TOL
+    assert _rel(hT, h_ref) <= TOL
