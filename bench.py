@@ -54,6 +54,9 @@ def parse_args():
     p.add_argument("--backward-steps", type=int, default=3)
     p.add_argument("--cpu-seconds", type=float, default=12.0,
                    help="target CPU time of the oracle sample (0 skips the CPU baseline)")
+    p.add_argument("--profile-range", action="store_true",
+                   help="after the warm-up, run one long-context step between cudaProfilerStart and "
+                        "cudaProfilerStop and exit (for a profiler's range replay of the whole concurrent call)")
     p.add_argument("--seq-len", type=int, default=131072,
                    help="override T of the long-context workload (small cases for profiler captures)")
     return p.parse_args()
@@ -399,6 +402,16 @@ def gpu_arm(args):
         step()
     torch.cuda.synchronize(dev)
     assert kda.kda_get_status(ws) == 0, "device status after warm-up"
+    if args.profile_range:  # one step inside a profiler range (both kernels of the call, concurrent)
+        torch.cuda.cudart().cudaProfilerStart()
+        step()
+        torch.cuda.synchronize(dev)
+        torch.cuda.cudart().cudaProfilerStop()
+        assert kda.kda_get_status(ws) == 0, "device status after the profiled step"
+        print(json.dumps({"profile_range": shp.name, "T": T, "H": H, "tokens": B * T}))
+        if world > 1:
+            dist.destroy_process_group()
+        return
 
     clocks = ClockSampler(dev.index)
     barrier()

@@ -233,6 +233,12 @@ kda_decode_multi_kernel(const T *__restrict__ q, const T *__restrict__ k, const 
             }
             __syncthreads();
         }
+        // alpha = 2^{log_alpha log2 e} once per staged (token, row) instead of once per warp and lane
+        for (int e = threadIdx.x; e < nt * D; e += kMultiWarps * 32) {
+            float *p = &sla[buf][e / D][e % D];
+            *p = ex2f(*p * kLog2e);
+        }
+        __syncthreads();
         for (int tt = 0; tt < nt; ++tt) {
             // decay, then this lane's partial row sums of S^T k, S^T q (its CPL columns) and k . q
             float2 pa[CP2], pb[CP2];
@@ -245,7 +251,7 @@ kda_decode_multi_kernel(const T *__restrict__ q, const T *__restrict__ k, const 
                 const int i = rg + 8 * r;
                 const float ki = to_f(sk[buf][tt][i]);
                 const float qi = to_f(sq[buf][tt][i]);
-                const float ai = ex2f(sla[buf][tt][i] * kLog2e);  // alpha_i by the hardware exp2
+                const float ai = sla[buf][tt][i];  // alpha_i (the hardware exp2, applied above)
                 kr[r] = ki;
                 pqk = fmaf(qi, ki, pqk);
                 const float2 a2 = make_float2(ai, ai), k2 = make_float2(ki, ki), q2 = make_float2(qi, qi);
