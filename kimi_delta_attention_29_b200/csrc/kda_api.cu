@@ -292,7 +292,7 @@ size_t kda_chunk_bwd_workspace_size(int B, int T, int H, int dk, int dv, int num
     const bool varlen = (B == 1 && num_seqs > 1);
     if (check_prefill_shape(B, T, H, dk, dv, num_seqs, varlen, chunk_size) != KDA_OK) return 0;
     if (dk != dv) return 0;
-    return kda::chunk_bwd_workspace_bytes(B, T, H, dk, num_seqs);
+    return kda::chunk_bwd_workspace_bytes(B, T, H, dk, num_seqs, dtype);
 }
 
 int kda_chunk_bwd(const void *q, const void *k, const void *v, const float *log_alpha, const float *beta,
@@ -313,7 +313,7 @@ int kda_chunk_bwd(const void *q, const void *k, const void *v, const float *log_
     for (const void *p : ptrs)
         if (p && !aligned16(p)) return KDA_ERR_MISALIGNED;
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return KDA_ERR_MISALIGNED;
-    const size_t need = kda::chunk_bwd_workspace_bytes(B, T, H, dk, num_seqs);
+    const size_t need = kda::chunk_bwd_workspace_bytes(B, T, H, dk, num_seqs, dtype);
     if (workspace_bytes < need) return KDA_ERR_WORKSPACE_TOO_SMALL;
     const size_t es = elem_size(dtype), tk = (size_t)tokens * H, sb = (size_t)num_seqs * H * dk * dv * 4;
     const Range in[] = {range_of(q, tk * dk * es), range_of(k, tk * dk * es), range_of(v, tk * dv * es),

@@ -221,7 +221,7 @@ kda_bwd_state_kernel(const T *__restrict__ v, const float *__restrict__ beta, co
                      const int32_t *__restrict__ cu_seqlens, const int *__restrict__ chunk_base, int num_seqs,
                      int T_len, int H, const T *__restrict__ dout, const float *__restrict__ dhT,
                      const float *__restrict__ ops, float *__restrict__ recs, T *__restrict__ dv_out,
-                     float *__restrict__ dh0, int *status) {
+                     float *__restrict__ dh0, int *status, bool have_states) {
     using SM = StateSmem<D>;
     constexpr int DKP = SM::DKP;
     using R = BwdRec<D>;
@@ -314,8 +314,8 @@ kda_bwd_state_kernel(const T *__restrict__ v, const float *__restrict__ beta, co
         __syncthreads();
     };
 
-    // ---- forward: chunk-start states into the records
-    for (int ch = 0; ch < nch; ++ch) {
+    // ---- forward: chunk-start states into the records (unless the tensor-core forward wrote them)
+    for (int ch = 0; ch < (have_states ? 0 : nch); ++ch) {
         const int64_t t0 = start + (int64_t)ch * kC;
         const int L = (int)min((int64_t)kC, len - (int64_t)ch * kC);
         float *rec = recs + ((size_t)(cbase + ch) * H + h) * R::floats;
@@ -692,12 +692,17 @@ kda_bwd_chunk_kernel(const T *__restrict__ q, const T *__restrict__ k, const flo
     }
 }
 
+// The first error recorded in src goes to dst when dst holds none.
+__global__ void kda_status_merge_kernel(int *dst, const int *src) {
+    if (threadIdx.x == 0 && src[0] != 0 && dst[0] == 0) dst[0] = src[0];
+}
+
 template <int D, typename T>
 cudaError_t launch_t(const void *q, const void *k, const void *v, const float *la, const float *beta,
                      const float *h0, const int32_t *cu, int num_seqs, int B, int T_len, int H, const void *dout,
                      const float *dhT, void *dq, void *dk, void *dv, float *dla, float *dbeta, float *dh0,
                      int *status, int *base, int4 *table, float *ops, float *recs, int64_t max_chunks,
-                     cudaStream_t stream) {
+                     void *fwd_ws, size_t fwd_ws_bytes, cudaStream_t stream) {
     auto kp = kda_bwd_prep_kernel<D, T>;
     auto ks = kda_bwd_state_kernel<D, T>;
     auto kc = kda_bwd_chunk_kernel<D, T>;
@@ -724,9 +729,22 @@ cudaError_t launch_t(const void *q, const void *k, const void *v, const float *l
         trace_after(stream);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
+    // bf16, D = 128: the tensor-core forward writes every chunk's incoming state straight into the
+    // records, so the state pass below runs only its reverse sweep
+    const bool have_states = fwd_ws != nullptr;
+    if (have_states) {
+        const StateSave save{recs + BwdRec<D>::St, cu ? base : nullptr, nc, (long long)BwdRec<D>::floats};
+        const Prologue none{0u, nullptr, nullptr};
+        if ((e = launch_prefill_tc(q, k, v, la, beta, h0, cu, num_seqs, B, T_len, H, nullptr, nullptr, fwd_ws,
+                                   fwd_ws_bytes, none, stream, nullptr, &save)) != cudaSuccess)
+            return e;
+        kda_status_merge_kernel<<<1, 32, 0, stream>>>(status, static_cast<const int *>(fwd_ws));
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
     trace_before(kKernBwdState, stream);
     ks<<<(unsigned)((int64_t)num_seqs * H * (D / kNV)), kBTs, StateSmem<D>::bytes, stream>>>(
-        vt, beta, h0, cu, base, num_seqs, T_len, H, dot, dhT, ops, recs, static_cast<T *>(dv), dh0, status);
+        vt, beta, h0, cu, base, num_seqs, T_len, H, dot, dhT, ops, recs, static_cast<T *>(dv), dh0, status,
+        have_states);
     trace_after(stream);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if (chunks == 0) return cudaSuccess;
@@ -739,11 +757,13 @@ cudaError_t launch_t(const void *q, const void *k, const void *v, const float *l
 }
 
 struct BwdLayout {
-    size_t base_off, table_off, ops_off, rec_off, total;
+    size_t base_off, table_off, ops_off, rec_off, fwd_off, fwd_bytes, total;
     int64_t max_chunks;
 };
+// The tensor-core forward provides the chunk-start states for bf16 inputs with D = 128.
+bool bwd_uses_tc_forward(int D, kda_dtype dtype) { return D == 128 && dtype == KDA_BF16; }
 // One bound for both modes: B ceil(T / C) chunks without cu_seqlens, at most B T / C + N with it.
-BwdLayout bwd_layout(int B, int T, int H, int D, int num_seqs) {
+BwdLayout bwd_layout(int B, int T, int H, int D, int num_seqs, kda_dtype dtype) {
     auto up = [](size_t x) { return (x + 1023) / 1024 * 1024; };
     BwdLayout l;
     l.max_chunks = ((int64_t)B * T + kC - 1) / kC + num_seqs;
@@ -753,21 +773,24 @@ BwdLayout bwd_layout(int B, int T, int H, int D, int num_seqs) {
     const size_t ops_floats = D == 128 ? BwdOps<128>::floats : BwdOps<64>::floats;
     l.rec_off = up(l.ops_off + (size_t)l.max_chunks * H * ops_floats * sizeof(float));
     const size_t rec_floats = D == 128 ? BwdRec<128>::floats : BwdRec<64>::floats;
-    l.total = l.rec_off + (size_t)l.max_chunks * H * rec_floats * sizeof(float);
+    l.fwd_off = up(l.rec_off + (size_t)l.max_chunks * H * rec_floats * sizeof(float));
+    // the tensor-core forward's own workspace (its chunk table, ready words and records) at the end
+    l.fwd_bytes = bwd_uses_tc_forward(D, dtype) ? prefill_tc_workspace_bytes(B, T, H, num_seqs, true) : 0;
+    l.total = l.fwd_off + l.fwd_bytes;
     return l;
 }
 
 }  // namespace
 
-size_t chunk_bwd_workspace_bytes(int B, int T, int H, int D, int num_seqs) {
-    return bwd_layout(B, T, H, D, num_seqs).total;
+size_t chunk_bwd_workspace_bytes(int B, int T, int H, int D, int num_seqs, kda_dtype dtype) {
+    return bwd_layout(B, T, H, D, num_seqs, dtype).total;
 }
 
 cudaError_t launch_chunk_bwd(const void *q, const void *k, const void *v, const float *la, const float *beta,
                              const float *h0, const int32_t *cu, int num_seqs, int B, int T, int H, int D,
                              kda_dtype dtype, const void *dout, const float *dhT, void *dq, void *dk, void *dv,
                              float *dla, float *dbeta, float *dh0, void *workspace, cudaStream_t stream) {
-    const BwdLayout lay = bwd_layout(B, T, H, D, num_seqs);
+    const BwdLayout lay = bwd_layout(B, T, H, D, num_seqs, dtype);
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     int *status = reinterpret_cast<int *>(ws);
     int *base = reinterpret_cast<int *>(ws + lay.base_off);
@@ -776,17 +799,18 @@ cudaError_t launch_chunk_bwd(const void *q, const void *k, const void *v, const 
     float *recs = reinterpret_cast<float *>(ws + lay.rec_off);
     cudaError_t e = cudaMemsetAsync(ws, 0, 256, stream);
     if (e != cudaSuccess) return e;
+    void *fwd = lay.fwd_bytes ? static_cast<void *>(ws + lay.fwd_off) : nullptr;
     if (dtype == KDA_BF16)
         return D == 128 ? launch_t<128, __nv_bfloat16>(q, k, v, la, beta, h0, cu, num_seqs, B, T, H, dout, dhT, dq, dk,
                                                        dv, dla, dbeta, dh0, status, base, table, ops, recs,
-                                                       lay.max_chunks, stream)
+                                                       lay.max_chunks, fwd, lay.fwd_bytes, stream)
                         : launch_t<64, __nv_bfloat16>(q, k, v, la, beta, h0, cu, num_seqs, B, T, H, dout, dhT, dq, dk,
                                                       dv, dla, dbeta, dh0, status, base, table, ops, recs, lay.max_chunks,
-                                                      stream);
+                                                      nullptr, 0, stream);
     return D == 128 ? launch_t<128, float>(q, k, v, la, beta, h0, cu, num_seqs, B, T, H, dout, dhT, dq, dk, dv, dla,
-                                           dbeta, dh0, status, base, table, ops, recs, lay.max_chunks, stream)
+                                           dbeta, dh0, status, base, table, ops, recs, lay.max_chunks, nullptr, 0, stream)
                     : launch_t<64, float>(q, k, v, la, beta, h0, cu, num_seqs, B, T, H, dout, dhT, dq, dk, dv, dla,
-                                          dbeta, dh0, status, base, table, ops, recs, lay.max_chunks, stream);
+                                          dbeta, dh0, status, base, table, ops, recs, lay.max_chunks, nullptr, 0, stream);
 }
 
 }  // namespace kda

@@ -131,7 +131,7 @@ cudaError_t launch_chunk_table(const int32_t *cu_seqlens, int num_seqs, int T, i
                                int4 *table, cudaStream_t stream);
 
 // CUDA-core chunkwise backward (dk = dv = D in {64, 128}).
-size_t chunk_bwd_workspace_bytes(int B, int T, int H, int D, int num_seqs);
+size_t chunk_bwd_workspace_bytes(int B, int T, int H, int D, int num_seqs, kda_dtype dtype);
 cudaError_t launch_chunk_bwd(const void *q, const void *k, const void *v, const float *la, const float *beta,
                              const float *h0, const int32_t *cu, int num_seqs, int B, int T, int H, int D,
                              kda_dtype dtype, const void *dout, const float *dhT, void *dq, void *dk, void *dv,
@@ -143,10 +143,19 @@ unsigned long long current_context_id();
 // Tensor-core (tcgen05) chunkwise forward: bf16, dk = dv = 128.  With map_out [H, 128, 256] (one
 // sequence, h0 and h_T NULL, o optional) it writes the sequence's affine state map [M | b] instead:
 // b = final state from zero (outputs to o when given), M = final state with v = 0 from the identity.
+// With save.dst set it also writes every chunk's incoming state S (fp32, transposed: S^T[j][c] at
+// dst + (chunk * H + h) * stride + j * 128 + c), chunk = base[n] + i for chunk i of sequence n (n * nc + i
+// without base): the chunk-start states a backward pass needs.
+struct StateSave {
+    float *dst;
+    const int *base;
+    int nc;
+    long long stride;
+};
 size_t prefill_tc_workspace_bytes(int B, int T, int H, int num_seqs, bool varlen);
 cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const float *log_alpha,
                               const float *beta, const float *h0, const int32_t *cu_seqlens,
                               int num_seqs, int B, int T, int H, void *o, float *h_T, void *workspace,
                               size_t workspace_bytes, const Prologue &pro, cudaStream_t stream,
-                              float *map_out = nullptr);
+                              float *map_out = nullptr, const StateSave *save = nullptr);
 }  // namespace kda

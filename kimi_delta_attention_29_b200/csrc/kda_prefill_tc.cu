@@ -777,7 +777,7 @@ kda_tc_state_kernel(const __grid_constant__ CUtensorMap tm_o, const uint8_t *__r
                     const int *__restrict__ flags, const float *__restrict__ h0, const int *__restrict__ base,
                     const int4 *__restrict__ table, const int *__restrict__ order, int num_units, int nc, int T_len,
                     int H, __nv_bfloat16 *__restrict__ o, float *__restrict__ h_T, float *__restrict__ Mb,
-                    int *status, int *unit_counter) {
+                    const StateSave save, int *status, int *unit_counter) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = align1024(smem_raw);
     uint64_t *full = reinterpret_cast<uint64_t *>(sm + ST_BAR);  // [2] record landed in the stage
@@ -951,6 +951,15 @@ kda_tc_state_kernel(const __grid_constant__ CUtensorMap tm_o, const uint8_t *__r
                 arrive(b_d2);
                 return true;
             };
+            // chunk i's incoming S^T row j, channels 32 g .. 32 g + 31 (fp32), for a backward pass
+            auto save_state = [&](int i, const float (&v)[32]) {
+                if (!save.dst) return;
+                const long long ci = (save.base ? (long long)save.base[n] : (long long)n * save.nc) + i;
+                float *p = save.dst + (ci * H + h) * save.stride + (size_t)j * D + 32 * g;
+#pragma unroll
+                for (int x = 0; x < 8; ++x)
+                    *reinterpret_cast<float4 *>(p + 4 * x) = make_float4(v[4 * x], v[4 * x + 1], v[4 * x + 2], v[4 * x + 3]);
+            };
             bool ok = true;
             float sv[32];
 #pragma unroll
@@ -964,6 +973,7 @@ kda_tc_state_kernel(const __grid_constant__ CUtensorMap tm_o, const uint8_t *__r
             } else {
                 store_as(sv);
                 ok = store_d2(gc0, sv);
+                save_state(0, sv);
                 for (int i = 0; i < nchunks && ok; ++i) {
                     const uint32_t gc = gc0 + i, b = gc & 1;
                     // Delta^T -> bf16 operand
@@ -988,6 +998,7 @@ kda_tc_state_kernel(const __grid_constant__ CUtensorMap tm_o, const uint8_t *__r
                     if (i + 1 < nchunks) {
                         store_as(nv);
                         if (!store_d2(gc + 1, nv)) { ok = false; break; }
+                        save_state(i + 1, nv);
                     } else if (hT_col) {
 #pragma unroll
                         for (int kk = 0; kk < 32; ++kk) hT_col[(size_t)(32 * g + kk) * hT_ld] = nv[kk];
@@ -1239,7 +1250,7 @@ size_t prefill_tc_workspace_bytes(int B, int T, int H, int num_seqs, bool varlen
 cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const float *log_alpha,
                               const float *beta, const float *h0, const int32_t *cu_seqlens, int num_seqs,
                               int B, int T, int H, void *o, float *h_T, void *workspace, size_t workspace_bytes,
-                              const Prologue &pro, cudaStream_t stream, float *map_out) {
+                              const Prologue &pro, cudaStream_t stream, float *map_out, const StateSave *save_in) {
     (void)workspace_bytes;
     const TcLayout lay = tc_layout(B, T, H, num_seqs);
     uint8_t *ws = static_cast<uint8_t *>(workspace);
@@ -1275,6 +1286,7 @@ cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const
         (o && (e = encode_token_map(&tm_o, o, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, tokens, H, D, CU_TENSOR_MAP_SWIZZLE_NONE)) != cudaSuccess)))
         return e;
     auto *ob = static_cast<__nv_bfloat16 *>(o);
+    const StateSave save = save_in ? *save_in : StateSave{nullptr, nullptr, 0, 0};
     const bool varlen = cu_seqlens != nullptr;
     // map mode (one sequence): a zero-start unit and an identity-start unit per head
     const int num_units = map_out ? 2 * H : (varlen ? num_seqs : B) * H;
@@ -1297,7 +1309,7 @@ cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const
     if (prep_ctas == 0) {  // no tokens: the state kernel alone writes h_T
         trace_before(kKernTcState, stream);
         kda_tc_state_kernel<<<(unsigned)state_grid, kStateThreads, STATE_SMEM, stream>>>(
-            tm_o, records, flags, h0, bas, tbl, ord, num_units, nc, T, H, ob, h_T, map_out, status, status + 2);
+            tm_o, records, flags, h0, bas, tbl, ord, num_units, nc, T, H, ob, h_T, map_out, save, status, status + 2);
         trace_after(stream);
         return cudaGetLastError();
     }
@@ -1318,7 +1330,7 @@ cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
         trace_before(kKernTcState, stream);
         kda_tc_state_kernel<<<(unsigned)state_grid, kStateThreads, STATE_SMEM, stream>>>(
-            tm_o, records, flags, h0, bas, tbl, ord, num_units, nc, T, H, ob, h_T, map_out, status, status + 2);
+            tm_o, records, flags, h0, bas, tbl, ord, num_units, nc, T, H, ob, h_T, map_out, save, status, status + 2);
         trace_after(stream);
         return cudaGetLastError();
     }
@@ -1333,7 +1345,7 @@ cudaError_t launch_prefill_tc(const void *q, const void *k, const void *v, const
     if ((e = cudaEventRecord(side->fork, stream)) != cudaSuccess) return e;
     if ((e = cudaStreamWaitEvent(side->stream, side->fork, 0)) != cudaSuccess) return e;
     kda_tc_state_kernel<<<(unsigned)state_grid, kStateThreads, STATE_SMEM, side->stream>>>(
-        tm_o, records, flags, h0, bas, tbl, ord, num_units, nc, T, H, ob, h_T, map_out, status, status + 2);
+        tm_o, records, flags, h0, bas, tbl, ord, num_units, nc, T, H, ob, h_T, map_out, save, status, status + 2);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if ((e = cudaEventRecord(side->join, side->stream)) != cudaSuccess) return e;
     prep<<<(unsigned)prep_ctas, kPrepThreads, PREP_SMEM, stream>>>(tm_q, tm_k, tm_v, tm_g, pro, beta, T, H, nc,
