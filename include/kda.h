@@ -289,7 +289,10 @@ KDA_API const char *kda_status_string(int status);
  * (kernel id, milliseconds) into kernel_ids / ms and returns how many kernels were recorded (or
  * KDA_ERR_CUDA).  Kernel ids: 0 varlen chunk table, 1 intra-chunk WY kernel (tensor cores),
  * 2 state-passing kernel (tensor cores), 3 chunkwise kernel (CUDA cores), 4 decode step,
- * 5 multi-token decode.
+ * 5 multi-token decode, 6 output epilogue, 7 backward state pass, 8 backward chunk kernel,
+ * 9 backward chunk operands, 10 segment-map composition, 11 the tensor-core prefill's two kernels
+ * running concurrently (one entry: its events bracket the fork of the side stream and the join;
+ * ids 1 and 2 appear instead when KDA_PREFILL_SERIAL=1 runs them back to back).
  * Process-wide and not thread-safe; events are owned by the library. */
 KDA_API int kda_trace_begin(int max_kernels);
 KDA_API int kda_trace_end(int *kernel_ids, float *ms, int capacity);

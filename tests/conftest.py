@@ -26,15 +26,27 @@ def cuda_device():
 PARITY_RECORDS: list[tuple[str, float, float, float]] = []
 
 
+GRAD_RECORDS: list[tuple[str, dict, float]] = []
+
+
 @pytest.fixture(scope="session")
 def parity_log():
     """Tests call parity_log(label, err_o, err_h, tol) to put an achieved error on record."""
     return lambda label, eo, eh, tol: PARITY_RECORDS.append((label, eo, eh, tol))
 
 
+@pytest.fixture(scope="session")
+def grad_log():
+    """Backward tests call grad_log(label, {gradient: error}, tol) to put achieved errors on record."""
+    return lambda label, errs, tol: GRAD_RECORDS.append((label, dict(errs), tol))
+
+
 def pytest_terminal_summary(terminalreporter, exitstatus, config):
-    if not PARITY_RECORDS:
+    if not PARITY_RECORDS and not GRAD_RECORDS:
         return
     terminalreporter.section("achieved parity (max |gpu - oracle| / max |oracle|)")
     for label, eo, eh, tol in PARITY_RECORDS:
         terminalreporter.write_line(f"{label}: o {eo:.3e}  h_T {eh:.3e}  (tolerance {tol:.0e})")
+    for label, errs, tol in GRAD_RECORDS:
+        body = "  ".join(f"{k} {v:.2e}" for k, v in errs.items())
+        terminalreporter.write_line(f"{label}: {body}  (tolerance {tol:.0e})")

@@ -41,6 +41,7 @@ def oracle_grads(x, do, dhT):
 
 
 def check(got, ref, tol, names=NAMES):
+    errs = {}
     for name in names:
         r = ref[name]
         den = float(np.abs(r).max())
@@ -48,6 +49,8 @@ def check(got, ref, tol, names=NAMES):
         err = float(np.abs(np64(got[name]) - r).max() / den)
         assert np.isfinite(np64(got[name])).all(), name
         assert err <= tol, f"{name}: {err:.3e} > {tol:.1e}"
+        errs[name] = err
+    return errs
 
 
 def run(x, do, dhT):
@@ -58,12 +61,13 @@ def run(x, do, dhT):
 @pytest.mark.parametrize("dtype,d,T", [(torch.bfloat16, 128, 200), (torch.bfloat16, 128, 64),
                                        (torch.float32, 64, 130), (torch.float32, 128, 97),
                                        (torch.bfloat16, 64, 1)])
-def test_backward_matches_oracle(cuda_device, dtype, d, T):
+def test_backward_matches_oracle(cuda_device, grad_log, dtype, d, T):
     x = gen.make_prefill(2, T, 2, d, d, dtype, gate_shift=1.0, h0_std=0.2, seed=50 + T, device=cuda_device)
     do, dhT = upstream(x, 2, cuda_device, seed=T)
     got = run(x, do, dhT)
     torch.cuda.synchronize(cuda_device)
-    check(got, oracle_grads(x, do, dhT), TOL[dtype])
+    errs = check(got, oracle_grads(x, do, dhT), TOL[dtype])
+    grad_log(f"backward {'bf16' if dtype == torch.bfloat16 else 'fp32'} d={d} B=2 H=2 T={T}", errs, TOL[dtype])
 
 
 def test_backward_no_h0_no_dhT(cuda_device):
@@ -124,11 +128,12 @@ def test_backward_empty(cuda_device):
     assert torch.equal(got["dh0"], dhT)
 
 
-def test_backward_train_shape_heads(cuda_device):
+def test_backward_train_shape_heads(cuda_device, grad_log):
     """The training workload's sequence length (T = 4096, d = 128, bf16), two heads, full comparison."""
     x = gen.make_prefill(1, 4096, 2, 128, 128, torch.bfloat16, gate_shift=2.0, h0_std=0.0, seed=66,
                          device=cuda_device)
     do, dhT = upstream(x, 1, cuda_device, seed=9)
     got = run(x, do, dhT)
     torch.cuda.synchronize(cuda_device)
-    check(got, oracle_grads(x, do, dhT), TOL[torch.bfloat16])
+    errs = check(got, oracle_grads(x, do, dhT), TOL[torch.bfloat16])
+    grad_log("backward bf16 d=128 T=4096 (training length, 2 heads)", errs, TOL[torch.bfloat16])
