@@ -497,24 +497,19 @@ kda_tc_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     const float2 eE = ex2v(make_float2(Eown.x + kSplitBias, Eown.y + kSplitBias));
     const float2 eGL = ex2v(make_float2(gl.x - Eown.x + kSplitBias, gl.y - Eown.y + kSplitBias));
 
-    // ---- operands: X, R^(b) for b >= own block, K o 2^G (smem); Q o 2^G and K o 2^{G63-G} (record).
+    // ---- operands: X, R^(b) for b >= own block (smem) first; then, while the Gram products run,
+    // K o 2^G (smem) and Q o 2^G, K o 2^{G63-G} (record), their factors formed again from G.
     // The factors are rounded to bf16 and applied with packed bf16 multiplies on the bf16 inputs.
 #pragma unroll
-    for (int m = 0; m < 16; ++m) {
+    for (int m = 0; m < 16; ++m) {  // pass 1: the Gram operands X and R^(b)
         const int r = 16 * qr + m;
         const float2 F = ex2v(sub2(g[m], Eown));
         const float2 Rf = ex2v(sub2(Eown, g[m]));
-        const float2 Fs = make_float2(F.x * kSplitDown, F.y * kSplitDown);
         const float2 Rs = make_float2(Rf.x * kSplitDown, Rf.y * kSplitDown);
         const __nv_bfloat162 k2 = as_bf2(kk[m]), q2 = as_bf2(qq[m]);
         const __nv_bfloat162 fx = bf2_of(F);
-        const __nv_bfloat162 fe = bf2_of(make_float2(Fs.x * eE.x, Fs.y * eE.y));
-        const __nv_bfloat162 frg = bf2_of(make_float2(Rs.x * eGL.x, Rs.y * eGL.y));
         st_bf2(X + sw128_off(32 * qr + m, c0, 128), __hmul2(k2, fx));
         st_bf2(X + sw128_off(32 * qr + 16 + m, c0, 128), __hmul2(q2, fx));
-        st_bf2(KT + sw128_off(r, c0, 64), __hmul2(k2, fe));
-        st_bf2(rec + REC_AQ + sw128_off(64 + r, c0, 128), __hmul2(q2, fe));
-        st_bf2(rec + REC_KH + sw128_off(r, c0, 64), __hmul2(k2, frg));
 #pragma unroll
         for (int b = 0; b < 4; ++b)
             if (b >= qr)
@@ -537,6 +532,21 @@ kda_tc_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         }
         mma_commit(mbar + 1);
     }
+#pragma unroll
+    for (int m = 0; m < 16; ++m) {  // pass 2, while the Gram products run: K o 2^G, Q o 2^G, K o 2^{G63-G}
+        const int r = 16 * qr + m;
+        const float2 F = ex2v(sub2(g[m], Eown));
+        const float2 Rf = ex2v(sub2(Eown, g[m]));
+        const float2 Fs = make_float2(F.x * kSplitDown, F.y * kSplitDown);
+        const float2 Rs = make_float2(Rf.x * kSplitDown, Rf.y * kSplitDown);
+        const __nv_bfloat162 k2 = as_bf2(kk[m]), q2 = as_bf2(qq[m]);
+        const __nv_bfloat162 fe = bf2_of(make_float2(Fs.x * eE.x, Fs.y * eE.y));
+        const __nv_bfloat162 frg = bf2_of(make_float2(Rs.x * eGL.x, Rs.y * eGL.y));
+        st_bf2(KT + sw128_off(r, c0, 64), __hmul2(k2, fe));
+        st_bf2(rec + REC_AQ + sw128_off(64 + r, c0, 128), __hmul2(q2, fe));
+        st_bf2(rec + REC_KH + sw128_off(r, c0, 64), __hmul2(k2, frg));
+    }
+    fence_async_smem();
     if (tid < D) reinterpret_cast<float *>(rec + REC_GL)[tid] = ex2(s_gl[tid]);
     bool ok = mbar_wait(mbar + 1, 0) && in_ok;
     ok = __syncthreads_and(ok);
@@ -737,7 +747,8 @@ kda_tc_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
 //   D1[2]  per chunk parity: preloaded with [U^T | 0]; P1 adds S^T [-W; Q~]^T -> [Delta^T | (Q~ S)^T]
 //          and P2b adds Delta^T P^T to the second half -> O^T
 // Per chunk:
-//   P1:  D1 += A_S [-W; Q~]^T       (M=128, N=128, K=128) onto [U^T | 0] = [Delta^T | (Q~ S)^T]
+//   P1:  D1 += A_S [-W; Q~]^T       (M=128, K=128) onto [U^T | 0] = [Delta^T | (Q~ S)^T], as two N=64
+//        halves: the -W half first and committed on its own, so the chain waits only for Delta
 //   P2a: D2 += A_D K^               (M=128, N=128, K=64)  = S_next^T = S^T Diag(e^{G_63}) + Delta^T K^
 //   P2b: D1[:, 64:] += A_D P^T      (M=128, N=64,  K=64)  = O^T = (Q~ S + P Delta)^T
 // Warps:
@@ -882,7 +893,7 @@ kda_tc_state_kernel(const __grid_constant__ CUtensorMap tm_o, const uint8_t *__r
         } else if (warp == kMmaWarp) {
             // ------------------------------------------------ MMA issue (one thread)
             if (lane == 0) {
-                const uint32_t id_p1 = idesc_bf16_f32(128, 128, 0, 0);
+                const uint32_t id_p1h = idesc_bf16_f32(128, 64, 0, 0);
                 const uint32_t id_p2a = idesc_bf16_f32(128, 128, 0, 1);
                 const uint32_t id_p2b = idesc_bf16_f32(128, 64, 0, 1);
                 // operand descriptors of stage 0; stage 1 is REC_BYTES / 16 further in the start field
@@ -906,9 +917,12 @@ kda_tc_state_kernel(const __grid_constant__ CUtensorMap tm_o, const uint8_t *__r
                     if (!ok) { *s_abort = 1; break; }
                     tc_fence_after();
 #pragma unroll
-                    for (int ks = 0; ks < 8; ++ks)  // [-W; Q~] as one N=128 product onto [U^T | 0]
-                        mma_bf16_ts(d1, tmem + TM_AS + 8 * ks, dw[ks] + so, id_p1, 1);
+                    for (int ks = 0; ks < 8; ++ks)  // -W S first: the chain waits only for Delta
+                        mma_bf16_ts(d1, tmem + TM_AS + 8 * ks, dw[ks] + so, id_p1h, 1);
                     mma_commit(b_p1);
+#pragma unroll
+                    for (int ks = 0; ks < 8; ++ks)  // then Q~ S, rows 64.. of the operand
+                        mma_bf16_ts(d1 + 64, tmem + TM_AS + 8 * ks, dw[ks] + so + (8192 >> 4), id_p1h, 1);
                     ok = mbar_wait_or_abort(b_dr, gc & 1, s_abort) && mbar_wait_or_abort(b_d2, gc & 1, s_abort);
                     if (!ok) { *s_abort = 1; break; }
                     tc_fence_after();
