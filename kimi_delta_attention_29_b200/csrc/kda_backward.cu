@@ -204,10 +204,13 @@ kda_bwd_prep_kernel(const T *__restrict__ q, const T *__restrict__ k, const floa
     for (int c = tid; c < D; c += kBT) rec[O::eGL + c] = ex2f(gl[c]);
 }
 
+// The operand tiles' rows are padded by 4 floats: 16-byte aligned, so they are staged with 16-byte
+// copies, and rows r, r + 1 start 4 banks apart (the loops below read at most two rows per warp).
 template <int D>
 struct StateSmem {
-    static constexpr int DKP = D + 1;
-    static constexpr size_t floats = 2 * (size_t)kC * CP     // sT, sP
+    static constexpr int DKP = D + 4;
+    static constexpr int CPS = kC + 4;
+    static constexpr size_t floats = 2 * (size_t)kC * CPS    // sT, sP
                                      + 3 * (size_t)kC * DKP  // sKt, sKh, sQt
                                      + 6 * (size_t)kC * kNV  // Vs, dOs, X1, Dl, dDl, Zs
                                      + 3 * (size_t)D * kSP   // Ss, dSs, dSn
@@ -223,7 +226,7 @@ kda_bwd_state_kernel(const T *__restrict__ v, const float *__restrict__ beta, co
                      const float *__restrict__ ops, float *__restrict__ recs, T *__restrict__ dv_out,
                      float *__restrict__ dh0, int *status, bool have_states) {
     using SM = StateSmem<D>;
-    constexpr int DKP = SM::DKP;
+    constexpr int DKP = SM::DKP, CP = SM::CPS;
     using R = BwdRec<D>;
     using O = BwdOps<D>;
     extern __shared__ float smem[];
@@ -266,16 +269,16 @@ kda_bwd_state_kernel(const T *__restrict__ v, const float *__restrict__ beta, co
 
     // the chunk's operands (from the prep kernel) and V / dO slices; ends with a barrier
     auto stage = [&](const float *op, int64_t t0, int L, bool bwd) {
-        for (int p = tid; p < kC * kC; p += kBTs) {  // operand tiles by cp.async: all in flight at once
-            const int r = p / kC, i = p % kC;
-            cp_async4(sT + r * CP + i, op + O::Tm + p);
-            if (bwd) cp_async4(sP + r * CP + i, op + O::Pm + p);
+        for (int p = tid; p < kC * kC / 4; p += kBTs) {  // operand tiles by 16-byte cp.async, all in flight
+            const int r = p / (kC / 4), i = 4 * (p % (kC / 4));
+            cp_async16(sT + r * CP + i, op + O::Tm + r * kC + i);
+            if (bwd) cp_async16(sP + r * CP + i, op + O::Pm + r * kC + i);
         }
-        for (int idx = tid; idx < kC * D; idx += kBTs) {
-            const int r = idx / D, c = idx % D;
-            cp_async4(sKt + r * DKP + c, op + O::Kt + idx);
-            cp_async4(sKh + r * DKP + c, op + O::Kh + idx);
-            if (bwd) cp_async4(sQt + r * DKP + c, op + O::Qt + idx);
+        for (int idx = tid; idx < kC * D / 4; idx += kBTs) {
+            const int r = idx / (D / 4), c = 4 * (idx % (D / 4));
+            cp_async16(sKt + r * DKP + c, op + O::Kt + r * D + c);
+            cp_async16(sKh + r * DKP + c, op + O::Kh + r * D + c);
+            if (bwd) cp_async16(sQt + r * DKP + c, op + O::Qt + r * D + c);
         }
         for (int c = tid; c < D; c += kBTs) cp_async4(egl + c, op + O::eGL + c);
         cp_async_commit();
@@ -494,13 +497,13 @@ kda_bwd_chunk_kernel(const T *__restrict__ q, const T *__restrict__ k, const flo
         Gb[r * kCBP + cc] = lv;
     }
     // ---- phase 1 staging: dDelta [C][D], X1^T [D][C], Z [C][D], S^T block [D][kCB]
-    for (int idx = tid; idx < kC * D; idx += kBT2) {
-        cp_async4(U0 + idx, rec + R::dD + idx);
-        cp_async4(U1 + idx, rec + R::X1t + idx);
-        cp_async4(U2 + idx, rec + R::Z + idx);
+    for (int idx = 4 * tid; idx < kC * D; idx += 4 * kBT2) {  // 16-byte pieces of contiguous tiles
+        cp_async16(U0 + idx, rec + R::dD + idx);
+        cp_async16(U1 + idx, rec + R::X1t + idx);
+        cp_async16(U2 + idx, rec + R::Z + idx);
     }
-    for (int idx = tid; idx < D * kCB; idx += kBT2)
-        cp_async4(Ub + idx, rec + R::St + (size_t)(idx / kCB) * D + cb * kCB + idx % kCB);
+    for (int idx = 4 * tid; idx < D * kCB; idx += 4 * kBT2)
+        cp_async16(Ub + idx, rec + R::St + (size_t)(idx / kCB) * D + cb * kCB + idx % kCB);
     cp_async_commit();
     cp_async_wait<0>();
     __syncthreads();
