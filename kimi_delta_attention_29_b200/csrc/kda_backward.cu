@@ -554,9 +554,9 @@ kda_bwd_chunk_kernel(const T *__restrict__ q, const T *__restrict__ k, const flo
     for (int m = 0; m < kRowsPerWarp; ++m) dKt[m] *= -bt[warp + m * (kBT2 / 32)];
     __syncthreads();
     // ---- phase 2 staging: dO [C][D], Delta^T [D][C], dS'^T block [D][kCB] (S^T block stays)
-    for (int idx = tid; idx < kC * D; idx += kBT2) cp_async4(U1 + idx, rec + R::Dt + idx);
-    for (int idx = tid; idx < D * kCB; idx += kBT2)
-        cp_async4(U2 + idx, rec + R::dSt + (size_t)(idx / kCB) * D + cb * kCB + idx % kCB);
+    for (int idx = 4 * tid; idx < kC * D; idx += 4 * kBT2) cp_async16(U1 + idx, rec + R::Dt + idx);
+    for (int idx = 4 * tid; idx < D * kCB; idx += 4 * kBT2)
+        cp_async16(U2 + idx, rec + R::dSt + (size_t)(idx / kCB) * D + cb * kCB + idx % kCB);
     cp_async_commit();
     for (int idx = tid; idx < kC * D; idx += kBT2) {
         const int r = idx / D, j = idx % D;

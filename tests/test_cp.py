@@ -178,3 +178,33 @@ def test_segment_map_one_pass(cuda_device, T, want_o, gate_shift):
     assert rel(f(Mb[:, :, d:]), f(b2[0])) <= 2e-2
     if check_m:
         assert rel(f(Mb[:, :, :d]), f(M2[0])) <= 2e-2
+
+
+@pytest.mark.gpu
+def test_segment_map_full_segment_sampled(cuda_device, parity_log):
+    """The map of one eighth of the long-context sequence (T = 16,384, H = 32, d = 128), the segment
+    one of eight ranks holds: every head on the GPU, four heads against the oracle (b, M and o0).
+    Over 16,384 tokens the delta rule's own contraction takes M below 1e-40 even with weak decay
+    (gate shift -6), under fp32's normal range: M is compared on the scale of the identity it starts
+    from (what an error in M does to an incoming state of that scale), b and o0 relative to their
+    own maximum."""
+    import oracle
+    import kimi_delta_attention_29_b200 as kda
+    from kimi_delta_attention_29_b200 import inputs as gen
+    T, H, d = 16384, 32, 128
+    x = gen.make_prefill(1, T, H, d, d, torch.bfloat16, gate_shift=-6.0, seed=95, device=cuda_device)
+    o0, Mb = kda.kda_segment_map(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"])
+    torch.cuda.synchronize(cuda_device)
+    heads = [0, 9, 22, 31]
+    f = lambda a: a.detach().float().cpu().numpy().astype(np.float64)
+    sub = {n: f(x[n][:, :, heads]) for n in ("q", "k", "v", "log_alpha", "beta")}
+    o_ref, b_ref = oracle.recurrent(sub["q"], sub["k"], sub["v"], sub["log_alpha"], sub["beta"], None)
+    eye = np.broadcast_to(np.eye(d), (1, len(heads), d, d)).copy()
+    _, M_ref = oracle.recurrent(sub["q"], sub["k"], np.zeros_like(sub["v"]), sub["log_alpha"], sub["beta"], eye)
+    rel = lambda a, b: float(np.abs(a - b).max() / np.abs(b).max())
+    Mb_s = f(Mb[heads])
+    e_o, e_b = rel(f(o0[:, :, heads]), o_ref), rel(Mb_s[:, :, d:], b_ref[0])
+    e_m = float(np.abs(Mb_s[:, :, :d] - M_ref[0]).max() / max(np.abs(M_ref).max(), 1.0))
+    parity_log("segment map T=16384 H=32 (4 heads; h_T column: b)", e_o, e_b, 2e-2)
+    assert e_o <= 2e-2 and e_b <= 2e-2 and e_m <= 2e-2, (e_o, e_b, e_m)
+    assert torch.isfinite(Mb).all()
