@@ -117,11 +117,35 @@ kda_decode_kernel(const T *__restrict__ q, const T *__restrict__ k, const T *__r
 // Tq tokens per state, the state kept in registers between them: read once from slot_in, written
 // once to slot_out.  The columns of S evolve independently (each column j only meets u_j and the
 // sums over the rows of column j), so warp w owns columns 16 w .. 16 w + 15 for every token and
-// never waits for another warp: lane (rg, cg) = (lane >> 2, lane & 3) holds rows rg + 8 r (r < D/8)
-// of columns 16 w + 4 cg .. + 3, the row sums S^T k and S^T q of a token are warp shuffles over the
+// never waits for another warp: lane (rg, cg) = (lane >> 2, lane & 3) holds the D/8 consecutive
+// rows D/8 rg .. of columns 16 w + 4 cg .. + 3 (so a token's k, q and alpha for those rows are a few
+// 16-byte shared loads), the row sums S^T k and S^T q of a token are warp shuffles over the
 // 8 row groups, and u is handed back to the row groups by shuffles too.  The token data (q, k, v,
 // log_alpha, beta) is staged in shared memory with cp.async, kTokBatch tokens at a time (half for
 // fp32) and double-buffered; the CTA meets at a barrier once per batch, not per token.
+// N consecutive elements (16-byte aligned) of a staged row into fp32 registers with 16-byte loads.
+template <int N>
+__device__ __forceinline__ void ld_rows(const float *p, float (&o)[N]) {
+#pragma unroll
+    for (int x = 0; x < N / 4; ++x) {
+        const float4 v = reinterpret_cast<const float4 *>(p)[x];
+        o[4 * x] = v.x; o[4 * x + 1] = v.y; o[4 * x + 2] = v.z; o[4 * x + 3] = v.w;
+    }
+}
+template <int N>
+__device__ __forceinline__ void ld_rows(const __nv_bfloat16 *p, float (&o)[N]) {
+#pragma unroll
+    for (int x = 0; x < N / 8; ++x) {
+        const uint4 v = reinterpret_cast<const uint4 *>(p)[x];
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {  // bf16 -> fp32 is exact: the bf16 bits are the high half
+            o[8 * x + 2 * e] = __uint_as_float(w[e] << 16);
+            o[8 * x + 2 * e + 1] = __uint_as_float(w[e] & 0xFFFF0000u);
+        }
+    }
+}
+
 constexpr int kMultiWarps = 8;
 constexpr int kTokBatch = 8;
 __device__ __forceinline__ float to_f(float x) { return x; }
@@ -137,7 +161,7 @@ kda_decode_multi_kernel(const T *__restrict__ q, const T *__restrict__ k, const 
                         float *__restrict__ S_pool, int num_slots, const int32_t *__restrict__ slot_in,
                         const int32_t *__restrict__ slot_out, int Tq, int H, T *__restrict__ o,
                         int *__restrict__ status, const Prologue pro) {
-    constexpr int RPL = D / 8;                   // rows per lane: rg + 8 r
+    constexpr int RPL = D / 8;                   // rows per lane: RPL rg + r
     constexpr int CPW = D / kMultiWarps;         // columns per warp
     constexpr int CPL = CPW / 4;                 // columns per lane (4 for D = 128, 2 for D = 64)
     constexpr int VEC = D / 32;                  // prologue: elements of a q / k row per lane
@@ -188,10 +212,11 @@ kda_decode_multi_kernel(const T *__restrict__ q, const T *__restrict__ k, const 
     const int col0 = CPW * warp + CPL * cg;  // this lane's first column
     constexpr int CP2 = CPL / 2;  // column pairs per lane: the state math runs on packed fp32 pairs
     float2 s[RPL][CP2];
+    const int row0 = RPL * rg;
 #pragma unroll
     for (int r = 0; r < RPL; ++r) {
         float x[CPL];
-        VecIO<CPL>::load(Sin + (size_t)(rg + 8 * r) * D + col0, x);
+        VecIO<CPL>::load(Sin + (size_t)(row0 + r) * D + col0, x);
 #pragma unroll
         for (int c = 0; c < CP2; ++c) s[r][c] = make_float2(x[2 * c], x[2 * c + 1]);
     }
@@ -242,17 +267,16 @@ kda_decode_multi_kernel(const T *__restrict__ q, const T *__restrict__ k, const 
         for (int tt = 0; tt < nt; ++tt) {
             // decay, then this lane's partial row sums of S^T k, S^T q (its CPL columns) and k . q
             float2 pa[CP2], pb[CP2];
-            float kr[RPL];
+            float kr[RPL], qr[RPL], ar[RPL];  // this lane's rows of k, q and alpha (the hardware exp2, applied above)
+            ld_rows<RPL>(&sk[buf][tt][row0], kr);
+            ld_rows<RPL>(&sq[buf][tt][row0], qr);
+            ld_rows<RPL>(&sla[buf][tt][row0], ar);
 #pragma unroll
             for (int c = 0; c < CP2; ++c) pa[c] = pb[c] = make_float2(0.f, 0.f);
             float pqk = 0.f;
 #pragma unroll
             for (int r = 0; r < RPL; ++r) {
-                const int i = rg + 8 * r;
-                const float ki = to_f(sk[buf][tt][i]);
-                const float qi = to_f(sq[buf][tt][i]);
-                const float ai = sla[buf][tt][i];  // alpha_i (the hardware exp2, applied above)
-                kr[r] = ki;
+                const float ki = kr[r], qi = qr[r], ai = ar[r];
                 pqk = fmaf(qi, ki, pqk);
                 const float2 a2 = make_float2(ai, ai), k2 = make_float2(ki, ki), q2 = make_float2(qi, qi);
 #pragma unroll
@@ -305,7 +329,7 @@ kda_decode_multi_kernel(const T *__restrict__ q, const T *__restrict__ k, const 
             x[2 * c] = s[r][c].x;
             x[2 * c + 1] = s[r][c].y;
         }
-        VecIO<CPL>::store(Sout + (size_t)(rg + 8 * r) * D + col0, x);
+        VecIO<CPL>::store(Sout + (size_t)(row0 + r) * D + col0, x);
     }
 }
 

@@ -96,3 +96,20 @@ def test_noalloc_varlen_matches_workspace_entry_point(cuda_device):
     assert torch.isfinite(o.float()).all() and torch.isfinite(hT).all()
     assert _rel(o, o_ref) <= TOL
     assert _rel(hT, h_ref) <= TOL
+
+
+def test_noalloc_repeat_call_allocates_nothing(cuda_device):
+    """After the first call on the device (which loads the library's device code and scratch), a call
+    leaves the device's free memory exactly where it was: nothing is allocated, not even by CUDA."""
+    fn = _noalloc_fn()
+    stream = torch.cuda.current_stream(cuda_device)
+    x = gen.make_prefill(1, 640, 8, 128, 128, torch.bfloat16, gate_shift=2.0, h0_std=0.1, seed=25, device=cuda_device)
+    o = torch.empty_like(x["v"])
+    hT = torch.empty(1, 8, 128, 128, device=cuda_device)
+    assert _call_noalloc(fn, x, o, hT, stream) == _lib.KDA_OK  # first call of this test (others ran before)
+    torch.cuda.synchronize(cuda_device)
+    free0 = torch.cuda.mem_get_info(cuda_device)[0]
+    for _ in range(3):
+        assert _call_noalloc(fn, x, o, hT, stream) == _lib.KDA_OK
+    torch.cuda.synchronize(cuda_device)
+    assert torch.cuda.mem_get_info(cuda_device)[0] == free0
