@@ -286,31 +286,52 @@ kda_decode_multi_kernel(const T *__restrict__ q, const T *__restrict__ k, const 
                     pb[c] = __ffma2_rn(s[r][c], q2, pb[c]);
                 }
             }
-            // sums over the 8 row groups (lane bits 2..4): each lane ends with the totals of every
-            // one of its columns
+            // Sums over the 8 row groups (lane bits 2..4), halving at each level: the 2 CPL partial
+            // sums [S^T k of the CPL columns | S^T q of them] are split between the two partner lanes,
+            // each keeping one half, so after the levels a lane holds one total, number li; k . q by a
+            // plain butterfly.
+            constexpr int NV = 2 * CPL;
+            float cur[NV];
 #pragma unroll
-            for (int off = 4; off < 32; off <<= 1) {
+            for (int c = 0; c < CP2; ++c) {
+                cur[2 * c] = pa[c].x; cur[2 * c + 1] = pa[c].y;
+                cur[CPL + 2 * c] = pb[c].x; cur[CPL + 2 * c + 1] = pb[c].y;
+            }
+            int li = 0;
 #pragma unroll
-                for (int c = 0; c < CP2; ++c) {
-                    pa[c].x += __shfl_xor_sync(0xffffffffu, pa[c].x, off);
-                    pa[c].y += __shfl_xor_sync(0xffffffffu, pa[c].y, off);
-                    pb[c].x += __shfl_xor_sync(0xffffffffu, pb[c].x, off);
-                    pb[c].y += __shfl_xor_sync(0xffffffffu, pb[c].y, off);
+            for (int lvl = 0, half = NV / 2; lvl < 3; ++lvl, half /= 2) {
+                const int off = 4 << lvl;
+                const bool upper = (lane & off) != 0;
+                if (half >= 1) {
+#pragma unroll
+                    for (int j = 0; j < (half >= 1 ? half : 1); ++j) {
+                        const float keep = upper ? cur[half + j] : cur[j];
+                        const float send = upper ? cur[j] : cur[half + j];
+                        cur[j] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+                    }
+                    li += upper ? half : 0;
+                } else {
+                    cur[0] += __shfl_xor_sync(0xffffffffu, cur[0], off);
                 }
                 pqk += __shfl_xor_sync(0xffffffffu, pqk, off);
             }
-            // u_j = beta (v_j - (S'^T k)_j); o_j = (S'^T q)_j + (k . q) u_j, with S' the decayed state
+            // u_j = beta (v_j - (S'^T k)_j) in the lanes holding an S^T k total (lane bit 2 clear);
+            // o_j = (S'^T q)_j + (k . q) u_j in their partners (bit 2 set, the same column)
+            const int cc = li % CPL;
             const float bt = sb[buf][tt];
+            const float u_here = bt * (to_f(sv[buf][tt][col0 + cc]) - cur[0]);
+            const float u_pair = __shfl_xor_sync(0xffffffffu, u_here, 4);
+            if (li >= CPL && (CPL == 4 || (lane & 16) == 0))  // one writer per column
+                Elem<T>::store(o + tok_of(t0 + tt) * D + col0 + cc, fmaf(pqk, u_pair, cur[0]));
+            // every lane needs u of its CPL columns: column c's total sits in row group rg(c)
             float2 uu[CP2];
 #pragma unroll
             for (int c = 0; c < CP2; ++c) {
-                uu[c] = make_float2(bt * (to_f(sv[buf][tt][col0 + 2 * c]) - pa[c].x),
-                                    bt * (to_f(sv[buf][tt][col0 + 2 * c + 1]) - pa[c].y));
-                if (rg == 0) {  // row group 0 writes the warp's columns of o
-                    T *orow = o + tok_of(t0 + tt) * D + col0 + 2 * c;
-                    Elem<T>::store(orow, fmaf(pqk, uu[c].x, pb[c].x));
-                    Elem<T>::store(orow + 1, fmaf(pqk, uu[c].y, pb[c].y));
-                }
+                const int c0i = 2 * c, c1i = 2 * c + 1;
+                const int rg0 = CPL == 4 ? 2 * (c0i >> 1) + 4 * (c0i & 1) : 2 * c0i;
+                const int rg1 = CPL == 4 ? 2 * (c1i >> 1) + 4 * (c1i & 1) : 2 * c1i;
+                uu[c] = make_float2(__shfl_sync(0xffffffffu, u_here, 4 * rg0 + cg),
+                                    __shfl_sync(0xffffffffu, u_here, 4 * rg1 + cg));
             }
 #pragma unroll
             for (int r = 0; r < RPL; ++r) {
