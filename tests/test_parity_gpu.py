@@ -283,6 +283,18 @@ def test_train_shape_sampled(cuda_device, parity_log):
                    label="training shape B=4 H=16 T=4096 (6 heads x 16 columns)", log=parity_log)
 
 
+def test_train_shape_full(cuda_device, parity_log):
+    """B=4, H=16, T=4096, d=128, bf16: every output element and every final state against the
+    oracle (4 x 16 units, all 128 value columns; about a second of oracle time on 16 threads)."""
+    x = gen.make_prefill_for(gen.TRAIN, seed=1, device=cuda_device)
+    o, hT = run_fwd(x)
+    torch.cuda.synchronize()
+    o_ref, h_ref = oracle_fwd(x)
+    eo, eh = rel_err(o, o_ref), rel_err(hT, h_ref)
+    parity_log("training shape B=4 H=16 T=4096, every element (all 64 units x 128 columns)", eo, eh, 2e-2)
+    assert eo <= 2e-2 and eh <= 2e-2, (eo, eh)
+
+
 def test_long_context_sampled(cuda_device, parity_log):
     """B=1, H=32, T=131072, d=128, bf16, h0 ~ N(0, 0.02): the prefill the benchmark times."""
     x = gen.make_prefill_for(gen.LONG, seed=0, device=cuda_device)
