@@ -608,9 +608,10 @@ def backward_bench(args, dev, stream, barrier, max_over_ranks, world):
 
 
 def cp_bench(x, dev, stream, single_ms):
-    """Context parallelism on the long-context sequence: the work ONE rank does for R segments (two
-    passes for its map [M | b], the composition of R maps, one pass from its incoming state), timed on
-    this GPU for the last segment.  The all-gather between GPUs is not part of it."""
+    """Context parallelism on the long-context sequence: the work ONE rank does for R segments (its map
+    [M | b] in one pass, the composition of R maps, one pass from its incoming state), timed on this GPU
+    for the last segment, with the time of each of the three steps.  The all-gather between GPUs is not
+    part of it."""
     import torch
     import kimi_delta_attention_29_b200 as kda
     from kimi_delta_attention_29_b200 import cp
@@ -620,24 +621,41 @@ def cp_bench(x, dev, stream, single_ms):
         a, e = T - T // R, T
         part = [x[n][:, a:e].contiguous() for n in ("q", "k", "v", "log_alpha", "beta")]
         Mb_all = torch.zeros(R, x["q"].shape[2], 128, 256, device=dev)
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        split = [0.0, 0.0, 0.0]
 
-        def rank_work():
-            _, Mb = cp.segment_map(*part, stream=stream)
+        def rank_work(timed):
+            if timed:
+                ev[0].record(stream)
+            _, Mb = cp.segment_map(*part, stream=stream, want_o=False)  # a rank > 0 keeps no map-pass outputs
             Mb_all[R - 1].copy_(Mb)
+            if timed:
+                ev[1].record(stream)
             S_in, _ = kda.kda_state_compose(Mb_all, None, stream=stream)
-            return cp.segment_from(*part, S_in[R - 1], stream=stream)
+            if timed:
+                ev[2].record(stream)
+            o = cp.segment_from(*part, S_in[R - 1], stream=stream)
+            if timed:
+                ev[3].record(stream)
+                torch.cuda.synchronize(dev)
+                for i in range(3):
+                    split[i] += ev[i].elapsed_time(ev[i + 1])
+            return o
 
-        rank_work()
+        rank_work(False)
         torch.cuda.synchronize(dev)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         for _ in range(3):
-            rank_work()
+            rank_work(False)
         e1.record(stream)
         torch.cuda.synchronize(dev)
         ms = e0.elapsed_time(e1) / 3
+        for _ in range(3):
+            rank_work(True)
         rows.append({"R": R, "segment_tokens": e - a, "rank_ms": ms, "single_gpu_ms": single_ms,
-                     "rank_over_single": ms / single_ms})
+                     "rank_over_single": ms / single_ms, "map_pass_ms": split[0] / 3, "compose_ms": split[1] / 3,
+                     "rerun_ms": split[2] / 3})
     return {"workload": "long_B1_H32_T131072_d128 split into R segments", "per_rank": rows,
             "exchange": "all-gather of [M | b] (32 x 128 x 256 fp32 = 4 MiB per rank) not measured: one GPU"}
 
