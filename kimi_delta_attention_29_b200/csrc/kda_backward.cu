@@ -41,7 +41,7 @@ namespace kda {
 namespace {
 
 constexpr int kC = kChunk;
-constexpr int kBT = 256;   // threads per CTA of the prep kernel
+constexpr int kBT = 512;   // threads per CTA of the prep kernel (one CTA per SM: shared memory)
 constexpr int kBTs = 512;  // threads per CTA of the state pass
 constexpr int kNV = 16;    // value columns per state-pass CTA
 constexpr int kSP = kNV + 1;  // padded row stride of the [D][kNV] state tiles
@@ -102,13 +102,17 @@ __device__ __forceinline__ void decayed_grams(const float *Kc, const float *Qc, 
     for (int p = threadIdx.x; p < kC * kC; p += kBT) {
         const int r = p / kC, i = p % kC;
         float sa = 0.f, sp = 0.f;
-        if (i <= r) {
+        if (i <= r) {  // four partial sums per product, so consecutive channels do not wait on each other
             const float *gr = Gc + r * DKP, *gi = Gc + i * DKP;
+            float pa[4] = {0.f, 0.f, 0.f, 0.f}, pp[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
             for (int c = 0; c < D; ++c) {
                 const float kd = Kc[i * DKP + c] * ex2f(gr[c] - gi[c]);
-                sa = fmaf(Kc[r * DKP + c], kd, sa);
-                if (Pm) sp = fmaf(Qc[r * DKP + c], kd, sp);
+                pa[c & 3] = fmaf(Kc[r * DKP + c], kd, pa[c & 3]);
+                if (Pm) pp[c & 3] = fmaf(Qc[r * DKP + c], kd, pp[c & 3]);
             }
+            sa = (pa[0] + pa[1]) + (pa[2] + pa[3]);
+            sp = (pp[0] + pp[1]) + (pp[2] + pp[3]);
         }
         Am[r * CP + i] = i < r ? (scale_beta ? bt[r] * sa : sa) : 0.f;
         if (Pm) Pm[r * CP + i] = i <= r ? sp : 0.f;
