@@ -120,15 +120,46 @@ __device__ __forceinline__ void decayed_grams(const float *Kc, const float *Qc, 
     __syncthreads();
 }
 
-// T = (I + A)^-1 for strictly lower A (row stride CP), by forward substitution one row at a time.
-__device__ __forceinline__ void ut_inverse(const float *Am, float *Tm) {
-    for (int r = 0; r < kC; ++r) {
-        if (threadIdx.x < kC) {
-            const int j = threadIdx.x;
-            float t = (j == r) ? 1.f : 0.f;
-            if (j < r)
-                for (int i = j; i < r; ++i) t = fmaf(-Am[r * CP + i], Tm[i * CP + j], t);
-            Tm[r * CP + j] = (j <= r) ? t : 0.f;
+// T = (I + A)^-1 for strictly lower A (row stride CP) into Tm, blocked: the four 16 x 16 diagonal
+// blocks by forward substitution (one column per thread), then each block row b as
+// T_ba = -T_bb sum_{c=a}^{b-1} A_bc T_ca (a < b) in two stages, with Ms ([16][48]) as scratch.  Seven
+// barriers instead of one per row.  Tm's upper triangle is written as zeros.
+__device__ __forceinline__ void ut_inverse(const float *Am, float *Tm, float *Ms) {
+    const int tid = threadIdx.x;
+    for (int p = tid; p < kC * kC; p += kBT) {  // zeros outside the diagonal blocks (written below)
+        const int r = p / kC, i = p % kC;
+        if (r / 16 != i / 16) Tm[r * CP + i] = 0.f;
+    }
+    if (tid < kC) {  // diagonal blocks: column j of (I + A_bb)^-1
+        const int o = 16 * (tid >> 4), j = tid & 15;
+        float x[16];
+#pragma unroll
+        for (int rr = 0; rr < 16; ++rr) {
+            float t = rr == j ? 1.f : 0.f;
+#pragma unroll
+            for (int i = 0; i < rr; ++i)
+                if (i >= j) t = fmaf(-Am[(o + rr) * CP + o + i], x[i], t);
+            x[rr] = rr < j ? 0.f : t;
+        }
+#pragma unroll
+        for (int rr = 0; rr < 16; ++rr) Tm[(o + rr) * CP + o + j] = x[rr];
+    }
+    __syncthreads();
+    for (int b = 1; b < 4; ++b) {
+        const int o = 16 * b;
+        for (int p = tid; p < 16 * 16 * b; p += kBT) {  // stage 1: M[rr][16a + jj] = sum_i A[o + rr][i] T[i][16a + jj]
+            const int rr = p / (16 * b), col = p % (16 * b), a = col / 16;
+            float acc = 0.f;
+            for (int i = 16 * a; i < o; ++i) acc = fmaf(Am[(o + rr) * CP + i], Tm[i * CP + col], acc);
+            Ms[rr * 48 + col] = acc;
+        }
+        __syncthreads();
+        for (int p = tid; p < 16 * 16 * b; p += kBT) {  // stage 2: T[o + rr][col] = -sum_kk T_bb[rr][kk] M[kk][col]
+            const int rr = p / (16 * b), col = p % (16 * b);
+            float acc = 0.f;
+#pragma unroll
+            for (int kk = 0; kk < 16; ++kk) acc = fmaf(Tm[(o + rr) * CP + o + kk], Ms[kk * 48 + col], acc);
+            Tm[(o + rr) * CP + col] = -acc;
         }
         __syncthreads();
     }
@@ -196,7 +227,7 @@ kda_bwd_prep_kernel(const T *__restrict__ q, const T *__restrict__ k, const floa
         rec[O::Pm + p] = Pm[r * CP + i];
     }
     __syncthreads();
-    ut_inverse(Xm, Pm);  // T into the P buffer (P is already stored)
+    ut_inverse(Xm, Pm, Am);  // T into the P buffer (P is already stored), Abar's buffer as scratch
     for (int p = tid; p < kC * kC; p += kBT) rec[O::Tm + p] = Pm[(p / kC) * CP + p % kC];
     for (int idx = tid; idx < kC * D; idx += kBT) {
         const int r = idx / D, c = idx % D;
