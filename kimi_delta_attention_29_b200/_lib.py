@@ -34,7 +34,7 @@ KDA_PROLOGUE_L2NORM_QK = 1
 KDA_PROLOGUE_GATE = 2
 
 # Every entry point include/kda.h declares.
-EXPORTED = ("kda_chunk_fwd_workspace_size", "kda_chunk_fwd", "kda_chunk_fwd_ex", "kda_decode_step",
+EXPORTED = ("kda_chunk_fwd_workspace_size", "kda_chunk_fwd", "kda_chunk_fwd_noalloc", "kda_chunk_fwd_ex", "kda_decode_step",
             "kda_decode_multi", "kda_decode_multi_ex", "kda_output_gate_norm", "kda_chunk_bwd_workspace_size",
             "kda_chunk_bwd", "kda_state_compose", "kda_segment_map", "kda_get_status",
             "kda_status_string", "kda_version", "kda_trace_begin", "kda_trace_end")
@@ -62,6 +62,8 @@ def load() -> ctypes.CDLL:
     lib.kda_chunk_fwd_workspace_size.restype = sz
     lib.kda_chunk_fwd.argtypes = [vp, vp, vp, fp, fp, fp, ip, i, i, i, i, i, i, i, i, vp, fp, vp, sz, vp]
     lib.kda_chunk_fwd.restype = i
+    lib.kda_chunk_fwd_noalloc.argtypes = [vp, vp, vp, fp, fp, fp, ip, i, i, i, i, i, i, i, i, vp, fp, vp]
+    lib.kda_chunk_fwd_noalloc.restype = i
     lib.kda_decode_step.argtypes = [vp, vp, vp, fp, fp, fp, i, i, i, i, i, vp, vp]
     lib.kda_decode_step.restype = i
     lib.kda_decode_multi.argtypes = [vp, vp, vp, fp, fp, fp, i, ip, ip, i, i, i, i, i, i, vp, ip, vp]
