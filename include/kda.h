@@ -292,7 +292,8 @@ KDA_API const char *kda_status_string(int status);
  * 5 multi-token decode, 6 output epilogue, 7 backward state pass, 8 backward chunk kernel,
  * 9 backward chunk operands, 10 segment-map composition, 11 the tensor-core prefill's two kernels
  * running concurrently (one entry: its events bracket the fork of the side stream and the join;
- * ids 1 and 2 appear instead when KDA_PREFILL_SERIAL=1 runs them back to back).
+ * ids 1 and 2 appear instead when KDA_PREFILL_SERIAL=1 runs them back to back), 12 backward
+ * chunk-pair products (dT, dP, dA, dbeta once per chunk and head).
  * Process-wide and not thread-safe; events are owned by the library. */
 KDA_API int kda_trace_begin(int max_kernels);
 KDA_API int kda_trace_end(int *kernel_ids, float *ms, int capacity);

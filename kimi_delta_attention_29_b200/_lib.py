@@ -43,7 +43,7 @@ KERNEL_NAMES = {0: "kda_chunk_table_kernel", 1: "kda_tc_prep_kernel", 2: "kda_tc
                 3: "kda_prefill_simt_kernel", 4: "kda_decode_kernel", 5: "kda_decode_multi_kernel",
                 6: "kda_output_gate_norm_kernel", 7: "kda_bwd_state_kernel", 8: "kda_bwd_chunk_kernel",
                 9: "kda_bwd_prep_kernel", 10: "kda_state_compose_kernel",
-                11: "kda_tc_prefill (state kernel and intra-chunk kernel, concurrent)"}
+                11: "kda_tc_prefill (state kernel and intra-chunk kernel, concurrent)", 12: "kda_bwd_pair_kernel"}
 
 _lib = None
 

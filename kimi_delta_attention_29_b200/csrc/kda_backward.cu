@@ -20,18 +20,20 @@
 // channel, and dlog_alpha is the reverse running sum of dG over the chunk.  (The derivation is
 // checked against the token-by-token adjoint in the tests.)
 //
-// Three kernels, the forward's split between chunk-parallel and sequential work:
+// Four kernels, the forward's split between chunk-parallel and sequential work:
 //  * kda_bwd_prep_kernel - one CTA per (chunk, head), all chunks in parallel: Abar, P, T and the
 //    decayed rows K o 2^G, Q o 2^G, K o 2^{G_L - G} of the chunk, once.
 //  * kda_bwd_state_kernel - one CTA per (sequence, head, 16 value columns), sequential over chunks:
 //    recomputes the chunk-start states (forward pass), then walks the chunks backwards carrying dS,
 //    with only its 16-column products per chunk.  Value columns of S and dS evolve independently,
 //    so slices need no communication.  Per chunk it writes dv and a record of S, dS', Z, dDelta,
-//    X1 and Delta for the chunk kernel.
+//    X1 and Delta for the pair and chunk kernels.
+//  * kda_bwd_pair_kernel - one CTA per (chunk, head), all chunks in parallel: the chunk's 64 x 64
+//    products dT, dP, W and dA from the record and the prep kernel's T, once per chunk-head; writes
+//    dbeta, and dA, dP into the record.
 //  * kda_bwd_chunk_kernel - one CTA per (chunk, head, 32 key channels), all chunks in parallel:
-//    forms dT, dP, dA from the record and the prep kernel's T and Abar, and writes dq, dk,
-//    dlog_alpha (and dbeta from the first channel block).  Every output element has one writer:
-//    deterministic.
+//    the per-channel state products and decayed Gram terms; writes dq, dk and dlog_alpha.
+//    Every output element has one writer: deterministic.
 // Decay factors are single exponentials of differences that are <= 0 where they are used, with
 // each step's base-2 gate clamped at kMinLog2DecaySimt as in the CUDA-core forward (the gradient
 // of a clamped step's log gate is zero).
@@ -57,6 +59,11 @@ template <int D> struct BwdRec {
     static constexpr size_t X1t = dD + (size_t)kC * D;    // [dv][C]  X1^T
     static constexpr size_t Dt = X1t + (size_t)D * kC;    // [dv][C]  Delta^T
     static constexpr size_t floats = Dt + (size_t)D * kC;
+    // dA (strictly lower) and dP (lower) [C][C], written by the pair kernel over dDelta and X1^T,
+    // of which it is the only reader
+    static constexpr size_t dA = dD;
+    static constexpr size_t dP = dD + (size_t)kC * kC;
+    static_assert(dP + (size_t)kC * kC <= Dt, "dA and dP must fit in the dDelta and X1^T slots");
 };
 
 // Chunk loader shared by both kernels: raw K, Q (fp32), the clamped base-2 running gate G and beta
@@ -466,96 +473,54 @@ kda_bwd_state_kernel(const T *__restrict__ v, const float *__restrict__ beta, co
         }
 }
 
-constexpr int kBT2 = 512;            // chunk kernel: threads per CTA
+constexpr int kBT2 = 512;            // pair and chunk kernels: threads per CTA
 constexpr int kCBP = kCB + 1;        // padded row stride of the [C][kCB] channel-block tiles
 constexpr int kRowsPerWarp = kC / (kBT2 / 32);
 
-// Shared memory of the chunk kernel (floats): the channel block's K, Q, G; T, Abar, dT / dA, dP;
-// a staging area for the record tiles (two phases), reused for W and for dG.
+// Shared memory of the pair kernel (floats): T, dT / dA, W; three staged [C][D]-sized record tiles.
 template <int D>
-struct ChunkSmem {
-    static constexpr size_t kbq = 3 * (size_t)kC * kCBP;          // Kb, Qb, Gb
-    static constexpr size_t cc = 4 * (size_t)kC * CP;             // Tm, Am, Mm, Pm
-    static constexpr size_t stage = 3 * (size_t)kC * D + (size_t)D * kCB;  // 3 [C][D]-sized tiles + a [D][kCB] block
-    static constexpr size_t floats = kbq + cc + stage + 2 * (size_t)kC + 2 * (size_t)kCB;
+struct PairSmem {
+    static constexpr size_t floats = 3 * (size_t)kC * CP + 3 * (size_t)kC * D + 2 * (size_t)kC;
     static constexpr size_t bytes = floats * sizeof(float);
 };
 
+// The chunk's 64 x 64 products, once per (chunk, head): dT, dP, W = dT T^T, dA = -strict_lower(T^T W)
+// and dbeta.  dA and dP go to the record for the chunk kernel's channel blocks.  The products are
+// register-blocked: thread t owns rows 4 (t / 32) .. + 3 (warp-uniform, so their operands are
+// broadcast) and columns i0 = t % 32, i0 + 32: six shared loads feed eight FMAs.
 template <int D, typename T>
 __global__ void __launch_bounds__(kBT2, 1)
-kda_bwd_chunk_kernel(const T *__restrict__ q, const T *__restrict__ k, const float *__restrict__ la,
-                     const float *__restrict__ beta, const int4 *__restrict__ table, const int *__restrict__ n_chunks,
-                     int nc, int T_len, int H, const T *__restrict__ dout, const float *__restrict__ ops,
-                     const float *__restrict__ recs, T *__restrict__ dq, T *__restrict__ dk, float *__restrict__ dla,
-                     float *__restrict__ dbeta) {
-    using SM = ChunkSmem<D>;
+kda_bwd_pair_kernel(const float *__restrict__ beta, const int4 *__restrict__ table, const int *__restrict__ n_chunks,
+                    int nc, int T_len, int H, const T *__restrict__ dout, const float *__restrict__ ops,
+                    float *__restrict__ recs, float *__restrict__ dbeta) {
     using R = BwdRec<D>;
     using O = BwdOps<D>;
     extern __shared__ float smem[];
-    float *Kb = smem, *Qb = Kb + kC * kCBP, *Gb = Qb + kC * kCBP;
-    float *Tm = Gb + kC * kCBP, *Am = Tm + kC * CP, *Mm = Am + kC * CP, *Pm = Mm + kC * CP;
-    float *U = Pm + kC * CP;                                   // staging area
-    float *U0 = U, *U1 = U + kC * D, *U2 = U1 + kC * D, *Ub = U2 + kC * D;  // three [C][D] tiles, one [D][kCB]
-    float *bt = U + SM::stage, *dbs = bt + kC, *glb = dbs + kC, *sds = glb + kCB;
+    float *Tm = smem, *Mm = Tm + kC * CP, *Wm = Mm + kC * CP;
+    float *U0 = Wm + kC * CP, *U1 = U0 + kC * D, *U2 = U1 + kC * D;
+    float *bt = U2 + kC * D, *dbs = bt + kC;
 
-    constexpr int blocks = D / kCB;
-    int bid = blockIdx.x;
-    const int cb = bid % blocks;
-    bid /= blocks;
-    const int h = bid % H, ci = bid / H;
+    const int h = blockIdx.x % H, ci = blockIdx.x / H;
     int64_t t0;
     int L;
     if (!chunk_of(ci, table, n_chunks, nc, T_len, t0, L)) return;
-    const float *rec = recs + ((size_t)ci * H + h) * R::floats;
+    float *rec = recs + ((size_t)ci * H + h) * R::floats;
     const float *op = ops + ((size_t)ci * H + h) * O::floats;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int c = cb * kCB + lane;  // this lane's channel in the per-(row, channel) phase
+    const int rb = 4 * warp, i0 = lane;
 
-    // ---- phase 0: T, Abar (prep kernel); beta; K, Q and the clamped base-2 running gate of this block
-    for (int p = tid; p < kC * kC; p += kBT2) {
-        const int r = p / kC, i = p % kC;
-        cp_async4(Tm + r * CP + i, op + O::Tm + p);
-        cp_async4(Am + r * CP + i, op + O::Ab + p);
-    }
-    if (tid < kC) bt[tid] = tid < L ? __ldg(beta + (size_t)(t0 + tid) * H + h) : 0.f;
-    for (int idx = tid; idx < kC * kCB; idx += kBT2) {
-        const int r = idx / kCB, cc = idx % kCB;
-        float kv = 0.f, qv = 0.f, lv = 0.f;
-        if (r < L) {
-            const size_t off = ((size_t)(t0 + r) * H + h) * D + cb * kCB + cc;
-            kv = Elem<T>::load(k + off);
-            qv = Elem<T>::load(q + off);
-            lv = fmaxf(__ldg(la + off) * kLog2e, kMinLog2DecaySimt);
-        }
-        Kb[r * kCBP + cc] = kv;
-        Qb[r * kCBP + cc] = qv;
-        Gb[r * kCBP + cc] = lv;
-    }
-    // ---- phase 1 staging: dDelta [C][D], X1^T [D][C], Z [C][D], S^T block [D][kCB]
+    // ---- staging: T (prep kernel); dDelta [C][D], X1^T [D][C], Z [C][D] (state pass); beta
+    for (int p = tid; p < kC * kC; p += kBT2) cp_async4(Tm + (p / kC) * CP + p % kC, op + O::Tm + p);
     for (int idx = 4 * tid; idx < kC * D; idx += 4 * kBT2) {  // 16-byte pieces of contiguous tiles
         cp_async16(U0 + idx, rec + R::dD + idx);
         cp_async16(U1 + idx, rec + R::X1t + idx);
         cp_async16(U2 + idx, rec + R::Z + idx);
     }
-    for (int idx = 4 * tid; idx < D * kCB; idx += 4 * kBT2)
-        cp_async16(Ub + idx, rec + R::St + (size_t)(idx / kCB) * D + cb * kCB + idx % kCB);
     cp_async_commit();
+    if (tid < kC) bt[tid] = tid < L ? __ldg(beta + (size_t)(t0 + tid) * H + h) : 0.f;
     cp_async_wait<0>();
     __syncthreads();
-    if (tid < kCB) {  // running gate per channel of the block
-        float acc = 0.f;
-        for (int r = 0; r < kC; ++r) {
-            acc += Gb[r * kCBP + tid];
-            Gb[r * kCBP + tid] = acc;
-        }
-        glb[tid] = acc;
-    }
-    // The 64 x 64 products below are register-blocked: thread t owns rows 4 (t / 32) .. + 3 (warp-
-    // uniform, so their operands are broadcast) and columns i0 = t % 32, i0 + 32: six shared loads
-    // feed eight FMAs.
-    const int rb = 4 * warp, i0 = lane;
-    // dT[r][i] = beta_i sum_j dDelta[r][j] X1[i][j]
-    {
+    {  // dT[r][i] = beta_i sum_j dDelta[r][j] X1[i][j]
         float acc[4][2] = {};
         for (int j = 0; j < D; ++j) {
             const float x0 = U1[j * kC + i0], x1 = U1[j * kC + i0 + 32];
@@ -572,68 +537,23 @@ kda_bwd_chunk_kernel(const T *__restrict__ q, const T *__restrict__ k, const flo
             Mm[(rb + m) * CP + i0 + 32] = bt[i0 + 32] * acc[m][1];
         }
     }
-    if (cb == 0 && tid < kC) {  // dbeta, X1 part: sum_j Z[r][j] X1[r][j]
+    if (tid < kC) {  // dbeta, X1 part: sum_j Z[r][j] X1[r][j], j rotated by the lane (no bank conflicts)
         float acc = 0.f;
-        for (int j = 0; j < D; ++j) acc = fmaf(U2[tid * D + j], U1[j * kC + tid], acc);
+        for (int jj = 0; jj < D; ++jj) {
+            const int j = (jj + lane) & (D - 1);
+            acc = fmaf(U2[tid * D + j], U1[j * kC + tid], acc);
+        }
         dbs[tid] = acc;
     }
-    // per-(row, channel) state products: this lane's channel, rows warp + 16 m; each S value is
-    // loaded once for the four rows
-    float dKt[kRowsPerWarp] = {}, dQt[kRowsPerWarp] = {}, dKh[kRowsPerWarp] = {};
-    for (int j = 0; j < D; ++j) {  // dK~ = -beta_r (Z S^T)[r][c]
-        const float sv = Ub[j * kCB + lane];
-#pragma unroll
-        for (int m = 0; m < kRowsPerWarp; ++m) dKt[m] = fmaf(U2[(warp + m * (kBT2 / 32)) * D + j], sv, dKt[m]);
-    }
-#pragma unroll
-    for (int m = 0; m < kRowsPerWarp; ++m) dKt[m] *= -bt[warp + m * (kBT2 / 32)];
-    __syncthreads();
-    // ---- phase 2 staging: dO [C][D], Delta^T [D][C], dS'^T block [D][kCB] (S^T block stays)
+    __syncthreads();  // dT complete; dDelta and X1^T no longer read
+    // ---- staging: Delta^T [D][C] over X1^T, dO [C][D] over dDelta; W = dT T^T meanwhile
     for (int idx = 4 * tid; idx < kC * D; idx += 4 * kBT2) cp_async16(U1 + idx, rec + R::Dt + idx);
-    for (int idx = 4 * tid; idx < D * kCB; idx += 4 * kBT2)
-        cp_async16(U2 + idx, rec + R::dSt + (size_t)(idx / kCB) * D + cb * kCB + idx % kCB);
     cp_async_commit();
     for (int idx = tid; idx < kC * D; idx += kBT2) {
         const int r = idx / D, j = idx % D;
         U0[idx] = r < L ? Elem<T>::load(dout + ((size_t)(t0 + r) * H + h) * D + j) : 0.f;
     }
-    cp_async_wait<0>();
-    __syncthreads();
-    {  // dP[r][i] = sum_j dO[r][j] Delta[i][j]  (i <= r), register-blocked as dT
-        float acc[4][2] = {};
-        for (int j = 0; j < D; ++j) {
-            const float x0 = U1[j * kC + i0], x1 = U1[j * kC + i0 + 32];
-#pragma unroll
-            for (int m = 0; m < 4; ++m) {
-                const float a = U0[(rb + m) * D + j];
-                acc[m][0] = fmaf(a, x0, acc[m][0]);
-                acc[m][1] = fmaf(a, x1, acc[m][1]);
-            }
-        }
-#pragma unroll
-        for (int m = 0; m < 4; ++m) {
-            Pm[(rb + m) * CP + i0] = i0 <= rb + m ? acc[m][0] : 0.f;
-            Pm[(rb + m) * CP + i0 + 32] = i0 + 32 <= rb + m ? acc[m][1] : 0.f;
-        }
-    }
-    for (int j = 0; j < D; ++j) {  // dQ~ = (dO S^T)[r][c],  dK^ = (Delta dS'^T)[r][c]
-        const float sv = Ub[j * kCB + lane], dsv = U2[j * kCB + lane];
-#pragma unroll
-        for (int m = 0; m < kRowsPerWarp; ++m) {
-            const int r = warp + m * (kBT2 / 32);
-            dQt[m] = fmaf(U0[r * D + j], sv, dQt[m]);
-            dKh[m] = fmaf(U1[j * kC + r], dsv, dKh[m]);
-        }
-    }
-    if (warp == 0) {  // sum_j S[c][j] dS'[c][j] for the state-decay term of dG_L
-        float acc = 0.f;
-        for (int j = 0; j < D; ++j) acc = fmaf(Ub[j * kCB + lane], U2[j * kCB + lane], acc);
-        sds[lane] = acc;
-    }
-    __syncthreads();
-    // ---- W = dT T^T (T lower: m <= i) into the staging area, then dA = -strict_lower(T^T W)
-    float *Wm = U;
-    {  // T is stored with zeros above its diagonal, so the sums run over all m
+    {  // W = dT T^T (T is stored with zeros above its diagonal, so the sums run over all m)
         float acc[4][2] = {};
         for (int m = 0; m < kC; ++m) {
             const float t0v = Tm[i0 * CP + m], t1v = Tm[(i0 + 32) * CP + m];
@@ -650,8 +570,26 @@ kda_bwd_chunk_kernel(const T *__restrict__ q, const T *__restrict__ k, const flo
             Wm[(rb + q2) * CP + i0 + 32] = acc[q2][1];
         }
     }
-    __syncthreads();
-    {  // dA[r][i] = -sum_{m >= r} T[m][r] W[m][i] for i < r (T[m][r] = 0 for m < r)
+    cp_async_wait<0>();
+    __syncthreads();  // W, dO and Delta^T in place; dT no longer read
+    {  // dP[r][i] = sum_j dO[r][j] Delta[i][j] (i <= r, zero above) into the record
+        float acc[4][2] = {};
+        for (int j = 0; j < D; ++j) {
+            const float x0 = U1[j * kC + i0], x1 = U1[j * kC + i0 + 32];
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+                const float a = U0[(rb + m) * D + j];
+                acc[m][0] = fmaf(a, x0, acc[m][0]);
+                acc[m][1] = fmaf(a, x1, acc[m][1]);
+            }
+        }
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+            rec[R::dP + (size_t)(rb + m) * kC + i0] = i0 <= rb + m ? acc[m][0] : 0.f;
+            rec[R::dP + (size_t)(rb + m) * kC + i0 + 32] = i0 + 32 <= rb + m ? acc[m][1] : 0.f;
+        }
+    }
+    {  // dA[r][i] = -sum_{m >= r} T[m][r] W[m][i] for i < r (T[m][r] = 0 for m < r), into Mm and the record
         float acc[4][2] = {};
         for (int m = rb; m < kC; ++m) {
             const float w0 = Wm[m * CP + i0], w1 = Wm[m * CP + i0 + 32];
@@ -664,21 +602,130 @@ kda_bwd_chunk_kernel(const T *__restrict__ q, const T *__restrict__ k, const flo
         }
 #pragma unroll
         for (int q2 = 0; q2 < 4; ++q2) {
-            Mm[(rb + q2) * CP + i0] = i0 < rb + q2 ? -acc[q2][0] : 0.f;
-            Mm[(rb + q2) * CP + i0 + 32] = i0 + 32 < rb + q2 ? -acc[q2][1] : 0.f;
+            const float a0 = i0 < rb + q2 ? -acc[q2][0] : 0.f, a1 = i0 + 32 < rb + q2 ? -acc[q2][1] : 0.f;
+            Mm[(rb + q2) * CP + i0] = a0;
+            Mm[(rb + q2) * CP + i0 + 32] = a1;
+            rec[R::dA + (size_t)(rb + q2) * kC + i0] = a0;
+            rec[R::dA + (size_t)(rb + q2) * kC + i0 + 32] = a1;
         }
     }
     __syncthreads();
-    if (cb == 0) {  // dbeta_r = sum_j Z[r][j] X1[r][j] + sum_{i<r} dA[r][i] Abar[r][i]  (one warp per row)
-        for (int r = warp; r < L; r += kBT2 / 32) {
-            float acc = 0.f;
-            for (int i = lane; i < r; i += 32) acc = fmaf(Mm[r * CP + i], Am[r * CP + i], acc);
+    // dbeta_r = sum_j Z[r][j] X1[r][j] + sum_{i<r} dA[r][i] Abar[r][i]  (one warp per row)
+    for (int r = warp; r < L; r += kBT2 / 32) {
+        float acc = 0.f;
+        for (int i = lane; i < r; i += 32) acc = fmaf(Mm[r * CP + i], __ldg(op + O::Ab + r * kC + i), acc);
 #pragma unroll
-            for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-            if (lane == 0) dbeta[(size_t)(t0 + r) * H + h] = acc + dbs[r];
+        for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+        if (lane == 0) dbeta[(size_t)(t0 + r) * H + h] = acc + dbs[r];
+    }
+}
+
+// Shared memory of the chunk kernel (floats): the channel block's K, Q, G; dA, dP (pair kernel); the
+// record tiles dO, Delta^T, Z and the S^T, dS'^T blocks, all staged at once; the first tile is
+// reused for dG.
+template <int D>
+struct ChunkSmem {
+    static constexpr size_t kbq = 3 * (size_t)kC * kCBP;                          // Kb, Qb, Gb
+    static constexpr size_t cc = 2 * (size_t)kC * CP;                             // Mm (dA), Pm (dP)
+    static constexpr size_t stage = 3 * (size_t)kC * D + 2 * (size_t)D * kCB;     // 3 [C][D] tiles, 2 [D][kCB] blocks
+    static constexpr size_t floats = kbq + cc + stage + (size_t)kC + 2 * (size_t)kCB;
+    static constexpr size_t bytes = floats * sizeof(float);
+};
+
+template <int D, typename T>
+__global__ void __launch_bounds__(kBT2, 1)
+kda_bwd_chunk_kernel(const T *__restrict__ q, const T *__restrict__ k, const float *__restrict__ la,
+                     const float *__restrict__ beta, const int4 *__restrict__ table, const int *__restrict__ n_chunks,
+                     int nc, int T_len, int H, const T *__restrict__ dout, const float *__restrict__ recs,
+                     T *__restrict__ dq, T *__restrict__ dk, float *__restrict__ dla) {
+    using SM = ChunkSmem<D>;
+    using R = BwdRec<D>;
+    extern __shared__ float smem[];
+    float *Kb = smem, *Qb = Kb + kC * kCBP, *Gb = Qb + kC * kCBP;
+    float *Mm = Gb + kC * kCBP, *Pm = Mm + kC * CP;
+    float *U = Pm + kC * CP;                                   // staging area
+    float *U0 = U, *U1 = U + kC * D, *U2 = U1 + kC * D;        // dO [C][D], Delta^T [D][C], Z [C][D]
+    float *Ub = U2 + kC * D, *Ud = Ub + D * kCB;               // S^T and dS'^T blocks [D][kCB]
+    float *bt = U + SM::stage, *glb = bt + kC, *sds = glb + kCB;
+
+    constexpr int blocks = D / kCB;
+    int bid = blockIdx.x;
+    const int cb = bid % blocks;
+    bid /= blocks;
+    const int h = bid % H, ci = bid / H;
+    int64_t t0;
+    int L;
+    if (!chunk_of(ci, table, n_chunks, nc, T_len, t0, L)) return;
+    const float *rec = recs + ((size_t)ci * H + h) * R::floats;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int c = cb * kCB + lane;  // this lane's channel in the per-(row, channel) phase
+
+    // ---- staging, all in flight at once: dA, dP (pair kernel); Delta^T, Z and the S^T, dS'^T
+    // blocks (state pass) by cp.async; beta, dO and this block's K, Q and clamped base-2 log gate
+    for (int p = tid; p < kC * kC; p += kBT2) {
+        const int r = p / kC, i = p % kC;
+        cp_async4(Mm + r * CP + i, rec + R::dA + p);
+        cp_async4(Pm + r * CP + i, rec + R::dP + p);
+    }
+    for (int idx = 4 * tid; idx < kC * D; idx += 4 * kBT2) {  // 16-byte pieces of contiguous tiles
+        cp_async16(U1 + idx, rec + R::Dt + idx);
+        cp_async16(U2 + idx, rec + R::Z + idx);
+    }
+    for (int idx = 4 * tid; idx < D * kCB; idx += 4 * kBT2) {
+        const size_t off = (size_t)(idx / kCB) * D + cb * kCB + idx % kCB;
+        cp_async16(Ub + idx, rec + R::St + off);
+        cp_async16(Ud + idx, rec + R::dSt + off);
+    }
+    cp_async_commit();
+    if (tid < kC) bt[tid] = tid < L ? __ldg(beta + (size_t)(t0 + tid) * H + h) : 0.f;
+    for (int idx = tid; idx < kC * kCB; idx += kBT2) {
+        const int r = idx / kCB, cc = idx % kCB;
+        float kv = 0.f, qv = 0.f, lv = 0.f;
+        if (r < L) {
+            const size_t off = ((size_t)(t0 + r) * H + h) * D + cb * kCB + cc;
+            kv = Elem<T>::load(k + off);
+            qv = Elem<T>::load(q + off);
+            lv = fmaxf(__ldg(la + off) * kLog2e, kMinLog2DecaySimt);
+        }
+        Kb[r * kCBP + cc] = kv;
+        Qb[r * kCBP + cc] = qv;
+        Gb[r * kCBP + cc] = lv;
+    }
+    for (int idx = tid; idx < kC * D; idx += kBT2) {
+        const int r = idx / D, j = idx % D;
+        U0[idx] = r < L ? Elem<T>::load(dout + ((size_t)(t0 + r) * H + h) * D + j) : 0.f;
+    }
+    cp_async_wait<0>();
+    __syncthreads();
+    if (tid < kCB) {  // running gate per channel of the block
+        float acc = 0.f;
+        for (int r = 0; r < kC; ++r) {
+            acc += Gb[r * kCBP + tid];
+            Gb[r * kCBP + tid] = acc;
+        }
+        glb[tid] = acc;
+    }
+    // per-(row, channel) state products: this lane's channel, rows warp + 16 m; each S and dS' value
+    // is loaded once for the four rows
+    float dKt[kRowsPerWarp] = {}, dQt[kRowsPerWarp] = {}, dKh[kRowsPerWarp] = {};
+    for (int j = 0; j < D; ++j) {  // dK~ = -beta_r (Z S^T)[r][c],  dQ~ = (dO S^T)[r][c],  dK^ = (Delta dS'^T)[r][c]
+        const float sv = Ub[j * kCB + lane], dsv = Ud[j * kCB + lane];
+#pragma unroll
+        for (int m = 0; m < kRowsPerWarp; ++m) {
+            const int r = warp + m * (kBT2 / 32);
+            dKt[m] = fmaf(U2[r * D + j], sv, dKt[m]);
+            dQt[m] = fmaf(U0[r * D + j], sv, dQt[m]);
+            dKh[m] = fmaf(U1[j * kC + r], dsv, dKh[m]);
         }
     }
-
+#pragma unroll
+    for (int m = 0; m < kRowsPerWarp; ++m) dKt[m] *= -bt[warp + m * (kBT2 / 32)];
+    if (warp == 0) {  // sum_j S[c][j] dS'[c][j] for the state-decay term of dG_L
+        float acc = 0.f;
+        for (int j = 0; j < D; ++j) acc = fmaf(Ub[j * kCB + lane], Ud[j * kCB + lane], acc);
+        sds[lane] = acc;
+    }
+    __syncthreads();  // running gate in place; dO, Delta^T and Z no longer read
     // ---- per (row r, channel c): decayed Gram terms and the factor terms; lane = channel
     float *dGs = U;  // [C][kCBP]
     float *dGLw = U + kC * kCBP;  // [warps][kCB]
@@ -743,10 +790,14 @@ cudaError_t launch_t(const void *q, const void *k, const void *v, const float *l
                      void *fwd_ws, size_t fwd_ws_bytes, cudaStream_t stream) {
     auto kp = kda_bwd_prep_kernel<D, T>;
     auto ks = kda_bwd_state_kernel<D, T>;
+    auto kpair = kda_bwd_pair_kernel<D, T>;
     auto kc = kda_bwd_chunk_kernel<D, T>;
     cudaError_t e = cudaFuncSetAttribute(kp, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)PrepSmem<D>::bytes);
     if (e != cudaSuccess) return e;
     if ((e = cudaFuncSetAttribute(ks, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)StateSmem<D>::bytes)) !=
+        cudaSuccess)
+        return e;
+    if ((e = cudaFuncSetAttribute(kpair, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)PairSmem<D>::bytes)) !=
         cudaSuccess)
         return e;
     if ((e = cudaFuncSetAttribute(kc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ChunkSmem<D>::bytes)) !=
@@ -786,10 +837,14 @@ cudaError_t launch_t(const void *q, const void *k, const void *v, const float *l
     trace_after(stream);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if (chunks == 0) return cudaSuccess;
+    trace_before(kKernBwdPair, stream);
+    kpair<<<(unsigned)(chunks * H), kBT2, PairSmem<D>::bytes, stream>>>(beta, tab, cnt, nc, T_len, H, dot, ops, recs,
+                                                                      dbeta);
+    trace_after(stream);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
     trace_before(kKernBwdChunk, stream);
     kc<<<(unsigned)(chunks * H * (D / kCB)), kBT2, ChunkSmem<D>::bytes, stream>>>(
-        qt, kt, la, beta, tab, cnt, nc, T_len, H, dot, ops, recs, static_cast<T *>(dq), static_cast<T *>(dk), dla,
-        dbeta);
+        qt, kt, la, beta, tab, cnt, nc, T_len, H, dot, recs, static_cast<T *>(dq), static_cast<T *>(dk), dla);
     trace_after(stream);
     return cudaGetLastError();
 }

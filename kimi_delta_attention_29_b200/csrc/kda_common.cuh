@@ -100,7 +100,7 @@ namespace kda {
 // Kernel ids reported by kda_trace_end.
 enum KernelId { kKernChunkTable = 0, kKernTcPrep = 1, kKernTcState = 2, kKernSimt = 3, kKernDecode = 4,
                 kKernDecodeMulti = 5, kKernOutputGateNorm = 6, kKernBwdState = 7, kKernBwdChunk = 8,
-                kKernBwdPrep = 9, kKernStateCompose = 10, kKernTcPrefill = 11 };
+                kKernBwdPrep = 9, kKernStateCompose = 10, kKernTcPrefill = 11, kKernBwdPair = 12 };
 // Diagnostics: bracket one kernel launch with trace events when kda_trace_begin is active.
 void trace_before(int kernel_id, cudaStream_t stream);
 void trace_after(cudaStream_t stream);
