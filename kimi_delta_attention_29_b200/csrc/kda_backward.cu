@@ -248,6 +248,19 @@ kda_bwd_prep_kernel(const T *__restrict__ q, const T *__restrict__ k, const floa
 
 // The operand tiles' rows are padded by 4 floats: 16-byte aligned, so they are staged with 16-byte
 // copies, and rows r, r + 1 start 4 banks apart (the loops below read at most two rows per warp).
+// N consecutive floats from 16-byte (N = 4) or 8-byte (N = 2) aligned shared memory.
+template <int N>
+__device__ __forceinline__ void load_vec(const float *p, float (&out)[N]) {
+    static_assert(N == 2 || N == 4, "two or four floats");
+    if constexpr (N == 4) {
+        const float4 v = *reinterpret_cast<const float4 *>(p);
+        out[0] = v.x, out[1] = v.y, out[2] = v.z, out[3] = v.w;
+    } else {
+        const float2 v = *reinterpret_cast<const float2 *>(p);
+        out[0] = v.x, out[1] = v.y;
+    }
+}
+
 template <int D>
 struct StateSmem {
     static constexpr int DKP = D + 4;
@@ -258,6 +271,10 @@ struct StateSmem {
                                      + 3 * (size_t)D * kSP   // Ss, dSs, dSn
                                      + kC + (size_t)D;       // bt, egl
     static constexpr size_t bytes = floats * sizeof(float);
+    // 16-byte rows and offsets for the cp.async staging and the vector loads of T, K rows and beta
+    static_assert(DKP % 4 == 0 && CPS % 4 == 0, "row strides");
+    static_assert((2 * (size_t)kC * CPS + 3 * (size_t)kC * DKP + 6 * (size_t)kC * kNV + 3 * (size_t)D * kSP) % 4 == 0,
+                  "beta offset");
 };
 
 template <int D, typename T>
@@ -335,24 +352,54 @@ kda_bwd_state_kernel(const T *__restrict__ v, const float *__restrict__ beta, co
         __syncthreads();
     };
     // Register blocking (512 threads): for [C][kNV] tiles a thread owns column jj = tid % 16 of
-    // rows rp = tid / 16 and rp + 32; for [D][kNV] tiles column jj of channels cq + 32 k.
+    // rows rp = tid / 16 and rp + 32; for [D][kNV] tiles column jj of channels rp + 32 k (forward
+    // sweep) or of the D / 32 adjacent channels from (D / 32) rp (reverse sweep).
     const int jj = tid % kNV, rp = tid / kNV;
     constexpr int kCq = D / 32;
+    // The row operands of the dot loops (rows of K o 2^G, K o 2^{G_L - G}, T: two per warp) are read
+    // 16 bytes at a time along the reduction index; the column operands one value per step.
     auto x1_delta = [&]() {  // X1 = V - (K o 2^G) S;  Delta = T Diag(beta) X1
         float a0 = Vs[rp * kNV + jj], a1 = Vs[(rp + 32) * kNV + jj];
-        for (int c = 0; c < D; ++c) {
-            const float sv = Ss[c * kSP + jj];
-            a0 = fmaf(-sKt[rp * DKP + c], sv, a0);
-            a1 = fmaf(-sKt[(rp + 32) * DKP + c], sv, a1);
+        {
+            const float4 *kr0 = reinterpret_cast<const float4 *>(sKt + rp * DKP);
+            const float4 *kr1 = reinterpret_cast<const float4 *>(sKt + (rp + 32) * DKP);
+            for (int c4 = 0; c4 < D / 4; ++c4) {
+                const float4 x = kr0[c4], y = kr1[c4];
+                const float *sv = Ss + 4 * c4 * kSP + jj;
+                const float s0 = sv[0], s1 = sv[kSP], s2 = sv[2 * kSP], s3 = sv[3 * kSP];
+                a0 = fmaf(-x.x, s0, a0);
+                a1 = fmaf(-y.x, s0, a1);
+                a0 = fmaf(-x.y, s1, a0);
+                a1 = fmaf(-y.y, s1, a1);
+                a0 = fmaf(-x.z, s2, a0);
+                a1 = fmaf(-y.z, s2, a1);
+                a0 = fmaf(-x.w, s3, a0);
+                a1 = fmaf(-y.w, s3, a1);
+            }
         }
         X1[rp * kNV + jj] = a0;
         X1[(rp + 32) * kNV + jj] = a1;
         __syncthreads();
-        float d0 = 0.f, d1 = 0.f;  // T is zero above its diagonal
-        for (int i = 0; i <= rp + 32; ++i) {
-            const float xb = bt[i] * X1[i * kNV + jj];
-            d0 = fmaf(sT[rp * CP + i], xb, d0);
-            d1 = fmaf(sT[(rp + 32) * CP + i], xb, d1);
+        // T is zero above its diagonal, so the last group of four may reach past row rp + 32's diagonal
+        // (and both rows run to the same bound: (rp + 32) / 4 is the same for the warp's two rp)
+        float d0 = 0.f, d1 = 0.f;
+        {
+            const float4 *tr0 = reinterpret_cast<const float4 *>(sT + rp * CP);
+            const float4 *tr1 = reinterpret_cast<const float4 *>(sT + (rp + 32) * CP);
+            const float4 *b4 = reinterpret_cast<const float4 *>(bt);
+            for (int i4 = 0; i4 <= (rp + 32) / 4; ++i4) {
+                const float4 u = tr0[i4], w = tr1[i4], b = b4[i4];
+                const float *xs = X1 + 4 * i4 * kNV + jj;
+                const float x0 = b.x * xs[0], x1 = b.y * xs[kNV], x2 = b.z * xs[2 * kNV], x3 = b.w * xs[3 * kNV];
+                d0 = fmaf(u.x, x0, d0);
+                d1 = fmaf(w.x, x0, d1);
+                d0 = fmaf(u.y, x1, d0);
+                d1 = fmaf(w.y, x1, d1);
+                d0 = fmaf(u.z, x2, d0);
+                d1 = fmaf(w.z, x2, d1);
+                d0 = fmaf(u.w, x3, d0);
+                d1 = fmaf(w.w, x3, d1);
+            }
         }
         Dl[rp * kNV + jj] = d0;
         Dl[(rp + 32) * kNV + jj] = d1;
@@ -407,10 +454,20 @@ kda_bwd_state_kernel(const T *__restrict__ v, const float *__restrict__ beta, co
         x1_delta();
         {  // dDelta = (K o 2^{G_L - G}) dS + P^T dO  (P is zero above its diagonal)
             float a0 = 0.f, a1 = 0.f;
-            for (int c = 0; c < D; ++c) {
-                const float ds = dSs[c * kSP + jj];
-                a0 = fmaf(sKh[rp * DKP + c], ds, a0);
-                a1 = fmaf(sKh[(rp + 32) * DKP + c], ds, a1);
+            const float4 *kr0 = reinterpret_cast<const float4 *>(sKh + rp * DKP);
+            const float4 *kr1 = reinterpret_cast<const float4 *>(sKh + (rp + 32) * DKP);
+            for (int c4 = 0; c4 < D / 4; ++c4) {
+                const float4 x = kr0[c4], y = kr1[c4];
+                const float *dsv = dSs + 4 * c4 * kSP + jj;
+                const float s0 = dsv[0], s1 = dsv[kSP], s2 = dsv[2 * kSP], s3 = dsv[3 * kSP];
+                a0 = fmaf(x.x, s0, a0);
+                a1 = fmaf(y.x, s0, a1);
+                a0 = fmaf(x.y, s1, a0);
+                a1 = fmaf(y.y, s1, a1);
+                a0 = fmaf(x.z, s2, a0);
+                a1 = fmaf(y.z, s2, a1);
+                a0 = fmaf(x.w, s3, a0);
+                a1 = fmaf(y.w, s3, a1);
             }
             for (int i = rp; i < kC; ++i) {
                 const float dov = dOs[i * kNV + jj];
@@ -444,20 +501,25 @@ kda_bwd_state_kernel(const T *__restrict__ v, const float *__restrict__ beta, co
             rec[R::X1t + (size_t)(j0 + jj) * kC + r] = X1[r * kNV + jj];
             rec[R::Dt + (size_t)(j0 + jj) * kC + r] = Dl[r * kNV + jj];
         }
-        {  // dS <- 2^{G_L} dS + (Q o 2^G)^T dO - (K o 2^G)^T Diag(beta) Z
+        {  // dS <- 2^{G_L} dS + (Q o 2^G)^T dO - (K o 2^G)^T Diag(beta) Z, for the kCq adjacent
+           // channels kCq rp .. (one 8- or 16-byte load of each operand row per step)
+            const int ch0 = kCq * rp;
             float acc[kCq];
 #pragma unroll
-            for (int q2 = 0; q2 < kCq; ++q2) acc[q2] = egl[rp + 32 * q2] * dSs[(rp + 32 * q2) * kSP + jj];
+            for (int q2 = 0; q2 < kCq; ++q2) acc[q2] = egl[ch0 + q2] * dSs[(ch0 + q2) * kSP + jj];
             for (int r = 0; r < kC; ++r) {
                 const float dov = dOs[r * kNV + jj], zb = -bt[r] * Zs[r * kNV + jj];
+                float qv[kCq], kv[kCq];
+                load_vec<kCq>(sQt + r * DKP + ch0, qv);
+                load_vec<kCq>(sKt + r * DKP + ch0, kv);
 #pragma unroll
                 for (int q2 = 0; q2 < kCq; ++q2) {
-                    acc[q2] = fmaf(sQt[r * DKP + rp + 32 * q2], dov, acc[q2]);
-                    acc[q2] = fmaf(sKt[r * DKP + rp + 32 * q2], zb, acc[q2]);
+                    acc[q2] = fmaf(qv[q2], dov, acc[q2]);
+                    acc[q2] = fmaf(kv[q2], zb, acc[q2]);
                 }
             }
 #pragma unroll
-            for (int q2 = 0; q2 < kCq; ++q2) dSn[(rp + 32 * q2) * kSP + jj] = acc[q2];
+            for (int q2 = 0; q2 < kCq; ++q2) dSn[(ch0 + q2) * kSP + jj] = acc[q2];
         }
         __syncthreads();
         for (int idx = tid; idx < D * kNV; idx += kBTs) {
