@@ -172,12 +172,14 @@ __device__ __forceinline__ void ut_inverse(const float *Am, float *Tm, float *Ms
     }
 }
 
-// Per chunk-head chunk-level operands (fp32), written once by the prep kernel and read by both
-// other kernels (the state pass re-reads them for every 16-column slice).
+// Per chunk-head chunk-level operands (fp32), written once by the prep kernel and read by the
+// state pass (once for every 16-column slice) and the pair kernel.  T and P are also stored
+// transposed, so that every product reads its operand rows along the reduction index.
 template <int D> struct BwdOps {
-    static constexpr size_t Tm = 0;                          // [C][C]  (I + Diag(beta) Abar)^-1
-    static constexpr size_t Pm = Tm + (size_t)kC * kC;       // [C][C]  decayed q-k Gram, i <= r
-    static constexpr size_t Ab = Pm + (size_t)kC * kC;       // [C][C]  Abar, i < r
+    static constexpr size_t Tm = 0;                          // [C][C]  T = (I + Diag(beta) Abar)^-1 (lower)
+    static constexpr size_t Tt = Tm + (size_t)kC * kC;       // [C][C]  T^T
+    static constexpr size_t Pt = Tt + (size_t)kC * kC;       // [C][C]  P^T (P: decayed q-k Gram, i <= r)
+    static constexpr size_t Ab = Pt + (size_t)kC * kC;       // [C][C]  Abar, i < r
     static constexpr size_t Kt = Ab + (size_t)kC * kC;       // [C][D]  K o 2^G
     static constexpr size_t Qt = Kt + (size_t)kC * D;        // [C][D]  Q o 2^G
     static constexpr size_t Kh = Qt + (size_t)kC * D;        // [C][D]  K o 2^{G_L - G}
@@ -231,11 +233,15 @@ kda_bwd_prep_kernel(const T *__restrict__ q, const T *__restrict__ k, const floa
         const int r = p / kC, i = p % kC;
         Xm[r * CP + i] = bt[r] * Am[r * CP + i];  // A = Diag(beta) Abar
         rec[O::Ab + p] = Am[r * CP + i];
-        rec[O::Pm + p] = Pm[r * CP + i];
+        rec[O::Pt + p] = Pm[i * CP + r];
     }
     __syncthreads();
     ut_inverse(Xm, Pm, Am);  // T into the P buffer (P is already stored), Abar's buffer as scratch
-    for (int p = tid; p < kC * kC; p += kBT) rec[O::Tm + p] = Pm[(p / kC) * CP + p % kC];
+    for (int p = tid; p < kC * kC; p += kBT) {
+        const int r = p / kC, i = p % kC;
+        rec[O::Tm + p] = Pm[r * CP + i];
+        rec[O::Tt + p] = Pm[i * CP + r];
+    }
     for (int idx = tid; idx < kC * D; idx += kBT) {
         const int r = idx / D, c = idx % D;
         const float g = Gc[r * DKP + c], e = ex2f(g);
@@ -246,8 +252,6 @@ kda_bwd_prep_kernel(const T *__restrict__ q, const T *__restrict__ k, const floa
     for (int c = tid; c < D; c += kBT) rec[O::eGL + c] = ex2f(gl[c]);
 }
 
-// The operand tiles' rows are padded by 4 floats: 16-byte aligned, so they are staged with 16-byte
-// copies, and rows r, r + 1 start 4 banks apart (the loops below read at most two rows per warp).
 // N consecutive floats from 16-byte (N = 4) or 8-byte (N = 2) aligned shared memory.
 template <int N>
 __device__ __forceinline__ void load_vec(const float *p, float (&out)[N]) {
@@ -261,11 +265,13 @@ __device__ __forceinline__ void load_vec(const float *p, float (&out)[N]) {
     }
 }
 
+// The operand tiles' rows are padded by 4 floats: 16-byte aligned, so they are staged with 16-byte
+// copies, and rows r, r + 1 start 4 banks apart (the loops below read at most two rows per warp).
 template <int D>
 struct StateSmem {
     static constexpr int DKP = D + 4;
     static constexpr int CPS = kC + 4;
-    static constexpr size_t floats = 2 * (size_t)kC * CPS    // sT, sP
+    static constexpr size_t floats = 3 * (size_t)kC * CPS    // sT, sPt, sTt
                                      + 3 * (size_t)kC * DKP  // sKt, sKh, sQt
                                      + 6 * (size_t)kC * kNV  // Vs, dOs, X1, Dl, dDl, Zs
                                      + 3 * (size_t)D * kSP   // Ss, dSs, dSn
@@ -273,7 +279,7 @@ struct StateSmem {
     static constexpr size_t bytes = floats * sizeof(float);
     // 16-byte rows and offsets for the cp.async staging and the vector loads of T, K rows and beta
     static_assert(DKP % 4 == 0 && CPS % 4 == 0, "row strides");
-    static_assert((2 * (size_t)kC * CPS + 3 * (size_t)kC * DKP + 6 * (size_t)kC * kNV + 3 * (size_t)D * kSP) % 4 == 0,
+    static_assert((3 * (size_t)kC * CPS + 3 * (size_t)kC * DKP + 6 * (size_t)kC * kNV + 3 * (size_t)D * kSP) % 4 == 0,
                   "beta offset");
 };
 
@@ -289,8 +295,8 @@ kda_bwd_state_kernel(const T *__restrict__ v, const float *__restrict__ beta, co
     using R = BwdRec<D>;
     using O = BwdOps<D>;
     extern __shared__ float smem[];
-    float *sT = smem, *sP = sT + kC * CP;
-    float *sKt = sP + kC * CP, *sKh = sKt + kC * DKP, *sQt = sKh + kC * DKP;
+    float *sT = smem, *sPt = sT + kC * CP, *sTt = sPt + kC * CP;
+    float *sKt = sTt + kC * CP, *sKh = sKt + kC * DKP, *sQt = sKh + kC * DKP;
     float *Vs = sQt + kC * DKP, *dOs = Vs + kC * kNV, *X1 = dOs + kC * kNV, *Dl = X1 + kC * kNV;
     float *dDl = Dl + kC * kNV, *Zs = dDl + kC * kNV;
     float *Ss = Zs + kC * kNV, *dSs = Ss + D * kSP, *dSn = dSs + D * kSP;
@@ -326,17 +332,30 @@ kda_bwd_state_kernel(const T *__restrict__ v, const float *__restrict__ beta, co
         dSs[c * kSP + jj] = dhT ? dhT[soff + (size_t)c * D + j0 + jj] : 0.f;
     }
 
-    // the chunk's operands (from the prep kernel) and V / dO slices; ends with a barrier
-    auto stage = [&](const float *op, int64_t t0, int L, bool bwd) {
-        for (int p = tid; p < kC * kC / 4; p += kBTs) {  // operand tiles by 16-byte cp.async, all in flight
+    // A chunk's operands (from the prep kernel) by 16-byte cp.async, in two parts.  Part A (T, K^ and,
+    // for the reverse sweep, P^T and T^T) is no longer read once the reverse sweep has formed Z, so
+    // the next chunk's copy of it is issued there and lands while the dS update runs.  Part B (K~,
+    // Q~, 2^{G_L}), the V / dO slices and beta come at the start of the chunk, whose wait covers
+    // every copy in flight; it ends with a barrier.
+    auto stage_a = [&](const float *op, bool bwd) {
+        for (int p = tid; p < kC * kC / 4; p += kBTs) {
             const int r = p / (kC / 4), i = 4 * (p % (kC / 4));
             cp_async16(sT + r * CP + i, op + O::Tm + r * kC + i);
-            if (bwd) cp_async16(sP + r * CP + i, op + O::Pm + r * kC + i);
+            if (bwd) {
+                cp_async16(sPt + r * CP + i, op + O::Pt + r * kC + i);
+                cp_async16(sTt + r * CP + i, op + O::Tt + r * kC + i);
+            }
         }
         for (int idx = tid; idx < kC * D / 4; idx += kBTs) {
             const int r = idx / (D / 4), c = 4 * (idx % (D / 4));
-            cp_async16(sKt + r * DKP + c, op + O::Kt + r * D + c);
             cp_async16(sKh + r * DKP + c, op + O::Kh + r * D + c);
+        }
+        cp_async_commit();
+    };
+    auto stage_b = [&](const float *op, int64_t t0, int L, bool bwd) {
+        for (int idx = tid; idx < kC * D / 4; idx += kBTs) {
+            const int r = idx / (D / 4), c = 4 * (idx % (D / 4));
+            cp_async16(sKt + r * DKP + c, op + O::Kt + r * D + c);
             if (bwd) cp_async16(sQt + r * DKP + c, op + O::Qt + r * D + c);
         }
         for (int c = tid; c < D; c += kBTs) cp_async4(egl + c, op + O::eGL + c);
@@ -417,7 +436,8 @@ kda_bwd_state_kernel(const T *__restrict__ v, const float *__restrict__ beta, co
             const int jj = idx / D, c = idx % D;
             rec[R::St + (size_t)(j0 + jj) * D + c] = Ss[c * kSP + jj];
         }
-        stage(op, t0, L, false);
+        stage_a(op, false);
+        stage_b(op, t0, L, false);
         x1_delta();
         {  // S <- 2^{G_L} S + (K o 2^{G_L - G})^T Delta
             float acc[kCq];
@@ -439,6 +459,7 @@ kda_bwd_state_kernel(const T *__restrict__ v, const float *__restrict__ beta, co
     }
 
     // ---- backward over the chunks, carrying dS (= dL/d state after the chunk)
+    if (nch > 0) stage_a(ops + ((size_t)(cbase + nch - 1) * H + h) * O::floats, true);
     for (int ch = nch - 1; ch >= 0; --ch) {
         const int64_t t0 = start + (int64_t)ch * kC;
         const int L = (int)min((int64_t)kC, len - (int64_t)ch * kC);
@@ -447,10 +468,10 @@ kda_bwd_state_kernel(const T *__restrict__ v, const float *__restrict__ beta, co
         __syncthreads();
         for (int idx = tid; idx < kNV * D; idx += kBTs) {
             const int jj = idx / D, c = idx % D;
-            Ss[c * kSP + jj] = rec[R::St + (size_t)(j0 + jj) * D + c];
+            cp_async4(Ss + c * kSP + jj, rec + R::St + (size_t)(j0 + jj) * D + c);
             rec[R::dSt + (size_t)(j0 + jj) * D + c] = dSs[c * kSP + jj];
         }
-        stage(op, t0, L, true);
+        stage_b(op, t0, L, true);
         x1_delta();
         {  // dDelta = (K o 2^{G_L - G}) dS + P^T dO  (P is zero above its diagonal)
             float a0 = 0.f, a1 = 0.f;
@@ -469,21 +490,43 @@ kda_bwd_state_kernel(const T *__restrict__ v, const float *__restrict__ beta, co
                 a0 = fmaf(x.w, s3, a0);
                 a1 = fmaf(y.w, s3, a1);
             }
-            for (int i = rp; i < kC; ++i) {
-                const float dov = dOs[i * kNV + jj];
-                a0 = fmaf(sP[i * CP + rp], dov, a0);
-                a1 = fmaf(sP[i * CP + rp + 32], dov, a1);
+            {  // rows rp, rp + 32 of P^T from the warp's common start rp / 4 (P^T[r][i] = 0 for i < r)
+                const float4 *pr0 = reinterpret_cast<const float4 *>(sPt + rp * CP);
+                const float4 *pr1 = reinterpret_cast<const float4 *>(sPt + (rp + 32) * CP);
+                for (int i4 = rp / 4; i4 < kC / 4; ++i4) {
+                    const float4 x = pr0[i4], y = pr1[i4];
+                    const float *dov = dOs + 4 * i4 * kNV + jj;
+                    const float e0 = dov[0], e1 = dov[kNV], e2 = dov[2 * kNV], e3 = dov[3 * kNV];
+                    a0 = fmaf(x.x, e0, a0);
+                    a1 = fmaf(y.x, e0, a1);
+                    a0 = fmaf(x.y, e1, a0);
+                    a1 = fmaf(y.y, e1, a1);
+                    a0 = fmaf(x.z, e2, a0);
+                    a1 = fmaf(y.z, e2, a1);
+                    a0 = fmaf(x.w, e3, a0);
+                    a1 = fmaf(y.w, e3, a1);
+                }
             }
             dDl[rp * kNV + jj] = a0;
             dDl[(rp + 32) * kNV + jj] = a1;
         }
         __syncthreads();
-        {  // Z = T^T dDelta;  dV = Diag(beta) Z  (T[i][r] = 0 for i < r)
+        {  // Z = T^T dDelta;  dV = Diag(beta) Z  (rows of T^T from rp / 4: T^T[r][i] = 0 for i < r)
             float z0 = 0.f, z1 = 0.f;
-            for (int i = rp; i < kC; ++i) {
-                const float dd = dDl[i * kNV + jj];
-                z0 = fmaf(sT[i * CP + rp], dd, z0);
-                z1 = fmaf(sT[i * CP + rp + 32], dd, z1);
+            const float4 *tr0 = reinterpret_cast<const float4 *>(sTt + rp * CP);
+            const float4 *tr1 = reinterpret_cast<const float4 *>(sTt + (rp + 32) * CP);
+            for (int i4 = rp / 4; i4 < kC / 4; ++i4) {
+                const float4 x = tr0[i4], y = tr1[i4];
+                const float *dd = dDl + 4 * i4 * kNV + jj;
+                const float e0 = dd[0], e1 = dd[kNV], e2 = dd[2 * kNV], e3 = dd[3 * kNV];
+                z0 = fmaf(x.x, e0, z0);
+                z1 = fmaf(y.x, e0, z1);
+                z0 = fmaf(x.y, e1, z0);
+                z1 = fmaf(y.y, e1, z1);
+                z0 = fmaf(x.z, e2, z0);
+                z1 = fmaf(y.z, e2, z1);
+                z0 = fmaf(x.w, e3, z0);
+                z1 = fmaf(y.w, e3, z1);
             }
             Zs[rp * kNV + jj] = z0;
             Zs[(rp + 32) * kNV + jj] = z1;
@@ -491,6 +534,7 @@ kda_bwd_state_kernel(const T *__restrict__ v, const float *__restrict__ beta, co
             if (rp + 32 < L) Elem<T>::store(dv_out + ((size_t)(t0 + rp + 32) * H + h) * D + j0 + jj, bt[rp + 32] * z1);
         }
         __syncthreads();
+        if (ch > 0) stage_a(ops + ((size_t)(cbase + ch - 1) * H + h) * O::floats, true);  // the next chunk's part A
         for (int idx = tid; idx < kC * kNV; idx += kBTs) {  // record rows: Z, dDelta ([C][dv])
             const int r = idx / kNV, jj = idx % kNV;
             rec[R::Z + (size_t)r * D + j0 + jj] = Zs[idx];
