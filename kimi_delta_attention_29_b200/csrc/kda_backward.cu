@@ -58,9 +58,12 @@ template <int D> struct BwdRec {
     static constexpr size_t dD = Z + (size_t)kC * D;      // [C][dv]  dDelta
     static constexpr size_t X1t = dD + (size_t)kC * D;    // [dv][C]  X1^T
     static constexpr size_t Dt = X1t + (size_t)D * kC;    // [dv][C]  Delta^T
-    static constexpr size_t floats = Dt + (size_t)D * kC;
+    static constexpr size_t Dr = Dt + (size_t)D * kC;     // [C][dv]  Delta
+    static constexpr size_t dAt = Dr + (size_t)kC * D;    // [C][C]   dA^T (pair kernel)
+    static constexpr size_t dPt = dAt + (size_t)kC * kC;  // [C][C]   dP^T (pair kernel)
+    static constexpr size_t floats = dPt + (size_t)kC * kC;
     // dA (strictly lower) and dP (lower) [C][C], written by the pair kernel over dDelta and X1^T,
-    // of which it is the only reader
+    // of which it is the only reader (their transposes have slots of their own)
     static constexpr size_t dA = dD;
     static constexpr size_t dP = dD + (size_t)kC * kC;
     static_assert(dP + (size_t)kC * kC <= Dt, "dA and dP must fit in the dDelta and X1^T slots");
@@ -535,10 +538,11 @@ kda_bwd_state_kernel(const T *__restrict__ v, const float *__restrict__ beta, co
         }
         __syncthreads();
         if (ch > 0) stage_a(ops + ((size_t)(cbase + ch - 1) * H + h) * O::floats, true);  // the next chunk's part A
-        for (int idx = tid; idx < kC * kNV; idx += kBTs) {  // record rows: Z, dDelta ([C][dv])
+        for (int idx = tid; idx < kC * kNV; idx += kBTs) {  // record rows: Z, dDelta, Delta ([C][dv])
             const int r = idx / kNV, jj = idx % kNV;
             rec[R::Z + (size_t)r * D + j0 + jj] = Zs[idx];
             rec[R::dD + (size_t)r * D + j0 + jj] = dDl[idx];
+            rec[R::Dr + (size_t)r * D + j0 + jj] = Dl[idx];
         }
         for (int idx = tid; idx < kNV * kC; idx += kBTs) {  // transposed: X1^T, Delta^T ([dv][C])
             const int jj = idx / kC, r = idx % kC;
@@ -582,11 +586,13 @@ kda_bwd_state_kernel(const T *__restrict__ v, const float *__restrict__ beta, co
 constexpr int kBT2 = 512;            // pair and chunk kernels: threads per CTA
 constexpr int kCBP = kCB + 1;        // padded row stride of the [C][kCB] channel-block tiles
 constexpr int kRowsPerWarp = kC / (kBT2 / 32);
+constexpr int CP4 = kC + 4;          // 16-byte aligned row stride of the chunk kernel's [C][C] tiles
 
-// Shared memory of the pair kernel (floats): T, dT / dA, W; three staged [C][D]-sized record tiles.
+// Shared memory of the pair kernel (floats): T, dT / dA, W; three staged [C][D]-sized record tiles;
+// Abar.
 template <int D>
 struct PairSmem {
-    static constexpr size_t floats = 3 * (size_t)kC * CP + 3 * (size_t)kC * D + 2 * (size_t)kC;
+    static constexpr size_t floats = 3 * (size_t)kC * CP + 3 * (size_t)kC * D + 2 * (size_t)kC + (size_t)kC * kC;
     static constexpr size_t bytes = floats * sizeof(float);
 };
 
@@ -604,7 +610,7 @@ kda_bwd_pair_kernel(const float *__restrict__ beta, const int4 *__restrict__ tab
     extern __shared__ float smem[];
     float *Tm = smem, *Mm = Tm + kC * CP, *Wm = Mm + kC * CP;
     float *U0 = Wm + kC * CP, *U1 = U0 + kC * D, *U2 = U1 + kC * D;
-    float *bt = U2 + kC * D, *dbs = bt + kC;
+    float *bt = U2 + kC * D, *dbs = bt + kC, *Abs = dbs + kC;
 
     const int h = blockIdx.x % H, ci = blockIdx.x / H;
     int64_t t0;
@@ -615,8 +621,9 @@ kda_bwd_pair_kernel(const float *__restrict__ beta, const int4 *__restrict__ tab
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int rb = 4 * warp, i0 = lane;
 
-    // ---- staging: T (prep kernel); dDelta [C][D], X1^T [D][C], Z [C][D] (state pass); beta
+    // ---- staging: T, Abar (prep kernel); dDelta [C][D], X1^T [D][C], Z [C][D] (state pass); beta
     for (int p = tid; p < kC * kC; p += kBT2) cp_async4(Tm + (p / kC) * CP + p % kC, op + O::Tm + p);
+    for (int p = 4 * tid; p < kC * kC; p += 4 * kBT2) cp_async16(Abs + p, op + O::Ab + p);
     for (int idx = 4 * tid; idx < kC * D; idx += 4 * kBT2) {  // 16-byte pieces of contiguous tiles
         cp_async16(U0 + idx, rec + R::dD + idx);
         cp_async16(U1 + idx, rec + R::X1t + idx);
@@ -678,6 +685,9 @@ kda_bwd_pair_kernel(const float *__restrict__ beta, const int4 *__restrict__ tab
     }
     cp_async_wait<0>();
     __syncthreads();  // W, dO and Delta^T in place; dT no longer read
+    // dP [C][C] over Z (read only by dbs, before the first barrier), row stride kC with the column
+    // XOR-ed by the row's low five bits: row writes and column reads both hit 32 distinct banks
+    float *Ps = U2;
     {  // dP[r][i] = sum_j dO[r][j] Delta[i][j] (i <= r, zero above) into the record
         float acc[4][2] = {};
         for (int j = 0; j < D; ++j) {
@@ -691,8 +701,11 @@ kda_bwd_pair_kernel(const float *__restrict__ beta, const int4 *__restrict__ tab
         }
 #pragma unroll
         for (int m = 0; m < 4; ++m) {
-            rec[R::dP + (size_t)(rb + m) * kC + i0] = i0 <= rb + m ? acc[m][0] : 0.f;
-            rec[R::dP + (size_t)(rb + m) * kC + i0 + 32] = i0 + 32 <= rb + m ? acc[m][1] : 0.f;
+            const float p0 = i0 <= rb + m ? acc[m][0] : 0.f, p1 = i0 + 32 <= rb + m ? acc[m][1] : 0.f;
+            rec[R::dP + (size_t)(rb + m) * kC + i0] = p0;
+            rec[R::dP + (size_t)(rb + m) * kC + i0 + 32] = p1;
+            Ps[(rb + m) * kC + (i0 ^ ((rb + m) & 31))] = p0;
+            Ps[(rb + m) * kC + ((i0 + 32) ^ ((rb + m) & 31))] = p1;
         }
     }
     {  // dA[r][i] = -sum_{m >= r} T[m][r] W[m][i] for i < r (T[m][r] = 0 for m < r), into Mm and the record
@@ -716,25 +729,30 @@ kda_bwd_pair_kernel(const float *__restrict__ beta, const int4 *__restrict__ tab
         }
     }
     __syncthreads();
+    for (int p = tid; p < kC * kC; p += kBT2) {  // dA^T, dP^T: coalesced rows, conflict-free column reads
+        const int i = p / kC, r = p % kC;
+        rec[R::dAt + p] = Mm[r * CP + i];
+        rec[R::dPt + p] = Ps[r * kC + (i ^ (r & 31))];
+    }
     // dbeta_r = sum_j Z[r][j] X1[r][j] + sum_{i<r} dA[r][i] Abar[r][i]  (one warp per row)
     for (int r = warp; r < L; r += kBT2 / 32) {
         float acc = 0.f;
-        for (int i = lane; i < r; i += 32) acc = fmaf(Mm[r * CP + i], __ldg(op + O::Ab + r * kC + i), acc);
+        for (int i = lane; i < r; i += 32) acc = fmaf(Mm[r * CP + i], Abs[r * kC + i], acc);
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
         if (lane == 0) dbeta[(size_t)(t0 + r) * H + h] = acc + dbs[r];
     }
 }
 
-// Shared memory of the chunk kernel (floats): the channel block's K, Q, G; dA, dP (pair kernel); the
-// record tiles dO, Delta^T, Z and the S^T, dS'^T blocks, all staged at once; the first tile is
-// reused for dG.
+// Shared memory of the chunk kernel (floats): the channel block's K, Q, G; dA, dP and their
+// transposes (pair kernel); the record tiles dO, Delta, Z and the S^T, dS'^T blocks, all staged at
+// once; the first tile is reused for dG.
 template <int D>
 struct ChunkSmem {
     static constexpr size_t kbq = 3 * (size_t)kC * kCBP;                          // Kb, Qb, Gb
-    static constexpr size_t cc = 2 * (size_t)kC * CP;                             // Mm (dA), Pm (dP)
+    static constexpr size_t cc = 4 * (size_t)kC * CP4;                            // dA, dP, dA^T, dP^T
     static constexpr size_t stage = 3 * (size_t)kC * D + 2 * (size_t)D * kCB;     // 3 [C][D] tiles, 2 [D][kCB] blocks
-    static constexpr size_t floats = kbq + cc + stage + (size_t)kC + 2 * (size_t)kCB;
+    static constexpr size_t floats = kbq + cc + stage + 2 * (size_t)kC + 2 * (size_t)kCB;  // + beta, clamp masks
     static constexpr size_t bytes = floats * sizeof(float);
 };
 
@@ -748,12 +766,14 @@ kda_bwd_chunk_kernel(const T *__restrict__ q, const T *__restrict__ k, const flo
     using R = BwdRec<D>;
     extern __shared__ float smem[];
     float *Kb = smem, *Qb = Kb + kC * kCBP, *Gb = Qb + kC * kCBP;
-    float *Mm = Gb + kC * kCBP, *Pm = Mm + kC * CP;
-    float *U = Pm + kC * CP;                                   // staging area
-    float *U0 = U, *U1 = U + kC * D, *U2 = U1 + kC * D;        // dO [C][D], Delta^T [D][C], Z [C][D]
+    float *Mm = Gb + kC * kCBP, *Pm = Mm + kC * CP4, *Mt = Pm + kC * CP4, *Pt = Mt + kC * CP4;
+    float *U = Pt + kC * CP4;                                  // staging area
+    float *U0 = U, *U1 = U + kC * D, *U2 = U1 + kC * D;        // dO, Delta, Z: [C][D]
     float *Ub = U2 + kC * D, *Ud = Ub + D * kCB;               // S^T and dS'^T blocks [D][kCB]
     float *bt = U + SM::stage, *glb = bt + kC, *sds = glb + kCB;
+    unsigned *cmask = reinterpret_cast<unsigned *>(sds + kCB);  // [C]: bit cc set where row r's gate was clamped
 
+    static_assert(kCB == 32, "one warp per row of the channel block");
     constexpr int blocks = D / kCB;
     int bid = blockIdx.x;
     const int cb = bid % blocks;
@@ -766,15 +786,17 @@ kda_bwd_chunk_kernel(const T *__restrict__ q, const T *__restrict__ k, const flo
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int c = cb * kCB + lane;  // this lane's channel in the per-(row, channel) phase
 
-    // ---- staging, all in flight at once: dA, dP (pair kernel); Delta^T, Z and the S^T, dS'^T
-    // blocks (state pass) by cp.async; beta, dO and this block's K, Q and clamped base-2 log gate
-    for (int p = tid; p < kC * kC; p += kBT2) {
-        const int r = p / kC, i = p % kC;
-        cp_async4(Mm + r * CP + i, rec + R::dA + p);
-        cp_async4(Pm + r * CP + i, rec + R::dP + p);
+    // ---- staging, all in flight at once: dA, dP (pair kernel); Delta, Z and the S^T, dS'^T blocks
+    // (state pass) by cp.async; beta, dO and this block's K, Q and clamped base-2 log gate
+    for (int p = tid; p < kC * kC / 4; p += kBT2) {
+        const int r = p / (kC / 4), i = 4 * (p % (kC / 4));
+        cp_async16(Mm + r * CP4 + i, rec + R::dA + r * kC + i);
+        cp_async16(Pm + r * CP4 + i, rec + R::dP + r * kC + i);
+        cp_async16(Mt + r * CP4 + i, rec + R::dAt + r * kC + i);
+        cp_async16(Pt + r * CP4 + i, rec + R::dPt + r * kC + i);
     }
     for (int idx = 4 * tid; idx < kC * D; idx += 4 * kBT2) {  // 16-byte pieces of contiguous tiles
-        cp_async16(U1 + idx, rec + R::Dt + idx);
+        cp_async16(U1 + idx, rec + R::Dr + idx);
         cp_async16(U2 + idx, rec + R::Z + idx);
     }
     for (int idx = 4 * tid; idx < D * kCB; idx += 4 * kBT2) {
@@ -784,18 +806,23 @@ kda_bwd_chunk_kernel(const T *__restrict__ q, const T *__restrict__ k, const flo
     }
     cp_async_commit();
     if (tid < kC) bt[tid] = tid < L ? __ldg(beta + (size_t)(t0 + tid) * H + h) : 0.f;
-    for (int idx = tid; idx < kC * kCB; idx += kBT2) {
+    for (int idx = tid; idx < kC * kCB; idx += kBT2) {  // warp-uniform row r, lane = channel cc
         const int r = idx / kCB, cc = idx % kCB;
         float kv = 0.f, qv = 0.f, lv = 0.f;
+        bool clamped = false;
         if (r < L) {
             const size_t off = ((size_t)(t0 + r) * H + h) * D + cb * kCB + cc;
             kv = Elem<T>::load(k + off);
             qv = Elem<T>::load(q + off);
-            lv = fmaxf(__ldg(la + off) * kLog2e, kMinLog2DecaySimt);
+            const float l2 = __ldg(la + off) * kLog2e;
+            clamped = l2 < kMinLog2DecaySimt;
+            lv = fmaxf(l2, kMinLog2DecaySimt);
         }
         Kb[r * kCBP + cc] = kv;
         Qb[r * kCBP + cc] = qv;
         Gb[r * kCBP + cc] = lv;
+        const unsigned cm = __ballot_sync(0xffffffffu, clamped);
+        if (cc == 0) cmask[r] = cm;
     }
     for (int idx = tid; idx < kC * D; idx += kBT2) {
         const int r = idx / D, j = idx % D;
@@ -811,17 +838,29 @@ kda_bwd_chunk_kernel(const T *__restrict__ q, const T *__restrict__ k, const flo
         }
         glb[tid] = acc;
     }
-    // per-(row, channel) state products: this lane's channel, rows warp + 16 m; each S and dS' value
-    // is loaded once for the four rows
+    // per-(row, channel) state products: this lane's channel, rows warp + 16 m; four S and dS'
+    // values per step serve the four rows, whose Z, dO and Delta entries come as 16-byte broadcasts
     float dKt[kRowsPerWarp] = {}, dQt[kRowsPerWarp] = {}, dKh[kRowsPerWarp] = {};
-    for (int j = 0; j < D; ++j) {  // dK~ = -beta_r (Z S^T)[r][c],  dQ~ = (dO S^T)[r][c],  dK^ = (Delta dS'^T)[r][c]
-        const float sv = Ub[j * kCB + lane], dsv = Ud[j * kCB + lane];
+    for (int j4 = 0; j4 < D / 4; ++j4) {  // dK~ = -beta_r (Z S^T)[r][c],  dQ~ = (dO S^T)[r][c],  dK^ = (Delta dS'^T)[r][c]
+        float sv[4], dsv[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            sv[u] = Ub[(4 * j4 + u) * kCB + lane];
+            dsv[u] = Ud[(4 * j4 + u) * kCB + lane];
+        }
 #pragma unroll
         for (int m = 0; m < kRowsPerWarp; ++m) {
             const int r = warp + m * (kBT2 / 32);
-            dKt[m] = fmaf(U2[r * D + j], sv, dKt[m]);
-            dQt[m] = fmaf(U0[r * D + j], sv, dQt[m]);
-            dKh[m] = fmaf(U1[j * kC + r], dsv, dKh[m]);
+            float z[4], o[4], d[4];
+            load_vec<4>(U2 + r * D + 4 * j4, z);
+            load_vec<4>(U0 + r * D + 4 * j4, o);
+            load_vec<4>(U1 + r * D + 4 * j4, d);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                dKt[m] = fmaf(z[u], sv[u], dKt[m]);
+                dQt[m] = fmaf(o[u], sv[u], dQt[m]);
+                dKh[m] = fmaf(d[u], dsv[u], dKh[m]);
+            }
         }
     }
 #pragma unroll
@@ -831,7 +870,7 @@ kda_bwd_chunk_kernel(const T *__restrict__ q, const T *__restrict__ k, const flo
         for (int j = 0; j < D; ++j) acc = fmaf(Ub[j * kCB + lane], Ud[j * kCB + lane], acc);
         sds[lane] = acc;
     }
-    __syncthreads();  // running gate in place; dO, Delta^T and Z no longer read
+    __syncthreads();  // running gate in place; dO, Delta and Z no longer read
     // ---- per (row r, channel c): decayed Gram terms and the factor terms; lane = channel
     float *dGs = U;  // [C][kCBP]
     float *dGLw = U + kC * kCBP;  // [warps][kCB]
@@ -843,15 +882,34 @@ kda_bwd_chunk_kernel(const T *__restrict__ q, const T *__restrict__ k, const flo
         const float g = Gb[r * kCBP + lane], kc = Kb[r * kCBP + lane], qc = Qb[r * kCBP + lane];
         const float er = ex2f(g), eL = ex2f(glc - g);
         float xa = 0.f, yq = 0.f, zk = 0.f;
-        for (int i = 0; i <= r; ++i) {  // this row as the later index
-            const float kd = Kb[i * kCBP + lane] * ex2f(g - Gb[i * kCBP + lane]);
-            if (i < r) xa = fmaf(Mm[r * CP + i], kd, xa);
-            yq = fmaf(Pm[r * CP + i], kd, yq);
+        // Both loops take dA, dP (rows of the tiles or of their transposes) and beta four at a time, so
+        // the group of four holding r also runs over indices on the other side of r, where dA and dP
+        // are zero (dA[r][r] too); there the decay exponent, <= 0 on the valid side since G only
+        // falls, is clamped at 0 so that the factor stays finite and the term exactly zero.
+        for (int i4 = 0; i4 <= r / 4; ++i4) {  // this row as the later index: i <= r
+            float a[4], pq[4];
+            load_vec<4>(Mm + r * CP4 + 4 * i4, a);
+            load_vec<4>(Pm + r * CP4 + 4 * i4, pq);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int i = 4 * i4 + u;
+                const float kd = Kb[i * kCBP + lane] * ex2f(fminf(g - Gb[i * kCBP + lane], 0.f));
+                xa = fmaf(a[u], kd, xa);
+                yq = fmaf(pq[u], kd, yq);
+            }
         }
-        for (int mm = r; mm < kC; ++mm) {  // this row as the earlier index
-            const float e = ex2f(Gb[mm * kCBP + lane] - g);
-            if (mm > r) zk = fmaf(bt[mm] * Mm[mm * CP + r] * Kb[mm * kCBP + lane], e, zk);
-            zk = fmaf(Pm[mm * CP + r] * Qb[mm * kCBP + lane], e, zk);
+        for (int m4 = r / 4; m4 < kC / 4; ++m4) {  // this row as the earlier index: mm >= r
+            float at[4], pt[4], b[4];
+            load_vec<4>(Mt + r * CP4 + 4 * m4, at);  // dA^T[r][mm] = dA[mm][r]
+            load_vec<4>(Pt + r * CP4 + 4 * m4, pt);
+            load_vec<4>(bt + 4 * m4, b);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int mm = 4 * m4 + u;
+                const float e = ex2f(fminf(Gb[mm * kCBP + lane] - g, 0.f));
+                zk = fmaf(b[u] * at[u] * Kb[mm * kCBP + lane], e, zk);
+                zk = fmaf(pt[u] * Qb[mm * kCBP + lane], e, zk);
+            }
         }
         const float dkv = dKt[m] * er + dKh[m] * eL + bt[r] * xa + zk;
         const float dqv = dQt[m] * er + yq;
@@ -876,9 +934,7 @@ kda_bwd_chunk_kernel(const T *__restrict__ q, const T *__restrict__ k, const flo
         float run = 0.f;
         for (int r = L - 1; r >= 0; --r) {
             run += dGs[r * kCBP + lane];
-            const size_t off = ((size_t)(t0 + r) * H + h) * D + c;
-            const bool clamped = __ldg(la + off) * kLog2e < kMinLog2DecaySimt;
-            dla[off] = clamped ? 0.f : run;
+            dla[((size_t)(t0 + r) * H + h) * D + c] = (cmask[r] >> lane) & 1u ? 0.f : run;
         }
     }
 }
