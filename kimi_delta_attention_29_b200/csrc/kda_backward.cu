@@ -69,14 +69,15 @@ template <int D> struct BwdRec {
     static_assert(dP + (size_t)kC * kC <= Dt, "dA and dP must fit in the dDelta and X1^T slots");
 };
 
-// Chunk loader shared by both kernels: raw K, Q (fp32), the clamped base-2 running gate G and beta
-// of one chunk; rows >= L are the neutral token (k = q = 0, log gate 0, beta 0).  Ends with a
-// barrier; gl[c] = G at the last row.
+// Chunk loader of the prep kernel: raw K, Q (fp32), the clamped base-2 running gate G and beta of
+// one chunk in rows of D + 4 floats (16-byte aligned), then K and G transposed ([D][C]); rows >= L
+// are the neutral token (k = q = 0, log gate 0, beta 0).  Ends with a barrier; gl[c] = G at the
+// last row.
 template <int D, typename T>
 __device__ __forceinline__ void load_chunk(const T *q, const T *k, const float *la, const float *beta, int64_t t0,
                                            int L, int H, int h, bool want_q, float *Kc, float *Qc, float *Gc,
-                                           float *bt, float *gl) {
-    constexpr int DKP = D + 1;
+                                           float *KT, float *GT, float *bt, float *gl) {
+    constexpr int DKP = D + 4;
     const int tid = threadIdx.x;
     for (int idx = tid; idx < kC * D; idx += kBT) {
         const int r = idx / D, c = idx % D;
@@ -102,30 +103,45 @@ __device__ __forceinline__ void load_chunk(const T *q, const T *k, const float *
         gl[c] = acc;
     }
     __syncthreads();
+    for (int idx = tid; idx < kC * D; idx += kBT) {  // consecutive threads: consecutive rows i
+        const int c = idx / kC, i = idx % kC;
+        KT[idx] = Kc[i * DKP + c];
+        GT[idx] = Gc[i * DKP + c];
+    }
+    __syncthreads();
 }
 
-// Abar[r][i] (i < r, else 0) into Am, optionally times beta_r; P (i <= r) into Pm when Pm != null.
+// Abar[r][i] (i < r, else 0) into Am and P (i <= r) into Pm.  The warp shares r: its K, Q and G
+// rows come as 16-byte broadcasts, and each lane's row i from the transposed K and G.
 template <int D>
-__device__ __forceinline__ void decayed_grams(const float *Kc, const float *Qc, const float *Gc, const float *bt,
-                                              bool scale_beta, float *Am, float *Pm) {
-    constexpr int DKP = D + 1;
+__device__ __forceinline__ void decayed_grams(const float *Kc, const float *Qc, const float *Gc, const float *KT,
+                                              const float *GT, float *Am, float *Pm) {
+    constexpr int DKP = D + 4;
     for (int p = threadIdx.x; p < kC * kC; p += kBT) {
         const int r = p / kC, i = p % kC;
         float sa = 0.f, sp = 0.f;
         if (i <= r) {  // four partial sums per product, so consecutive channels do not wait on each other
-            const float *gr = Gc + r * DKP, *gi = Gc + i * DKP;
+            const float4 *kr = reinterpret_cast<const float4 *>(Kc + r * DKP);
+            const float4 *qr = reinterpret_cast<const float4 *>(Qc + r * DKP);
+            const float4 *gr = reinterpret_cast<const float4 *>(Gc + r * DKP);
             float pa[4] = {0.f, 0.f, 0.f, 0.f}, pp[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 4
-            for (int c = 0; c < D; ++c) {
-                const float kd = Kc[i * DKP + c] * ex2f(gr[c] - gi[c]);
-                pa[c & 3] = fmaf(Kc[r * DKP + c], kd, pa[c & 3]);
-                if (Pm) pp[c & 3] = fmaf(Qc[r * DKP + c], kd, pp[c & 3]);
+            for (int c4 = 0; c4 < D / 4; ++c4) {
+                const float4 kv = kr[c4], qv = qr[c4], gv = gr[c4];
+                const float *ki = KT + 4 * c4 * kC + i, *gi = GT + 4 * c4 * kC + i;
+                const float kra[4] = {kv.x, kv.y, kv.z, kv.w}, qra[4] = {qv.x, qv.y, qv.z, qv.w};
+                const float gra[4] = {gv.x, gv.y, gv.z, gv.w};
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const float kd = ki[u * kC] * ex2f(gra[u] - gi[u * kC]);
+                    pa[u] = fmaf(kra[u], kd, pa[u]);
+                    pp[u] = fmaf(qra[u], kd, pp[u]);
+                }
             }
             sa = (pa[0] + pa[1]) + (pa[2] + pa[3]);
             sp = (pp[0] + pp[1]) + (pp[2] + pp[3]);
         }
-        Am[r * CP + i] = i < r ? (scale_beta ? bt[r] * sa : sa) : 0.f;
-        if (Pm) Pm[r * CP + i] = i <= r ? sp : 0.f;
+        Am[r * CP + i] = i < r ? sa : 0.f;
+        Pm[r * CP + i] = i <= r ? sp : 0.f;
     }
     __syncthreads();
 }
@@ -208,8 +224,8 @@ __device__ __forceinline__ bool chunk_of(int ci, const int4 *table, const int *n
 
 template <int D>
 struct PrepSmem {
-    static constexpr int DKP = D + 1;
-    static constexpr size_t floats = 3 * (size_t)kC * DKP + 3 * (size_t)kC * CP + kC + D;
+    static constexpr int DKP = D + 4;  // K, Q, G rows (16-byte aligned); K^T, G^T [D][C] besides
+    static constexpr size_t floats = 3 * (size_t)kC * DKP + 2 * (size_t)D * kC + 3 * (size_t)kC * CP + kC + D;
     static constexpr size_t bytes = floats * sizeof(float);
 };
 
@@ -223,15 +239,15 @@ kda_bwd_prep_kernel(const T *__restrict__ q, const T *__restrict__ k, const floa
     constexpr int DKP = SM::DKP;
     using O = BwdOps<D>;
     extern __shared__ float smem[];
-    float *Kc = smem, *Qc = Kc + kC * DKP, *Gc = Qc + kC * DKP;
-    float *Am = Gc + kC * DKP, *Pm = Am + kC * CP, *Xm = Pm + kC * CP, *bt = Xm + kC * CP, *gl = bt + kC;
+    float *Kc = smem, *Qc = Kc + kC * DKP, *Gc = Qc + kC * DKP, *KT = Gc + kC * DKP, *GT = KT + D * kC;
+    float *Am = GT + D * kC, *Pm = Am + kC * CP, *Xm = Pm + kC * CP, *bt = Xm + kC * CP, *gl = bt + kC;
     const int h = blockIdx.x % H, ci = blockIdx.x / H, tid = threadIdx.x;
     int64_t t0;
     int L;
     if (!chunk_of(ci, table, n_chunks, nc, T_len, t0, L)) return;
     float *rec = ops + ((size_t)ci * H + h) * O::floats;
-    load_chunk<D, T>(q, k, la, beta, t0, L, H, h, true, Kc, Qc, Gc, bt, gl);
-    decayed_grams<D>(Kc, Qc, Gc, bt, false, Am, Pm);
+    load_chunk<D, T>(q, k, la, beta, t0, L, H, h, true, Kc, Qc, Gc, KT, GT, bt, gl);
+    decayed_grams<D>(Kc, Qc, Gc, KT, GT, Am, Pm);
     for (int p = tid; p < kC * kC; p += kBT) {
         const int r = p / kC, i = p % kC;
         Xm[r * CP + i] = bt[r] * Am[r * CP + i];  // A = Diag(beta) Abar
