@@ -46,7 +46,6 @@ constexpr int kC = kChunk;
 constexpr int kBT = 512;   // threads per CTA of the prep kernel (one CTA per SM: shared memory)
 constexpr int kBTs = 512;  // threads per CTA of the state pass
 constexpr int kNV = 16;    // value columns per state-pass CTA
-constexpr int kSP = kNV + 1;  // padded row stride of the [D][kNV] state tiles
 constexpr int kCB = 32;    // key channels per chunk-kernel CTA
 constexpr int CP = kC + 1;
 
@@ -293,12 +292,13 @@ struct StateSmem {
     static constexpr size_t floats = 3 * (size_t)kC * CPS    // sT, sPt, sTt
                                      + 3 * (size_t)kC * DKP  // sKt, sKh, sQt
                                      + 6 * (size_t)kC * kNV  // Vs, dOs, X1, Dl, dDl, Zs
-                                     + 3 * (size_t)D * kSP   // Ss, dSs, dSn
+                                     + 2 * (size_t)kC * kNV  // DZ: (dO, -beta Z) pairs
+                                     + 3 * (size_t)kNV * DKP // Ss, dSs, dSn transposed: [kNV][D + 4]
                                      + kC + (size_t)D;       // bt, egl
     static constexpr size_t bytes = floats * sizeof(float);
     // 16-byte rows and offsets for the cp.async staging and the vector loads of T, K rows and beta
     static_assert(DKP % 4 == 0 && CPS % 4 == 0, "row strides");
-    static_assert((3 * (size_t)kC * CPS + 3 * (size_t)kC * DKP + 6 * (size_t)kC * kNV + 3 * (size_t)D * kSP) % 4 == 0,
+    static_assert((3 * (size_t)kC * CPS + 3 * (size_t)kC * DKP + 8 * (size_t)kC * kNV + 3 * (size_t)kNV * DKP) % 4 == 0,
                   "beta offset");
 };
 
@@ -317,9 +317,12 @@ kda_bwd_state_kernel(const T *__restrict__ v, const float *__restrict__ beta, co
     float *sT = smem, *sPt = sT + kC * CP, *sTt = sPt + kC * CP;
     float *sKt = sTt + kC * CP, *sKh = sKt + kC * DKP, *sQt = sKh + kC * DKP;
     float *Vs = sQt + kC * DKP, *dOs = Vs + kC * kNV, *X1 = dOs + kC * kNV, *Dl = X1 + kC * kNV;
-    float *dDl = Dl + kC * kNV, *Zs = dDl + kC * kNV;
-    float *Ss = Zs + kC * kNV, *dSs = Ss + D * kSP, *dSn = dSs + D * kSP;
-    float *bt = dSn + D * kSP, *egl = bt + kC;
+    float *dDl = Dl + kC * kNV, *Zs = dDl + kC * kNV, *DZ = Zs + kC * kNV;
+    // The state slices are stored transposed (row jj = value column j0 + jj, D + 4 floats), so the
+    // dot loops read them 16 bytes at a time along the key channels; dSn and dSs (and in the forward
+    // sweep dSn and Ss) swap roles after each chunk instead of being copied.
+    float *Ss = DZ + 2 * kC * kNV, *dSs = Ss + kNV * DKP, *dSn = dSs + kNV * DKP;
+    float *bt = dSn + kNV * DKP, *egl = bt + kC;
 
     constexpr int slices = D / kNV;
     int bid = blockIdx.x;
@@ -347,8 +350,8 @@ kda_bwd_state_kernel(const T *__restrict__ v, const float *__restrict__ beta, co
     const size_t soff = ((size_t)n * H + h) * D * D;
     for (int idx = tid; idx < D * kNV; idx += kBTs) {
         const int c = idx / kNV, jj = idx % kNV;
-        Ss[c * kSP + jj] = h0 ? h0[soff + (size_t)c * D + j0 + jj] : 0.f;
-        dSs[c * kSP + jj] = dhT ? dhT[soff + (size_t)c * D + j0 + jj] : 0.f;
+        Ss[jj * DKP + c] = h0 ? h0[soff + (size_t)c * D + j0 + jj] : 0.f;
+        dSs[jj * DKP + c] = dhT ? dhT[soff + (size_t)c * D + j0 + jj] : 0.f;
     }
 
     // A chunk's operands (from the prep kernel) by 16-byte cp.async, in two parts.  Part A (T, K^ and,
@@ -383,15 +386,19 @@ kda_bwd_state_kernel(const T *__restrict__ v, const float *__restrict__ beta, co
             const int r = idx / kNV, jj = idx % kNV;
             const size_t off = ((size_t)(t0 + r) * H + h) * D + j0 + jj;
             Vs[idx] = r < L ? Elem<T>::load(v + off) : 0.f;
-            if (bwd) dOs[idx] = r < L ? Elem<T>::load(dout + off) : 0.f;
+            if (bwd) {
+                const float dov = r < L ? Elem<T>::load(dout + off) : 0.f;
+                dOs[idx] = dov;
+                DZ[2 * idx] = dov;
+            }
         }
         if (tid < kC) bt[tid] = tid < L ? __ldg(beta + (size_t)(t0 + tid) * H + h) : 0.f;
         cp_async_wait<0>();
         __syncthreads();
     };
     // Register blocking (512 threads): for [C][kNV] tiles a thread owns column jj = tid % 16 of
-    // rows rp = tid / 16 and rp + 32; for [D][kNV] tiles column jj of channels rp + 32 k (forward
-    // sweep) or of the D / 32 adjacent channels from (D / 32) rp (reverse sweep).
+    // rows rp = tid / 16 and rp + 32; for the transposed state slices, row jj at channels rp + 32 k
+    // (forward sweep) or the D / 32 adjacent channels from (D / 32) rp (reverse sweep).
     const int jj = tid % kNV, rp = tid / kNV;
     constexpr int kCq = D / 32;
     // The row operands of the dot loops (rows of K o 2^G, K o 2^{G_L - G}, T: two per warp) are read
@@ -403,8 +410,8 @@ kda_bwd_state_kernel(const T *__restrict__ v, const float *__restrict__ beta, co
             const float4 *kr1 = reinterpret_cast<const float4 *>(sKt + (rp + 32) * DKP);
             for (int c4 = 0; c4 < D / 4; ++c4) {
                 const float4 x = kr0[c4], y = kr1[c4];
-                const float *sv = Ss + 4 * c4 * kSP + jj;
-                const float s0 = sv[0], s1 = sv[kSP], s2 = sv[2 * kSP], s3 = sv[3 * kSP];
+                const float4 sv = *reinterpret_cast<const float4 *>(Ss + jj * DKP + 4 * c4);
+                const float s0 = sv.x, s1 = sv.y, s2 = sv.z, s3 = sv.w;
                 a0 = fmaf(-x.x, s0, a0);
                 a1 = fmaf(-y.x, s0, a1);
                 a0 = fmaf(-x.y, s1, a0);
@@ -453,7 +460,7 @@ kda_bwd_state_kernel(const T *__restrict__ v, const float *__restrict__ beta, co
         __syncthreads();  // the previous chunk's reads of the staged tiles are done
         for (int idx = tid; idx < kNV * D; idx += kBTs) {
             const int jj = idx / D, c = idx % D;
-            rec[R::St + (size_t)(j0 + jj) * D + c] = Ss[c * kSP + jj];
+            rec[R::St + (size_t)(j0 + jj) * D + c] = Ss[jj * DKP + c];
         }
         stage_a(op, false);
         stage_b(op, t0, L, false);
@@ -461,20 +468,19 @@ kda_bwd_state_kernel(const T *__restrict__ v, const float *__restrict__ beta, co
         {  // S <- 2^{G_L} S + (K o 2^{G_L - G})^T Delta
             float acc[kCq];
 #pragma unroll
-            for (int q2 = 0; q2 < kCq; ++q2) acc[q2] = egl[rp + 32 * q2] * Ss[(rp + 32 * q2) * kSP + jj];
+            for (int q2 = 0; q2 < kCq; ++q2) acc[q2] = egl[rp + 32 * q2] * Ss[jj * DKP + rp + 32 * q2];
             for (int r = 0; r < kC; ++r) {
                 const float dl = Dl[r * kNV + jj];
 #pragma unroll
                 for (int q2 = 0; q2 < kCq; ++q2) acc[q2] = fmaf(sKh[r * DKP + rp + 32 * q2], dl, acc[q2]);
             }
 #pragma unroll
-            for (int q2 = 0; q2 < kCq; ++q2) dSn[(rp + 32 * q2) * kSP + jj] = acc[q2];
+            for (int q2 = 0; q2 < kCq; ++q2) dSn[jj * DKP + rp + 32 * q2] = acc[q2];
         }
         __syncthreads();
-        for (int idx = tid; idx < D * kNV; idx += kBTs) {
-            const int c = idx / kNV, jj = idx % kNV;
-            Ss[c * kSP + jj] = dSn[c * kSP + jj];
-        }
+        float *const s_next = dSn;  // the new state becomes S; its old buffer takes the next one
+        dSn = Ss;
+        Ss = s_next;
     }
 
     // ---- backward over the chunks, carrying dS (= dL/d state after the chunk)
@@ -485,10 +491,11 @@ kda_bwd_state_kernel(const T *__restrict__ v, const float *__restrict__ beta, co
         float *rec = recs + ((size_t)(cbase + ch) * H + h) * R::floats;
         const float *op = ops + ((size_t)(cbase + ch) * H + h) * O::floats;
         __syncthreads();
-        for (int idx = tid; idx < kNV * D; idx += kBTs) {
-            const int jj = idx / D, c = idx % D;
-            cp_async4(Ss + c * kSP + jj, rec + R::St + (size_t)(j0 + jj) * D + c);
-            rec[R::dSt + (size_t)(j0 + jj) * D + c] = dSs[c * kSP + jj];
+        for (int idx = tid; idx < kNV * D / 4; idx += kBTs) {  // S^T, dS'^T rows of the slice, 16 bytes at a time
+            const int jj = idx / (D / 4), c = 4 * (idx % (D / 4));
+            cp_async16(Ss + jj * DKP + c, rec + R::St + (size_t)(j0 + jj) * D + c);
+            *reinterpret_cast<float4 *>(rec + R::dSt + (size_t)(j0 + jj) * D + c) =
+                *reinterpret_cast<const float4 *>(dSs + jj * DKP + c);
         }
         stage_b(op, t0, L, true);
         x1_delta();
@@ -498,8 +505,8 @@ kda_bwd_state_kernel(const T *__restrict__ v, const float *__restrict__ beta, co
             const float4 *kr1 = reinterpret_cast<const float4 *>(sKh + (rp + 32) * DKP);
             for (int c4 = 0; c4 < D / 4; ++c4) {
                 const float4 x = kr0[c4], y = kr1[c4];
-                const float *dsv = dSs + 4 * c4 * kSP + jj;
-                const float s0 = dsv[0], s1 = dsv[kSP], s2 = dsv[2 * kSP], s3 = dsv[3 * kSP];
+                const float4 dsv = *reinterpret_cast<const float4 *>(dSs + jj * DKP + 4 * c4);
+                const float s0 = dsv.x, s1 = dsv.y, s2 = dsv.z, s3 = dsv.w;
                 a0 = fmaf(x.x, s0, a0);
                 a1 = fmaf(y.x, s0, a1);
                 a0 = fmaf(x.y, s1, a0);
@@ -549,6 +556,8 @@ kda_bwd_state_kernel(const T *__restrict__ v, const float *__restrict__ beta, co
             }
             Zs[rp * kNV + jj] = z0;
             Zs[(rp + 32) * kNV + jj] = z1;
+            DZ[2 * (rp * kNV + jj) + 1] = -bt[rp] * z0;
+            DZ[2 * ((rp + 32) * kNV + jj) + 1] = -bt[rp + 32] * z1;
             if (rp < L) Elem<T>::store(dv_out + ((size_t)(t0 + rp) * H + h) * D + j0 + jj, bt[rp] * z0);
             if (rp + 32 < L) Elem<T>::store(dv_out + ((size_t)(t0 + rp + 32) * H + h) * D + j0 + jj, bt[rp + 32] * z1);
         }
@@ -569,10 +578,12 @@ kda_bwd_state_kernel(const T *__restrict__ v, const float *__restrict__ beta, co
            // channels kCq rp .. (one 8- or 16-byte load of each operand row per step)
             const int ch0 = kCq * rp;
             float acc[kCq];
+            load_vec<kCq>(dSs + jj * DKP + ch0, acc);
 #pragma unroll
-            for (int q2 = 0; q2 < kCq; ++q2) acc[q2] = egl[ch0 + q2] * dSs[(ch0 + q2) * kSP + jj];
+            for (int q2 = 0; q2 < kCq; ++q2) acc[q2] *= egl[ch0 + q2];
             for (int r = 0; r < kC; ++r) {
-                const float dov = dOs[r * kNV + jj], zb = -bt[r] * Zs[r * kNV + jj];
+                const float2 dz = *reinterpret_cast<const float2 *>(DZ + 2 * (r * kNV + jj));
+                const float dov = dz.x, zb = dz.y;
                 float qv[kCq], kv[kCq];
                 load_vec<kCq>(sQt + r * DKP + ch0, qv);
                 load_vec<kCq>(sKt + r * DKP + ch0, kv);
@@ -583,19 +594,18 @@ kda_bwd_state_kernel(const T *__restrict__ v, const float *__restrict__ beta, co
                 }
             }
 #pragma unroll
-            for (int q2 = 0; q2 < kCq; ++q2) dSn[(ch0 + q2) * kSP + jj] = acc[q2];
+            for (int q2 = 0; q2 < kCq; ++q2) dSn[jj * DKP + ch0 + q2] = acc[q2];
         }
         __syncthreads();
-        for (int idx = tid; idx < D * kNV; idx += kBTs) {
-            const int c = idx / kNV, jj = idx % kNV;
-            dSs[c * kSP + jj] = dSn[c * kSP + jj];
-        }
+        float *const ds_next = dSn;  // the new dS becomes dS; its old buffer takes the next one
+        dSn = dSs;
+        dSs = ds_next;
     }
     __syncthreads();
     if (dh0)
         for (int idx = tid; idx < D * kNV; idx += kBTs) {
             const int c = idx / kNV, jj = idx % kNV;
-            dh0[soff + (size_t)c * D + j0 + jj] = dSs[c * kSP + jj];
+            dh0[soff + (size_t)c * D + j0 + jj] = dSs[jj * DKP + c];
         }
 }
 
