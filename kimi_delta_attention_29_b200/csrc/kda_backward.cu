@@ -614,6 +614,41 @@ constexpr int kCBP = kCB + 1;        // padded row stride of the [C][kCB] channe
 constexpr int kRowsPerWarp = kC / (kBT2 / 32);
 constexpr int CP4 = kC + 4;          // 16-byte aligned row stride of the chunk kernel's [C][C] tiles
 
+// dO rows t0 .. t0 + L - 1 of head h as fp32 [C][D] in dst (rows >= L zero), staged by 16-byte
+// cp.async (each row starts 16-byte aligned: the entry point checks dout, and a row is D elements).
+// stage_dout_issue goes before the caller's commit; stage_dout_finish after its wait and barrier.
+// fp32 rows land in place; bf16 rows land in dst's upper half and are widened in place (through
+// registers, with a barrier between the reads and the writes, and one at the end).
+template <int D, typename T>
+__device__ __forceinline__ void stage_dout_issue(const T *dout, int64_t t0, int L, int H, int h, float *dst) {
+    constexpr int kPieces = D * (int)sizeof(T) / 16;
+    char *raw = reinterpret_cast<char *>(dst) + (sizeof(T) == 2 ? (size_t)kC * D * 2 : 0);
+    for (int p = threadIdx.x; p < L * kPieces; p += kBT2) {
+        const int r = p / kPieces, b = p % kPieces;
+        cp_async16(raw + ((size_t)r * kPieces + b) * 16,
+                   reinterpret_cast<const char *>(dout + ((size_t)(t0 + r) * H + h) * D) + 16 * b);
+    }
+    if constexpr (sizeof(T) == 4)
+        for (int idx = L * D + threadIdx.x; idx < kC * D; idx += kBT2) dst[idx] = 0.f;
+}
+template <int D, typename T>
+__device__ __forceinline__ void stage_dout_finish(int L, float *dst) {
+    if constexpr (sizeof(T) == 2) {
+        constexpr int kPer = kC * D / kBT2;
+        const __nv_bfloat16 *raw = reinterpret_cast<const __nv_bfloat16 *>(dst + kC * D / 2);
+        float w[kPer];
+#pragma unroll
+        for (int u = 0; u < kPer; ++u) {
+            const int idx = threadIdx.x + u * kBT2;
+            w[u] = idx < L * D ? __bfloat162float(raw[idx]) : 0.f;
+        }
+        __syncthreads();
+#pragma unroll
+        for (int u = 0; u < kPer; ++u) dst[threadIdx.x + u * kBT2] = w[u];
+        __syncthreads();
+    }
+}
+
 // Shared memory of the pair kernel (floats): T, dT / dA, W; three staged [C][D]-sized record tiles;
 // Abar.
 template <int D>
@@ -685,13 +720,10 @@ kda_bwd_pair_kernel(const float *__restrict__ beta, const int4 *__restrict__ tab
         dbs[tid] = acc;
     }
     __syncthreads();  // dT complete; dDelta and X1^T no longer read
-    // ---- staging: Delta^T [D][C] over X1^T, dO [C][D] over dDelta; W = dT T^T meanwhile
+    // ---- staging: Delta^T [D][C] over X1^T, dO [C][D] over dDelta (cp.async); W = dT T^T meanwhile
     for (int idx = 4 * tid; idx < kC * D; idx += 4 * kBT2) cp_async16(U1 + idx, rec + R::Dt + idx);
+    stage_dout_issue<D, T>(dout, t0, L, H, h, U0);
     cp_async_commit();
-    for (int idx = tid; idx < kC * D; idx += kBT2) {
-        const int r = idx / D, j = idx % D;
-        U0[idx] = r < L ? Elem<T>::load(dout + ((size_t)(t0 + r) * H + h) * D + j) : 0.f;
-    }
     {  // W = dT T^T (T is stored with zeros above its diagonal, so the sums run over all m)
         float acc[4][2] = {};
         for (int m = 0; m < kC; ++m) {
@@ -710,7 +742,8 @@ kda_bwd_pair_kernel(const float *__restrict__ beta, const int4 *__restrict__ tab
         }
     }
     cp_async_wait<0>();
-    __syncthreads();  // W, dO and Delta^T in place; dT no longer read
+    __syncthreads();  // W and Delta^T in place; dT no longer read
+    stage_dout_finish<D, T>(L, U0);
     // dP [C][C] over Z (read only by dbs, before the first barrier), row stride kC with the column
     // XOR-ed by the row's low five bits: row writes and column reads both hit 32 distinct banks
     float *Ps = U2;
@@ -813,7 +846,7 @@ kda_bwd_chunk_kernel(const T *__restrict__ q, const T *__restrict__ k, const flo
     const int c = cb * kCB + lane;  // this lane's channel in the per-(row, channel) phase
 
     // ---- staging, all in flight at once: dA, dP (pair kernel); Delta, Z and the S^T, dS'^T blocks
-    // (state pass) by cp.async; beta, dO and this block's K, Q and clamped base-2 log gate
+    // (state pass) and dO by cp.async; beta and this block's K, Q and clamped base-2 log gate
     for (int p = tid; p < kC * kC / 4; p += kBT2) {
         const int r = p / (kC / 4), i = 4 * (p % (kC / 4));
         cp_async16(Mm + r * CP4 + i, rec + R::dA + r * kC + i);
@@ -830,6 +863,7 @@ kda_bwd_chunk_kernel(const T *__restrict__ q, const T *__restrict__ k, const flo
         cp_async16(Ub + idx, rec + R::St + off);
         cp_async16(Ud + idx, rec + R::dSt + off);
     }
+    stage_dout_issue<D, T>(dout, t0, L, H, h, U0);
     cp_async_commit();
     if (tid < kC) bt[tid] = tid < L ? __ldg(beta + (size_t)(t0 + tid) * H + h) : 0.f;
     for (int idx = tid; idx < kC * kCB; idx += kBT2) {  // warp-uniform row r, lane = channel cc
@@ -850,12 +884,9 @@ kda_bwd_chunk_kernel(const T *__restrict__ q, const T *__restrict__ k, const flo
         const unsigned cm = __ballot_sync(0xffffffffu, clamped);
         if (cc == 0) cmask[r] = cm;
     }
-    for (int idx = tid; idx < kC * D; idx += kBT2) {
-        const int r = idx / D, j = idx % D;
-        U0[idx] = r < L ? Elem<T>::load(dout + ((size_t)(t0 + r) * H + h) * D + j) : 0.f;
-    }
     cp_async_wait<0>();
     __syncthreads();
+    stage_dout_finish<D, T>(L, U0);
     if (tid < kCB) {  // running gate per channel of the block
         float acc = 0.f;
         for (int r = 0; r < kC; ++r) {
