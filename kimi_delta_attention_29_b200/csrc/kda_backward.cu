@@ -24,13 +24,14 @@
 //  * kda_bwd_prep_kernel - one CTA per (chunk, head), all chunks in parallel: Abar, P, T and the
 //    decayed rows K o 2^G, Q o 2^G, K o 2^{G_L - G} of the chunk, once.
 //  * kda_bwd_state_kernel - one CTA per (sequence, head, 16 value columns), sequential over chunks:
-//    recomputes the chunk-start states (forward pass), then walks the chunks backwards carrying dS,
+//    recomputes the chunk-start states (a forward sweep, unless the tensor-core forward saved them
+//    into the records), then walks the chunks backwards carrying dS,
 //    with only its 16-column products per chunk.  Value columns of S and dS evolve independently,
 //    so slices need no communication.  Per chunk it writes dv and a record of S, dS', Z, dDelta,
 //    X1 and Delta for the pair and chunk kernels.
 //  * kda_bwd_pair_kernel - one CTA per (chunk, head), all chunks in parallel: the chunk's 64 x 64
 //    products dT, dP, W and dA from the record and the prep kernel's T, once per chunk-head; writes
-//    dbeta, and dA, dP into the record.
+//    dbeta, and dA, dP and their transposes into the record.
 //  * kda_bwd_chunk_kernel - one CTA per (chunk, head, 32 key channels), all chunks in parallel:
 //    the per-channel state products and decayed Gram terms; writes dq, dk and dlog_alpha.
 //    Every output element has one writer: deterministic.
